@@ -1,0 +1,237 @@
+/*
+ * tri_evict.h -- C ABI of a B200 (sm_100a) library for TriAttention-style
+ * KV-cache eviction: fold the offset average into one weight per band, score
+ * every cached key, keep the top B keys per (layer, KV head, sequence) and
+ * compact K and V to the survivors.
+ *
+ * Method source: the page "The future-offset average in TriAttention can be
+ * precomputed" (hozhoke.com); budget default from the TriAttention README
+ * (github.com/WeianMao/triattention).
+ *
+ * Conventions used by every call:
+ *  - "device" pointers are CUDA global memory of the device that owns the
+ *    cache (the library launches on the device of desc->k, or of q_center for
+ *    the fold); "host" pointers are ordinary CPU memory read during the call.
+ *  - The caller allocates and owns every buffer.  The library never allocates
+ *    or frees memory and never synchronises the stream, except
+ *    tri_read_device_status, which reads a status word and waits for it.
+ *  - Device calls are asynchronous on `stream` (NULL = legacy default stream).
+ *    Pointers must stay valid until the stream reaches the work.
+ *  - Arguments are checked on the host before anything is launched; a call
+ *    that returns an error has launched nothing (TRI_ERR_CUDA excepted, which
+ *    reports a launch failure).  Device code never traps: problems it can only
+ *    see on the device (a page id out of range, a non-finite center, a wait
+ *    that timed out) set bits in a per-device status word read by
+ *    tri_read_device_status.
+ *  - bf16 tensors hold IEEE binary32 values truncated to their top 16 bits
+ *    (round-to-nearest-even when produced), head_dim = 128 contiguous
+ *    elements per row, rows 16-byte aligned.
+ *
+ * A "unit" is one (layer l, KV head h, sequence b).  Units are numbered
+ *     u = (l * num_kv_heads + h) * batch + b.
+ * Per-unit outputs (scores, kept indices, compacted rows) are stored in that
+ * order.
+ */
+#ifndef TRI_EVICT_H
+#define TRI_EVICT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the same pointer type). */
+typedef struct CUstream_st* tri_stream_t;
+
+typedef enum tri_status {
+  TRI_OK = 0,
+  TRI_ERR_INVALID_ARG = 1,    /* null pointer, bad size, bad alignment, inconsistent lengths */
+  TRI_ERR_UNSUPPORTED = 2,    /* a valid request outside what the kernels implement (head_dim != 128, ...) */
+  TRI_ERR_WORKSPACE = 3,      /* workspace smaller than tri_workspace_size() */
+  TRI_ERR_CUDA = 4,           /* a CUDA runtime call failed; see tri_last_cuda_error() */
+  TRI_ERR_DEVICE_CHECK = 5,   /* tri_read_device_status: a device-side check failed */
+  TRI_ERR_DEVICE_TIMEOUT = 6  /* tri_read_device_status: a bounded device wait gave up */
+} tri_status;
+
+/* Which two coordinates of a head vector form rotary band f (0 <= f < d/2).
+ * The page says only that the rotation turns two coordinates at a time.
+ * HALF: (f, f + d/2), the rotate-half convention of Llama/Qwen checkpoints.
+ * INTERLEAVED: (2f, 2f + 1). */
+typedef enum tri_pairing { TRI_PAIRING_HALF = 0, TRI_PAIRING_INTERLEAVED = 1 } tri_pairing;
+
+typedef enum tri_layout {
+  /* Row (l, h, b, i) at element  l*stride_layer + h*stride_head + b*stride_seq + i*128.
+   * Every sequence has seq_len keys. */
+  TRI_LAYOUT_CONTIG = 0,
+  /* Row (l, h, b, i) at element  l*stride_layer + h*stride_head + (cu_seqlens[b] + i)*128.
+   * Sequence b has cu_seqlens[b+1] - cu_seqlens[b] keys. */
+  TRI_LAYOUT_RAGGED = 1,
+  /* Pages of block_size tokens, each page [block_size][num_kv_heads][128] contiguous.
+   * Row (l, h, b, i) at element
+   *   l*stride_layer + block_table[b*max_blocks_per_seq + i/block_size]*stride_block
+   *   + (i % block_size)*num_kv_heads*128 + h*128.
+   * Sequence b has seq_lens[b] keys. */
+  TRI_LAYOUT_PAGED = 2
+} tri_layout;
+
+typedef enum tri_compact_mode {
+  /* k_out/v_out [units][B][128]: row j of unit u is the unit's kept[u][j]-th
+   * row.  Rows j >= kept_count[u] are left untouched. */
+  TRI_COMPACT_OUT_OF_PLACE = 0,
+  /* In place, in the cache itself ("hole fill"): in a unit with n > B keys,
+   * the kept keys with index < B stay where they are, and the evicted
+   * positions below B, in ascending order, receive the kept keys with index
+   * >= B, in ascending order.  Afterwards the unit's first B rows are its
+   * survivors; the caller shortens the sequence to B (and may release whole
+   * pages past it).  Units with n <= B are not touched. */
+  TRI_COMPACT_IN_PLACE_HOLEFILL = 1
+} tri_compact_mode;
+
+/* Parameters of the offline fold. */
+typedef struct tri_fold_params {
+  int head_dim;            /* d; must be 128 */
+  double theta;            /* rotary base; omega_f = theta^(-2f/d); > 0 */
+  const double* offsets;   /* HOST array: the offset schedule D (a multiset; finite values) */
+  int n_offsets;           /* |D|, 1 .. TRI_MAX_OFFSETS */
+  double delta0;           /* the kept distance Delta of the score, one scalar per event (0 by default) */
+  tri_pairing pairing;
+} tri_fold_params;
+
+#define TRI_MAX_OFFSETS 2048
+#define TRI_MAX_BATCH 256
+#define TRI_HEAD_DIM 128
+
+/* Where the cache lives.  All strides are in bf16 elements and must be
+ * multiples of 8 (16 bytes).  V uses the same layout and strides as K. */
+typedef struct tri_cache_desc {
+  tri_layout layout;
+  int num_layers;          /* L >= 1 */
+  int num_kv_heads;        /* H >= 1 (PAGED: H divides 16 and block_size*H <= 128) */
+  int head_dim;            /* must be 128 */
+  int batch;               /* sequences, 1 .. TRI_MAX_BATCH */
+  int max_seq_len;         /* capacity of a score row; 0 = the longest sequence */
+  const void* k;           /* device bf16 key cache (16-byte aligned) */
+  const void* v;           /* device bf16 value cache; may be NULL for scoring/selection */
+  int64_t stride_layer;
+  int64_t stride_head;     /* CONTIG / RAGGED */
+  int64_t stride_seq;      /* CONTIG */
+  int64_t stride_block;    /* PAGED: elements between pages (>= block_size*H*128) */
+  int seq_len;             /* CONTIG: keys per unit (>= 0) */
+  const int32_t* cu_seqlens;   /* RAGGED: HOST [batch+1], cu_seqlens[0] = 0, non-decreasing */
+  const int32_t* seq_lens;     /* PAGED: HOST [batch] keys per sequence */
+  const int32_t* block_table;  /* PAGED: DEVICE [batch][max_blocks_per_seq] page ids */
+  int max_blocks_per_seq;  /* PAGED */
+  int block_size;          /* PAGED: tokens per page */
+  int num_blocks;          /* PAGED: pages in the pool; ids outside [0, num_blocks) are
+                              skipped on the device and flagged (TRI_ERR_DEVICE_CHECK) */
+} tri_cache_desc;
+
+/* ---------------------------------------------------------------- fold */
+
+/* Fold the offset average into one real weight vector per center
+ * (page "The future-offset average in TriAttention can be precomputed",
+ * section "The averaging step - the one we improve": the offset weight
+ * W_f = (1/|D|) sum_{delta in D} e^{i omega_f delta}, the offset-averaged center
+ * mu'_f = E[q_f] W_f, and the real 2x2 per-band map of its closing remark).
+ *
+ * For each center c and band f (coordinates re(f), im(f) per `pairing`):
+ *     a_f = E[q_f] * W_f * e^{i omega_f delta0},   E[q_f] = q[re] + i q[im]
+ *     w[c][re(f)] = Re a_f,   w[c][im(f)] = Im a_f
+ * so that for a key k, Re sum_f a_f conj(k_f) = sum_j w[j] k[j] is the
+ * offset-averaged trigonometric score.  Computed on the device in fp64,
+ * stored as fp32.
+ *
+ * q_center: device fp32 [n_centers][128]; w_out: device fp32 [n_centers][128].
+ * Centers are indexed (l * num_kv_heads + h) by the other calls.
+ * A non-finite center sets TRI_ERR_DEVICE_CHECK in the status word. */
+tri_status tri_fold_weights(const tri_fold_params* params, const float* q_center,
+                            int n_centers, float* w_out, tri_stream_t stream);
+
+/* ---------------------------------------------------------------- score */
+
+/* Row stride (in floats) of the score matrix for `desc`: the longest row
+ * rounded up to a multiple of 4.  Scores are [units][stride]. */
+int64_t tri_score_row_stride(const tri_cache_desc* desc);
+
+/* Score every cached key (page above, the folded form: one evaluation per key
+ * instead of one per offset):
+ *     scores[u][i] = sum_{j<128} w[l*H + h][j] * float(K_u[i][j])
+ * an fp32 dot product of the unit's folded weight vector with the bf16 key,
+ * i.e. the offset-averaged trigonometric score S~_trig of the key.
+ * w: device fp32 [L*H][128] from tri_fold_weights.  scores: device fp32
+ * [units][tri_score_row_stride(desc)]; entries i >= n_u are not written. */
+tri_status tri_score_keys(const tri_cache_desc* desc, const float* w, float* scores,
+                          tri_stream_t stream);
+
+/* ---------------------------------------------------------------- select */
+
+/* Keep the highest-scoring keys (same page, opening section: the cache keeps
+ * the highest-scoring keys within a budget; the budget B is TriAttention's KV
+ * budget, default 2048).  Per unit with n keys: the top min(B, n) keys in the
+ * order (score descending, index ascending), NaN ranked lowest and -0 equal to
+ * +0, written as ASCENDING key indices to kept[u][0 .. min(B,n)), and
+ * kept_count[u] = min(B, n).  Entries past kept_count are not written.
+ * scores: device fp32 [units][tri_score_row_stride(desc)].
+ * kept: device int32 [units][B]; kept_count: device int32 [units].
+ * B >= 1.  Needs no workspace. */
+tri_status tri_select_topk(const tri_cache_desc* desc, const float* scores, int B,
+                           int32_t* kept, int32_t* kept_count, tri_stream_t stream);
+
+/* ---------------------------------------------------------------- compact */
+
+/* Compact K and V to the kept keys (bit copies).  See tri_compact_mode for
+ * the two layouts.  kept / kept_count as written by tri_select_topk with the
+ * same desc and B.  OUT_OF_PLACE: k_out, v_out device bf16 [units][B][128]
+ * (16-byte aligned).  IN_PLACE_HOLEFILL: k_out and v_out must be NULL; the
+ * cache (desc->k, desc->v) is modified, so they must point to writable
+ * memory; B <= 16384.  desc->v must be non-NULL. */
+tri_status tri_compact_kv(const tri_cache_desc* desc, const int32_t* kept,
+                          const int32_t* kept_count, int B, tri_compact_mode mode,
+                          void* k_out, void* v_out, tri_stream_t stream);
+
+/* ---------------------------------------------------------------- fused */
+
+/* Bytes of workspace tri_compress needs for `desc` (the score matrix). */
+tri_status tri_workspace_size(const tri_cache_desc* desc, int B, size_t* bytes);
+
+/* score -> select -> compact in one call (three kernels, no host sync).
+ * Same arguments as the three calls; the scores live in `workspace`
+ * (device, >= tri_workspace_size bytes, 256-byte aligned). */
+tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B,
+                        tri_compact_mode mode, int32_t* kept, int32_t* kept_count,
+                        void* k_out, void* v_out, void* workspace, size_t workspace_bytes,
+                        tri_stream_t stream);
+
+/* ---------------------------------------------------------------- status */
+
+/* Device-side status bits (OR-ed by kernels). */
+#define TRI_DEVFLAG_BAD_PAGE      0x1u  /* a page id outside [0, num_blocks) was skipped */
+#define TRI_DEVFLAG_NONFINITE     0x2u  /* a non-finite center or offset in the fold */
+#define TRI_DEVFLAG_TIMEOUT       0x4u  /* a bounded wait inside a kernel gave up */
+#define TRI_DEVFLAG_BAD_KEPT      0x8u  /* compaction met a kept index outside [0, n) */
+
+/* Wait for `stream`, then read the status word of the device that owns
+ * `stream` (the current device for NULL) into *flags, and zero it if `clear`.
+ * Returns TRI_ERR_DEVICE_TIMEOUT if the timeout bit is set, else
+ * TRI_ERR_DEVICE_CHECK if any bit is set, else TRI_OK. */
+tri_status tri_read_device_status(tri_stream_t stream, uint32_t* flags, int clear);
+
+/* Human-readable name of a status code (static string). */
+const char* tri_status_string(tri_status status);
+
+/* The cudaError_t behind the most recent TRI_ERR_CUDA on this thread (0 if none). */
+int tri_last_cuda_error(void);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t tri_kernel_launches(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* tri_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRI_EVICT_H */

@@ -1,0 +1,65 @@
+"""Build libtri_evict.so in-tree with nvcc for sm_100a.
+
+    python -m rope_aware_key_b200.build [--force] [-D NAME=VALUE ...]
+
+One translation unit (csrc/tri_evict.cu includes the kernel headers), static
+CUDA runtime, -lineinfo.  ptxas resource usage goes to _build/ptxas.txt.
+"""
+from __future__ import annotations
+
+import glob
+import os
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+LIB = os.path.join(PKG, "libtri_evict.so")
+INCLUDE = os.path.join(ROOT, "include")
+MAIN = os.path.join(PKG, "csrc", "tri_evict.cu")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def _sources():
+    return (glob.glob(os.path.join(PKG, "csrc", "*.cu")) + glob.glob(os.path.join(PKG, "csrc", "*.cuh"))
+            + glob.glob(os.path.join(INCLUDE, "*.h")))
+
+
+def _nvcc() -> str:
+    for c in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", "nvcc"):
+        if c and (os.path.sep not in c or os.path.exists(c)):
+            return c
+    return "nvcc"
+
+
+def needs_build(out: str = LIB) -> bool:
+    if not os.path.exists(out):
+        return True
+    t = os.path.getmtime(out)
+    return any(os.path.getmtime(s) > t for s in _sources())
+
+
+def build(force: bool = False, defines=(), out: str = LIB, verbose: bool = False) -> str:
+    if not force and not defines and not needs_build(out):
+        return out
+    os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared",
+           "-cudart", "static", "-Xptxas", "-v", "-I", INCLUDE, "-I", os.path.join(PKG, "csrc"),
+           *[f"-D{d}" for d in defines], "-o", tmp, MAIN]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    with open(os.path.join(ROOT, "_build", "ptxas.txt"), "w") as f:
+        f.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError(f"nvcc failed ({res.returncode})")
+    if verbose:
+        sys.stdout.write(res.stderr)
+    os.replace(tmp, out)
+    return out
+
+
+if __name__ == "__main__":
+    args = sys.argv[1:]
+    defs = [args[i + 1] for i, a in enumerate(args) if a == "-D"]
+    build(force="--force" in args or bool(defs), defines=defs, verbose=True)

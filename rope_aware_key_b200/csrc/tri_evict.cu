@@ -1,0 +1,397 @@
+// C ABI of the library (declared in include/tri_evict.h): argument checks on
+// the host, geometry packing, and the kernel launches.  Everything runs on
+// the caller's stream; nothing is allocated, freed or synchronised here
+// (tri_read_device_status excepted, which waits for its own small copy).
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "tri_evict.h"
+#include "common.cuh"
+#include "fold.cuh"
+#include "score.cuh"
+#include "select.cuh"
+#include "compact.cuh"
+
+namespace {
+
+using tri::Geom;
+
+std::atomic<uint64_t> g_launches{0};
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int score_blocks_per_sm = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+tri_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return TRI_ERR_CUDA;
+}
+
+#define TRI_CUDA(call)                               \
+  do {                                               \
+    cudaError_t e_ = (call);                         \
+    if (e_ != cudaSuccess) return cuda_fail(e_);     \
+  } while (0)
+
+// Make the device that owns `ptr` current (the library's runtime keeps its
+// own notion of the current device), and set up per-device state once.
+tri_status use_device_of(const void* ptr, int* dev_out) {
+  int dev = -1;
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, ptr);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return TRI_ERR_INVALID_ARG;
+  dev = attr.device;
+  if (dev < 0 || dev >= kMaxDevices) return TRI_ERR_UNSUPPORTED;
+  int cur = -1;
+  TRI_CUDA(cudaGetDevice(&cur));
+  if (cur != dev) TRI_CUDA(cudaSetDevice(dev));
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    TRI_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    TRI_CUDA(cudaFuncSetAttribute(tri::score::score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tri::score::kSmemBytes)));
+    TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.score_blocks_per_sm, tri::score::score_kernel,
+                                                           tri::score::kThreads, tri::score::kSmemBytes));
+    if (d.score_blocks_per_sm < 1) return TRI_ERR_UNSUPPORTED;
+    const int fill_smem = ((tri::compact::kMaxFillBudget + 31) / 32 + tri::compact::kMaxFillBudget) * 4;
+    TRI_CUDA(cudaFuncSetAttribute(tri::compact::holefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  fill_smem));
+    d.ready = true;
+  }
+  *dev_out = dev;
+  return TRI_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validate `c` and fill `g` (everything except the per-call pointers the
+// kernels take separately).  `need_v`: compaction needs V.
+tri_status make_geom(const tri_cache_desc* c, bool need_v, Geom* g) {
+  if (!c || !g) return TRI_ERR_INVALID_ARG;
+  if (c->head_dim != TRI_HEAD_DIM) return TRI_ERR_UNSUPPORTED;
+  if (c->num_layers < 1 || c->num_kv_heads < 1 || c->batch < 1) return TRI_ERR_INVALID_ARG;
+  if (c->batch > TRI_MAX_BATCH) return TRI_ERR_UNSUPPORTED;
+  if (!c->k || !aligned16(c->k)) return TRI_ERR_INVALID_ARG;
+  if (need_v && (!c->v || !aligned16(c->v))) return TRI_ERR_INVALID_ARG;
+  if (c->v && !aligned16(c->v)) return TRI_ERR_INVALID_ARG;
+  const int64_t L = c->num_layers, H = c->num_kv_heads, Bt = c->batch;
+  if ((L * H * Bt) > (int64_t{1} << 31) - 1) return TRI_ERR_UNSUPPORTED;
+  if (c->stride_layer < 0 || (c->stride_layer % 8) != 0) return TRI_ERR_INVALID_ARG;
+  if (L > 1 && c->stride_layer == 0) return TRI_ERR_INVALID_ARG;
+
+  std::memset(g, 0, sizeof(*g));
+  g->layout = c->layout;
+  g->L = c->num_layers;
+  g->H = c->num_kv_heads;
+  g->batch = c->batch;
+  g->sL = c->stride_layer;
+  g->k = static_cast<const uint16_t*>(c->k);
+  g->v = static_cast<const uint16_t*>(c->v);
+
+  int64_t max_len = 0;
+  switch (c->layout) {
+    case TRI_LAYOUT_CONTIG: {
+      if (c->seq_len < 0) return TRI_ERR_INVALID_ARG;
+      if (c->stride_head < 0 || c->stride_seq < 0 || (c->stride_head % 8) || (c->stride_seq % 8))
+        return TRI_ERR_INVALID_ARG;
+      if ((H > 1 && c->stride_head == 0) || (Bt > 1 && c->stride_seq == 0)) return TRI_ERR_INVALID_ARG;
+      for (int b = 0; b < c->batch; ++b) g->len[b] = c->seq_len;
+      g->sH = c->stride_head;
+      g->sB = c->stride_seq;
+      max_len = c->seq_len;
+      break;
+    }
+    case TRI_LAYOUT_RAGGED: {
+      if (!c->cu_seqlens) return TRI_ERR_INVALID_ARG;
+      if (c->cu_seqlens[0] != 0) return TRI_ERR_INVALID_ARG;
+      if (c->stride_head < 0 || (c->stride_head % 8)) return TRI_ERR_INVALID_ARG;
+      if (H > 1 && c->stride_head == 0) return TRI_ERR_INVALID_ARG;
+      for (int b = 0; b < c->batch; ++b) {
+        const int32_t n = c->cu_seqlens[b + 1] - c->cu_seqlens[b];
+        if (n < 0) return TRI_ERR_INVALID_ARG;
+        g->len[b] = n;
+        g->start[b] = c->cu_seqlens[b];
+        if (n > max_len) max_len = n;
+      }
+      g->sH = c->stride_head;
+      break;
+    }
+    case TRI_LAYOUT_PAGED: {
+      if (!c->seq_lens || !c->block_table) return TRI_ERR_INVALID_ARG;
+      if (c->block_size < 1 || c->max_blocks_per_seq < 1 || c->num_blocks < 1) return TRI_ERR_INVALID_ARG;
+      if (16 % c->num_kv_heads != 0 || c->block_size * c->num_kv_heads > tri::score::kTileRows)
+        return TRI_ERR_UNSUPPORTED;
+      const int64_t page = int64_t{c->block_size} * c->num_kv_heads * TRI_HEAD_DIM;
+      if (c->stride_block < page || (c->stride_block % 8)) return TRI_ERR_INVALID_ARG;
+      for (int b = 0; b < c->batch; ++b) {
+        const int32_t n = c->seq_lens[b];
+        if (n < 0 || int64_t{n} > int64_t{c->max_blocks_per_seq} * c->block_size) return TRI_ERR_INVALID_ARG;
+        g->len[b] = n;
+        if (n > max_len) max_len = n;
+      }
+      g->block_size = c->block_size;
+      g->max_blocks = c->max_blocks_per_seq;
+      g->num_blocks = c->num_blocks;
+      g->sB = c->stride_block;
+      g->block_table = c->block_table;
+      if (reinterpret_cast<uintptr_t>(c->block_table) & 3u) return TRI_ERR_INVALID_ARG;
+      break;
+    }
+    default:
+      return TRI_ERR_INVALID_ARG;
+  }
+  if (c->max_seq_len < 0) return TRI_ERR_INVALID_ARG;
+  if (c->max_seq_len > 0 && c->max_seq_len < max_len) return TRI_ERR_INVALID_ARG;
+  const int64_t cap = c->max_seq_len > 0 ? c->max_seq_len : max_len;
+  if (cap > (int64_t{1} << 30)) return TRI_ERR_UNSUPPORTED;
+  g->score_stride = (cap + 3) & ~int64_t{3};
+  return TRI_OK;
+}
+
+// Score tiles: per sequence, 128-key chunks (CONTIG / RAGGED) or pages (PAGED).
+int64_t fill_tile_prefix(Geom* g) {
+  int32_t acc = 0;
+  for (int b = 0; b < g->batch; ++b) {
+    g->tile_prefix[b] = acc;
+    const int per = g->layout == TRI_LAYOUT_PAGED ? g->block_size : tri::score::kTileRows;
+    acc += (g->len[b] + per - 1) / per;
+  }
+  g->tile_prefix[g->batch] = acc;
+  const int64_t outer = g->layout == TRI_LAYOUT_PAGED ? g->L : int64_t{g->L} * g->H;
+  return outer * acc;
+}
+
+tri_status launch_score(const Geom& g0, const float* w, float* scores, int dev, cudaStream_t s) {
+  Geom g = g0;
+  const int64_t ntiles = fill_tile_prefix(&g);
+  if (ntiles == 0) return TRI_OK;
+  if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].score_blocks_per_sm;
+  const int grid = static_cast<int>(ntiles < resident ? ntiles : resident);
+  tri::score::score_kernel<<<grid, tri::score::kThreads, tri::score::kSmemBytes, s>>>(
+      g, w, scores, static_cast<int>(ntiles));
+  ++g_launches;
+  TRI_CUDA(cudaGetLastError());
+  return TRI_OK;
+}
+
+tri_status launch_select(const Geom& g, const float* scores, int B, int32_t* kept, int32_t* kept_count,
+                         cudaStream_t s) {
+  const int units = g.L * g.H * g.batch;
+  tri::select::Args a{scores, kept, kept_count, B};
+  if (g.score_stride >= 8192) {
+    tri::select::select_kernel<1024><<<units, 1024, 0, s>>>(g, a);
+  } else {
+    tri::select::select_kernel<256><<<units, 256, 0, s>>>(g, a);
+  }
+  ++g_launches;
+  TRI_CUDA(cudaGetLastError());
+  return TRI_OK;
+}
+
+tri_status launch_compact(const Geom& g, const int32_t* kept, const int32_t* kept_count, int B,
+                          tri_compact_mode mode, void* k_out, void* v_out, int dev, cudaStream_t s) {
+  const int units = g.L * g.H * g.batch;
+  if (mode == TRI_COMPACT_OUT_OF_PLACE) {
+    const int64_t rows = int64_t{units} * B;
+    if (rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+    const int64_t want = (rows * 16 + tri::compact::kGatherThreads - 1) / tri::compact::kGatherThreads;
+    const int64_t cap = int64_t{g_dev[dev].sms} * 8 * 4;
+    const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+    tri::compact::gather_kernel<<<grid, tri::compact::kGatherThreads, 0, s>>>(
+        g, kept, kept_count, B, static_cast<uint16_t*>(k_out), static_cast<uint16_t*>(v_out), rows);
+  } else {
+    const size_t smem = static_cast<size_t>((B + 31) / 32 + B) * 4;
+    tri::compact::holefill_kernel<<<units, tri::compact::kFillThreads, smem, s>>>(
+        g, kept, B, const_cast<uint16_t*>(g.k), const_cast<uint16_t*>(g.v));
+  }
+  ++g_launches;
+  TRI_CUDA(cudaGetLastError());
+  return TRI_OK;
+}
+
+tri_status check_compact_args(const tri_cache_desc* desc, const int32_t* kept, const int32_t* kept_count,
+                              int B, tri_compact_mode mode, void* k_out, void* v_out) {
+  if (!kept || !kept_count || B < 1) return TRI_ERR_INVALID_ARG;
+  if (mode == TRI_COMPACT_OUT_OF_PLACE) {
+    if (!k_out || !v_out || !aligned16(k_out) || !aligned16(v_out)) return TRI_ERR_INVALID_ARG;
+  } else if (mode == TRI_COMPACT_IN_PLACE_HOLEFILL) {
+    if (k_out || v_out) return TRI_ERR_INVALID_ARG;
+    if (B > tri::compact::kMaxFillBudget) return TRI_ERR_UNSUPPORTED;
+  } else {
+    return TRI_ERR_INVALID_ARG;
+  }
+  (void)desc;
+  return TRI_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tri_status tri_fold_weights(const tri_fold_params* p, const float* q_center, int n_centers, float* w_out,
+                            tri_stream_t stream) {
+  if (!p || !q_center || !w_out || n_centers < 1) return TRI_ERR_INVALID_ARG;
+  if (p->head_dim != TRI_HEAD_DIM) return TRI_ERR_UNSUPPORTED;
+  if (!p->offsets || p->n_offsets < 1) return TRI_ERR_INVALID_ARG;
+  if (p->n_offsets > TRI_MAX_OFFSETS) return TRI_ERR_UNSUPPORTED;
+  if (!(p->theta > 0.0) || !std::isfinite(p->theta) || !std::isfinite(p->delta0)) return TRI_ERR_INVALID_ARG;
+  if (p->pairing != TRI_PAIRING_HALF && p->pairing != TRI_PAIRING_INTERLEAVED) return TRI_ERR_INVALID_ARG;
+  for (int t = 0; t < p->n_offsets; ++t)
+    if (!std::isfinite(p->offsets[t])) return TRI_ERR_INVALID_ARG;
+  if (!aligned16(q_center) || !aligned16(w_out)) return TRI_ERR_INVALID_ARG;
+  int dev;
+  tri_status st = use_device_of(q_center, &dev);
+  if (st != TRI_OK) return st;
+  static tri::fold::Args a;   // large parameter block: built in static storage, copied by the launch
+  static std::mutex m;
+  std::lock_guard<std::mutex> lock(m);
+  a.q = q_center;
+  a.w = w_out;
+  a.n_centers = n_centers;
+  a.pairing = p->pairing;
+  a.theta = p->theta;
+  a.delta0 = p->delta0;
+  a.n_offsets = p->n_offsets;
+  std::memcpy(a.offsets, p->offsets, sizeof(double) * p->n_offsets);
+  tri::fold::fold_kernel<<<1, tri::fold::kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  ++g_launches;
+  TRI_CUDA(cudaGetLastError());
+  return TRI_OK;
+}
+
+int64_t tri_score_row_stride(const tri_cache_desc* desc) {
+  Geom g;
+  if (make_geom(desc, false, &g) != TRI_OK) return -1;
+  return g.score_stride;
+}
+
+tri_status tri_score_keys(const tri_cache_desc* desc, const float* w, float* scores, tri_stream_t stream) {
+  Geom g;
+  tri_status st = make_geom(desc, false, &g);
+  if (st != TRI_OK) return st;
+  if (!w || !scores || !aligned16(w) || !aligned16(scores)) return TRI_ERR_INVALID_ARG;
+  int dev;
+  st = use_device_of(desc->k, &dev);
+  if (st != TRI_OK) return st;
+  return launch_score(g, w, scores, dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+tri_status tri_select_topk(const tri_cache_desc* desc, const float* scores, int B, int32_t* kept,
+                           int32_t* kept_count, tri_stream_t stream) {
+  Geom g;
+  tri_status st = make_geom(desc, false, &g);
+  if (st != TRI_OK) return st;
+  if (!scores || !aligned16(scores) || !kept || !kept_count || B < 1) return TRI_ERR_INVALID_ARG;
+  int dev;
+  st = use_device_of(desc->k, &dev);
+  if (st != TRI_OK) return st;
+  return launch_select(g, scores, B, kept, kept_count, reinterpret_cast<cudaStream_t>(stream));
+}
+
+tri_status tri_compact_kv(const tri_cache_desc* desc, const int32_t* kept, const int32_t* kept_count, int B,
+                          tri_compact_mode mode, void* k_out, void* v_out, tri_stream_t stream) {
+  Geom g;
+  tri_status st = make_geom(desc, true, &g);
+  if (st != TRI_OK) return st;
+  st = check_compact_args(desc, kept, kept_count, B, mode, k_out, v_out);
+  if (st != TRI_OK) return st;
+  int dev;
+  st = use_device_of(desc->k, &dev);
+  if (st != TRI_OK) return st;
+  return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+tri_status tri_workspace_size(const tri_cache_desc* desc, int B, size_t* bytes) {
+  if (!bytes || B < 1) return TRI_ERR_INVALID_ARG;
+  Geom g;
+  tri_status st = make_geom(desc, false, &g);
+  if (st != TRI_OK) return st;
+  const int64_t units = int64_t{g.L} * g.H * g.batch;
+  *bytes = static_cast<size_t>(units * g.score_stride * 4 + 256);
+  return TRI_OK;
+}
+
+tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B, tri_compact_mode mode, int32_t* kept,
+                        int32_t* kept_count, void* k_out, void* v_out, void* workspace, size_t workspace_bytes,
+                        tri_stream_t stream) {
+  Geom g;
+  tri_status st = make_geom(desc, true, &g);
+  if (st != TRI_OK) return st;
+  if (!w || !aligned16(w)) return TRI_ERR_INVALID_ARG;
+  st = check_compact_args(desc, kept, kept_count, B, mode, k_out, v_out);
+  if (st != TRI_OK) return st;
+  size_t need = 0;
+  st = tri_workspace_size(desc, B, &need);
+  if (st != TRI_OK) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return TRI_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return TRI_ERR_WORKSPACE;
+  int dev;
+  st = use_device_of(desc->k, &dev);
+  if (st != TRI_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* scores = static_cast<float*>(workspace);
+  st = launch_score(g, w, scores, dev, s);
+  if (st != TRI_OK) return st;
+  st = launch_select(g, scores, B, kept, kept_count, s);
+  if (st != TRI_OK) return st;
+  return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, s);
+}
+
+tri_status tri_read_device_status(tri_stream_t stream, uint32_t* flags, int clear) {
+  if (!flags) return TRI_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (s) {
+    int dev = -1;
+    TRI_CUDA(cudaStreamGetDevice(s, &dev));
+    int cur = -1;
+    TRI_CUDA(cudaGetDevice(&cur));
+    if (cur != dev) TRI_CUDA(cudaSetDevice(dev));
+  }
+  unsigned int v = 0;
+  TRI_CUDA(cudaMemcpyFromSymbolAsync(&v, tri::g_status, sizeof(v), 0, cudaMemcpyDeviceToHost, s));
+  TRI_CUDA(cudaStreamSynchronize(s));
+  if (clear) {
+    const unsigned int zero = 0;
+    TRI_CUDA(cudaMemcpyToSymbolAsync(tri::g_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s));
+    TRI_CUDA(cudaStreamSynchronize(s));
+  }
+  *flags = v;
+  if (v & TRI_DEVFLAG_TIMEOUT) return TRI_ERR_DEVICE_TIMEOUT;
+  if (v) return TRI_ERR_DEVICE_CHECK;
+  return TRI_OK;
+}
+
+const char* tri_status_string(tri_status st) {
+  switch (st) {
+    case TRI_OK: return "TRI_OK";
+    case TRI_ERR_INVALID_ARG: return "TRI_ERR_INVALID_ARG";
+    case TRI_ERR_UNSUPPORTED: return "TRI_ERR_UNSUPPORTED";
+    case TRI_ERR_WORKSPACE: return "TRI_ERR_WORKSPACE";
+    case TRI_ERR_CUDA: return "TRI_ERR_CUDA";
+    case TRI_ERR_DEVICE_CHECK: return "TRI_ERR_DEVICE_CHECK";
+    case TRI_ERR_DEVICE_TIMEOUT: return "TRI_ERR_DEVICE_TIMEOUT";
+  }
+  return "TRI_ERR_UNKNOWN";
+}
+
+int tri_last_cuda_error(void) { return g_last_cuda_error; }
+
+uint64_t tri_kernel_launches(void) { return g_launches.load(); }
+
+const char* tri_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,278 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Small cases compare every key of every unit with the oracle's literal
+per-offset average; the full-size workloads run in the launch configuration
+the bench times (fold, then the fused score -> select -> compact call) and
+compare sampled units key by key, plus properties on every unit.
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import gen
+import oracle
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(autouse=True)
+def _cleanup():
+    yield
+    gc.collect()
+    if torch.cuda.is_available():
+        torch.cuda.empty_cache()
+
+
+def tri():
+    import rope_aware_key_b200 as t
+    return t
+
+
+def check_every_unit(cache, res, pairing=0, delta0=None, literal=True, before=None, after=None):
+    w64 = parity.check_fold(res, cache, pairing, delta0)
+    wl = cache.wl
+    reports = []
+    for l in range(wl.num_layers):
+        for h in range(wl.num_kv_heads):
+            for b in range(wl.batch):
+                kw = {}
+                if before is not None:
+                    kw = dict(before_k=before[(l, h, b)][0], before_v=before[(l, h, b)][1],
+                              after_k=after[(l, h, b)][0], after_v=after[(l, h, b)][1])
+                reports.append(parity.check_unit(cache, res, l, h, b, w64[l * wl.num_kv_heads + h],
+                                                 literal=literal, pairing=pairing, delta0=delta0, **kw))
+    parity.check_all_units_properties(cache, res)
+    assert res.status == 0
+    return reports
+
+
+def snapshot(cache, units):
+    out = {}
+    for (l, h, b) in units:
+        out[(l, h, b)] = (parity.bits16(gen.unit_rows(cache, cache.k, l, h, b)),
+                          parity.bits16(gen.unit_rows(cache, cache.v, l, h, b)))
+    return out
+
+
+def all_units(wl):
+    return [(l, h, b) for l in range(wl.num_layers) for h in range(wl.num_kv_heads) for b in range(wl.batch)]
+
+
+# ------------------------------------------------------------------ small, every key
+
+def test_tiny_single_head():
+    cache = gen.make_cache(gen.WORKLOADS["tiny"], seed=0, device=DEV)
+    res = parity.run_gpu(cache)
+    reps = check_every_unit(cache, res)
+    assert reps[0].max_err_over_l1 < 1e-5
+
+
+def test_qwen3_layer_8x32768():
+    cache = gen.make_cache(gen.WORKLOADS["qwen3_layer"], seed=0, device=DEV)
+    res = parity.run_gpu(cache, fused=True)
+    check_every_unit(cache, res)
+
+
+@pytest.mark.parametrize("pairing,delta0", [(0, 0.0), (1, 5.0), (0, 1234.5)])
+def test_contig_batch_ragged_tail(pairing, delta0):
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=2, num_kv_heads=3, batch=3, seq_len=1000, budget=100,
+                    theta=1e6)
+    cache = gen.make_cache(wl, seed=3, device=DEV)
+    res = parity.run_gpu(cache, pairing=pairing, delta0=delta0)
+    check_every_unit(cache, res, pairing=pairing, delta0=delta0)
+
+
+def test_ragged_edge_lengths():
+    wl = gen.scaled(gen.WORKLOADS["qwen3_ragged"], num_layers=2, num_kv_heads=2, batch=7, budget=128)
+    lens = [1, 127, 128, 129, 300, 0, 2049]
+    cache = gen.make_cache(wl, seed=5, device=DEV, lens=lens)
+    for fused in (False, True):
+        res = parity.run_gpu(cache, fused=fused)
+        check_every_unit(cache, res)
+
+
+@pytest.mark.parametrize("H", [1, 2, 4, 8])
+def test_paged_out_of_place(H):
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=H, batch=5, budget=64,
+                    spare_blocks_per_seq=1)
+    cache = gen.make_cache(wl, seed=H, device=DEV, lens=[5, 16, 17, 300, 1000])
+    res = parity.run_gpu(cache, mode=tri().COMPACT_OUT_OF_PLACE)
+    check_every_unit(cache, res)
+
+
+@pytest.mark.parametrize("H,fused", [(4, False), (8, True), (1, True)])
+def test_paged_in_place_holefill(H, fused):
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=H, batch=5, budget=64,
+                    spare_blocks_per_seq=1)
+    cache = gen.make_cache(wl, seed=10 + H, device=DEV, lens=[5, 64, 65, 300, 1000])
+    units = all_units(wl)
+    before = snapshot(cache, units)
+    res = parity.run_gpu(cache, mode=tri().COMPACT_IN_PLACE_HOLEFILL, fused=fused)
+    after = snapshot(cache, units)
+    check_every_unit(cache, res, before=before, after=after)
+
+
+def test_contig_in_place_holefill():
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=2, seq_len=777, budget=200)
+    cache = gen.make_cache(wl, seed=4, device=DEV)
+    units = all_units(wl)
+    before = snapshot(cache, units)
+    res = parity.run_gpu(cache, mode=tri().COMPACT_IN_PLACE_HOLEFILL)
+    after = snapshot(cache, units)
+    check_every_unit(cache, res, before=before, after=after)
+
+
+@pytest.mark.parametrize("B", [1, 2, 999, 1000, 1005])
+def test_budget_edges(B):
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=1000, budget=B)
+    cache = gen.make_cache(wl, seed=6, device=DEV)
+    res = parity.run_gpu(cache)
+    check_every_unit(cache, res)
+
+
+def test_exact_ties_go_to_lower_index():
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=3000, budget=700)
+    cache = gen.make_cache(wl, seed=7, device=DEV)
+    # 37 distinct rows repeated: every score appears ~81 times, exactly
+    base = cache.k[0, 0, 0, :37].clone()
+    cache.k[0, 0, 0] = base.repeat(82, 1)[:3000]
+    res = parity.run_gpu(cache)
+    check_every_unit(cache, res)
+    s = res.scores[0, :3000].cpu().numpy()
+    kept = res.kept[0].cpu().numpy()
+    t = s[kept].min()
+    eq = np.flatnonzero(s == t)
+    kept_eq = np.intersect1d(eq, kept)
+    assert len(kept_eq) < len(eq) and np.array_equal(kept_eq, eq[: len(kept_eq)])
+
+
+def test_all_scores_equal():
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=4100, budget=333)
+    cache = gen.make_cache(wl, seed=8, device=DEV)
+    cache.k[0, 0, 0] = cache.k[0, 0, 0, :1].expand(4100, -1)
+    res = parity.run_gpu(cache)
+    check_every_unit(cache, res)
+    assert np.array_equal(res.kept[0].cpu().numpy(), np.arange(333))
+
+
+def test_nonfinite_keys_rank_lowest():
+    """NaN scores rank lowest; +/-inf keys give +/-inf or NaN scores."""
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=600, budget=590)
+    cache = gen.make_cache(wl, seed=9, device=DEV)
+    k = cache.k[0, 0, 0]
+    k[10] = float("nan")
+    k[20, 5] = float("inf")
+    k[30, 7] = float("-inf")
+    k[40] = 0.0
+    res = parity.run_gpu(cache)
+    s = res.scores[0, :600].cpu().numpy()
+    assert np.isnan(s[10])
+    kept = res.kept[0, :590].cpu().numpy()
+    np.testing.assert_array_equal(kept, oracle.select(s, 590))
+    assert 10 not in set(kept.tolist())
+    # finite keys: scores within tolerance of the oracle
+    w64 = parity.check_fold(res, cache)
+    keys = parity.bits16(k)
+    fin = np.all(np.isfinite(k.float().cpu().numpy()), axis=1)
+    ref = oracle.score_literal(keys[fin], cache.query_center[0, 0].numpy(), wl.theta, wl.offsets)
+    parity.check_scores(keys[fin], s[fin], ref, w64[0])
+
+
+def test_score_row_padding():
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=513, budget=64)
+    cache = gen.make_cache(wl, seed=11, device=DEV)
+    res = parity.run_gpu(cache, max_seq_len=1001)
+    assert res.scores.shape[1] == 1004
+    assert torch.isnan(res.scores[:, 513:]).all()      # padding never written
+    check_every_unit(cache, res)
+
+
+def test_bad_page_is_flagged_not_fatal():
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=1, num_kv_heads=4, batch=2, budget=16,
+                    spare_blocks_per_seq=0)
+    cache = gen.make_cache(wl, seed=12, device=DEV, lens=[40, 40])
+    nb = cache.k.shape[1]
+    cache.block_table[1, 1] = nb + 1000            # out of the pool
+    res = parity.run_gpu(cache)
+    assert res.status & tri().DEVFLAG_BAD_PAGE
+    # the intact sequence is still right
+    w64 = parity.check_fold(res, cache)
+    for h in range(4):
+        parity.check_unit(cache, res, 0, h, 0, w64[h])
+    assert tri().read_device_status() == 0           # cleared
+
+
+def test_launch_count_and_status_clean():
+    t = tri()
+    cache = gen.make_cache(gen.WORKLOADS["tiny"], seed=0, device=DEV)
+    n0 = t.kernel_launches()
+    parity.run_gpu(cache, fused=True)
+    assert t.kernel_launches() - n0 == 4            # fold, score, select, compact
+
+
+# ------------------------------------------------------------------ full size, sampled
+
+def sample_units(wl, k, seed):
+    rng = np.random.default_rng(seed)
+    units = {(0, 0, 0), (wl.num_layers - 1, wl.num_kv_heads - 1, wl.batch - 1)}
+    while len(units) < k:
+        units.add((int(rng.integers(wl.num_layers)), int(rng.integers(wl.num_kv_heads)),
+                   int(rng.integers(wl.batch))))
+    return sorted(units)
+
+
+def check_sampled(cache, res, units, before=None, after=None, literal_subset=512):
+    w64 = parity.check_fold(res, cache)
+    H = cache.wl.num_kv_heads
+    for (l, h, b) in units:
+        kw = {}
+        if before is not None:
+            kw = dict(before_k=before[(l, h, b)][0], before_v=before[(l, h, b)][1],
+                      after_k=after[(l, h, b)][0], after_v=after[(l, h, b)][1])
+        parity.check_unit(cache, res, l, h, b, w64[l * H + h], literal=False, literal_subset=literal_subset, **kw)
+    parity.check_all_units_properties(cache, res)
+    assert res.status == 0
+
+
+def test_full_qwen3_36x8x32768():
+    """The bench workload."""
+    wl = gen.WORKLOADS["qwen3_full"]
+    cache = gen.make_cache(wl, seed=0, device=DEV)
+    res = parity.run_gpu(cache, fused=True)
+    check_sampled(cache, res, sample_units(wl, 5, 1))
+
+
+def test_full_qwen3_ragged_batch8():
+    wl = gen.WORKLOADS["qwen3_ragged"]
+    cache = gen.make_cache(wl, seed=0, device=DEV)
+    res = parity.run_gpu(cache, fused=True)
+    check_sampled(cache, res, sample_units(wl, 5, 2))
+
+
+def test_full_llama3_long_uniform_schedule():
+    wl = gen.WORKLOADS["llama3_long"]
+    cache = gen.make_cache(wl, seed=0, device=DEV)
+    res = parity.run_gpu(cache, fused=True)
+    check_sampled(cache, res, sample_units(wl, 3, 3), literal_subset=256)
+
+
+def test_full_paged_incremental_rounds():
+    """Initial compression of the paged cache, then rounds of 128 appended
+    tokens per sequence re-compressed in place down to B."""
+    wl = gen.WORKLOADS["qwen25_paged"]
+    cache = gen.make_cache(wl, seed=0, device=DEV)
+    t = tri()
+    for rnd in range(3):
+        if rnd > 0:
+            gen.append_tokens(cache, 128, step=rnd)
+        units = sample_units(wl, 4, 10 + rnd)
+        before = snapshot(cache, units)
+        res = parity.run_gpu(cache, mode=t.COMPACT_IN_PLACE_HOLEFILL, fused=True)
+        after = snapshot(cache, units)
+        check_sampled(cache, res, units, before=before, after=after)
+        gen.release_tail_blocks(cache, [min(wl.budget, n) for n in cache.lens])
