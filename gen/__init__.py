@@ -111,6 +111,9 @@ WORKLOADS: Dict[str, Workload] = {
     # full Qwen3-8B-shaped cache, 36 layers x 8 heads x 32768 keys, batch 1
     "qwen3_full": Workload("qwen3_full", 36, 8, 128, 1e6, _GEO17, 2048,
                            "contig", batch=1, seq_len=32768),
+    # 8 of those 36 layers: a smaller case of the same shape (profiling)
+    "qwen3_8layers": Workload("qwen3_8layers", 8, 8, 128, 1e6, _GEO17, 2048, "contig",
+                              batch=1, seq_len=32768),
     # 36 x 8, batch 8 ragged sequences of U{8192..32768} tokens
     "qwen3_ragged": Workload("qwen3_ragged", 36, 8, 128, 1e6, _GEO17, 2048,
                              "ragged", batch=8, len_lo=8192, len_hi=32768),

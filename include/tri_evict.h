@@ -108,7 +108,7 @@ typedef struct tri_fold_params {
 typedef struct tri_cache_desc {
   tri_layout layout;
   int num_layers;          /* L >= 1 */
-  int num_kv_heads;        /* H >= 1 (PAGED: H divides 16 and block_size*H <= 128) */
+  int num_kv_heads;        /* H >= 1 (PAGED: H divides 8 and block_size*H <= 128) */
   int head_dim;            /* must be 128 */
   int batch;               /* sequences, 1 .. TRI_MAX_BATCH */
   int max_seq_len;         /* capacity of a score row; 0 = the longest sequence */

@@ -12,8 +12,10 @@
 //     a_f = E[q_f] W_f e^{i w_f delta0},   w[re(f)] = Re a_f,  w[im(f)] = Im a_f,
 // and Re sum_f a_f conj(k_f) = sum_j w[j] k[j].
 //
-// One CTA; fp64 throughout (w_f * delta reaches 2^16 rad for the default
-// schedule, far beyond what fp32 phases can hold), fp32 output.
+// Grid: one CTA per (band f, block of kThreads centers).  Each CTA sums W_f
+// over the schedule with a fixed-order fp64 tree, then maps its centers'
+// band f.  fp64 throughout (w_f * delta reaches 2^16 rad for the default
+// schedule, far beyond what fp32 phases can hold); fp32 output.
 #pragma once
 
 #include "common.cuh"
@@ -21,7 +23,7 @@
 namespace tri {
 namespace fold {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kBands = kD / 2;
 
 struct Args {
@@ -36,62 +38,64 @@ struct Args {
 };
 
 __global__ void __launch_bounds__(kThreads) fold_kernel(const __grid_constant__ Args a) {
-  __shared__ double s_wre[kBands], s_wim[kBands], s_omega[kBands];
+  __shared__ double s_c[kThreads / 32], s_s[kThreads / 32];
+  const int f = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int kWarps = kThreads / 32;
+  const double omega = pow(a.theta, -2.0 * f / kD);
 
-  // W_f: warp-per-band sums over the schedule, fixed reduction order.
-  for (int f = warp; f < kBands; f += kWarps) {
-    const double omega = pow(a.theta, -2.0 * f / kD);
-    double c = 0.0, s = 0.0;
-    for (int t = lane; t < a.n_offsets; t += 32) {
-      double sn, cs;
-      sincos(omega * a.offsets[t], &sn, &cs);
-      c += cs;
-      s += sn;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      c += __shfl_xor_sync(0xffffffffu, c, o);
-      s += __shfl_xor_sync(0xffffffffu, s, o);
-    }
-    if (lane == 0) {
-      s_wre[f] = c / a.n_offsets;
-      s_wim[f] = s / a.n_offsets;
-      s_omega[f] = omega;
-    }
+  // W_f = mean over the schedule of e^{i omega delta}
+  double c = 0.0, s = 0.0;
+  for (int t = threadIdx.x; t < a.n_offsets; t += kThreads) {
+    double sn, cs;
+    sincos(omega * a.offsets[t], &sn, &cs);
+    c += cs;
+    s += sn;
   }
-  if (threadIdx.x == 0) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+  }
+  if (lane == 0) {
+    s_c[warp] = c;
+    s_s[warp] = s;
+  }
+  __syncthreads();
+  double wre = 0.0, wim = 0.0;
+  for (int i = 0; i < kThreads / 32; ++i) {
+    wre += s_c[i];
+    wim += s_s[i];
+  }
+  wre /= a.n_offsets;
+  wim /= a.n_offsets;
+
+  if (f == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     bool finite = isfinite(a.theta) && isfinite(a.delta0);
     for (int t = 0; t < a.n_offsets; ++t) finite = finite && isfinite(a.offsets[t]);
     if (!finite) flag(TRI_DEVFLAG_NONFINITE);
   }
-  __syncthreads();
 
-  // a_f for every (center, band).
-  const int total = a.n_centers * kBands;
-  for (int idx = threadIdx.x; idx < total; idx += kThreads) {
-    const int c = idx / kBands, f = idx - c * kBands;
-    const int re = a.pairing == TRI_PAIRING_HALF ? f : 2 * f;
-    const int im = a.pairing == TRI_PAIRING_HALF ? f + kBands : 2 * f + 1;
-    const float* q = a.q + static_cast<int64_t>(c) * kD;
-    const float qr_f = q[re], qi_f = q[im];
-    if (!isfinite(qr_f) || !isfinite(qi_f)) flag(TRI_DEVFLAG_NONFINITE);
-    const double qr = qr_f, qi = qi_f;
-    // mu' = E[q_f] W_f
-    const double mr = s_wre[f] * qr - s_wim[f] * qi;
-    const double mi = s_wim[f] * qr + s_wre[f] * qi;
-    double ar = mr, ai = mi;
-    if (a.delta0 != 0.0) {
-      double sn, cs;
-      sincos(s_omega[f] * a.delta0, &sn, &cs);
-      ar = cs * mr - sn * mi;
-      ai = sn * mr + cs * mi;
-    }
-    float* w = a.w + static_cast<int64_t>(c) * kD;
-    w[re] = static_cast<float>(ar);
-    w[im] = static_cast<float>(ai);
+  const int ci = blockIdx.y * kThreads + threadIdx.x;
+  if (ci >= a.n_centers) return;
+  const int re = a.pairing == TRI_PAIRING_HALF ? f : 2 * f;
+  const int im = a.pairing == TRI_PAIRING_HALF ? f + kBands : 2 * f + 1;
+  const float* q = a.q + static_cast<int64_t>(ci) * kD;
+  const float qr_f = q[re], qi_f = q[im];
+  if (!isfinite(qr_f) || !isfinite(qi_f)) flag(TRI_DEVFLAG_NONFINITE);
+  const double qr = qr_f, qi = qi_f;
+  // mu'_f = E[q_f] W_f
+  const double mr = wre * qr - wim * qi;
+  const double mi = wim * qr + wre * qi;
+  double ar = mr, ai = mi;
+  if (a.delta0 != 0.0) {
+    double sn, cs;
+    sincos(omega * a.delta0, &sn, &cs);
+    ar = cs * mr - sn * mi;
+    ai = sn * mr + cs * mi;
   }
+  float* w = a.w + static_cast<int64_t>(ci) * kD;
+  w[re] = static_cast<float>(ar);
+  w[im] = static_cast<float>(ai);
 }
 
 }  // namespace fold

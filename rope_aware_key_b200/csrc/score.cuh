@@ -6,83 +6,100 @@
 // offset.  128 FMAs per 256-byte key, so the kernel is bound by HBM: it is a
 // stream of the key cache through shared memory.
 //
-// Design (one persistent CTA per SM):
-//  * a producer thread issues 1-D bulk copies (cp.async.bulk, no multicast)
-//    of whole tiles -- up to 128 consecutive keys of one unit (CONTIG,
-//    RAGGED) or one page of all heads (PAGED) -- into a ring of
-//    TRI_SCORE_STAGES 32 KB shared-memory stages, each guarded by a
-//    full/empty mbarrier pair; keys are fetched with an L2 evict-first hint;
-//  * 8 consumer warps read the stage with 16-byte shared loads, a half-warp
-//    per key (16 lanes x 8 bf16), multiply with the unit's weight slice held
-//    in registers and reduce across the half-warp with shuffles;
+// Design (persistent, TRI_SCORE_CTAS_PER_SM CTAs per SM):
+//  * a producer thread decodes each tile once -- up to 128 consecutive keys
+//    of one unit (CONTIG, RAGGED) or one page of all heads (PAGED) -- writes
+//    its metadata next to the stage and issues one 1-D bulk copy
+//    (cp.async.bulk, no multicast, L2 evict-first) into a ring of
+//    TRI_SCORE_STAGES 32 KB shared-memory stages guarded by full/empty
+//    mbarriers;
+//  * 8 consumer warps read a stage with 16-byte shared loads, four lanes per
+//    key (32 bf16 each).  The two keys of a quarter-warp read opposite halves
+//    of the 128-byte bank window at every load (the odd key's chunk order is
+//    rotated), so the loads are conflict-free; each lane keeps its 32
+//    weights in registers in its own rotated order.  Two shuffles reduce a
+//    key;
 //  * every wait is bounded (about 2 s) and reported through the status word.
 #pragma once
 
 #include "common.cuh"
 
 #ifndef TRI_SCORE_STAGES
-#define TRI_SCORE_STAGES 4
+#define TRI_SCORE_STAGES 3
+#endif
+#ifndef TRI_SCORE_CTAS_PER_SM
+#define TRI_SCORE_CTAS_PER_SM 2
 #endif
 
 namespace tri {
 namespace score {
 
 constexpr int kTileRows = 128;
-constexpr int kTileBytes = kTileRows * kRowBytes;  // 32 KB
+constexpr int kTileBytes = kTileRows * kRowBytes;   // 32 KB
 constexpr int kStages = TRI_SCORE_STAGES;
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kIters = kTileRows / (2 * kConsumerWarps);   // rows per half-warp per tile
-constexpr size_t kSmemBytes = static_cast<size_t>(kStages) * kTileBytes + 2 * kStages * sizeof(uint64_t);
+constexpr int kRowsPerWarpPass = 8;                  // 4 lanes per key
+constexpr int kGroup = kRowsPerWarpPass * kConsumerWarps;   // rows per pass of all consumers
+constexpr int kIters = kTileRows / kGroup;
 
-struct Tile {
-  int l, h, b;     // h is meaningful for CONTIG / RAGGED only
-  int i0;          // first key index of the tile
-  int rows;        // rows held in the stage
-  int tvalid;      // PAGED: tokens of the page that belong to the sequence
-  int64_t src;     // element offset of the first row
-  bool ok;
+// Decoded tile, written by the producer next to its stage.
+struct TileInfo {
+  int rows;          // rows held in the stage (0: nothing to do)
+  int paged;         // rows interleave heads (PAGED)
+  int lh;            // layer*H + head of row 0 (CONTIG / RAGGED), layer*H (PAGED)
+  int tvalid;        // PAGED: tokens of the page inside the sequence
+  float* out;        // score of row 0 (CONTIG / RAGGED) or of head 0, token 0 (PAGED)
+  int64_t head_step; // PAGED: floats between the score rows of consecutive heads
 };
+
+constexpr size_t kBarOffset = static_cast<size_t>(kStages) * kTileBytes;
+constexpr size_t kInfoOffset = kBarOffset + 2 * kStages * sizeof(uint64_t);
+constexpr size_t kSmemBytes = kInfoOffset + kStages * sizeof(TileInfo);
 
 // Tiles are numbered layer-major: CONTIG / RAGGED per (layer, head) then
 // sequence then 128-key chunk; PAGED per layer then sequence then page.
-__device__ __forceinline__ Tile decode(const Geom& g, int t) {
-  Tile T;
+__device__ __forceinline__ void decode(const Geom& g, int t, float* scores, TileInfo* T, int64_t* src,
+                                       bool* ok) {
   const int per = g.tile_prefix[g.batch];
   const int outer = t / per;
   const int r = t - outer * per;
   const int b = find_seq(g.tile_prefix, g.batch, r);
   const int j = r - g.tile_prefix[b];
-  T.b = b;
-  T.ok = true;
+  *ok = true;
   if (g.layout == TRI_LAYOUT_PAGED) {
-    T.l = outer;
-    T.h = 0;
-    T.i0 = j * g.block_size;
-    T.rows = g.block_size * g.H;
-    T.tvalid = min(g.block_size, g.len[b] - T.i0);
+    const int l = outer;
+    const int i0 = j * g.block_size;
+    T->rows = g.block_size * g.H;
+    T->paged = 1;
+    T->lh = l * g.H;
+    T->tvalid = min(g.block_size, g.len[b] - i0);
+    T->head_step = static_cast<int64_t>(g.batch) * g.score_stride;
+    T->out = scores + (static_cast<int64_t>(l) * g.H * g.batch + b) * g.score_stride + i0;
     const int blk = g.block_table[static_cast<int64_t>(b) * g.max_blocks + j];
     if (static_cast<unsigned>(blk) >= static_cast<unsigned>(g.num_blocks)) {
-      T.ok = false;
-      T.src = 0;
+      *ok = false;
+      *src = 0;
     } else {
-      T.src = T.l * g.sL + static_cast<int64_t>(blk) * g.sB;
+      *src = l * g.sL + static_cast<int64_t>(blk) * g.sB;
     }
   } else {
-    T.l = outer / g.H;
-    T.h = outer - T.l * g.H;
-    T.i0 = j * kTileRows;
-    T.rows = min(kTileRows, g.len[b] - T.i0);
-    T.tvalid = T.rows;
-    bool ok = true;
-    T.src = row_elem(g, T.l, T.h, b, T.i0, &ok);
+    const int l = outer / g.H;
+    const int h = outer - l * g.H;
+    const int i0 = j * kTileRows;
+    T->rows = min(kTileRows, g.len[b] - i0);
+    T->paged = 0;
+    T->lh = outer;
+    T->tvalid = T->rows;
+    T->head_step = 0;
+    T->out = scores + (static_cast<int64_t>(outer) * g.batch + b) * g.score_stride + i0;
+    *src = row_elem(g, l, h, b, i0, ok);
   }
-  return T;
 }
 
 // Dot product of 8 bf16 (packed in x, element order) with 8 fp32 weights.
-__device__ __forceinline__ float dot8(const uint4 x, const float (&w)[8]) {
-  float a = __uint_as_float(x.x << 16) * w[0];
+__device__ __forceinline__ float dot8(const uint4 x, const float* w, float a) {
+  a = fmaf(__uint_as_float(x.x << 16), w[0], a);
   a = fmaf(__uint_as_float(x.x & 0xffff0000u), w[1], a);
   a = fmaf(__uint_as_float(x.y << 16), w[2], a);
   a = fmaf(__uint_as_float(x.y & 0xffff0000u), w[3], a);
@@ -93,19 +110,26 @@ __device__ __forceinline__ float dot8(const uint4 x, const float (&w)[8]) {
   return a;
 }
 
-__device__ __forceinline__ void load_w(const float* __restrict__ w, int lh, int l16, float (&wv)[8]) {
-  const float4* p = reinterpret_cast<const float4*>(w + static_cast<int64_t>(lh) * kD + l16 * 8);
-  const float4 a = __ldg(p), b = __ldg(p + 1);
-  wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w;
-  wv[4] = b.x; wv[5] = b.y; wv[6] = b.z; wv[7] = b.w;
+// The lane's 32 weights: chunk (4*(k ^ p) + c) of the head's 16 chunks of 8,
+// for k = 0..3 (the order in which the lane reads a key).
+__device__ __forceinline__ void load_w(const float* __restrict__ w, int lh, int c, int p, float (&wv)[32]) {
+  const float4* base = reinterpret_cast<const float4*>(w + static_cast<int64_t>(lh) * kD);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int ch = 4 * (k ^ p) + c;
+    const float4 a = __ldg(base + 2 * ch), b = __ldg(base + 2 * ch + 1);
+    wv[8 * k + 0] = a.x; wv[8 * k + 1] = a.y; wv[8 * k + 2] = a.z; wv[8 * k + 3] = a.w;
+    wv[8 * k + 4] = b.x; wv[8 * k + 5] = b.y; wv[8 * k + 6] = b.z; wv[8 * k + 7] = b.w;
+  }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, TRI_SCORE_CTAS_PER_SM)
 score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float* __restrict__ scores,
              int ntiles) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(kStages) * kTileBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
   uint64_t* empty = full + kStages;
+  TileInfo* info = reinterpret_cast<TileInfo*>(smem + kInfoOffset);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -118,20 +142,27 @@ score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float*
   __syncthreads();
 
   if (warp == kConsumerWarps) {
-    // ---------------- producer: one thread issues the bulk copies
+    // ---------------- producer: one thread decodes tiles and issues the copies
     if (lane != 0) return;
     const uint64_t policy = policy_evict_first();
     int k = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
       const int s = k % kStages, n = k / kStages;
       if (n > 0 && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) break;
-      const Tile T = decode(g, t);
-      if (T.ok) {
+      TileInfo T;
+      int64_t src;
+      bool ok;
+      decode(g, t, scores, &T, &src, &ok);
+      if (!ok) {
+        T.rows = 0;
+        flag(TRI_DEVFLAG_BAD_PAGE);
+      }
+      info[s] = T;
+      if (T.rows > 0) {
         const uint32_t bytes = static_cast<uint32_t>(T.rows) * kRowBytes;
         mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_g2s(smem + static_cast<size_t>(s) * kTileBytes, g.k + T.src, bytes, &full[s], policy);
+        bulk_g2s(smem + static_cast<size_t>(s) * kTileBytes, g.k + src, bytes, &full[s], policy);
       } else {
-        flag(TRI_DEVFLAG_BAD_PAGE);
         mbar_arrive(&full[s]);
       }
     }
@@ -144,56 +175,58 @@ score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float*
     return;
   }
 
-  // ---------------- consumers
-  const int half = lane >> 4, l16 = lane & 15;
-  const int slot = warp * 2 + half;       // 0..15: which row of each 16-row group
-  float wv[8];
+  // ---------------- consumers: 4 lanes per key
+  const int c = lane & 3;                 // which 4 of the row's 16 chunks
+  const int r8 = lane >> 2;               // key within the warp's group of 8
+  const int p = r8 & 1;                   // chunk-order rotation of odd keys
+  const int row0 = warp * kRowsPerWarpPass + r8;
+  float wv[32];
   int cur_lh = -1;
   int k = 0;
   for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
     const int s = k % kStages, n = k / kStages;
     if (!mbar_wait_bounded(&full[s], n & 1)) break;
-    const Tile T = decode(g, t);
-    if (T.ok) {
-      const unsigned char* buf = smem + static_cast<size_t>(s) * kTileBytes + l16 * 16;
-      int h, iters;
-      float* out;
-      if (g.layout == TRI_LAYOUT_PAGED) {
-        h = slot % g.H;                                // fixed per half-warp: 16 % H == 0
-        iters = (T.rows + 15) >> 4;
-      } else {
-        h = T.h;
-        iters = (T.rows + 15) >> 4;
-      }
-      const int lh = T.l * g.H + h;
+    const TileInfo T = info[s];
+    if (T.rows > 0) {
+      // PAGED rows interleave heads: row r is head r % H, and every row this
+      // lane reads has the same r % H (kGroup and the warp offset are multiples of 8, H | 8).
+      const int h = T.paged ? (row0 % g.H) : 0;
+      const int lh = T.lh + h;
       if (lh != cur_lh) {
-        load_w(w, lh, l16, wv);
+        load_w(w, lh, c, p, wv);
         cur_lh = lh;
       }
-      out = scores + (static_cast<int64_t>(lh) * g.batch + T.b) * g.score_stride + T.i0;
-
-      uint4 x[kIters];
-#pragma unroll
-      for (int it = 0; it < kIters; ++it)
-        if (it < iters) x[it] = *reinterpret_cast<const uint4*>(buf + (it * 16 + slot) * kRowBytes);
-      float acc[kIters];
-#pragma unroll
-      for (int it = 0; it < kIters; ++it) acc[it] = it < iters ? dot8(x[it], wv) : 0.f;
+      const unsigned char* buf = smem + static_cast<size_t>(s) * kTileBytes;
+      const int iters = (T.rows + kGroup - 1) / kGroup;
+      uint4 x[kIters][4];
 #pragma unroll
       for (int it = 0; it < kIters; ++it) {
-        if (it < iters) {    // warp-uniform
-          float a = acc[it];
-          a += __shfl_xor_sync(0xffffffffu, a, 8);
-          a += __shfl_xor_sync(0xffffffffu, a, 4);
-          a += __shfl_xor_sync(0xffffffffu, a, 2);
+        if (it < iters) {
+          const unsigned char* rowp = buf + (it * kGroup + row0) * kRowBytes;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            x[it][q] = *reinterpret_cast<const uint4*>(rowp + (4 * (q ^ p) + c) * 16);
+        }
+      }
+#pragma unroll
+      for (int it = 0; it < kIters; ++it) {
+        if (it < iters) {   // warp-uniform
+          // (d0 + d1) + (d2 + d3): the odd keys' rotation swaps d0/d1 and
+          // d2/d3, and fp32 addition commutes, so every key is summed in the
+          // same order whatever its position
+          float d[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) d[q] = dot8(x[it][q], wv + 8 * q, 0.f);
+          float a = (d[0] + d[1]) + (d[2] + d[3]);
           a += __shfl_xor_sync(0xffffffffu, a, 1);
-          const int r = it * 16 + slot;
-          if (l16 == 0 && r < T.rows) {
-            if (g.layout == TRI_LAYOUT_PAGED) {
+          a += __shfl_xor_sync(0xffffffffu, a, 2);
+          const int r = it * kGroup + row0;
+          if (c == 0 && r < T.rows) {
+            if (T.paged) {
               const int tok = r / g.H;
-              if (tok < T.tvalid) out[tok] = a;
+              if (tok < T.tvalid) T.out[h * T.head_step + tok] = a;
             } else {
-              out[r] = a;
+              T.out[r] = a;
             }
           }
         }

@@ -66,6 +66,14 @@ tri_status use_device_of(const void* ptr, int* dev_out) {
     TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.score_blocks_per_sm, tri::score::score_kernel,
                                                            tri::score::kThreads, tri::score::kSmemBytes));
     if (d.score_blocks_per_sm < 1) return TRI_ERR_UNSUPPORTED;
+    const int sel_cached = static_cast<int>(tri::select::smem_bytes(tri::select::kMaxCached, true));
+    const int sel_long = static_cast<int>(tri::select::smem_bytes(tri::select::kMaxLen, false));
+    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<1024, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, sel_cached));
+    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, sel_cached));
+    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<1024, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, sel_long));
     const int fill_smem = ((tri::compact::kMaxFillBudget + 31) / 32 + tri::compact::kMaxFillBudget) * 4;
     TRI_CUDA(cudaFuncSetAttribute(tri::compact::holefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   fill_smem));
@@ -132,7 +140,7 @@ tri_status make_geom(const tri_cache_desc* c, bool need_v, Geom* g) {
     case TRI_LAYOUT_PAGED: {
       if (!c->seq_lens || !c->block_table) return TRI_ERR_INVALID_ARG;
       if (c->block_size < 1 || c->max_blocks_per_seq < 1 || c->num_blocks < 1) return TRI_ERR_INVALID_ARG;
-      if (16 % c->num_kv_heads != 0 || c->block_size * c->num_kv_heads > tri::score::kTileRows)
+      if (8 % c->num_kv_heads != 0 || c->block_size * c->num_kv_heads > tri::score::kTileRows)
         return TRI_ERR_UNSUPPORTED;
       const int64_t page = int64_t{c->block_size} * c->num_kv_heads * TRI_HEAD_DIM;
       if (c->stride_block < page || (c->stride_block % 8)) return TRI_ERR_INVALID_ARG;
@@ -191,11 +199,17 @@ tri_status launch_score(const Geom& g0, const float* w, float* scores, int dev, 
 tri_status launch_select(const Geom& g, const float* scores, int B, int32_t* kept, int32_t* kept_count,
                          cudaStream_t s) {
   const int units = g.L * g.H * g.batch;
-  tri::select::Args a{scores, kept, kept_count, B};
-  if (g.score_stride >= 8192) {
-    tri::select::select_kernel<1024><<<units, 1024, 0, s>>>(g, a);
+  int max_len = 0;
+  for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
+  if (max_len > tri::select::kMaxLen) return TRI_ERR_UNSUPPORTED;
+  const int cap = (max_len + 3) & ~3;
+  tri::select::Args a{scores, kept, kept_count, B, cap};
+  if (cap > tri::select::kMaxCached) {
+    tri::select::select_kernel<1024, false><<<units, 1024, tri::select::smem_bytes(cap, false), s>>>(g, a);
+  } else if (cap >= 8192) {
+    tri::select::select_kernel<1024, true><<<units, 1024, tri::select::smem_bytes(cap, true), s>>>(g, a);
   } else {
-    tri::select::select_kernel<256><<<units, 256, 0, s>>>(g, a);
+    tri::select::select_kernel<256, true><<<units, 256, tri::select::smem_bytes(cap, true), s>>>(g, a);
   }
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
@@ -267,7 +281,8 @@ tri_status tri_fold_weights(const tri_fold_params* p, const float* q_center, int
   a.delta0 = p->delta0;
   a.n_offsets = p->n_offsets;
   std::memcpy(a.offsets, p->offsets, sizeof(double) * p->n_offsets);
-  tri::fold::fold_kernel<<<1, tri::fold::kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  const dim3 grid(tri::fold::kBands, (n_centers + tri::fold::kThreads - 1) / tri::fold::kThreads);
+  tri::fold::fold_kernel<<<grid, tri::fold::kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
   return TRI_OK;

@@ -160,6 +160,33 @@ def test_all_scores_equal():
     assert np.array_equal(res.kept[0].cpu().numpy(), np.arange(333))
 
 
+def test_heavy_duplicates_overflow_path():
+    """Three distinct scores over 10000 keys: the threshold's bin holds more
+    keys than the candidate list, so the selection takes its fallback path."""
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=10000, budget=4100)
+    cache = gen.make_cache(wl, seed=13, device=DEV)
+    for h in range(2):
+        base = cache.k[0, h, 0, :3].clone()
+        cache.k[0, h, 0] = base.repeat(3334, 1)[:10000]
+    res = parity.run_gpu(cache)
+    check_every_unit(cache, res)
+
+
+def test_single_finite_value_with_infinities():
+    """One finite score value plus +/-inf keys: no finite range to bin."""
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=3000, budget=1500)
+    cache = gen.make_cache(wl, seed=14, device=DEV)
+    k = cache.k[0, 0, 0]
+    k[:] = k[:1].clone()
+    k[100, :] = float("inf")
+    k[200, :] = float("-inf")
+    res = parity.run_gpu(cache)
+    s = res.scores[0, :3000].cpu().numpy()
+    kept = res.kept[0, :1500].cpu().numpy()
+    np.testing.assert_array_equal(kept, oracle.select(s, 1500))
+    assert res.status == 0
+
+
 def test_nonfinite_keys_rank_lowest():
     """NaN scores rank lowest; +/-inf keys give +/-inf or NaN scores."""
     wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=600, budget=590)
