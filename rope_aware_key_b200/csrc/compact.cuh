@@ -15,7 +15,16 @@
 namespace tri {
 namespace compact {
 
+#ifndef TRI_GATHER_ROWS
+#define TRI_GATHER_ROWS 2
+#endif
+#ifndef TRI_GATHER_BLOCKS_PER_SM
+#define TRI_GATHER_BLOCKS_PER_SM 16
+#endif
+
 constexpr int kGatherThreads = 256;
+constexpr int kGatherRows = TRI_GATHER_ROWS;
+constexpr int kGatherBlocksPerSm = TRI_GATHER_BLOCKS_PER_SM;
 constexpr int kFillThreads = 256;
 constexpr int kMaxFillBudget = 16384;
 
@@ -26,6 +35,8 @@ __device__ __forceinline__ void unit_coords(const Geom& g, int u, int* l, int* h
   *h = lh - *l * g.H;
 }
 
+// Each half-warp copies kGatherRows rows per step (all loads issued before
+// the stores, so 2 x kGatherRows x 16 bytes per lane are in flight).
 __global__ void __launch_bounds__(kGatherThreads)
 gather_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept,
               const int32_t* __restrict__ kept_count, int B, uint16_t* __restrict__ kout,
@@ -34,27 +45,41 @@ gather_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept,
   const int l16 = threadIdx.x & 15;
   const int hw = (blockIdx.x * kGatherThreads + threadIdx.x) >> 4;
   const int nhw = (gridDim.x * kGatherThreads) >> 4;
-  for (int row = hw; row < total_rows; row += nhw) {
-    const int u = row / B;
-    const int j = row - u * B;
-    if (j >= __ldg(kept_count + u)) continue;
-    const int i = __ldg(kept + row);
-    int l, h, b;
-    unit_coords(g, u, &l, &h, &b);
-    if (static_cast<unsigned>(i) >= static_cast<unsigned>(g.len[b])) {
-      if (l16 == 0) flag(TRI_DEVFLAG_BAD_KEPT);
-      continue;
+  for (int base = hw; base < total_rows; base += nhw * kGatherRows) {
+    uint4 kx[kGatherRows], vx[kGatherRows];
+    bool live[kGatherRows];
+#pragma unroll
+    for (int r = 0; r < kGatherRows; ++r) {
+      const int row = base + r * nhw;
+      live[r] = false;
+      if (row >= total_rows) continue;
+      const int u = row / B;
+      const int j = row - u * B;
+      if (j >= __ldg(kept_count + u)) continue;
+      const int i = __ldg(kept + row);
+      int l, h, b;
+      unit_coords(g, u, &l, &h, &b);
+      if (static_cast<unsigned>(i) >= static_cast<unsigned>(g.len[b])) {
+        if (l16 == 0) flag(TRI_DEVFLAG_BAD_KEPT);
+        continue;
+      }
+      bool ok = true;
+      const int64_t e = row_elem(g, l, h, b, i, &ok);
+      if (!ok) {
+        if (l16 == 0) flag(TRI_DEVFLAG_BAD_PAGE);
+        continue;
+      }
+      kx[r] = ld_nc_v4(g.k + e + l16 * 8);
+      vx[r] = ld_nc_v4(g.v + e + l16 * 8);
+      live[r] = true;
     }
-    bool ok = true;
-    const int64_t e = row_elem(g, l, h, b, i, &ok);
-    if (!ok) {
-      if (l16 == 0) flag(TRI_DEVFLAG_BAD_PAGE);
-      continue;
+#pragma unroll
+    for (int r = 0; r < kGatherRows; ++r) {
+      if (!live[r]) continue;
+      const int64_t row = base + r * nhw;
+      reinterpret_cast<uint4*>(kout + row * kD)[l16] = kx[r];
+      reinterpret_cast<uint4*>(vout + row * kD)[l16] = vx[r];
     }
-    const uint4 kx = ld_nc_v4(g.k + e + l16 * 8);
-    const uint4 vx = ld_nc_v4(g.v + e + l16 * 8);
-    reinterpret_cast<uint4*>(kout + static_cast<int64_t>(row) * kD)[l16] = kx;
-    reinterpret_cast<uint4*>(vout + static_cast<int64_t>(row) * kD)[l16] = vx;
   }
 }
 

@@ -8,24 +8,22 @@
 // One CTA per unit, on the unit's row of the score matrix (L2-resident right
 // after scoring).  Every decision is made on an order-preserving uint32 key
 // of the fp32 score (NaN -> 0, the lowest; -0 -> +0), so it is exact:
-//  1. rows of up to kMaxCached scores are held in shared memory as keys
-//     (longer rows are re-read from global memory each pass); min / max of
-//     all keys and of the finite ones;
-//  2. a histogram over kBins equal-width bins of the finite value range
-//     (monotone in the key) finds the bin holding the B-th largest key; a
-//     warp-parallel 32-ary search turns that bin into its key interval
-//     [cmin, cmax];
-//  3. one ballot pass writes a bitmap of the keys above cmax (all kept) and
-//     collects the few keys inside [cmin, cmax] with their indices;
-//  4. radix select (12-bit digits) over that short list gives the threshold
-//     T, the B-th largest key, and `need`, how many keys equal to T are kept;
-//     keys above T join the bitmap, keys equal to T go to a second bitmap of
-//     which only the `need` lowest indices are kept;
-//  5. the kept bitmap is written out in index order (popcounts, one block
-//     scan), so the output is ascending and never depends on the order of
-//     atomics.
-// When the candidate list would overflow (heavy duplication), step 4 runs
-// the radix over all keys instead and step 3 is redone against T.
+//  1. evenly spaced samples of the row give a key L such that, for any but a
+//     pathological order of the scores, between B and lcap keys are >= L
+//     (the sample's (B/n share + 5 sigma)-quantile, via a value histogram);
+//  2. one pass lists every key >= L with its index (warp-aggregated appends
+//     into shared memory);
+//  3. radix select (11-bit digits) over the list gives the threshold T, the
+//     B-th largest key, and `need`, how many keys equal to T are kept; kept
+//     keys are marked in a bitmap, keys equal to T in a tie bitmap;
+//  4. the `need` lowest-index ties join the bitmap, which is written out in
+//     index order (popcounts, block scans): the output is ascending and never
+//     depends on the order of atomics.
+// If the count of keys >= L falls outside [B, lcap], an exact path over the
+// whole row replaces steps 1-3: a value histogram finds the bin of the B-th
+// largest key, a ballot pass marks everything above the bin and lists the
+// bin's keys, and the radix runs on that list (or on the whole row if the
+// bin is too crowded).
 #pragma once
 
 #include "common.cuh"
@@ -33,45 +31,49 @@
 namespace tri {
 namespace select {
 
-constexpr int kDigitBits = 12;
+constexpr int kDigitBits = 11;
 constexpr int kBins = 1 << kDigitBits;
-constexpr int kMaxCached = 45056;          // keys held in shared memory (176 KB)
-constexpr int kMaxLen = 655360;            // longest row (its two bitmaps must fit in shared memory)
-constexpr int kMaxCand = 2048;             // candidate list capacity
+constexpr int kSamples = 4096;             // evenly spaced scores that bound the threshold
+constexpr int kMaxShared = 200 * 1024;     // dynamic shared memory one CTA may use
 constexpr uint32_t kKeyNegInf = 0x007fffffu;
 constexpr uint32_t kKeyPosInf = 0xff800000u;
 
 __device__ __forceinline__ uint32_t order_key(float s) {
   uint32_t u = __float_as_uint(s);
-  if (s != s) return 0u;               // NaN ranks lowest
-  if (u == 0x80000000u) u = 0u;        // -0 ranks with +0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  const bool nan = (u & 0x7fffffffu) > 0x7f800000u;      // NaN ranks lowest
+  u = u == 0x80000000u ? 0u : u;                         // -0 ranks with +0
+  const uint32_t k = u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
+  return nan ? 0u : k;
 }
 
 __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Value bin of a key: equal-width bins over [lo, lo + kBins/scale]; keys
-// below lo (NaN, -inf) go to bin 0, +inf (and the unused patterns above it)
-// to the last bin.  Non-decreasing over all 2^32 keys.
-__device__ __forceinline__ int value_bin(uint32_t key, float lo, float scale) {
-  if (key >= kKeyPosInf) return kBins - 1;
-  const float v = key_value(key);
-  if (!(v >= lo)) return 0;
-  const float t = (v - lo) * scale;
-  return t < static_cast<float>(kBins) ? static_cast<int>(t) : kBins - 1;
+// Value bin of a real key (one that order_key can produce): equal-width bins,
+// bin = clamp(trunc(v * scale - lo_s), 0, kBins - 1).  The fused multiply-add
+// and the saturating conversion are monotone, NaN converts to 0 and -inf / +inf
+// saturate to the first / last bin, so the bin never decreases with the key.
+__device__ __forceinline__ int value_bin(uint32_t key, float scale, float lo_s) {
+  const int t = __float2int_rz(fmaf(key_value(key), scale, -lo_s));
+  return min(max(t, 0), kBins - 1);
+}
+
+// The same over all 2^32 bit patterns (the unused ones above +inf's key go to
+// the last bin), for the key-space search.
+__device__ __forceinline__ int value_bin_any(uint32_t key, float scale, float lo_s) {
+  return key >= kKeyPosInf ? kBins - 1 : value_bin(key, scale, lo_s);
 }
 
 // Warp-collective: the smallest key k with value_bin(k) >= target, or 2^32.
-__device__ __forceinline__ uint64_t first_key_in_bin(int target, float lo, float scale) {
+__device__ __forceinline__ uint64_t first_key_in_bin(int target, float scale, float lo_s) {
   const int lane = threadIdx.x & 31;
   uint64_t a = 0, b = uint64_t{1} << 32;       // the answer lies in [a, b]; b == 2^32 means none
   while (a < b) {
     const uint64_t step = (b - a + 31) / 32;
     const uint64_t x = a + static_cast<uint64_t>(lane) * step;
     const bool valid = x < b;
-    const bool p = valid ? value_bin(static_cast<uint32_t>(x), lo, scale) >= target : true;
+    const bool p = valid ? value_bin_any(static_cast<uint32_t>(x), scale, lo_s) >= target : true;
     const uint32_t m = __ballot_sync(0xffffffffu, p);
     if (m == 0u) {                             // every probe below: answer after the last one
       a = a + 31 * step + 1;
@@ -95,13 +97,9 @@ struct Args {
   int32_t* kept;
   int32_t* kept_count;
   int B;
-  int cap;          // >= every row length, a multiple of 4: sizes the shared-memory arrays
+  int cap;          // >= every row length, a multiple of 4: sizes the shared-memory bitmaps
+  int lcap;         // capacity of the shared-memory key list
 };
-
-template <bool CACHED>
-__device__ __forceinline__ uint32_t key_at(const float* __restrict__ row, const uint32_t* skeys, int i) {
-  return CACHED ? skeys[i] : order_key(row[i]);
-}
 
 // Block-wide: find the digit d with (count above d) < need <= (count above d) + hist[d],
 // scanning bins from the top.  Returns d; *above gets the count above d.
@@ -194,101 +192,68 @@ __device__ __forceinline__ uint32_t radix_threshold(Visit visit, uint32_t lo_key
   return prefix;
 }
 
-template <int NT, bool CACHED>
-__global__ void __launch_bounds__(NT) select_kernel(const __grid_constant__ Geom g, const Args a) {
-  constexpr int NW = NT / 32;
-  extern __shared__ uint4 select_dyn[];
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t scan_sh[NW];
-  __shared__ uint32_t red[4][NW];
-  __shared__ uint32_t s_pair[2];
-  __shared__ uint32_t s_bounds[2];
-  __shared__ uint32_t s_ncand;
+// Shared-memory layout of one CTA (dynamic part), all 32-bit words:
+//   list_key[max(lcap, kSamples)] list_idx[lcap] keepmap[wcap] tiemap[wcap];
+// the samples live in list_key until the list is filled.
+struct Smem {
+  uint32_t* list_key;
+  int32_t* list_idx;
+  uint32_t* keepmap;
+  uint32_t* tiemap;
+  uint32_t* samples;
+};
 
-  const int u = blockIdx.x;
-  const int b = u % g.batch;
-  const int n = g.len[b];
-  const int B = a.B;
-  const float* __restrict__ row = a.scores + static_cast<int64_t>(u) * g.score_stride;
-  int32_t* __restrict__ kept = a.kept + static_cast<int64_t>(u) * B;
+// Exact threshold over the whole row (read from global memory): value-bin
+// histogram, the bin's key interval, a ballot pass that writes the kept
+// bitmap above the interval and lists the keys inside it, then radix select
+// over that list (or over the whole row if the list would overflow).  Marks
+// keys above T in keepmap and keys equal to T in tiemap; returns `need`, the
+// number of ties to keep.
+template <int NT>
+__device__ __forceinline__ uint32_t exact_path(const float* __restrict__ row, int n, int B, int lcap, const Smem& m,
+                                               uint32_t* hist, uint32_t* scan_sh, uint32_t (*red)[NT / 32],
+                                               uint32_t* s_pair, uint32_t* s_bounds, uint32_t* s_count) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-
-  if (threadIdx.x == 0) a.kept_count[u] = min(n, B);
-  if (n <= B) {
-    for (int i = threadIdx.x; i < n; i += NT) kept[i] = i;
-    return;
-  }
-
-  // dynamic shared memory: [keys (CACHED)] [kept bitmap] [tie bitmap] [candidate keys] [candidate indices]
-  const int cap = a.cap;
   const int words = (n + 31) >> 5;
-  const int wcap = (cap + 31) >> 5;
-  uint32_t* skeys = reinterpret_cast<uint32_t*>(select_dyn);
-  uint32_t* keepmap = skeys + (CACHED ? cap : 0);
-  uint32_t* tiemap = keepmap + wcap;
-  uint32_t* cand_key = tiemap + wcap;
-  int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_key + kMaxCand);
-
-  // ---- 1. keys, min / max of all keys and of the finite ones
+  __syncthreads();                                 // the sampled path is done with the shared arrays
+  // min / max of all keys and of the finite ones
   uint32_t mm[4] = {0xffffffffu, 0u, 0xffffffffu, 0u};
-  for (int i = threadIdx.x * 4; i < n; i += NT * 4) {
-    uint32_t t[4];
-    if (i + 3 < n) {
-      const float4 v = *reinterpret_cast<const float4*>(row + i);
-      t[0] = order_key(v.x); t[1] = order_key(v.y); t[2] = order_key(v.z); t[3] = order_key(v.w);
-      if (CACHED) *reinterpret_cast<uint4*>(skeys + i) = make_uint4(t[0], t[1], t[2], t[3]);
-    } else {
-      for (int e = 0; e < 4; ++e) {
-        t[e] = i + e < n ? order_key(row[i + e]) : 0u;
-        if (CACHED && i + e < n) skeys[i + e] = t[e];
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      if (i + e < n) {
-        mm[0] = min(mm[0], t[e]);
-        mm[1] = max(mm[1], t[e]);
-        if (t[e] > kKeyNegInf && t[e] < kKeyPosInf) {
-          mm[2] = min(mm[2], t[e]);
-          mm[3] = max(mm[3], t[e]);
-        }
-      }
+  for (int i = threadIdx.x; i < n; i += NT) {
+    const uint32_t k = order_key(row[i]);
+    mm[0] = min(mm[0], k);
+    mm[1] = max(mm[1], k);
+    if (k > kKeyNegInf && k < kKeyPosInf) {
+      mm[2] = min(mm[2], k);
+      mm[3] = max(mm[3], k);
     }
   }
-  for (int w = threadIdx.x; w < words; w += NT) tiemap[w] = 0u;
-  if (threadIdx.x == 0) s_ncand = 0;
+  for (int w = threadIdx.x; w < words; w += NT) m.tiemap[w] = 0u;
+  if (threadIdx.x == 0) *s_count = 0;
   block_minmax4<NT>(mm, red);
-  const uint32_t kmin = mm[0], kmax = mm[1];
-
-  if (kmin == kmax) {                          // all scores equal: the B lowest indices
-    for (int j = threadIdx.x; j < B; j += NT) kept[j] = j;
-    return;
-  }
-
-  // ---- 2. the bin of the B-th largest key and its key interval
-  uint32_t need = static_cast<uint32_t>(B);   // still to take inside [cmin, cmax]
-  uint32_t cmin = kmin, cmax = kmax;
-  uint32_t ncand_expected = static_cast<uint32_t>(n);
-  float lo = 0.f, scale = 0.f;
+  uint32_t need = static_cast<uint32_t>(B);
+  uint32_t cmin = mm[0], cmax = mm[1];
+  uint32_t ncand = static_cast<uint32_t>(n);
+  float scale = 0.f, lo_s = 0.f;
   bool binned = false;
   if (mm[2] < mm[3]) {
-    lo = key_value(mm[2]);
+    const float lo = key_value(mm[2]);
     const float width = key_value(mm[3]) - lo;
     scale = static_cast<float>(kBins) / width;
-    binned = width > 0.f && isfinite(width) && isfinite(scale) && scale > 0.f;
+    lo_s = lo * scale;
+    binned = width > 0.f && isfinite(width) && isfinite(scale) && scale > 0.f && isfinite(lo_s);
   }
   if (binned) {
     for (int i = threadIdx.x; i < kBins; i += NT) hist[i] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += NT) atomicAdd(&hist[value_bin(key_at<CACHED>(row, skeys, i), lo, scale)], 1u);
+    for (int i = threadIdx.x; i < n; i += NT) atomicAdd(&hist[value_bin(order_key(row[i]), scale, lo_s)], 1u);
     __syncthreads();
     uint32_t above;
     const int bin = find_digit<NT>(hist, kBins, need, scan_sh, s_pair, &above);
     need -= above;
-    ncand_expected = hist[bin];
+    ncand = hist[bin];
     if (warp == 0) {
-      const uint64_t k0 = first_key_in_bin(bin, lo, scale);
-      const uint64_t k1 = bin + 1 < kBins ? first_key_in_bin(bin + 1, lo, scale) : (uint64_t{1} << 32);
+      const uint64_t k0 = first_key_in_bin(bin, scale, lo_s);
+      const uint64_t k1 = bin + 1 < kBins ? first_key_in_bin(bin + 1, scale, lo_s) : (uint64_t{1} << 32);
       if (lane == 0) {
         s_bounds[0] = static_cast<uint32_t>(k0);
         s_bounds[1] = static_cast<uint32_t>(k1 - 1);
@@ -298,95 +263,259 @@ __global__ void __launch_bounds__(NT) select_kernel(const __grid_constant__ Geom
     cmin = s_bounds[0];
     cmax = s_bounds[1];
   }
-  const bool listed = ncand_expected <= static_cast<uint32_t>(kMaxCand);
-
-  // ---- 3. bitmap of the keys above cmax; candidates in [cmin, cmax]
+  const bool listed = ncand <= static_cast<uint32_t>(lcap);
   for (int base = warp * 32; base < n; base += NT) {
     const int i = base + lane;
-    const uint32_t k = i < n ? key_at<CACHED>(row, skeys, i) : 0u;
     const bool in = i < n;
-    const uint32_t m = __ballot_sync(0xffffffffu, in && k > cmax);
-    if (lane == 0) keepmap[base >> 5] = m;
+    const uint32_t k = in ? order_key(row[i]) : 0u;
+    const uint32_t bits = __ballot_sync(0xffffffffu, in && k > cmax);
+    if (lane == 0) m.keepmap[base >> 5] = bits;
     if (listed && in && k >= cmin && k <= cmax) {
-      const uint32_t pos = atomicAdd(&s_ncand, 1u);
-      cand_key[pos] = k;
-      cand_idx[pos] = i;
+      const uint32_t pos = atomicAdd(s_count, 1u);
+      m.list_key[pos] = k;
+      m.list_idx[pos] = i;
     }
   }
   __syncthreads();
-
-  // ---- 4. threshold among the candidates, then mark them
   if (listed) {
-    const int nc = static_cast<int>(s_ncand);
+    const int nc = static_cast<int>(*s_count);
     const uint32_t T = radix_threshold<NT>(
         [&](auto fn) {
-          for (int j = threadIdx.x; j < nc; j += NT) fn(cand_key[j]);
+          for (int j = threadIdx.x; j < nc; j += NT) fn(m.list_key[j]);
         },
         cmin, cmax, &need, hist, scan_sh, s_pair);
     for (int j = threadIdx.x; j < nc; j += NT) {
-      const uint32_t k = cand_key[j];
-      const int i = cand_idx[j];
-      if (k > T) atomicOr(&keepmap[i >> 5], 1u << (i & 31));
-      else if (k == T) atomicOr(&tiemap[i >> 5], 1u << (i & 31));
+      const uint32_t k = m.list_key[j];
+      const int i = m.list_idx[j];
+      if (k > T) atomicOr(&m.keepmap[i >> 5], 1u << (i & 31));
+      else if (k == T) atomicOr(&m.tiemap[i >> 5], 1u << (i & 31));
     }
   } else {
     const uint32_t T = radix_threshold<NT>(
         [&](auto fn) {
           for (int i = threadIdx.x; i < n; i += NT) {
-            const uint32_t k = key_at<CACHED>(row, skeys, i);
+            const uint32_t k = order_key(row[i]);
             if (k >= cmin && k <= cmax) fn(k);
           }
         },
         cmin, cmax, &need, hist, scan_sh, s_pair);
     for (int base = warp * 32; base < n; base += NT) {
       const int i = base + lane;
-      const uint32_t k = i < n ? key_at<CACHED>(row, skeys, i) : 0u;
+      const uint32_t k = i < n ? order_key(row[i]) : 0u;
       const uint32_t mk = __ballot_sync(0xffffffffu, i < n && k > T);
       const uint32_t mt = __ballot_sync(0xffffffffu, i < n && k == T);
       if (lane == 0) {
-        keepmap[base >> 5] = mk;
-        tiemap[base >> 5] = mt;
+        m.keepmap[base >> 5] = mk;
+        m.tiemap[base >> 5] = mt;
       }
     }
   }
   __syncthreads();
+  return need;
+}
 
-  // ---- 5. ties: keep the `need` lowest indices equal to T; then write out
+// Sampled path.  kSamples evenly spaced scores give a key L that at least
+// `r` samples reach, r chosen well above the B/n share of the samples, so
+// that (for any but a pathological order of the scores) between B and lcap
+// keys of the row are >= L.  One pass lists exactly those keys; the B-th
+// largest of the list is then the B-th largest of the row.  Returns false
+// (having written nothing) when the count falls outside [B, lcap].
+template <int NT>
+__device__ __forceinline__ bool sampled_path(const float* __restrict__ row, int n, int B, int lcap, const Smem& m,
+                                             uint32_t* hist, uint32_t* scan_sh, uint32_t (*red)[NT / 32],
+                                             uint32_t* s_pair, uint32_t* s_bounds, uint32_t* s_count,
+                                             uint32_t* need_out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int words = (n + 31) >> 5;
+  const int ms = min(n, kSamples);
+  uint32_t mm[4] = {0xffffffffu, 0u, 0xffffffffu, 0u};
+  for (int j = threadIdx.x; j < ms; j += NT) {
+    const int i = static_cast<int>(static_cast<int64_t>(j) * n / ms);
+    const uint32_t k = order_key(row[i]);
+    m.samples[j] = k;
+    if (k > kKeyNegInf && k < kKeyPosInf) {
+      mm[2] = min(mm[2], k);
+      mm[3] = max(mm[3], k);
+    }
+  }
+  for (int w = threadIdx.x; w < words; w += NT) {
+    m.keepmap[w] = 0u;
+    m.tiemap[w] = 0u;
+  }
+  if (threadIdx.x == 0) *s_count = 0;
+  block_minmax4<NT>(mm, red);
+  const float qm = static_cast<float>(B) * static_cast<float>(ms) / static_cast<float>(n);
+  const int r = static_cast<int>(ceilf(qm + 5.f * sqrtf(qm) + 20.f));
+  uint32_t L = 0u;                                 // r >= ms: every key is listed
+  if (r < ms) {
+    if (!(mm[2] < mm[3])) return false;            // no spread among the samples
+    const float lo = key_value(mm[2]);
+    const float width = key_value(mm[3]) - lo;
+    const float scale = static_cast<float>(kBins) / width;
+    const float lo_s = lo * scale;
+    if (!(width > 0.f && isfinite(width) && isfinite(scale) && scale > 0.f && isfinite(lo_s))) return false;
+    for (int i = threadIdx.x; i < kBins; i += NT) hist[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < ms; j += NT) atomicAdd(&hist[value_bin(m.samples[j], scale, lo_s)], 1u);
+    __syncthreads();
+    uint32_t above;
+    const int bin = find_digit<NT>(hist, kBins, static_cast<uint32_t>(r), scan_sh, s_pair, &above);
+    if (warp == 0) {
+      const uint64_t k0 = first_key_in_bin(bin, scale, lo_s);
+      if (lane == 0) s_bounds[0] = static_cast<uint32_t>(k0);
+    }
+    __syncthreads();
+    L = s_bounds[0];
+  }
+  // list every key >= L (warp-aggregated appends)
+  uint32_t lmax = 0u;
+  for (int base = warp * 128; base < n; base += NT * 4) {
+    const int i = base + lane * 4;
+    uint32_t k[4];
+    if (i + 3 < n) {
+      const float4 v = *reinterpret_cast<const float4*>(row + i);
+      k[0] = order_key(v.x); k[1] = order_key(v.y); k[2] = order_key(v.z); k[3] = order_key(v.w);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) k[e] = i + e < n ? order_key(row[i + e]) : 0u;
+    }
+    uint32_t flags = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool f = i + e < n && k[e] >= L;
+      flags |= static_cast<uint32_t>(f) << e;
+      lmax = f ? max(lmax, k[e]) : lmax;
+    }
+    const uint32_t c = __popc(flags);
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    uint32_t pos = 0;
+    if (lane == 0 && total) pos = atomicAdd(s_count, total);
+    pos = __shfl_sync(0xffffffffu, pos, 0) + incl - c;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (flags & (1u << e)) {
+        if (pos < static_cast<uint32_t>(lcap)) {
+          m.list_key[pos] = k[e];
+          m.list_idx[pos] = i + e;
+        }
+        ++pos;
+      }
+    }
+  }
+  lmax = __reduce_max_sync(0xffffffffu, lmax);
+  if (lane == 0) red[1][warp] = lmax;
+  __syncthreads();
+  const uint32_t c = *s_count;
+  const bool ok = c >= static_cast<uint32_t>(B) && c <= static_cast<uint32_t>(lcap);
+  __syncthreads();                                 // every thread has read s_count
+  if (!ok) return false;
+  uint32_t hi = 0u;
+  for (int w = 0; w < NT / 32; ++w) hi = max(hi, red[1][w]);
+  __syncthreads();
+  uint32_t need = static_cast<uint32_t>(B);
+  const int nc = static_cast<int>(c);
+  const uint32_t T = radix_threshold<NT>(
+      [&](auto fn) {
+        for (int j = threadIdx.x; j < nc; j += NT) fn(m.list_key[j]);
+      },
+      L, hi, &need, hist, scan_sh, s_pair);
+  for (int j = threadIdx.x; j < nc; j += NT) {
+    const uint32_t k = m.list_key[j];
+    const int i = m.list_idx[j];
+    if (k > T) atomicOr(&m.keepmap[i >> 5], 1u << (i & 31));
+    else if (k == T) atomicOr(&m.tiemap[i >> 5], 1u << (i & 31));
+  }
+  __syncthreads();
+  *need_out = need;
+  return true;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) select_kernel(const __grid_constant__ Geom g, const Args a) {
+  constexpr int NW = NT / 32;
+  extern __shared__ uint4 select_dyn[];
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t scan_sh[NW];
+  __shared__ uint32_t red[4][NW];
+  __shared__ uint32_t s_pair[2];
+  __shared__ uint32_t s_bounds[2];
+  __shared__ uint32_t s_count;
+
+  const int u = blockIdx.x;
+  const int b = u % g.batch;
+  const int n = g.len[b];
+  const int B = a.B;
+  const float* __restrict__ row = a.scores + static_cast<int64_t>(u) * g.score_stride;
+  int32_t* __restrict__ kept = a.kept + static_cast<int64_t>(u) * B;
+
+  if (threadIdx.x == 0) a.kept_count[u] = min(n, B);
+  if (n <= B) {
+    for (int i = threadIdx.x; i < n; i += NT) kept[i] = i;
+    return;
+  }
+
+  const int wcap = (a.cap + 31) >> 5;
+  Smem m;
+  m.list_key = reinterpret_cast<uint32_t*>(select_dyn);
+  m.samples = m.list_key;
+  m.list_idx = reinterpret_cast<int32_t*>(m.list_key + max(a.lcap, kSamples));
+  m.keepmap = reinterpret_cast<uint32_t*>(m.list_idx + a.lcap);
+  m.tiemap = m.keepmap + wcap;
+
+  uint32_t need;
+  if (!sampled_path<NT>(row, n, B, a.lcap, m, hist, scan_sh, red, s_pair, s_bounds, &s_count, &need))
+    need = exact_path<NT>(row, n, B, a.lcap, m, hist, scan_sh, red, s_pair, s_bounds, &s_count);
+
+  // ties: keep the `need` lowest indices equal to T; then write out in index order
+  const int words = (n + 31) >> 5;
   const int per = (words + NT - 1) / NT;              // words per thread, contiguous
   const int w0 = min(words, static_cast<int>(threadIdx.x) * per);
   const int w1 = min(words, w0 + per);
   uint32_t cnt = 0;
-  for (int w = w0; w < w1; ++w) cnt += __popc(tiemap[w]);
+  for (int w = w0; w < w1; ++w) cnt += __popc(m.tiemap[w]);
   uint32_t total;
   uint32_t before = block_exclusive_sum<NT>(cnt, scan_sh, &total);
   for (int w = w0; w < w1 && before < need; ++w) {
-    uint32_t m = tiemap[w], take = 0u;
-    while (m && before < need) {
-      const uint32_t bit = m & (~m + 1u);
+    uint32_t bits = m.tiemap[w], take = 0u;
+    while (bits && before < need) {
+      const uint32_t bit = bits & (~bits + 1u);
       take |= bit;
-      m ^= bit;
+      bits ^= bit;
       ++before;
     }
-    if (take) keepmap[w] |= take;
+    if (take) m.keepmap[w] |= take;
   }
   __syncthreads();
   cnt = 0;
-  for (int w = w0; w < w1; ++w) cnt += __popc(keepmap[w]);
+  for (int w = w0; w < w1; ++w) cnt += __popc(m.keepmap[w]);
   uint32_t slot = block_exclusive_sum<NT>(cnt, scan_sh, &total);
   for (int w = w0; w < w1; ++w) {
-    uint32_t m = keepmap[w];
-    while (m) {
-      const int bit = __ffs(m) - 1;
+    uint32_t bits = m.keepmap[w];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
       kept[slot++] = w * 32 + bit;
-      m &= m - 1u;
+      bits &= bits - 1u;
     }
   }
 }
 
-// Dynamic shared memory of select_kernel for rows of `cap` floats.
-inline size_t smem_bytes(int64_t cap, bool cached) {
-  const int64_t wcap = (cap + 31) / 32;
-  return static_cast<size_t>((cached ? cap : 0) + 2 * wcap + 2 * kMaxCand) * 4;
+// Capacity of the key list for budget B on rows of at most `cap` keys.
+inline int list_capacity(int B, int cap) {
+  const int64_t want = int64_t{B} + B / 2 + 2048;
+  return static_cast<int>(want < cap ? want : cap);
+}
+
+// Dynamic shared memory of select_kernel.
+inline size_t smem_bytes(int cap, int lcap) {
+  const int64_t wcap = (int64_t{cap} + 31) / 32;
+  const int64_t keys = lcap > kSamples ? lcap : kSamples;
+  return static_cast<size_t>(keys + int64_t{lcap} + 2 * wcap) * 4;
 }
 
 }  // namespace select

@@ -66,14 +66,10 @@ tri_status use_device_of(const void* ptr, int* dev_out) {
     TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.score_blocks_per_sm, tri::score::score_kernel,
                                                            tri::score::kThreads, tri::score::kSmemBytes));
     if (d.score_blocks_per_sm < 1) return TRI_ERR_UNSUPPORTED;
-    const int sel_cached = static_cast<int>(tri::select::smem_bytes(tri::select::kMaxCached, true));
-    const int sel_long = static_cast<int>(tri::select::smem_bytes(tri::select::kMaxLen, false));
-    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<1024, true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, sel_cached));
-    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256, true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, sel_cached));
-    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<1024, false>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, sel_long));
+    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  tri::select::kMaxShared));
+    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  tri::select::kMaxShared));
     const int fill_smem = ((tri::compact::kMaxFillBudget + 31) / 32 + tri::compact::kMaxFillBudget) * 4;
     TRI_CUDA(cudaFuncSetAttribute(tri::compact::holefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   fill_smem));
@@ -201,15 +197,15 @@ tri_status launch_select(const Geom& g, const float* scores, int B, int32_t* kep
   const int units = g.L * g.H * g.batch;
   int max_len = 0;
   for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
-  if (max_len > tri::select::kMaxLen) return TRI_ERR_UNSUPPORTED;
   const int cap = (max_len + 3) & ~3;
-  tri::select::Args a{scores, kept, kept_count, B, cap};
-  if (cap > tri::select::kMaxCached) {
-    tri::select::select_kernel<1024, false><<<units, 1024, tri::select::smem_bytes(cap, false), s>>>(g, a);
-  } else if (cap >= 8192) {
-    tri::select::select_kernel<1024, true><<<units, 1024, tri::select::smem_bytes(cap, true), s>>>(g, a);
+  const int lcap = tri::select::list_capacity(B, cap);
+  const size_t smem = tri::select::smem_bytes(cap, lcap);
+  if (smem > static_cast<size_t>(tri::select::kMaxShared)) return TRI_ERR_UNSUPPORTED;
+  tri::select::Args a{scores, kept, kept_count, B, cap, lcap};
+  if (cap >= 8192) {
+    tri::select::select_kernel<512><<<units, 512, smem, s>>>(g, a);
   } else {
-    tri::select::select_kernel<256, true><<<units, 256, tri::select::smem_bytes(cap, true), s>>>(g, a);
+    tri::select::select_kernel<256><<<units, 256, smem, s>>>(g, a);
   }
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
@@ -223,7 +219,7 @@ tri_status launch_compact(const Geom& g, const int32_t* kept, const int32_t* kep
     const int64_t rows = int64_t{units} * B;
     if (rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
     const int64_t want = (rows * 16 + tri::compact::kGatherThreads - 1) / tri::compact::kGatherThreads;
-    const int64_t cap = int64_t{g_dev[dev].sms} * 8 * 4;
+    const int64_t cap = int64_t{g_dev[dev].sms} * tri::compact::kGatherBlocksPerSm;
     const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
     tri::compact::gather_kernel<<<grid, tri::compact::kGatherThreads, 0, s>>>(
         g, kept, kept_count, B, static_cast<uint16_t*>(k_out), static_cast<uint16_t*>(v_out), rows);

@@ -160,6 +160,15 @@ def test_all_scores_equal():
     assert np.array_equal(res.kept[0].cpu().numpy(), np.arange(333))
 
 
+def test_long_rows_select_without_shared_cache():
+    """Rows longer than the shared-memory key cache take the uncached path."""
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=50001, budget=3000,
+                    theta=5e5)
+    cache = gen.make_cache(wl, seed=15, device=DEV)
+    res = parity.run_gpu(cache)
+    check_every_unit(cache, res, literal=False)
+
+
 def test_heavy_duplicates_overflow_path():
     """Three distinct scores over 10000 keys: the threshold's bin holds more
     keys than the candidate list, so the selection takes its fallback path."""
