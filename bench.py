@@ -49,6 +49,20 @@ def dist_env():
     return ws, rank, local
 
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank compresses its own cache: a different seed per rank."""
+    return seed + rank
+
+
+def max_over_ranks(ms: float, world_size: int, device) -> float:
+    """The job's time is the slowest rank's (device-timed) time."""
+    if world_size <= 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_hbm_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -69,7 +83,7 @@ def score_kernel_fingerprint():
 
 def ncu_traffic(workload):
     """Per-launch DRAM bytes of the scoring kernel from the committed ncu summary, if current."""
-    p = os.path.join(ROOT, "profiles", "score_keys_traffic.json")
+    p = os.path.join(ROOT, "profiles", "score_keys_traffic.txt")
     try:
         with open(p) as f:
             d = json.load(f)
@@ -155,7 +169,7 @@ def run_ours(args):
     B = wl.budget
 
     t = time.time()
-    cache = gen.make_cache(wl, seed=args.seed + rank, device=dev)
+    cache = gen.make_cache(wl, seed=rank_seed(args.seed, rank), device=dev)
     torch.cuda.synchronize()
     log(f"[rank {rank}] generated {args.workload} in {time.time() - t:.1f}s")
     d = (tri.desc_contig(cache.k, cache.v) if wl.layout == "contig"
@@ -222,11 +236,7 @@ def run_ours(args):
     if st:
         raise RuntimeError(f"device status {st:#x} after the timed steps")
 
-    ms_max = ms
-    if ws > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(tt.item())
+    ms_max = max_over_ranks(ms, ws, dev)
     ms_step = ms_max / args.steps
     value = keys * ws * args.steps / (ms_max / 1e3)
 
@@ -312,11 +322,7 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
         one()
     end.record(stream)
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end)
-    if ws > 1:
-        tt = torch.tensor([ms], device=qc.device, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(start.elapsed_time(end), ws, qc.device)
     h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 4
     d2h = hkept.numel() * 4 + hcnt.numel() * 4 + hko.numel() * 2 + hvo.numel() * 2
     return {"value": keys * ws * steps / (ms / 1e3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
