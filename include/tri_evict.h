@@ -204,6 +204,38 @@ tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B,
                         void* k_out, void* v_out, void* workspace, size_t workspace_bytes,
                         tri_stream_t stream);
 
+/* ---------------------------------------------------------------- no allocation */
+
+/* Capacity, in floats, of the built-in score scratch of tri_compress_noalloc
+ * (16 MiB per device). */
+#define TRI_NOALLOC_MAX_SCORES (4 * 1024 * 1024)
+
+/* tri_compress without a caller-provided workspace.  The pages have no
+ * counterpart of this call: it exists for callers that cannot allocate
+ * device memory where they compress -- for instance a serving engine that
+ * hands nearly all free HBM to its KV-cache pool at start-up (a new
+ * cudaMalloc would fail or force cache blocks out), or a latency-critical
+ * loop that cannot take cudaMalloc's implicit device synchronisation.
+ *
+ * Same arguments, computation and results as tri_compress, except that the
+ * score matrix is kept in a fixed scratch array compiled into the library
+ * (TRI_NOALLOC_MAX_SCORES floats, 256-byte aligned, held by every device
+ * that loads the library until the process exits).  The call allocates and
+ * frees nothing.
+ *  - Limit: units * tri_score_row_stride(desc) must not exceed
+ *    TRI_NOALLOC_MAX_SCORES; larger requests return TRI_ERR_WORKSPACE
+ *    before anything is launched (split the cache, e.g. by layers).
+ *  - Set-up: the first call on a device looks up the scratch array's device
+ *    address (cudaGetSymbolAddress) with that device current; make that
+ *    first call before any stream capture.
+ *  - Sharing: every call on a device uses the same scratch array, and it
+ *    keeps the last call's contents (nothing in it needs to start at zero).
+ *    Calls that overlap on the GPU -- on different streams, or from several
+ *    host threads -- race on it: order them (one stream, or events). */
+tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int B, tri_compact_mode mode,
+                                int32_t* kept, int32_t* kept_count, void* k_out, void* v_out,
+                                tri_stream_t stream);
+
 /* ---------------------------------------------------------------- status */
 
 /* Device-side status bits (OR-ed by kernels). */

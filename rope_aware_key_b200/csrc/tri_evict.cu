@@ -81,6 +81,13 @@ tri_status use_device_of(const void* ptr, int* dev_out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Score matrix of tri_compress_noalloc: a fixed array in the module's device
+// memory (every device that loads the library holds it until exit), shared
+// by all calls.  Host code may not use the symbol as a device address; its
+// address is looked up once per device with that device current.
+static __device__ __align__(256) float g_noalloc_scores[TRI_NOALLOC_MAX_SCORES];
+float* g_noalloc_ptr[kMaxDevices] = {};
+
 // Validate `c` and fill `g` (everything except the per-call pointers the
 // kernels take separately).  `need_v`: compaction needs V.
 tri_status make_geom(const tri_cache_desc* c, bool need_v, Geom* g) {
@@ -355,6 +362,37 @@ tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B, tri_c
   if (st != TRI_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* scores = static_cast<float*>(workspace);
+  st = launch_score(g, w, scores, dev, s);
+  if (st != TRI_OK) return st;
+  st = launch_select(g, scores, B, kept, kept_count, s);
+  if (st != TRI_OK) return st;
+  return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, s);
+}
+
+tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int B, tri_compact_mode mode,
+                                int32_t* kept, int32_t* kept_count, void* k_out, void* v_out, tri_stream_t stream) {
+  Geom g;
+  tri_status st = make_geom(desc, true, &g);
+  if (st != TRI_OK) return st;
+  if (!w || !aligned16(w)) return TRI_ERR_INVALID_ARG;
+  st = check_compact_args(desc, kept, kept_count, B, mode, k_out, v_out);
+  if (st != TRI_OK) return st;
+  const int64_t units = int64_t{g.L} * g.H * g.batch;
+  if (units * g.score_stride > int64_t{TRI_NOALLOC_MAX_SCORES}) return TRI_ERR_WORKSPACE;
+  int dev;
+  st = use_device_of(desc->k, &dev);   // makes the cache's device current
+  if (st != TRI_OK) return st;
+  float* scores = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_noalloc_ptr[dev]) {
+      void* p = nullptr;
+      TRI_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scores));
+      g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    scores = g_noalloc_ptr[dev];
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   st = launch_score(g, w, scores, dev, s);
   if (st != TRI_OK) return st;
   st = launch_select(g, scores, B, kept, kept_count, s);
