@@ -542,7 +542,12 @@ __device__ __forceinline__ bool sampled_path(const float* row, int n, int B, int
   // warp-aggregated reservation per warp and pass step
   if (G::tid() == 0) S.count = 0;
   G::sync();
-  uint32_t lmax = 0u;
+  // key >= L as a float comparison: L = 0 takes every key (NaN included);
+  // L at or below -inf's key takes every number; otherwise key >= L exactly
+  // when score >= value(L) (-0 and +0 compare equal, NaN compares false).
+  const bool take_all = L == 0u;
+  const float Lv = L <= kKeyNegInf ? -INFINITY : key_value(L);
+  float lmaxf = -INFINITY;
   for (int w0 = warp * 32 * 4 * U; w0 < n; w0 += G::NT * 4 * U) {
     float4 v[U];
 #pragma unroll
@@ -559,10 +564,9 @@ __device__ __forceinline__ bool sampled_path(const float* row, int n, int B, int
       const float t[4] = {v[e].x, v[e].y, v[e].z, v[e].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const uint32_t k = order_key(t[q]);
-        const bool f = i + q < n && k >= L;
+        const bool f = i + q < n && (take_all || t[q] >= Lv);
         flags |= static_cast<uint32_t>(f) << (4 * e + q);
-        lmax = f ? max(lmax, k) : lmax;
+        lmaxf = fmaxf(lmaxf, f ? t[q] : -INFINITY);
       }
     }
     const uint32_t cnt = __popc(flags);
@@ -591,7 +595,8 @@ __device__ __forceinline__ bool sampled_path(const float* row, int n, int B, int
       }
     }
   }
-  lmax = __reduce_max_sync(0xffffffffu, lmax);
+  // the largest listed key (NaN keys are 0, below every bound)
+  const uint32_t lmax = __reduce_max_sync(0xffffffffu, max(order_key(lmaxf), L));
   if (lane == 0) S.red[1][warp] = lmax;
   G::sync();
   const uint32_t c = S.count;
@@ -656,7 +661,7 @@ __device__ __forceinline__ void select_row(const float* row, int n, int B, int l
 }
 
 template <int NT>
-__global__ void __launch_bounds__(NT) select_kernel(const __grid_constant__ Geom g, const Args a) {
+__global__ void __launch_bounds__(NT, 1024 / NT) select_kernel(const __grid_constant__ Geom g, const Args a) {
   using G = Group<NT, 0, 0>;
   extern __shared__ uint4 select_dyn[];
   __shared__ Scratch<G> S;
