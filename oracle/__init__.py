@@ -13,6 +13,7 @@ precomputed"):
 * ``score_literal``  O-ii  literal offset average of the complex form
 * ``score_folded``   O-iii folded complex form with W_f
 * ``score_polar``    O-iv  folded polar form with mu'_f = E[q_f] W_f
+* ``score_max_literal``    the max-over-offsets variant, per offset literally
 * ``fold_w`` + ``score_realdot``  O-v  the real 2x2 per-band map, then a dot
 * ``select``         keep-highest, ties to the lower index, ascending output
 * ``gather_rows`` / ``holefill``  compaction, out of place / paged in place
@@ -51,7 +52,8 @@ def _load():
     i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
     lib.orc_frequencies.argtypes = [dbl, i32, P]
     lib.orc_offset_weights.argtypes = [dbl, i32, P, i32, P, P]
-    for name in ("orc_score_cosine", "orc_score_literal", "orc_score_folded", "orc_score_polar"):
+    for name in ("orc_score_cosine", "orc_score_literal", "orc_score_folded", "orc_score_polar",
+                 "orc_score_max_literal"):
         getattr(lib, name).argtypes = [P, i64, i32, P, dbl, P, i32, dbl, i32, i32, P]
     lib.orc_fold_w.argtypes = [P, i32, i32, dbl, P, i32, dbl, i32, P]
     lib.orc_score_realdot.argtypes = [P, i64, i32, P, i32, P]
@@ -133,6 +135,11 @@ def score_cosine(keys, qc, theta, offsets, delta0=0.0, pairing=0, threads=None):
 
 def score_literal(keys, qc, theta, offsets, delta0=0.0, pairing=0, threads=None):
     return _score(_load().orc_score_literal, keys, qc, theta, offsets, delta0, pairing, threads)
+
+
+def score_max_literal(keys, qc, theta, offsets, delta0=0.0, pairing=0, threads=None):
+    """max over the schedule of the per-offset score (not foldable)."""
+    return _score(_load().orc_score_max_literal, keys, qc, theta, offsets, delta0, pairing, threads)
 
 
 def score_folded(keys, qc, theta, offsets, delta0=0.0, pairing=0, threads=None):

@@ -216,6 +216,31 @@ void orc_score_literal(const uint16_t* keys, int64_t n, int d, const float* qc, 
   });
 }
 
+// The max-over-offsets variant (same page, "What it saves, and what it does
+// not": a maximum over the offsets instead of the mean; not linear, so the
+// fold does not apply):
+//   s = max_{delta in D} Re sum_f q_f conj(k_f) e^{i omega_f (delta0 + delta)},
+// each offset's score evaluated literally.
+void orc_score_max_literal(const uint16_t* keys, int64_t n, int d, const float* qc, double theta,
+                           const double* D, int nD, double delta0, int pairing, int nthreads,
+                           double* out) {
+  const int F = d / 2;
+  std::vector<double> omega = frequencies(theta, d);
+  std::vector<cplx> q(F);
+  for (int f = 0; f < F; ++f) q[f] = band_of_center(qc, d, pairing, f);
+  parallel_for(n, nthreads, [&](int64_t i) {
+    const uint16_t* k = keys + i * d;
+    double best = -INFINITY;
+    for (int t = 0; t < nD; ++t) {
+      cplx s(0.0, 0.0);
+      for (int f = 0; f < F; ++f)
+        s += q[f] * std::conj(band_of_keys(k, d, pairing, f)) * std::polar(1.0, omega[f] * (delta0 + D[t]));
+      best = std::max(best, s.real());
+    }
+    out[i] = best;
+  });
+}
+
 // O-iii, the folded complex form:
 //   s = Re sum_f q_f conj(k_f) e^{i omega_f delta0} W_f.
 void orc_score_folded(const uint16_t* keys, int64_t n, int d, const float* qc, double theta,

@@ -378,3 +378,32 @@ def test_holefill_invariants(orc):
         assert moved == len(holes) == int(np.sum(kept >= B))
         src = [int(out[h, 0]) for h in holes]
         assert src == sorted(src) and all(x >= B for x in src)
+
+
+# ------------------------------------------------------------ max over offsets
+
+@pytest.mark.parametrize("pairing", [0, 1])
+def test_max_over_offsets_is_max_of_textbook_rope(orc, pairing):
+    """max_delta of RoPE(q at n + delta0 + delta) . RoPE(k at n), computed with
+    textbook RoPE in numpy, for a geometric schedule."""
+    bits, vals, q = rand_case(40, 128, seed=31)
+    theta, n_pos, delta0 = 1e6, 777, 5.0
+    D = [float(2 ** e) for e in range(17)]
+    kr = rope(vals, n_pos, theta, pairing)
+    per = np.stack([kr @ rope(q.astype(np.float64)[None, :], n_pos + delta0 + dl, theta, pairing)[0] for dl in D])
+    ref = per.max(axis=0)
+    got = orc.score_max_literal(bits, q, theta, D, delta0, pairing)
+    scale = np.abs(vals) @ np.abs(q.astype(np.float64))
+    assert np.all(np.abs(got - ref) <= 1e-9 * scale)
+
+
+def test_max_over_offsets_special_cases(orc):
+    bits, vals, q = rand_case(50, 128, seed=32)
+    D = [1.0, 64.0, 4096.0]
+    mx = orc.score_max_literal(bits, q, 1e4, D)
+    # a single offset: the literal score itself
+    np.testing.assert_allclose(orc.score_max_literal(bits, q, 1e4, [64.0]), orc.score_literal(bits, q, 1e4, [64.0]),
+                               rtol=1e-12, atol=1e-12)
+    # a repeated offset changes nothing; the max is at least the mean
+    np.testing.assert_allclose(orc.score_max_literal(bits, q, 1e4, D + [64.0, 1.0]), mx, rtol=0, atol=0)
+    assert np.all(mx >= orc.score_literal(bits, q, 1e4, D) - 1e-9)
