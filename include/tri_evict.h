@@ -149,6 +149,17 @@ typedef struct tri_cache_desc {
 tri_status tri_fold_weights(const tri_fold_params* params, const float* q_center,
                             int n_centers, float* w_out, tri_stream_t stream);
 
+/* Per-offset weights for the max-over-offsets score (no averaging): for each
+ * center c and offset t,
+ *     a_{f,t} = E[q_f] * e^{i omega_f (delta0 + delta_t)},
+ *     w_out[c][t][re(f)] = Re a_{f,t},   w_out[c][t][im(f)] = Im a_{f,t},
+ * i.e. the weight vector of the literal score at distance delta0 + delta_t
+ * (same page, "The same score, read as arrows in the plane").  Device fp64,
+ * stored as fp32.  q_center: device fp32 [n_centers][128];
+ * w_out: device fp32 [n_centers][n_offsets][128]. */
+tri_status tri_fold_offset_weights(const tri_fold_params* params, const float* q_center,
+                                   int n_centers, float* w_out, tri_stream_t stream);
+
 /* ---------------------------------------------------------------- score */
 
 /* Row stride (in floats) of the score matrix for `desc`: the longest row
@@ -164,6 +175,25 @@ int64_t tri_score_row_stride(const tri_cache_desc* desc);
  * [units][tri_score_row_stride(desc)]; entries i >= n_u are not written. */
 tri_status tri_score_keys(const tri_cache_desc* desc, const float* w, float* scores,
                           tri_stream_t stream);
+
+/* Longest offset schedule tri_score_keys_max accepts. */
+#define TRI_MAX_SCORE_OFFSETS 64
+
+/* The max-over-offsets variant of the score (same page, "What it saves, and
+ * what it does not": aggregating by a maximum over the offsets instead of
+ * the mean; it is not linear, so it does not fold):
+ *     scores[u][i] = max_{t < n_offsets} sum_j w[l*H + h][t][j] * float(K_u[i][j])
+ * with w from tri_fold_offset_weights (device fp32 [L*H][n_offsets][128]).
+ * Runs on the tensor cores (bf16 keys; each fp32 weight split into two bf16
+ * parts whose products accumulate in fp32, so the result keeps fp32-level
+ * accuracy).  Layouts: CONTIG and RAGGED caches whose units are packed back
+ * to back (stride_seq = seq_len*128, stride_head = batch*stride_seq,
+ * stride_layer = H*stride_head for CONTIG; stride_head = T*128 and
+ * stride_layer = H*stride_head for RAGGED with T = cu_seqlens[batch]);
+ * anything else, or n_offsets > TRI_MAX_SCORE_OFFSETS, is TRI_ERR_UNSUPPORTED.
+ * scores: as for tri_score_keys. */
+tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_offsets, float* scores,
+                              tri_stream_t stream);
 
 /* ---------------------------------------------------------------- select */
 

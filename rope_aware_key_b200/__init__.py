@@ -20,7 +20,8 @@ import torch
 
 __all__ = [
     "TriError", "lib", "Desc", "desc_contig", "desc_ragged", "desc_paged", "fold_weights", "score_keys",
-    "select_topk", "compact_kv", "compress", "workspace_size", "score_row_stride", "read_device_status",
+    "select_topk", "compact_kv", "fold_offset_weights", "score_keys_max", "compress", "workspace_size",
+    "score_row_stride", "read_device_status",
     "kernel_launches", "LAYOUT_CONTIG", "LAYOUT_RAGGED", "LAYOUT_PAGED", "PAIRING_HALF",
     "PAIRING_INTERLEAVED", "COMPACT_OUT_OF_PLACE", "COMPACT_IN_PLACE_HOLEFILL", "DEVFLAG_BAD_PAGE",
     "DEVFLAG_NONFINITE", "DEVFLAG_TIMEOUT", "DEVFLAG_BAD_KEPT",
@@ -82,6 +83,8 @@ def lib() -> ctypes.CDLL:
     P, I, I64, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     D = ctypes.POINTER(_CacheDesc)
     L.tri_fold_weights.argtypes = [ctypes.POINTER(_FoldParams), P, I, P, P]
+    L.tri_fold_offset_weights.argtypes = [ctypes.POINTER(_FoldParams), P, I, P, P]
+    L.tri_score_keys_max.argtypes = [D, P, I, P, P]
     L.tri_score_row_stride.argtypes = [D]
     L.tri_score_row_stride.restype = I64
     L.tri_score_keys.argtypes = [D, P, P, P]
@@ -95,8 +98,8 @@ def lib() -> ctypes.CDLL:
     L.tri_last_cuda_error.restype = I
     L.tri_kernel_launches.restype = ctypes.c_uint64
     L.tri_version.restype = ctypes.c_char_p
-    for name in ("tri_fold_weights", "tri_score_keys", "tri_select_topk", "tri_compact_kv",
-                 "tri_workspace_size", "tri_compress", "tri_read_device_status"):
+    for name in ("tri_fold_weights", "tri_fold_offset_weights", "tri_score_keys_max", "tri_score_keys",
+                 "tri_select_topk", "tri_compact_kv", "tri_workspace_size", "tri_compress", "tri_read_device_status"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -216,6 +219,34 @@ def fold_weights(q_center: torch.Tensor, theta: float, offsets: Sequence[float],
     _check(lib().tri_fold_weights(ctypes.byref(p), _ptr(q), q.shape[0], _ptr(out), _stream(stream)),
            "tri_fold_weights")
     return out
+
+
+def fold_offset_weights(q_center: torch.Tensor, theta: float, offsets: Sequence[float], delta0: float = 0.0,
+                        pairing: int = PAIRING_HALF, out: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """Per-offset (unaveraged) weights, fp32 [n][len(offsets)][128] on the device."""
+    q = q_center.reshape(-1, HEAD_DIM)
+    assert q.dtype == torch.float32 and q.is_cuda and q.is_contiguous()
+    offs = [float(x) for x in offsets]
+    if out is None:
+        out = torch.empty((q.shape[0], len(offs), HEAD_DIM), dtype=torch.float32, device=q.device)
+    arr = (ctypes.c_double * len(offs))(*offs)
+    p = _FoldParams(head_dim=HEAD_DIM, theta=float(theta), offsets=arr, n_offsets=len(offs),
+                    delta0=float(delta0), pairing=int(pairing))
+    _check(lib().tri_fold_offset_weights(ctypes.byref(p), _ptr(q), q.shape[0], _ptr(out), _stream(stream)),
+           "tri_fold_offset_weights")
+    return out
+
+
+def score_keys_max(d: Desc, w_offsets: torch.Tensor, scores: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Max over the offsets of the per-offset scores (tensor cores)."""
+    n_off = w_offsets.shape[-2]
+    if scores is None:
+        scores = torch.empty((d.units, score_row_stride(d)), dtype=torch.float32, device=w_offsets.device)
+    _check(lib().tri_score_keys_max(d.ref, _ptr(w_offsets), int(n_off), _ptr(scores), _stream(stream)),
+           "tri_score_keys_max")
+    return scores
 
 
 def score_row_stride(d: Desc) -> int:

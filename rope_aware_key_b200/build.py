@@ -20,6 +20,17 @@ MAIN = os.path.join(PKG, "csrc", "tri_evict.cu")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
+def _cute_include() -> str:
+    """CuTe headers (descriptor layouts for tcgen05): the copy vendored with flashinfer."""
+    import importlib.util
+    spec = importlib.util.find_spec("flashinfer")
+    if spec and spec.origin:
+        p = os.path.join(os.path.dirname(spec.origin), "data", "cutlass", "include")
+        if os.path.isdir(os.path.join(p, "cute")):
+            return p
+    raise RuntimeError("CuTe headers not found (flashinfer/data/cutlass/include)")
+
+
 def _sources():
     return (glob.glob(os.path.join(PKG, "csrc", "*.cu")) + glob.glob(os.path.join(PKG, "csrc", "*.cuh"))
             + glob.glob(os.path.join(INCLUDE, "*.h")))
@@ -46,6 +57,7 @@ def build(force: bool = False, defines=(), out: str = LIB, verbose: bool = False
     tmp = out + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared",
            "-cudart", "static", "-Xptxas", "-v", "-I", INCLUDE, "-I", os.path.join(PKG, "csrc"),
+           "-I", _cute_include(),
            *[f"-D{d}" for d in defines], "-o", tmp, MAIN]
     res = subprocess.run(cmd, capture_output=True, text=True)
     with open(os.path.join(ROOT, "_build", "ptxas.txt"), "w") as f:

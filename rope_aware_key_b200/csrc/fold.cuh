@@ -98,5 +98,32 @@ __global__ void __launch_bounds__(kThreads) fold_kernel(const __grid_constant__ 
   w[im] = static_cast<float>(ai);
 }
 
+// Per-offset weights for the max-over-offsets score (no averaging):
+//   a_{f,t} = E[q_f] e^{i w_f (delta0 + delta_t)},  w[c][t][re(f)] = Re, w[c][t][im(f)] = Im.
+// Grid: (band f, block of kThreads (center, offset) pairs); fp64, fp32 out.
+__global__ void __launch_bounds__(kThreads) fold_offsets_kernel(const __grid_constant__ Args a) {
+  const int f = blockIdx.x;
+  const double omega = pow(a.theta, -2.0 * f / kD);
+  if (f == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    bool finite = isfinite(a.theta) && isfinite(a.delta0);
+    for (int t = 0; t < a.n_offsets; ++t) finite = finite && isfinite(a.offsets[t]);
+    if (!finite) flag(TRI_DEVFLAG_NONFINITE);
+  }
+  const int idx = blockIdx.y * kThreads + threadIdx.x;
+  if (idx >= a.n_centers * a.n_offsets) return;
+  const int c = idx / a.n_offsets, t = idx - c * a.n_offsets;
+  const int re = a.pairing == TRI_PAIRING_HALF ? f : 2 * f;
+  const int im = a.pairing == TRI_PAIRING_HALF ? f + kBands : 2 * f + 1;
+  const float* q = a.q + static_cast<int64_t>(c) * kD;
+  const float qr_f = q[re], qi_f = q[im];
+  if (!isfinite(qr_f) || !isfinite(qi_f)) flag(TRI_DEVFLAG_NONFINITE);
+  double sn, cs;
+  sincos(omega * (a.delta0 + a.offsets[t]), &sn, &cs);
+  const double qr = qr_f, qi = qi_f;
+  float* w = a.w + static_cast<int64_t>(idx) * kD;
+  w[re] = static_cast<float>(cs * qr - sn * qi);
+  w[im] = static_cast<float>(sn * qr + cs * qi);
+}
+
 }  // namespace fold
 }  // namespace tri

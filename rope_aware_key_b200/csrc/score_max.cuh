@@ -1,0 +1,297 @@
+// Max-over-offsets scoring on the tensor cores:
+//     scores[u][i] = max_{t < |D|} sum_j w[l*H + h][t][j] * float(K_u[i][j]),
+// w[.][t] being the (unaveraged) weight vector of offset t.
+//
+// Page "The future-offset average in TriAttention can be precomputed",
+// section "What it saves, and what it does not": the fold relies on the
+// average being linear; a maximum over the offsets does not fold, so each
+// key needs one dot product per offset.  That is a skinny dense contraction
+// [keys x 128] x [128 x |D|], which is what the tensor cores are for:
+//  * warp 0 (one thread) streams 128-key tiles with 2-D TMA copies (two
+//    64-element boxes, 128-byte swizzle: the canonical K-major operand
+//    layout) into a ring of shared-memory stages;
+//  * warp 1 (one thread) issues tcgen05.mma kind::f16 (M = 128 keys,
+//    N = |D| rounded up to 16, K = 16 per instruction) with the keys as A and
+//    the weights as B.  bf16 weights alone would cost 2^-9 of relative
+//    accuracy, so every weight is split w = hi + lo into two bf16 parts and
+//    both products accumulate into the same fp32 accumulator in tensor memory
+//    (residual below 2^-16 of |w|); accumulators are double-buffered;
+//  * warps 2-5 read the accumulator rows (tcgen05.ld, one key per thread),
+//    take the max over the |D| columns and store the score.
+// The weights of a (layer, head) are converted and swizzled into shared memory
+// when a CTA's tile run reaches that head (runs are contiguous per CTA).
+#pragma once
+
+#include <cuda.h>
+#include <cute/arch/mma_sm100_desc.hpp>
+
+#include "common.cuh"
+#include "score.cuh"
+
+namespace tri {
+namespace smax {
+
+constexpr int kTileRows = score::kTileRows;     // 128 keys: the MMA's M
+constexpr int kStages = 4;
+constexpr int kStageBytes = kTileRows * kRowBytes;   // 32 KB: two 16 KB boxes
+constexpr int kBoxBytes = kStageBytes / 2;
+constexpr int kMaxOffsets = 64;
+constexpr int kThreads = 6 * 32;
+constexpr int kAccCols = 64;                      // columns per accumulator (N <= 64)
+constexpr uint32_t kTmemCols = 2 * kAccCols;
+constexpr int kBBytesMax = 2 * kMaxOffsets * kRowBytes;   // hi and lo parts, N <= 64
+constexpr size_t kBOffset = static_cast<size_t>(kStages) * kStageBytes;
+constexpr size_t kBarOffset = kBOffset + kBBytesMax;
+constexpr size_t kSmemBytes = kBarOffset + 256 + 1024;    // barriers, slot, alignment slack
+
+struct Args {
+  const float* w;        // [L*H][n_offsets][128]
+  float* scores;
+  int ntiles;
+  int n_offsets;         // 1 .. kMaxOffsets
+  int n_cols;            // n_offsets rounded up to 16
+};
+
+// ------------------------------------------------------------------ PTX
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+// K-major, 128-byte-swizzled operand: 8-row atoms of 1024 bytes (SBO), 16-byte
+// units along K; version 1 for sm_100.
+__device__ __forceinline__ uint64_t sw128_desc(const void* p) {
+  cute::UMMA::SmemDescriptor d;
+  d.desc_ = 0;
+  d.version_ = 1;
+  d.lbo_mode_ = 0;
+  d.layout_type_ = static_cast<uint8_t>(cute::UMMA::LayoutType::SWIZZLE_128B);
+  d.leading_byte_offset_ = 1;
+  d.stride_byte_offset_ = 1024 >> 4;
+  d.base_offset_ = 0;
+  d.start_address_ = static_cast<uint16_t>((smem_addr(p) & 0x3ffffu) >> 4);
+  return d.desc_;
+}
+
+// bf16 x bf16 -> fp32, both K-major, M = 128, N = n.
+__device__ __forceinline__ uint32_t instr_desc(int n) {
+  cute::UMMA::InstrDescriptor d;
+  d.desc_ = 0;
+  d.c_format_ = static_cast<uint8_t>(cute::UMMA::CFormat::F32);
+  d.a_format_ = static_cast<uint8_t>(cute::UMMA::F16F32Format::BF16);
+  d.b_format_ = static_cast<uint8_t>(cute::UMMA::F16F32Format::BF16);
+  d.a_major_ = static_cast<uint8_t>(cute::UMMA::Major::K);
+  d.b_major_ = static_cast<uint8_t>(cute::UMMA::Major::K);
+  d.m_dim_ = kTileRows >> 4;
+  d.n_dim_ = static_cast<uint8_t>(n >> 3);
+  return d.desc_;
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  const uint32_t no_mask = 0u;    // no output lanes disabled
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(no_mask)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this warp's 32 tensor-memory lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Byte offset of element (n, k) of a K-major operand with n_cols rows in two
+// 64-element boxes, 128-byte swizzle: 16-byte chunk index XOR (row mod 8).
+__device__ __forceinline__ uint32_t sw128_offset(int n, int k, int n_cols) {
+  const int box = k >> 6, kk = k & 63;
+  return static_cast<uint32_t>(box * n_cols * 128 + (n >> 3) * 1024 + (n & 7) * 128 +
+                               ((((kk >> 3) ^ (n & 7)) & 7) << 4) + (kk & 7) * 2);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtensorMap kmap, const Args a) {
+  extern __shared__ unsigned char smax_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smax_raw) + 1023) & ~uintptr_t{1023});
+  unsigned char* bhi = smem + kBOffset;
+  unsigned char* blo = bhi + a.n_cols * kRowBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // this CTA's contiguous run of tiles
+  const int t_begin = static_cast<int>(static_cast<int64_t>(a.ntiles) * blockIdx.x / gridDim.x);
+  const int t_end = static_cast<int>(static_cast<int64_t>(a.ntiles) * (blockIdx.x + 1) / gridDim.x);
+  const int per_lh = g.tile_prefix[g.batch];          // tiles of one (layer, head)
+  const uint32_t idesc = instr_desc(a.n_cols);
+  const uint64_t policy = policy_evict_first();
+  int k = 0, j = 0;                                   // stage-ring and accumulator counters
+  for (int t0 = t_begin; t0 < t_end;) {
+    const int lh = t0 / per_lh;
+    const int t1 = min(t_end, (lh + 1) * per_lh);
+
+    // weights of this head: bf16 hi / lo, swizzled (epilogue warps)
+    if (warp >= 2) {
+      const int kcol = threadIdx.x - 64;              // 0..127: one element column
+      for (int n = 0; n < a.n_cols; ++n) {
+        const float wv = n < a.n_offsets ? __ldg(a.w + (static_cast<int64_t>(lh) * a.n_offsets + n) * kD + kcol) : 0.f;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(wv);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(wv - __bfloat162float(hi));
+        const uint32_t off = sw128_offset(n, kcol, a.n_cols);
+        *reinterpret_cast<__nv_bfloat16*>(bhi + off) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(blo + off) = lo;
+      }
+      fence_async_smem();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+      // ---------------- producer
+      if (lane == 0) {
+        for (int t = t0; t < t1; ++t, ++k) {
+          const int s = k % kStages, n = k / kStages;
+          if (n > 0 && !*abort_flag && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) *abort_flag = 1;
+          if (*abort_flag) continue;
+          score::TileInfo T;
+          int64_t src;
+          bool ok;
+          score::decode(g, t, a.scores, &T, &src, &ok);
+          const int row = static_cast<int>(src / kD);
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          tma_load_2d(smem + static_cast<size_t>(s) * kStageBytes, &kmap, 0, row, &full[s], policy);
+          tma_load_2d(smem + static_cast<size_t>(s) * kStageBytes + kBoxBytes, &kmap, 64, row, &full[s], policy);
+        }
+      } else {
+        k += t1 - t0;
+      }
+    } else if (warp == 1) {
+      // ---------------- MMA issue
+      if (lane == 0) {
+        for (int t = t0; t < t1; ++t, ++k, ++j) {
+          const int s = k % kStages, n = k / kStages;
+          const int ab = j & 1, na = j >> 1;
+          if (!*abort_flag && !mbar_wait_bounded(&full[s], n & 1)) *abort_flag = 1;
+          if (!*abort_flag && na > 0 && !mbar_wait_bounded(&acc_empty[ab], (na - 1) & 1)) *abort_flag = 1;
+          if (*abort_flag) continue;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * kAccCols);
+          const unsigned char* stage = smem + static_cast<size_t>(s) * kStageBytes;
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            const unsigned char* b = part ? blo : bhi;
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint64_t da = sw128_desc(stage + (kk >> 2) * kBoxBytes + (kk & 3) * 32);
+              const uint64_t db = sw128_desc(b + (kk >> 2) * a.n_cols * 128 + (kk & 3) * 32);
+              mma_bf16(d_tmem, da, db, idesc, (part | kk) ? 1u : 0u);
+            }
+          }
+          mma_commit(&empty[s]);        // the stage is free once these MMAs have read it
+          mma_commit(&acc_full[ab]);    // the accumulator is ready
+        }
+      } else {
+        k += t1 - t0;
+        j += t1 - t0;
+      }
+    } else {
+      // ---------------- epilogue: one key per thread
+      const int quarter = warp & 3;                   // tensor-memory lanes 32*quarter ..
+      const int r = quarter * 32 + lane;
+      for (int t = t0; t < t1; ++t, ++j) {
+        const int ab = j & 1, na = j >> 1;
+        if (!*abort_flag && !mbar_wait_bounded(&acc_full[ab], na & 1)) *abort_flag = 1;
+        if (*abort_flag) continue;
+        tc_fence_after();
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(ab * kAccCols);
+        float v[32];
+        tmem_ld32(taddr, v);
+        float best = v[0];
+#pragma unroll
+        for (int c = 1; c < 32; ++c)
+          if (c < a.n_offsets) best = fmaxf(best, v[c]);
+        if (a.n_cols > 32) {
+          tmem_ld32(taddr + 32, v);
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (32 + c < a.n_offsets) best = fmaxf(best, v[c]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        score::TileInfo T;
+        int64_t src;
+        bool ok;
+        score::decode(g, t, a.scores, &T, &src, &ok);
+        if (r < T.rows) T.out[r] = best;
+      }
+    }
+    t0 = t1;
+    __syncthreads();   // the next head's weights overwrite bhi / blo
+  }
+
+  // never exit with copies in flight (only possible after an abort)
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    for (int s = 0; s < kStages && s < k; ++s) mbar_wait_bounded(&full[s], ((k - 1 - s) / kStages) & 1);
+  }
+  if (*abort_flag && threadIdx.x == 0) flag(TRI_DEVFLAG_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+}
+
+}  // namespace smax
+}  // namespace tri

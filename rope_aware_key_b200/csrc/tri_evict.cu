@@ -8,6 +8,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "tri_evict.h"
@@ -16,6 +18,7 @@
 #include "score.cuh"
 #include "select.cuh"
 #include "compact.cuh"
+#include "score_max.cuh"
 
 namespace {
 
@@ -70,6 +73,8 @@ tri_status use_device_of(const void* ptr, int* dev_out) {
                                   tri::select::kMaxShared));
     TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   tri::select::kMaxShared));
+    TRI_CUDA(cudaFuncSetAttribute(tri::smax::score_max_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tri::smax::kSmemBytes)));
     const int fill_smem = ((tri::compact::kMaxFillBudget + 31) / 32 + tri::compact::kMaxFillBudget) * 4;
     TRI_CUDA(cudaFuncSetAttribute(tri::compact::holefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   fill_smem));
@@ -255,12 +260,11 @@ tri_status check_compact_args(const tri_cache_desc* desc, const int32_t* kept, c
   return TRI_OK;
 }
 
-}  // namespace
 
-extern "C" {
-
-tri_status tri_fold_weights(const tri_fold_params* p, const float* q_center, int n_centers, float* w_out,
-                            tri_stream_t stream) {
+// Shared by the two fold calls: checks, then one launch with the schedule in
+// the kernel parameters (built in static storage under a lock).
+tri_status launch_fold(const tri_fold_params* p, const float* q_center, int n_centers, float* w_out,
+                       tri_stream_t stream, bool per_offset) {
   if (!p || !q_center || !w_out || n_centers < 1) return TRI_ERR_INVALID_ARG;
   if (p->head_dim != TRI_HEAD_DIM) return TRI_ERR_UNSUPPORTED;
   if (!p->offsets || p->n_offsets < 1) return TRI_ERR_INVALID_ARG;
@@ -270,6 +274,7 @@ tri_status tri_fold_weights(const tri_fold_params* p, const float* q_center, int
   for (int t = 0; t < p->n_offsets; ++t)
     if (!std::isfinite(p->offsets[t])) return TRI_ERR_INVALID_ARG;
   if (!aligned16(q_center) || !aligned16(w_out)) return TRI_ERR_INVALID_ARG;
+  if (per_offset && int64_t{n_centers} * p->n_offsets > INT32_MAX / 2) return TRI_ERR_UNSUPPORTED;
   int dev;
   tri_status st = use_device_of(q_center, &dev);
   if (st != TRI_OK) return st;
@@ -284,8 +289,98 @@ tri_status tri_fold_weights(const tri_fold_params* p, const float* q_center, int
   a.delta0 = p->delta0;
   a.n_offsets = p->n_offsets;
   std::memcpy(a.offsets, p->offsets, sizeof(double) * p->n_offsets);
-  const dim3 grid(tri::fold::kBands, (n_centers + tri::fold::kThreads - 1) / tri::fold::kThreads);
-  tri::fold::fold_kernel<<<grid, tri::fold::kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (per_offset) {
+    const int pairs = n_centers * p->n_offsets;
+    const dim3 grid(tri::fold::kBands, (pairs + tri::fold::kThreads - 1) / tri::fold::kThreads);
+    tri::fold::fold_offsets_kernel<<<grid, tri::fold::kThreads, 0, s>>>(a);
+  } else {
+    const dim3 grid(tri::fold::kBands, (n_centers + tri::fold::kThreads - 1) / tri::fold::kThreads);
+    tri::fold::fold_kernel<<<grid, tri::fold::kThreads, 0, s>>>(a);
+  }
+  ++g_launches;
+  TRI_CUDA(cudaGetLastError());
+  return TRI_OK;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Rows of the key cache as one 2-D bf16 tensor [rows][128] (256-byte rows),
+// when the layout packs the units back to back (CONTIG or RAGGED); 0 otherwise.
+int64_t packed_rows(const tri_cache_desc* c) {
+  const int64_t H = c->num_kv_heads, L = c->num_layers, Bt = c->batch;
+  if (c->layout == TRI_LAYOUT_CONTIG) {
+    const int64_t n = c->seq_len;
+    if (Bt > 1 && c->stride_seq != n * TRI_HEAD_DIM) return 0;
+    if (H > 1 && c->stride_head != Bt * n * TRI_HEAD_DIM) return 0;
+    if (L > 1 && c->stride_layer != H * Bt * n * TRI_HEAD_DIM) return 0;
+    return L * H * Bt * n;
+  }
+  if (c->layout == TRI_LAYOUT_RAGGED) {
+    const int64_t T = c->cu_seqlens[c->batch];
+    if (H > 1 && c->stride_head != T * TRI_HEAD_DIM) return 0;
+    if (L > 1 && c->stride_layer != H * T * TRI_HEAD_DIM) return 0;
+    return L * H * T;
+  }
+  return 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+tri_status tri_fold_weights(const tri_fold_params* p, const float* q_center, int n_centers, float* w_out,
+                            tri_stream_t stream) {
+  return launch_fold(p, q_center, n_centers, w_out, stream, false);
+}
+
+tri_status tri_fold_offset_weights(const tri_fold_params* p, const float* q_center, int n_centers, float* w_out,
+                                   tri_stream_t stream) {
+  return launch_fold(p, q_center, n_centers, w_out, stream, true);
+}
+
+tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_offsets, float* scores,
+                              tri_stream_t stream) {
+  Geom g;
+  tri_status st = make_geom(desc, false, &g);
+  if (st != TRI_OK) return st;
+  if (!w || !scores || !aligned16(w) || !aligned16(scores) || n_offsets < 1) return TRI_ERR_INVALID_ARG;
+  if (n_offsets > tri::smax::kMaxOffsets) return TRI_ERR_UNSUPPORTED;
+  const int64_t rows = packed_rows(desc);
+  if (rows <= 0 || rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  int dev;
+  st = use_device_of(desc->k, &dev);
+  if (st != TRI_OK) return st;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return TRI_ERR_UNSUPPORTED;
+  CUtensorMap map;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(TRI_HEAD_DIM), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(tri::kRowBytes)};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(tri::smax::kTileRows)};
+  cuuint32_t elem[2] = {1, 1};
+  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(desc->k), dims, strides, box,
+                       elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return TRI_ERR_INVALID_ARG;
+  const int64_t ntiles = fill_tile_prefix(&g);
+  if (ntiles == 0) return TRI_OK;
+  if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  tri::smax::Args a{w, scores, static_cast<int>(ntiles), n_offsets, (n_offsets + 15) & ~15};
+  const int grid = static_cast<int>(ntiles < g_dev[dev].sms ? ntiles : g_dev[dev].sms);
+  tri::smax::score_max_kernel<<<grid, tri::smax::kThreads, tri::smax::kSmemBytes,
+                                reinterpret_cast<cudaStream_t>(stream)>>>(g, map, a);
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
   return TRI_OK;

@@ -112,7 +112,7 @@ def paged(**kw):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(num_kv_heads=3, stride_block=16 * 3 * 128, stride_layer=100 * 16 * 3 * 128), 2),   # H must divide 16
+    (dict(num_kv_heads=3, stride_block=16 * 3 * 128, stride_layer=100 * 16 * 3 * 128), 2),   # H must divide 8
     (dict(block_size=64), 2),                     # block_size * H > 128
     (dict(stride_block=16 * 4 * 128 - 8), 1),     # pages overlap
     (dict(lens=(65, 1)), 1),                      # longer than max_blocks * block_size
@@ -182,3 +182,16 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(tri, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(ImportError):
         tri.lib()
+
+
+def test_score_max_checks(L):
+    P = ctypes.c_void_p
+    d = contig()                                   # packed [L][H][1][1000][128]
+    assert L.tri_score_keys_max(ctypes.byref(d), P(FAKE), 65, P(FAKE), None) == 2     # too many offsets
+    assert L.tri_score_keys_max(ctypes.byref(d), P(FAKE), 0, P(FAKE), None) == 1
+    loose = contig(stride_head=1000 * 128 + 64, stride_layer=8 * (1000 * 128 + 64))
+    assert L.tri_score_keys_max(ctypes.byref(loose), P(FAKE), 17, P(FAKE), None) == 2  # units not packed
+    pg = paged()
+    assert L.tri_score_keys_max(ctypes.byref(pg), P(FAKE), 17, P(FAKE), None) == 2     # paged: not supported
+    p = fold_params(offs=[1.0] * 3000)
+    assert L.tri_fold_offset_weights(ctypes.byref(p), P(FAKE), 4, P(FAKE), None) == 2

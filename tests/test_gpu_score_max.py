@@ -1,0 +1,121 @@
+"""The max-over-offsets score (tensor-core kernel) against the oracle's
+literal per-offset maximum, on the same seeded caches."""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import gen
+import oracle
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+GEO17 = [float(2 ** e) for e in range(17)]
+
+
+@pytest.fixture(autouse=True)
+def _cleanup():
+    yield
+    gc.collect()
+    if torch.cuda.is_available():
+        torch.cuda.empty_cache()
+
+
+def run_max(cache, offsets, delta0=0.0, pairing=0):
+    import rope_aware_key_b200 as tri
+    wl = cache.wl
+    qc = cache.query_center.reshape(-1, wl.head_dim).to(DEV).contiguous()
+    w = tri.fold_offset_weights(qc, wl.theta, offsets, delta0, pairing)
+    d = parity.make_desc(cache)
+    scores = torch.full((d.units, tri.score_row_stride(d)), float("nan"), device=DEV)
+    tri.score_keys_max(d, w, scores)
+    status = tri.read_device_status()
+    torch.cuda.synchronize()
+    return w, scores, status
+
+
+def check_offset_weights(w, cache, offsets, delta0, pairing):
+    wl = cache.wl
+    q = cache.query_center.reshape(-1, wl.head_dim)
+    got = w.cpu().numpy().astype(np.float64)
+    for t, dl in enumerate(offsets):
+        ref = oracle.fold_w(q, wl.theta, [dl], delta0, pairing)
+        err = np.abs(got[:, t] - ref)
+        assert np.all(err <= 2.0 ** -23 * np.abs(ref) + 1e-12 * np.abs(ref).max()), t
+    return got
+
+
+def check_unit_max(cache, scores, w64, l, h, b, offsets, delta0, pairing, subset=None):
+    """|s_gpu - s_ref| <= 1e-4 * max_t sum_j |w_t[j] k[j]| per key."""
+    wl = cache.wl
+    u = parity.unit_id(wl, l, h, b)
+    n = cache.lens[b]
+    keys = parity.bits16(gen.unit_rows(cache, cache.k, l, h, b))
+    s = scores[u, :n].cpu().numpy().astype(np.float64)
+    if subset:
+        idx = np.linspace(0, n - 1, num=min(n, subset)).astype(np.int64)
+        keys, s = keys[idx], s[idx]
+    ref = oracle.score_max_literal(keys, cache.query_center[l, h].numpy(), wl.theta, offsets, delta0, pairing)
+    lh = l * wl.num_kv_heads + h
+    scale = np.max(np.stack([oracle.abs_dot(keys, w64[lh, t]) for t in range(len(offsets))]), axis=0)
+    bad = np.flatnonzero(np.abs(s - ref) > parity.SCORE_TOL * scale)
+    assert bad.size == 0, (u, bad[:5], s[bad[:5]], ref[bad[:5]])
+    return float(np.max(np.abs(s - ref) / scale)) if n else 0.0
+
+
+@pytest.mark.parametrize("n_off,pairing,delta0", [(17, 0, 0.0), (1, 0, 0.0), (5, 1, 3.0), (33, 0, 0.0), (64, 0, 100.0)])
+def test_score_max_contig(n_off, pairing, delta0):
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=2, num_kv_heads=3, batch=2, seq_len=1000, theta=1e6)
+    cache = gen.make_cache(wl, seed=21, device=DEV, with_values=False)
+    offsets = GEO17[:n_off] if n_off <= 17 else [float(1 + 37 * i) for i in range(n_off)]
+    w, scores, status = run_max(cache, offsets, delta0, pairing)
+    assert status == 0
+    w64 = check_offset_weights(w, cache, offsets, delta0, pairing)
+    worst = 0.0
+    for l in range(wl.num_layers):
+        for h in range(wl.num_kv_heads):
+            for b in range(wl.batch):
+                worst = max(worst, check_unit_max(cache, scores, w64, l, h, b, offsets, delta0, pairing))
+    assert worst < 1e-5
+    assert torch.isnan(scores[:, 1000:]).all()          # row padding untouched
+
+
+def test_score_max_ragged_edges():
+    wl = gen.scaled(gen.WORKLOADS["qwen3_ragged"], num_layers=2, num_kv_heads=2, batch=7)
+    cache = gen.make_cache(wl, seed=22, device=DEV, with_values=False, lens=[1, 127, 128, 129, 300, 0, 2049])
+    w, scores, status = run_max(cache, GEO17)
+    assert status == 0
+    w64 = check_offset_weights(w, cache, GEO17, 0.0, 0)
+    for l in range(2):
+        for h in range(2):
+            for b in range(7):
+                check_unit_max(cache, scores, w64, l, h, b, GEO17, 0.0, 0)
+
+
+def test_score_max_selects_like_the_oracle():
+    """The kept set under the max score, through the same selection kernel."""
+    import rope_aware_key_b200 as tri
+    wl = gen.WORKLOADS["tiny"]
+    cache = gen.make_cache(wl, seed=23, device=DEV)
+    w, scores, status = run_max(cache, GEO17)
+    d = parity.make_desc(cache)
+    kept, cnt = tri.select_topk(d, scores, 512)
+    torch.cuda.synchronize()
+    s = scores[0, :4096].cpu().numpy()
+    np.testing.assert_array_equal(kept[0].cpu().numpy(), oracle.select(s, 512))
+
+
+def test_score_max_full_qwen3_sampled():
+    """The 36 x 8 x 32768 cache, sampled units (every CTA crosses head boundaries)."""
+    wl = gen.WORKLOADS["qwen3_full"]
+    cache = gen.make_cache(wl, seed=0, device=DEV, with_values=False)
+    w, scores, status = run_max(cache, GEO17)
+    assert status == 0
+    w64 = check_offset_weights(w, cache, GEO17, 0.0, 0)
+    for (l, h) in [(0, 0), (17, 5), (35, 7)]:
+        check_unit_max(cache, scores, w64, l, h, 0, GEO17, 0.0, 0, subset=2048)
+    # every key of every unit was written
+    assert not torch.isnan(scores).any()
