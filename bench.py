@@ -72,24 +72,31 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def score_kernel_fingerprint():
+# scoring kernel of each variant: (kernel name, its sources, committed traffic record)
+SCORE_KERNELS = {
+    "mean": ("score_kernel", ("common.cuh", "score.cuh"), "score_keys_traffic.txt"),
+    "max": ("score_max_kernel", ("common.cuh", "score.cuh", "score_max.cuh"), "score_max_traffic.txt"),
+}
+
+
+def score_kernel_fingerprint(variant="mean"):
     """Hash of the scoring kernel's sources: ncu traffic is only reported while it matches."""
     h = hashlib.sha256()
-    for name in ("common.cuh", "score.cuh"):
+    for name in SCORE_KERNELS[variant][1]:
         with open(os.path.join(ROOT, "rope_aware_key_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload):
+def ncu_traffic(workload, variant="mean"):
     """Per-launch DRAM bytes of the scoring kernel from the committed ncu summary, if current."""
-    p = os.path.join(ROOT, "profiles", "score_keys_traffic.txt")
+    p = os.path.join(ROOT, "profiles", SCORE_KERNELS[variant][2])
     try:
         with open(p) as f:
             d = json.load(f)
     except Exception:
         return None
-    if d.get("kernel_sources") != score_kernel_fingerprint() or d.get("workload") != workload:
+    if d.get("kernel_sources") != score_kernel_fingerprint(variant) or d.get("workload") != workload:
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -177,7 +184,10 @@ def run_ours(args):
     keys = sum(cache.lens) * wl.num_layers * wl.num_kv_heads
     moved = sum(min(B, n) for n in cache.lens) * wl.num_layers * wl.num_kv_heads
     qc = cache.query_center.reshape(-1, wl.head_dim).to(dev).contiguous()
-    w = torch.empty_like(qc)
+    if args.variant == "max":
+        w = torch.empty((qc.shape[0], len(wl.offsets), wl.head_dim), dtype=torch.float32, device=dev)
+    else:
+        w = torch.empty_like(qc)
     stride = tri.score_row_stride(d)
     scores = torch.empty((d.units, stride), dtype=torch.float32, device=dev)
     kept = torch.empty((d.units, B), dtype=torch.int32, device=dev)
@@ -189,10 +199,16 @@ def run_ours(args):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+        if args.variant == "max":
+            tri.fold_offset_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+        else:
+            tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        tri.score_keys(d, w, scores, stream=stream)
+        if args.variant == "max":
+            tri.score_keys_max(d, w, scores, stream=stream)
+        else:
+            tri.score_keys(d, w, scores, stream=stream)
         if ev is not None:
             ev[2].record(stream)
         tri.select_topk(d, scores, B, kept, cnt, stream=stream)
@@ -247,7 +263,7 @@ def run_ours(args):
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     step_bytes = keys * KEY_BYTES + moved * MOVE_BYTES
     step_gbs = step_bytes / (ms_step / 1e3) / 1e9
-    traffic = ncu_traffic(args.workload)
+    traffic = ncu_traffic(args.workload, args.variant)
 
     # end to end through the C ABI with host buffers (pinned), copies inside the timed region
     e2e = run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, keys, ws)
@@ -256,7 +272,9 @@ def run_ours(args):
     if rank == 0:
         cpu = cpu_baseline(wl, args) if ws == 1 and not args.no_cpu_baseline else None
         result = {
-            "metric": "keys scored+selected/s (fold + score + top-B select + K/V compaction)",
+            "metric": ("keys scored+selected/s (fold + score + top-B select + K/V compaction)" if args.variant == "mean"
+                       else "keys scored (max over offsets)+selected/s (per-offset fold + tensor-core score + "
+                            "top-B select + K/V compaction)"),
             "value": value, "unit": "keys/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16 keys/values, fp32 scores (fp64 fold)", "data": "synthetic (seeded generator)",
@@ -270,7 +288,7 @@ def run_ours(args):
                                   "select": float(per[:, 2].mean()), "compact": float(per[:, 3].mean())},
             "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_gbs,
                     "frac_of_measured": step_gbs / peak, "frac_of_8tbps_spec": step_gbs / SPEC_HBM_GBS},
-            "roofline": {"kernel": "score_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+            "roofline": {"kernel": SCORE_KERNELS[args.variant][0], "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "algorithmic_bytes_per_launch": score_bytes},
             "clocks": clocks,
@@ -303,8 +321,12 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
         cache.k.copy_(hk, non_blocking=True)
         cache.v.copy_(hv, non_blocking=True)
         qc.copy_(hq, non_blocking=True)
-        tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
-        tri.score_keys(d, w, scores, stream=stream)
+        if args.variant == "max":
+            tri.fold_offset_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+            tri.score_keys_max(d, w, scores, stream=stream)
+        else:
+            tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+            tri.score_keys(d, w, scores, stream=stream)
         tri.select_topk(d, scores, B, kept, cnt, stream=stream)
         tri.compact_kv(d, kept, cnt, B, tri.COMPACT_OUT_OF_PLACE, k_out, v_out, stream=stream)
         hkept.copy_(kept, non_blocking=True)
@@ -332,9 +354,11 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
 
 # ---------------------------------------------------------------- the oracle as a CPU baseline
 
-def oracle_unit_pipeline(orc, keys_bits, vals_bits, qc, wl, B, threads):
-    """The oracle's own path for one unit: literal per-offset average, keep-highest, gather."""
-    s = orc.score_literal(keys_bits, qc, wl.theta, wl.offsets, wl.delta0, 0, threads)
+def oracle_unit_pipeline(orc, keys_bits, vals_bits, qc, wl, B, threads, variant="mean"):
+    """The oracle's own path for one unit: literal per-offset average (or
+    maximum), keep-highest, gather."""
+    score = orc.score_max_literal if variant == "max" else orc.score_literal
+    s = score(keys_bits, qc, wl.theta, wl.offsets, wl.delta0, 0, threads)
     kept = orc.select(s, B)
     orc.gather_rows(keys_bits, kept)
     orc.gather_rows(vals_bits, kept)
@@ -362,13 +386,14 @@ def cpu_baseline(wl, args, budget_s=None):
     t0 = time.time()
     reps = 0
     while True:
-        done += oracle_unit_pipeline(orc, kb, vb, qc, wl, B, threads)
+        done += oracle_unit_pipeline(orc, kb, vb, qc, wl, B, threads, args.variant)
         reps += 1
         if time.time() - t0 >= budget_s:
             break
     dt = time.time() - t0
     return {"value": done / dt, "unit": "keys/s", "cores": threads, "kind": "oracle",
-            "sample": f"{reps} x one unit of {n} keys (literal average over |D|={len(wl.offsets)} offsets, "
+            "sample": f"{reps} x one unit of {n} keys (literal {'max' if args.variant == 'max' else 'average'} over "
+                      f"|D|={len(wl.offsets)} offsets, "
                       f"select B={B}, gather K and V), fp64, {dt:.1f}s"}
 
 
@@ -384,17 +409,17 @@ def run_reference(args):
     probe_n = 1024
     kb, vb, qc = cpu_sample(wl, probe_n, args.seed)
     t = time.time()
-    oracle_unit_pipeline(orc, kb, vb, qc, wl, min(wl.budget, probe_n), threads)
+    oracle_unit_pipeline(orc, kb, vb, qc, wl, min(wl.budget, probe_n), threads, args.variant)
     rate = probe_n / max(time.time() - t, 1e-6)
     per_step_s = min(1.0, 120.0 / max(1, args.steps + args.warmup))
     n = int(min(32768, max(256, rate * per_step_s)))
     kb, vb, qc = cpu_sample(wl, n, args.seed)
     B = min(wl.budget, n)
     for _ in range(args.warmup):
-        oracle_unit_pipeline(orc, kb, vb, qc, wl, B, threads)
+        oracle_unit_pipeline(orc, kb, vb, qc, wl, B, threads, args.variant)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_unit_pipeline(orc, kb, vb, qc, wl, B, threads)
+        oracle_unit_pipeline(orc, kb, vb, qc, wl, B, threads, args.variant)
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
     sample = (f"each step: one unit of {n} keys of the {args.workload} workload (literal average over "
@@ -419,6 +444,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", default="mean", choices=["mean", "max"],
+                    help="mean: the folded offset average (default); max: the max over the offsets")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -28,18 +28,28 @@
 #include "common.cuh"
 #include "score.cuh"
 
+#ifndef TRI_SMAX_STAGES
+#define TRI_SMAX_STAGES 4
+#endif
+#ifndef TRI_SMAX_MAX_OFFSETS
+#define TRI_SMAX_MAX_OFFSETS 64
+#endif
+#ifndef TRI_SMAX_CTAS_PER_SM
+#define TRI_SMAX_CTAS_PER_SM 1
+#endif
+
 namespace tri {
 namespace smax {
 
 constexpr int kTileRows = score::kTileRows;     // 128 keys: the MMA's M
-constexpr int kStages = 4;
+constexpr int kStages = TRI_SMAX_STAGES;
 constexpr int kStageBytes = kTileRows * kRowBytes;   // 32 KB: two 16 KB boxes
 constexpr int kBoxBytes = kStageBytes / 2;
-constexpr int kMaxOffsets = 64;
+constexpr int kMaxOffsets = TRI_SMAX_MAX_OFFSETS;
 constexpr int kThreads = 6 * 32;
-constexpr int kAccCols = 64;                      // columns per accumulator (N <= 64)
+constexpr int kAccCols = kMaxOffsets;             // columns per accumulator (N <= kMaxOffsets)
 constexpr uint32_t kTmemCols = 2 * kAccCols;
-constexpr int kBBytesMax = 2 * kMaxOffsets * kRowBytes;   // hi and lo parts, N <= 64
+constexpr int kBBytesMax = 2 * kMaxOffsets * kRowBytes;   // hi and lo parts, N <= kMaxOffsets
 constexpr size_t kBOffset = static_cast<size_t>(kStages) * kStageBytes;
 constexpr size_t kBarOffset = kBOffset + kBBytesMax;
 constexpr size_t kSmemBytes = kBarOffset + 256 + 1024;    // barriers, slot, alignment slack
@@ -135,7 +145,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int n, int k, int n_cols) {
                                ((((kk >> 3) ^ (n & 7)) & 7) << 4) + (kk & 7) * 2);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, TRI_SMAX_CTAS_PER_SM)
 score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtensorMap kmap, const Args a) {
   extern __shared__ unsigned char smax_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smax_raw) + 1023) & ~uintptr_t{1023});

@@ -32,6 +32,7 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   int score_blocks_per_sm = 0;
+  int smax_blocks_per_sm = 0;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -75,6 +76,9 @@ tri_status use_device_of(const void* ptr, int* dev_out) {
                                   tri::select::kMaxShared));
     TRI_CUDA(cudaFuncSetAttribute(tri::smax::score_max_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(tri::smax::kSmemBytes)));
+    TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.smax_blocks_per_sm, tri::smax::score_max_kernel,
+                                                           tri::smax::kThreads, tri::smax::kSmemBytes));
+    if (d.smax_blocks_per_sm < 1) return TRI_ERR_UNSUPPORTED;
     const int fill_smem = ((tri::compact::kMaxFillBudget + 31) / 32 + tri::compact::kMaxFillBudget) * 4;
     TRI_CUDA(cudaFuncSetAttribute(tri::compact::holefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   fill_smem));
@@ -378,7 +382,8 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   if (ntiles == 0) return TRI_OK;
   if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
   tri::smax::Args a{w, scores, static_cast<int>(ntiles), n_offsets, (n_offsets + 15) & ~15};
-  const int grid = static_cast<int>(ntiles < g_dev[dev].sms ? ntiles : g_dev[dev].sms);
+  const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].smax_blocks_per_sm;
+  const int grid = static_cast<int>(ntiles < resident ? ntiles : resident);
   tri::smax::score_max_kernel<<<grid, tri::smax::kThreads, tri::smax::kSmemBytes,
                                 reinterpret_cast<cudaStream_t>(stream)>>>(g, map, a);
   ++g_launches;
