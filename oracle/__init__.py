@@ -14,6 +14,7 @@ precomputed"):
 * ``score_folded``   O-iii folded complex form with W_f
 * ``score_polar``    O-iv  folded polar form with mu'_f = E[q_f] W_f
 * ``score_max_literal``    the max-over-offsets variant, per offset literally
+* ``score_at_positions``   the offset average at per-key distances (pre-RoPE cache)
 * ``fold_w`` + ``score_realdot``  O-v  the real 2x2 per-band map, then a dot
 * ``select``         keep-highest, ties to the lower index, ascending output
 * ``gather_rows`` / ``holefill``  compaction, out of place / paged in place
@@ -55,6 +56,7 @@ def _load():
     for name in ("orc_score_cosine", "orc_score_literal", "orc_score_folded", "orc_score_polar",
                  "orc_score_max_literal"):
         getattr(lib, name).argtypes = [P, i64, i32, P, dbl, P, i32, dbl, i32, i32, P]
+    lib.orc_score_at_positions.argtypes = [P, i64, i32, P, dbl, P, i32, P, i64, i32, i32, P]
     lib.orc_fold_w.argtypes = [P, i32, i32, dbl, P, i32, dbl, i32, P]
     lib.orc_score_realdot.argtypes = [P, i64, i32, P, i32, P]
     lib.orc_abs_dot.argtypes = [P, i64, i32, P, i32, P]
@@ -140,6 +142,19 @@ def score_literal(keys, qc, theta, offsets, delta0=0.0, pairing=0, threads=None)
 def score_max_literal(keys, qc, theta, offsets, delta0=0.0, pairing=0, threads=None):
     """max over the schedule of the per-offset score (not foldable)."""
     return _score(_load().orc_score_max_literal, keys, qc, theta, offsets, delta0, pairing, threads)
+
+
+def score_at_positions(keys, qc, theta, offsets, positions, t, pairing=0, threads=None):
+    """Offset average at per-key distances t - positions[i] (pre-RoPE cache)."""
+    k = _keys(keys)
+    q = _vec(qc, np.float32)
+    D = _vec(offsets, np.float64)
+    pos = _vec(positions, np.int64)
+    assert pos.shape[0] == k.shape[0]
+    out = np.empty(k.shape[0], dtype=np.float64)
+    _load().orc_score_at_positions(_ptr(k), k.shape[0], k.shape[1], _ptr(q), float(theta), _ptr(D), len(D),
+                                   _ptr(pos), int(t), int(pairing), int(threads or default_threads()), _ptr(out))
+    return out
 
 
 def score_folded(keys, qc, theta, offsets, delta0=0.0, pairing=0, threads=None):

@@ -216,6 +216,32 @@ void orc_score_literal(const uint16_t* keys, int64_t n, int d, const float* qc, 
   });
 }
 
+// Per-key distances (pre-RoPE cache): key i sits at position pos[i], the
+// query at position t, so its distance is t - pos[i]; the offset average is
+//   s_i = (1/|D|) sum_delta Re sum_f q_f conj(k_f) e^{i omega_f (t - pos[i] + delta)},
+// evaluated literally ("The averaging step - the one we improve", with the
+// distance carried per key).
+void orc_score_at_positions(const uint16_t* keys, int64_t n, int d, const float* qc, double theta,
+                            const double* D, int nD, const int64_t* pos, int64_t t, int pairing,
+                            int nthreads, double* out) {
+  const int F = d / 2;
+  std::vector<double> omega = frequencies(theta, d);
+  std::vector<cplx> q(F);
+  for (int f = 0; f < F; ++f) q[f] = band_of_center(qc, d, pairing, f);
+  parallel_for(n, nthreads, [&](int64_t i) {
+    const uint16_t* k = keys + i * d;
+    const double dist = static_cast<double>(t - pos[i]);
+    double total = 0.0;
+    for (int u = 0; u < nD; ++u) {
+      cplx s(0.0, 0.0);
+      for (int f = 0; f < F; ++f)
+        s += q[f] * std::conj(band_of_keys(k, d, pairing, f)) * std::polar(1.0, omega[f] * (dist + D[u]));
+      total += s.real();
+    }
+    out[i] = total / nD;
+  });
+}
+
 // The max-over-offsets variant (same page, "What it saves, and what it does
 // not": a maximum over the offsets instead of the mean; not linear, so the
 // fold does not apply):

@@ -407,3 +407,28 @@ def test_max_over_offsets_special_cases(orc):
     # a repeated offset changes nothing; the max is at least the mean
     np.testing.assert_allclose(orc.score_max_literal(bits, q, 1e4, D + [64.0, 1.0]), mx, rtol=0, atol=0)
     assert np.all(mx >= orc.score_literal(bits, q, 1e4, D) - 1e-9)
+
+
+# ------------------------------------------------------------ per-key distances
+
+@pytest.mark.parametrize("pairing", [0, 1])
+def test_per_key_distance_is_textbook_rope(orc, pairing):
+    """D = {delta}: key i at position p_i, query at t: RoPE(q, t + delta) . RoPE(k_i, p_i)."""
+    bits, vals, q = rand_case(30, 128, seed=41)
+    rng = np.random.default_rng(41)
+    pos = rng.integers(0, 100000, size=30)
+    t, delta, theta = 131000, 64.0, 5e5
+    qr = rope(q.astype(np.float64)[None, :], t + delta, theta, pairing)[0]
+    ref = np.array([rope(vals[i:i + 1], int(pos[i]), theta, pairing)[0] @ qr for i in range(30)])
+    got = orc.score_at_positions(bits, q, theta, [delta], pos, t, pairing)
+    scale = np.abs(vals) @ np.abs(q.astype(np.float64))
+    assert np.all(np.abs(got - ref) <= 1e-9 * scale)
+
+
+def test_per_key_distance_constant_positions(orc):
+    """Every key at the same position p: the single-distance average with delta0 = t - p."""
+    bits, vals, q = rand_case(40, 128, seed=42)
+    D = [float(2 ** e) for e in range(17)]
+    got = orc.score_at_positions(bits, q, 1e6, D, np.full(40, 1000), 4321)
+    ref = orc.score_literal(bits, q, 1e6, D, delta0=3321.0)
+    np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-10)
