@@ -76,6 +76,16 @@ def measured_hbm_peak():
 SCORE_KERNELS = {
     "mean": ("score_kernel", ("common.cuh", "score.cuh"), "score_keys_traffic.txt"),
     "max": ("score_max_kernel", ("common.cuh", "score.cuh", "score_max.cuh"), "score_max_traffic.txt"),
+    "pos": ("score_pos_kernel", ("common.cuh", "score.cuh", "score_pos.cuh"), "score_pos_traffic.txt"),
+}
+POS_SPREAD = 4             # pre-RoPE variant: keys keep 1 in 4 of the original positions
+
+METRICS = {
+    "mean": "keys scored+selected/s (fold + score + top-B select + K/V compaction)",
+    "max": ("keys scored (max over offsets)+selected/s (per-offset fold + tensor-core score + top-B select + "
+            "K/V compaction)"),
+    "pos": ("keys scored (per-key distance, pre-RoPE)+selected/s (fold + score at positions + top-B select + "
+            "K/V compaction)"),
 }
 
 
@@ -195,6 +205,10 @@ def run_ours(args):
     k_out = torch.empty((d.units, B, wl.head_dim), dtype=torch.bfloat16, device=dev)
     v_out = torch.empty_like(k_out)
     stream = torch.cuda.current_stream(dev)
+    positions = qpos = None
+    if args.variant == "pos":
+        positions, qpos = gen.key_positions(cache, seed=rank_seed(args.seed, rank), stride=stride,
+                                            spread=POS_SPREAD)
 
     def step(ev=None):
         if ev is not None:
@@ -207,6 +221,8 @@ def run_ours(args):
             ev[1].record(stream)
         if args.variant == "max":
             tri.score_keys_max(d, w, scores, stream=stream)
+        elif args.variant == "pos":
+            tri.score_keys_at_positions(d, w, wl.theta, qpos, positions, tri.PAIRING_HALF, scores, stream=stream)
         else:
             tri.score_keys(d, w, scores, stream=stream)
         if ev is not None:
@@ -259,22 +275,20 @@ def run_ours(args):
     # roofline of the dominant kernel (scoring) and of the whole step
     peak, peak_kind = measured_hbm_peak()
     score_ms = float(per[:, 1].mean())
-    score_bytes = keys * KEY_BYTES
+    score_bytes = keys * (KEY_BYTES + (4 if args.variant == "pos" else 0))   # + the positions read
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     step_bytes = keys * KEY_BYTES + moved * MOVE_BYTES
     step_gbs = step_bytes / (ms_step / 1e3) / 1e9
     traffic = ncu_traffic(args.workload, args.variant)
 
     # end to end through the C ABI with host buffers (pinned), copies inside the timed region
-    e2e = run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, keys, ws)
+    e2e = run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, keys, ws, positions, qpos)
 
     result = None
     if rank == 0:
         cpu = cpu_baseline(wl, args) if ws == 1 and not args.no_cpu_baseline else None
         result = {
-            "metric": ("keys scored+selected/s (fold + score + top-B select + K/V compaction)" if args.variant == "mean"
-                       else "keys scored (max over offsets)+selected/s (per-offset fold + tensor-core score + "
-                            "top-B select + K/V compaction)"),
+            "metric": METRICS[args.variant],
             "value": value, "unit": "keys/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16 keys/values, fp32 scores (fp64 fold)", "data": "synthetic (seeded generator)",
@@ -301,7 +315,7 @@ def run_ours(args):
     return result
 
 
-def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, keys, ws):
+def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, keys, ws, positions=None, qpos=None):
     """Same step with the cache in pinned host memory: H2D of K and V, the four
     calls, D2H of the kept indices, counts and compacted K/V, every step."""
     steps = max(1, min(args.steps, args.e2e_steps))
@@ -314,6 +328,7 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
     hko = torch.empty(k_out.shape, dtype=k_out.dtype, pin_memory=True)
     hvo = torch.empty(v_out.shape, dtype=v_out.dtype, pin_memory=True)
     hq = qc.cpu().pin_memory()
+    hpos = positions.cpu().pin_memory() if positions is not None else None
     B = kept.shape[1]
     scores = torch.empty((d.units, tri.score_row_stride(d)), dtype=torch.float32, device=qc.device)
 
@@ -321,9 +336,14 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
         cache.k.copy_(hk, non_blocking=True)
         cache.v.copy_(hv, non_blocking=True)
         qc.copy_(hq, non_blocking=True)
+        if hpos is not None:
+            positions.copy_(hpos, non_blocking=True)
         if args.variant == "max":
             tri.fold_offset_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
             tri.score_keys_max(d, w, scores, stream=stream)
+        elif args.variant == "pos":
+            tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+            tri.score_keys_at_positions(d, w, wl.theta, qpos, positions, tri.PAIRING_HALF, scores, stream=stream)
         else:
             tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
             tri.score_keys(d, w, scores, stream=stream)
@@ -345,7 +365,7 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
     end.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(start.elapsed_time(end), ws, qc.device)
-    h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 4
+    h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 4 + (hpos.numel() * 4 if hpos is not None else 0)
     d2h = hkept.numel() * 4 + hcnt.numel() * 4 + hko.numel() * 2 + hvo.numel() * 2
     return {"value": keys * ws * steps / (ms / 1e3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps,
@@ -357,8 +377,15 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
 def oracle_unit_pipeline(orc, keys_bits, vals_bits, qc, wl, B, threads, variant="mean"):
     """The oracle's own path for one unit: literal per-offset average (or
     maximum), keep-highest, gather."""
-    score = orc.score_max_literal if variant == "max" else orc.score_literal
-    s = score(keys_bits, qc, wl.theta, wl.offsets, wl.delta0, 0, threads)
+    if variant == "pos":
+        # a compacted pre-RoPE unit: sorted distinct positions in [0, POS_SPREAD * n), query at POS_SPREAD * n
+        n = keys_bits.shape[0]
+        rng = np.random.default_rng(n)
+        p = np.sort(rng.choice(POS_SPREAD * n, size=n, replace=False))
+        s = orc.score_at_positions(keys_bits, qc, wl.theta, wl.offsets, p, POS_SPREAD * n, 0, threads)
+    else:
+        score = orc.score_max_literal if variant == "max" else orc.score_literal
+        s = score(keys_bits, qc, wl.theta, wl.offsets, wl.delta0, 0, threads)
     kept = orc.select(s, B)
     orc.gather_rows(keys_bits, kept)
     orc.gather_rows(vals_bits, kept)
@@ -392,7 +419,8 @@ def cpu_baseline(wl, args, budget_s=None):
             break
     dt = time.time() - t0
     return {"value": done / dt, "unit": "keys/s", "cores": threads, "kind": "oracle",
-            "sample": f"{reps} x one unit of {n} keys (literal {'max' if args.variant == 'max' else 'average'} over "
+            "sample": f"{reps} x one unit of {n} keys (literal {'max' if args.variant == 'max' else 'average'} "
+                      f"{'at per-key distances ' if args.variant == 'pos' else ''}over "
                       f"|D|={len(wl.offsets)} offsets, "
                       f"select B={B}, gather K and V), fp64, {dt:.1f}s"}
 
@@ -422,9 +450,10 @@ def run_reference(args):
         oracle_unit_pipeline(orc, kb, vb, qc, wl, B, threads, args.variant)
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
-    sample = (f"each step: one unit of {n} keys of the {args.workload} workload (literal average over "
+    kind = {"mean": "literal average", "max": "literal max", "pos": "literal average at per-key distances"}
+    sample = (f"each step: one unit of {n} keys of the {args.workload} workload ({kind[args.variant]} over "
               f"|D|={len(wl.offsets)} offsets, select B={B}, gather K and V), fp64")
-    return {"impl": "reference", "metric": "keys scored+selected/s (fold + score + top-B select + K/V compaction)",
+    return {"impl": "reference", "metric": METRICS[args.variant],
             "value": value, "unit": "keys/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
@@ -444,8 +473,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", default="mean", choices=["mean", "max"],
-                    help="mean: the folded offset average (default); max: the max over the offsets")
+    ap.add_argument("--variant", default="mean", choices=["mean", "max", "pos"],
+                    help="mean: the folded offset average (default); max: the max over the offsets; "
+                         "pos: the offset average at per-key distances (pre-RoPE cache with positions)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -45,7 +45,7 @@ def _splitmix64(x: int) -> int:
 
 
 _TAGS = {"key_center": 1, "query_center": 2, "K": 3, "V": 4, "lens": 5,
-         "blocks": 6, "append_K": 7, "append_V": 8}
+         "blocks": 6, "append_K": 7, "append_V": 8, "positions": 9}
 
 
 def sub_seed(seed: int, tag: str, *idx: int) -> int:
@@ -259,6 +259,28 @@ def make_cache(wl: Workload, seed: int, device="cpu", with_values: bool = True,
     else:
         raise ValueError(f"unknown layout {wl.layout!r}")
     return c
+
+
+def key_positions(c: Cache, seed: int, stride: int, spread: int = 4, device=None):
+    """Positions of a pre-RoPE cache that was compacted before: for every unit
+    (order layer, head, sequence) its lens[b] keys keep a sorted random
+    sample of distinct original positions in [0, spread * lens[b]).  Returns
+    (int32 [units][stride], padding -1; the query position of each
+    sequence, spread * lens[b])."""
+    wl = c.wl
+    device = device or c.k.device
+    units = wl.num_layers * wl.num_kv_heads * wl.batch
+    pos = torch.full((units, stride), -1, dtype=torch.int32, device=device)
+    for l in range(wl.num_layers):
+        for h in range(wl.num_kv_heads):
+            for b, n in enumerate(c.lens):
+                if n == 0:
+                    continue
+                g = _gen(device, sub_seed(seed, "positions", l, h, b))
+                pick = torch.randperm(spread * n, generator=g, device=device)[:n]
+                u = (l * wl.num_kv_heads + h) * wl.batch + b
+                pos[u, :n] = torch.sort(pick).values.to(torch.int32)
+    return pos, [spread * n for n in c.lens]
 
 
 def paged_slots(table_row: torch.Tensor, n: int, bs: int) -> torch.Tensor:

@@ -176,6 +176,28 @@ int64_t tri_score_row_stride(const tri_cache_desc* desc);
 tri_status tri_score_keys(const tri_cache_desc* desc, const float* w, float* scores,
                           tri_stream_t stream);
 
+/* Score a pre-RoPE cache, where every key has its own distance to the query
+ * (same page, "The averaging step - the one we improve", with the kept
+ * distance taken per key, Delta_i = t_b - p_i, rather than one scalar):
+ *     scores[u][i] = Re sum_f a_f conj(k_f) e^{i omega_f (t_b - p_i)},
+ *     omega_f = theta^(-2f/128),  a_f = w[l*H + h][re(f)] + i w[l*H + h][im(f)]
+ * w: device fp32 [L*H][128], the folded weights of tri_fold_weights with
+ * delta0 = 0 (a nonzero delta0 adds to every key's distance).  theta and
+ * pairing must be the ones the weights were folded with.
+ * positions: device int32, 16-byte aligned, laid out like the scores
+ * ([units][row stride], entry i of unit u is the position p_i of key i), or
+ * NULL for p_i = i (a cache that has not been compacted yet); with a PAGED
+ * cache, block_size must then be a multiple of 4 (else TRI_ERR_UNSUPPORTED).  query_pos: HOST int64 [batch],
+ * the position t_b of the query of sequence b, 0 <= t_b < 2^31.
+ * Phases are reduced exactly in fixed point and evaluated with the fp32
+ * hardware sine/cosine on [-pi, pi): the result is within ~2e-6 of
+ * sum_f |a_f||k_f| of the exact value.  A key with |t_b - p_i| >= 2^31 gets
+ * a NaN score and sets TRI_DEVFLAG_BAD_POSITION.
+ * scores: as for tri_score_keys. */
+tri_status tri_score_keys_at_positions(const tri_cache_desc* desc, const float* w, double theta,
+                                       tri_pairing pairing, const int32_t* positions,
+                                       const int64_t* query_pos, float* scores, tri_stream_t stream);
+
 /* Longest offset schedule tri_score_keys_max accepts. */
 #define TRI_MAX_SCORE_OFFSETS 64
 
@@ -273,6 +295,7 @@ tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int 
 #define TRI_DEVFLAG_NONFINITE     0x2u  /* a non-finite center or offset in the fold */
 #define TRI_DEVFLAG_TIMEOUT       0x4u  /* a bounded wait inside a kernel gave up */
 #define TRI_DEVFLAG_BAD_KEPT      0x8u  /* compaction met a kept index outside [0, n) */
+#define TRI_DEVFLAG_BAD_POSITION  0x10u /* a key's distance t - p fell outside (-2^31, 2^31); its score is NaN */
 
 /* Wait for `stream`, then read the status word of the device that owns
  * `stream` (the current device for NULL) into *flags, and zero it if `clear`.

@@ -24,7 +24,8 @@ __all__ = [
     "score_row_stride", "read_device_status",
     "kernel_launches", "LAYOUT_CONTIG", "LAYOUT_RAGGED", "LAYOUT_PAGED", "PAIRING_HALF",
     "PAIRING_INTERLEAVED", "COMPACT_OUT_OF_PLACE", "COMPACT_IN_PLACE_HOLEFILL", "DEVFLAG_BAD_PAGE",
-    "DEVFLAG_NONFINITE", "DEVFLAG_TIMEOUT", "DEVFLAG_BAD_KEPT",
+    "DEVFLAG_NONFINITE", "DEVFLAG_TIMEOUT", "DEVFLAG_BAD_KEPT", "DEVFLAG_BAD_POSITION",
+    "score_keys_at_positions",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -34,6 +35,7 @@ LAYOUT_CONTIG, LAYOUT_RAGGED, LAYOUT_PAGED = 0, 1, 2
 PAIRING_HALF, PAIRING_INTERLEAVED = 0, 1
 COMPACT_OUT_OF_PLACE, COMPACT_IN_PLACE_HOLEFILL = 0, 1
 DEVFLAG_BAD_PAGE, DEVFLAG_NONFINITE, DEVFLAG_TIMEOUT, DEVFLAG_BAD_KEPT = 0x1, 0x2, 0x4, 0x8
+DEVFLAG_BAD_POSITION = 0x10
 MAX_OFFSETS, MAX_BATCH, HEAD_DIM = 2048, 256, 128
 
 _STATUS = {0: "TRI_OK", 1: "TRI_ERR_INVALID_ARG", 2: "TRI_ERR_UNSUPPORTED", 3: "TRI_ERR_WORKSPACE",
@@ -85,6 +87,7 @@ def lib() -> ctypes.CDLL:
     L.tri_fold_weights.argtypes = [ctypes.POINTER(_FoldParams), P, I, P, P]
     L.tri_fold_offset_weights.argtypes = [ctypes.POINTER(_FoldParams), P, I, P, P]
     L.tri_score_keys_max.argtypes = [D, P, I, P, P]
+    L.tri_score_keys_at_positions.argtypes = [D, P, ctypes.c_double, I, P, P, P, P]
     L.tri_score_row_stride.argtypes = [D]
     L.tri_score_row_stride.restype = I64
     L.tri_score_keys.argtypes = [D, P, P, P]
@@ -260,6 +263,23 @@ def score_keys(d: Desc, w: torch.Tensor, scores: Optional[torch.Tensor] = None, 
     if scores is None:
         scores = torch.empty((d.units, score_row_stride(d)), dtype=torch.float32, device=w.device)
     _check(lib().tri_score_keys(d.ref, _ptr(w), _ptr(scores), _stream(stream)), "tri_score_keys")
+    return scores
+
+
+def score_keys_at_positions(d: Desc, w: torch.Tensor, theta: float, query_pos: Sequence[int],
+                            positions: Optional[torch.Tensor] = None, pairing: int = PAIRING_HALF,
+                            scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Offset-averaged score of a pre-RoPE cache at each key's own distance
+    t_b - p_i.  positions: device int32 laid out like the scores, or None for
+    p_i = i; query_pos: one position per sequence."""
+    if scores is None:
+        scores = torch.empty((d.units, score_row_stride(d)), dtype=torch.float32, device=w.device)
+    if positions is not None:
+        assert positions.dtype == torch.int32 and positions.is_contiguous()
+    qp = (ctypes.c_int64 * max(1, len(query_pos)))(*[int(t) for t in query_pos])
+    _check(lib().tri_score_keys_at_positions(d.ref, _ptr(w), float(theta), int(pairing), _ptr(positions),
+                                             ctypes.cast(qp, ctypes.c_void_p), _ptr(scores), _stream(stream)),
+           "tri_score_keys_at_positions")
     return scores
 
 

@@ -49,6 +49,8 @@ struct TileInfo {
   int paged;         // rows interleave heads (PAGED)
   int lh;            // layer*H + head of row 0 (CONTIG / RAGGED), layer*H (PAGED)
   int tvalid;        // PAGED: tokens of the page inside the sequence
+  int b;             // sequence
+  int i0;            // index in the sequence of the tile's first key
   float* out;        // score of row 0 (CONTIG / RAGGED) or of head 0, token 0 (PAGED)
   int64_t head_step; // PAGED: floats between the score rows of consecutive heads
 };
@@ -67,9 +69,11 @@ __device__ __forceinline__ void decode(const Geom& g, int t, float* scores, Tile
   const int b = find_seq(g.tile_prefix, g.batch, r);
   const int j = r - g.tile_prefix[b];
   *ok = true;
+  T->b = b;
   if (g.layout == TRI_LAYOUT_PAGED) {
     const int l = outer;
     const int i0 = j * g.block_size;
+    T->i0 = i0;
     T->rows = g.block_size * g.H;
     T->paged = 1;
     T->lh = l * g.H;
@@ -87,6 +91,7 @@ __device__ __forceinline__ void decode(const Geom& g, int t, float* scores, Tile
     const int l = outer / g.H;
     const int h = outer - l * g.H;
     const int i0 = j * kTileRows;
+    T->i0 = i0;
     T->rows = min(kTileRows, g.len[b] - i0);
     T->paged = 0;
     T->lh = outer;
@@ -123,6 +128,61 @@ __device__ __forceinline__ void load_w(const float* __restrict__ w, int lh, int 
   }
 }
 
+// Nothing besides the keys travels with a tile.
+struct NoSideCopy {
+  __device__ __forceinline__ uint32_t bytes(const TileInfo&) const { return 0; }
+  __device__ __forceinline__ void issue(const TileInfo&, int, uint64_t*, uint64_t) const {}
+};
+
+// The producer thread: decodes this CTA's tiles in order, writes each one's
+// metadata next to its stage and issues its bulk copy (plus the side copies
+// of `side`, on the same barrier).  Before returning it waits (bounded) for
+// the last copy into every stage, so that no copy is in flight into the
+// shared memory of an exiting CTA.
+template <class Side = NoSideCopy>
+__device__ __forceinline__ void produce(const Geom& g, float* scores, unsigned char* smem, uint64_t* full,
+                                        uint64_t* empty, TileInfo* info, int ntiles, const Side& side = Side()) {
+  const uint64_t policy = policy_evict_first();
+  int k = 0;
+  for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
+    const int s = k % kStages, n = k / kStages;
+    if (n > 0 && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) break;
+    TileInfo T;
+    int64_t src;
+    bool ok;
+    decode(g, t, scores, &T, &src, &ok);
+    if (!ok) {
+      T.rows = 0;
+      flag(TRI_DEVFLAG_BAD_PAGE);
+    }
+    info[s] = T;
+    if (T.rows > 0) {
+      const uint32_t bytes = static_cast<uint32_t>(T.rows) * kRowBytes;
+      mbar_arrive_expect_tx(&full[s], bytes + side.bytes(T));
+      bulk_g2s(smem + static_cast<size_t>(s) * kTileBytes, g.k + src, bytes, &full[s], policy);
+      side.issue(T, s, &full[s], policy);
+    } else {
+      mbar_arrive(&full[s]);
+    }
+  }
+  for (int s = 0; s < kStages && s < k; ++s) {
+    const int last = (k - 1 - s) / kStages;   // issues on stage s: s, s+S, ... < k
+    mbar_wait_bounded(&full[s], last & 1);
+  }
+}
+
+// Barrier set-up shared by the score kernels.
+__device__ __forceinline__ void init_ring(uint64_t* full, uint64_t* empty) {
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kThreads, TRI_SCORE_CTAS_PER_SM)
 score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float* __restrict__ scores,
              int ntiles) {
@@ -132,46 +192,10 @@ score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float*
   TileInfo* info = reinterpret_cast<TileInfo*>(smem + kInfoOffset);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
+  init_ring(full, empty);
 
   if (warp == kConsumerWarps) {
-    // ---------------- producer: one thread decodes tiles and issues the copies
-    if (lane != 0) return;
-    const uint64_t policy = policy_evict_first();
-    int k = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
-      const int s = k % kStages, n = k / kStages;
-      if (n > 0 && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) break;
-      TileInfo T;
-      int64_t src;
-      bool ok;
-      decode(g, t, scores, &T, &src, &ok);
-      if (!ok) {
-        T.rows = 0;
-        flag(TRI_DEVFLAG_BAD_PAGE);
-      }
-      info[s] = T;
-      if (T.rows > 0) {
-        const uint32_t bytes = static_cast<uint32_t>(T.rows) * kRowBytes;
-        mbar_arrive_expect_tx(&full[s], bytes);
-        bulk_g2s(smem + static_cast<size_t>(s) * kTileBytes, g.k + src, bytes, &full[s], policy);
-      } else {
-        mbar_arrive(&full[s]);
-      }
-    }
-    // Never leave a copy in flight into shared memory of an exiting CTA:
-    // wait (bounded) for the latest issue on every stage.
-    for (int s = 0; s < kStages && s < k; ++s) {
-      const int last = (k - 1 - s) / kStages;   // issues on stage s: s, s+S, ... < k
-      mbar_wait_bounded(&full[s], last & 1);
-    }
+    if (lane == 0) produce(g, scores, smem, full, empty, info, ntiles);
     return;
   }
 

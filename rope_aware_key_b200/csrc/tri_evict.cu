@@ -19,6 +19,7 @@
 #include "select.cuh"
 #include "compact.cuh"
 #include "score_max.cuh"
+#include "score_pos.cuh"
 
 namespace {
 
@@ -33,6 +34,7 @@ struct DeviceInfo {
   int sms = 0;
   int score_blocks_per_sm = 0;
   int smax_blocks_per_sm = 0;
+  int pos_blocks_per_sm = 0;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -70,6 +72,17 @@ tri_status use_device_of(const void* ptr, int* dev_out) {
     TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.score_blocks_per_sm, tri::score::score_kernel,
                                                            tri::score::kThreads, tri::score::kSmemBytes));
     if (d.score_blocks_per_sm < 1) return TRI_ERR_UNSUPPORTED;
+    int pos_occ[2];
+    TRI_CUDA(cudaFuncSetAttribute(tri::score::score_pos_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tri::score::kPosSmemBytes)));
+    TRI_CUDA(cudaFuncSetAttribute(tri::score::score_pos_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tri::score::kPosSmemBytes)));
+    TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&pos_occ[0], tri::score::score_pos_kernel<0>,
+                                                           tri::score::kThreads, tri::score::kPosSmemBytes));
+    TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&pos_occ[1], tri::score::score_pos_kernel<1>,
+                                                           tri::score::kThreads, tri::score::kPosSmemBytes));
+    d.pos_blocks_per_sm = pos_occ[0] < pos_occ[1] ? pos_occ[0] : pos_occ[1];
+    if (d.pos_blocks_per_sm < 1) return TRI_ERR_UNSUPPORTED;
     TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   tri::select::kMaxShared));
     TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -386,6 +399,56 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   const int grid = static_cast<int>(ntiles < resident ? ntiles : resident);
   tri::smax::score_max_kernel<<<grid, tri::smax::kThreads, tri::smax::kSmemBytes,
                                 reinterpret_cast<cudaStream_t>(stream)>>>(g, map, a);
+  ++g_launches;
+  TRI_CUDA(cudaGetLastError());
+  return TRI_OK;
+}
+
+tri_status tri_score_keys_at_positions(const tri_cache_desc* desc, const float* w, double theta,
+                                       tri_pairing pairing, const int32_t* positions, const int64_t* query_pos,
+                                       float* scores, tri_stream_t stream) {
+  Geom g;
+  tri_status st = make_geom(desc, false, &g);
+  if (st != TRI_OK) return st;
+  if (!w || !scores || !aligned16(w) || !aligned16(scores) || !query_pos) return TRI_ERR_INVALID_ARG;
+  if (!(theta > 0.0) || !std::isfinite(theta)) return TRI_ERR_INVALID_ARG;
+  if (pairing != TRI_PAIRING_HALF && pairing != TRI_PAIRING_INTERLEAVED) return TRI_ERR_INVALID_ARG;
+  if (positions && !aligned16(positions)) return TRI_ERR_INVALID_ARG;
+  // a page's positions are copied in 16-byte pieces from a multiple of 4 tokens
+  if (positions && desc->layout == TRI_LAYOUT_PAGED && (desc->block_size % 4) != 0) return TRI_ERR_UNSUPPORTED;
+  static_assert(sizeof(tri::score::Rot) + sizeof(Geom) < 32000, "kernel parameters too large");
+  tri::score::Rot rot;
+  std::memset(&rot, 0, sizeof(rot));
+  rot.pos = positions;
+  for (int b = 0; b < g.batch; ++b) {
+    if (query_pos[b] < 0 || query_pos[b] > INT32_MAX) return TRI_ERR_INVALID_ARG;
+    rot.qpos[b] = static_cast<int32_t>(query_pos[b]);
+  }
+  // C_f = omega_f / (2 pi) * 2^55, rounded (omega_f <= 1 < 2 pi, so C_f < 2^53)
+  const long double two_pi = 6.283185307179586476925286766559L;
+  for (int f = 0; f < tri::score::kBands; ++f) {
+    const long double omega = std::pow(static_cast<long double>(theta), -2.0L * f / TRI_HEAD_DIM);
+    const long double turns = omega / two_pi;
+    if (!(turns >= 0.0L && turns < 1.0L)) return TRI_ERR_INVALID_ARG;
+    const uint64_t c = static_cast<uint64_t>(std::llround(std::ldexp(turns, 55)));
+    rot.c_hi[f] = static_cast<uint32_t>(c >> 32);
+    rot.c_lo[f] = static_cast<uint32_t>(c);
+  }
+  int dev;
+  st = use_device_of(desc->k, &dev);
+  if (st != TRI_OK) return st;
+  const int64_t ntiles = fill_tile_prefix(&g);
+  if (ntiles == 0) return TRI_OK;
+  if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].pos_blocks_per_sm;
+  const int grid = static_cast<int>(ntiles < resident ? ntiles : resident);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (pairing == TRI_PAIRING_HALF)
+    tri::score::score_pos_kernel<0><<<grid, tri::score::kThreads, tri::score::kPosSmemBytes, s>>>(
+        g, rot, w, scores, static_cast<int>(ntiles));
+  else
+    tri::score::score_pos_kernel<1><<<grid, tri::score::kThreads, tri::score::kPosSmemBytes, s>>>(
+        g, rot, w, scores, static_cast<int>(ntiles));
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
   return TRI_OK;

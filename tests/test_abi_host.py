@@ -195,3 +195,20 @@ def test_score_max_checks(L):
     assert L.tri_score_keys_max(ctypes.byref(pg), P(FAKE), 17, P(FAKE), None) == 2     # paged: not supported
     p = fold_params(offs=[1.0] * 3000)
     assert L.tri_fold_offset_weights(ctypes.byref(p), P(FAKE), 4, P(FAKE), None) == 2
+
+
+def test_score_positions_checks(L):
+    P = ctypes.c_void_p
+    d = contig()
+    fn = L.tri_score_keys_at_positions
+    qp = (ctypes.c_int64 * 1)(5000)
+    q = ctypes.cast(qp, P)
+    assert fn(ctypes.byref(d), P(FAKE), 0.0, 0, None, q, P(FAKE), None) == 1             # theta
+    assert fn(ctypes.byref(d), P(FAKE), float("inf"), 0, None, q, P(FAKE), None) == 1
+    assert fn(ctypes.byref(d), P(FAKE), 1e4, 2, None, q, P(FAKE), None) == 1             # pairing
+    assert fn(ctypes.byref(d), P(FAKE), 1e4, 0, None, None, P(FAKE), None) == 1          # no query positions
+    assert fn(ctypes.byref(d), P(FAKE), 1e4, 0, P(FAKE + 2), q, P(FAKE), None) == 1      # misaligned positions
+    for bad in (-1, 2 ** 31):
+        qb = (ctypes.c_int64 * 1)(bad)
+        assert fn(ctypes.byref(d), P(FAKE), 1e4, 0, None, ctypes.cast(qb, P), P(FAKE), None) == 1
+    assert fn(ctypes.byref(contig(head_dim=64)), P(FAKE), 1e4, 0, None, q, P(FAKE), None) == 2

@@ -116,3 +116,21 @@ def test_generator_recipe():
     assert abs(spread - wl.sigma) < 0.02
     lens = gen.seq_lengths(gen.WORKLOADS["qwen3_ragged"], 0)
     assert len(lens) == 8 and all(8192 <= n <= 32768 for n in lens)
+
+
+def test_key_positions_recipe():
+    """Positions of a compacted pre-RoPE cache: per unit sorted, distinct, inside
+    [0, spread * n), padded with -1, seeded."""
+    wl = gen.scaled(gen.WORKLOADS["qwen3_ragged"], num_layers=2, num_kv_heads=2, batch=3)
+    c = gen.make_cache(wl, seed=5, device="cpu", with_values=False, lens=[5, 0, 300])
+    pos, qpos = gen.key_positions(c, seed=5, stride=304, spread=3)
+    assert pos.shape == (12, 304) and qpos == [15, 0, 900]
+    for u in range(12):
+        b = u % 3
+        n = c.lens[b]
+        row = pos[u].numpy()
+        assert (row[n:] == -1).all()
+        assert (np.diff(row[:n]) > 0).all() and (row[:n] >= 0).all() and (row[:n] < qpos[b]).all()
+    again, _ = gen.key_positions(c, seed=5, stride=304, spread=3)
+    assert torch.equal(pos, again)
+    assert not torch.equal(pos[2], pos[5])           # units draw independently
