@@ -139,12 +139,14 @@ struct NoSideCopy {
 // of `side`, on the same barrier).  Before returning it waits (bounded) for
 // the last copy into every stage, so that no copy is in flight into the
 // shared memory of an exiting CTA.
+// The tiles a CTA takes are t_begin, t_begin + t_step, ... < t_end.
 template <class Side = NoSideCopy>
 __device__ __forceinline__ void produce(const Geom& g, float* scores, unsigned char* smem, uint64_t* full,
-                                        uint64_t* empty, TileInfo* info, int ntiles, const Side& side = Side()) {
+                                        uint64_t* empty, TileInfo* info, int t_begin, int t_end, int t_step,
+                                        const Side& side = Side()) {
   const uint64_t policy = policy_evict_first();
   int k = 0;
-  for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
+  for (int t = t_begin; t < t_end; t += t_step, ++k) {
     const int s = k % kStages, n = k / kStages;
     if (n > 0 && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) break;
     TileInfo T;
@@ -195,7 +197,7 @@ score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float*
   init_ring(full, empty);
 
   if (warp == kConsumerWarps) {
-    if (lane == 0) produce(g, scores, smem, full, empty, info, ntiles);
+    if (lane == 0) produce(g, scores, smem, full, empty, info, blockIdx.x, ntiles, gridDim.x);
     return;
   }
 

@@ -20,6 +20,7 @@
 #include "compact.cuh"
 #include "score_max.cuh"
 #include "score_pos.cuh"
+#include "score_pos_tma.cuh"
 
 namespace {
 
@@ -35,6 +36,7 @@ struct DeviceInfo {
   int score_blocks_per_sm = 0;
   int smax_blocks_per_sm = 0;
   int pos_blocks_per_sm = 0;
+  int pt_blocks_per_sm = 0;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -83,6 +85,16 @@ tri_status use_device_of(const void* ptr, int* dev_out) {
                                                            tri::score::kThreads, tri::score::kPosSmemBytes));
     d.pos_blocks_per_sm = pos_occ[0] < pos_occ[1] ? pos_occ[0] : pos_occ[1];
     if (d.pos_blocks_per_sm < 1) return TRI_ERR_UNSUPPORTED;
+    TRI_CUDA(cudaFuncSetAttribute(tri::score::score_pos_tma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tri::score::kPtSmemBytes)));
+    TRI_CUDA(cudaFuncSetAttribute(tri::score::score_pos_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tri::score::kPtSmemBytes)));
+    TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&pos_occ[0], tri::score::score_pos_tma_kernel<0>,
+                                                           tri::score::kPtThreads, tri::score::kPtSmemBytes));
+    TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&pos_occ[1], tri::score::score_pos_tma_kernel<1>,
+                                                           tri::score::kPtThreads, tri::score::kPtSmemBytes));
+    d.pt_blocks_per_sm = pos_occ[0] < pos_occ[1] ? pos_occ[0] : pos_occ[1];
+    if (d.pt_blocks_per_sm < 1) return TRI_ERR_UNSUPPORTED;
     TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   tri::select::kMaxShared));
     TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -354,6 +366,21 @@ int64_t packed_rows(const tri_cache_desc* c) {
   return 0;
 }
 
+// The key cache of a packed layout as a 2-D bf16 tensor [rows][128] for
+// tiled TMA loads: boxes of 64 elements x 128 rows, 128-byte swizzle.
+tri_status encode_key_map(const tri_cache_desc* desc, int64_t rows, CUtensorMap* map) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return TRI_ERR_UNSUPPORTED;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(TRI_HEAD_DIM), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(tri::kRowBytes)};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(tri::score::kTileRows)};
+  cuuint32_t elem[2] = {1, 1};
+  CUresult cr = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(desc->k), dims, strides, box,
+                       elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return cr == CUDA_SUCCESS ? TRI_OK : TRI_ERR_INVALID_ARG;
+}
+
 }  // namespace
 
 extern "C" {
@@ -380,17 +407,9 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   int dev;
   st = use_device_of(desc->k, &dev);
   if (st != TRI_OK) return st;
-  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
-  if (!encode) return TRI_ERR_UNSUPPORTED;
   CUtensorMap map;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(TRI_HEAD_DIM), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(tri::kRowBytes)};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(tri::smax::kTileRows)};
-  cuuint32_t elem[2] = {1, 1};
-  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(desc->k), dims, strides, box,
-                       elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return TRI_ERR_INVALID_ARG;
+  st = encode_key_map(desc, rows, &map);
+  if (st != TRI_OK) return st;
   const int64_t ntiles = fill_tile_prefix(&g);
   if (ntiles == 0) return TRI_OK;
   if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
@@ -440,9 +459,27 @@ tri_status tri_score_keys_at_positions(const tri_cache_desc* desc, const float* 
   const int64_t ntiles = fill_tile_prefix(&g);
   if (ntiles == 0) return TRI_OK;
   if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // units packed back to back: one lane per key over 2-D swizzled tiles
+  const int64_t rows = desc->layout == TRI_LAYOUT_PAGED ? 0 : packed_rows(desc);
+  if (rows > 0 && rows <= INT32_MAX) {
+    CUtensorMap map;
+    st = encode_key_map(desc, rows, &map);
+    if (st != TRI_OK) return st;
+    const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].pt_blocks_per_sm;
+    const int grid = static_cast<int>(ntiles < resident ? ntiles : resident);
+    if (pairing == TRI_PAIRING_HALF)
+      tri::score::score_pos_tma_kernel<0><<<grid, tri::score::kPtThreads, tri::score::kPtSmemBytes, s>>>(
+          g, map, rot, w, scores, static_cast<int>(ntiles));
+    else
+      tri::score::score_pos_tma_kernel<1><<<grid, tri::score::kPtThreads, tri::score::kPtSmemBytes, s>>>(
+          g, map, rot, w, scores, static_cast<int>(ntiles));
+    ++g_launches;
+    TRI_CUDA(cudaGetLastError());
+    return TRI_OK;
+  }
   const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].pos_blocks_per_sm;
   const int grid = static_cast<int>(ntiles < resident ? ntiles : resident);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (pairing == TRI_PAIRING_HALF)
     tri::score::score_pos_kernel<0><<<grid, tri::score::kThreads, tri::score::kPosSmemBytes, s>>>(
         g, rot, w, scores, static_cast<int>(ntiles));

@@ -215,3 +215,33 @@ def test_positions_full_qwen3_sampled():
     for (l, h) in [(0, 0), (17, 5), (35, 7)]:
         check_unit_pos(cache, scores, w64, None, qpos, l, h, 0, 0, subset=2048)
     assert not torch.isnan(scores).any()
+
+
+@pytest.mark.parametrize("pairing", [0, 1])
+def test_positions_unpacked_contig(pairing):
+    """A cache whose sequences are padded (not packed back to back) takes the
+    general scorer; it must agree with the oracle like the packed one."""
+    import rope_aware_key_b200 as tri
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=2, num_kv_heads=2, batch=2, seq_len=700, theta=1e6)
+    cache = gen.make_cache(wl, seed=36, device=DEV, with_values=False)
+    padded = torch.zeros((2, 2, 2, 712, 128), dtype=torch.bfloat16, device=DEV)
+    padded[..., :700, :] = cache.k
+    view = padded[..., :700, :]
+    d = tri.desc_contig(view, None)
+    qc = cache.query_center.reshape(-1, 128).to(DEV).contiguous()
+    w = tri.fold_weights(qc, wl.theta, wl.offsets, 0.0, pairing)
+    stride = tri.score_row_stride(d)
+    positions, qpos = gen.key_positions(cache, seed=36, stride=stride, spread=5)
+    scores = torch.full((d.units, stride), float("nan"), device=DEV)
+    tri.score_keys_at_positions(d, w, wl.theta, qpos, positions, pairing, scores)
+    assert tri.read_device_status() == 0
+    # the same cache packed: the fast scorer
+    packed = torch.full_like(scores, float("nan"))
+    tri.score_keys_at_positions(tri.desc_contig(cache.k, None), w, wl.theta, qpos, positions, pairing, packed)
+    torch.cuda.synchronize()
+    w64 = folded64(cache, pairing)
+    for l in range(2):
+        for h in range(2):
+            for b in range(2):
+                check_unit_pos(cache, scores, w64, positions, qpos, l, h, b, pairing)
+                check_unit_pos(cache, packed, w64, positions, qpos, l, h, b, pairing)
