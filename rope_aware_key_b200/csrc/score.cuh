@@ -51,6 +51,7 @@ struct TileInfo {
   int tvalid;        // PAGED: tokens of the page inside the sequence
   int b;             // sequence
   int i0;            // index in the sequence of the tile's first key
+  int tq;            // distance scorers: the query position of sequence b
   float* out;        // score of row 0 (CONTIG / RAGGED) or of head 0, token 0 (PAGED)
   int64_t head_step; // PAGED: floats between the score rows of consecutive heads
 };
@@ -130,6 +131,7 @@ __device__ __forceinline__ void load_w(const float* __restrict__ w, int lh, int 
 
 // Nothing besides the keys travels with a tile.
 struct NoSideCopy {
+  __device__ __forceinline__ void annotate(TileInfo&) const {}
   __device__ __forceinline__ uint32_t bytes(const TileInfo&) const { return 0; }
   __device__ __forceinline__ void issue(const TileInfo&, int, uint64_t*, uint64_t) const {}
 };
@@ -157,6 +159,7 @@ __device__ __forceinline__ void produce(const Geom& g, float* scores, unsigned c
       T.rows = 0;
       flag(TRI_DEVFLAG_BAD_PAGE);
     }
+    side.annotate(T);
     info[s] = T;
     if (T.rows > 0) {
       const uint32_t bytes = static_cast<uint32_t>(T.rows) * kRowBytes;

@@ -93,6 +93,8 @@ struct PosCopy {
   const float* w;
   unsigned char* smem;
   int H, block_size;
+  const int32_t* qpos;
+  __device__ __forceinline__ void annotate(TileInfo& T) const { T.tq = qpos[T.b]; }
   __device__ __forceinline__ uint32_t w_bytes(const TileInfo& T) const {
     return static_cast<uint32_t>(T.paged ? H : 1) * kD * 4;
   }
@@ -187,7 +189,7 @@ score_pos_kernel(const __grid_constant__ Geom g, const __grid_constant__ Rot rot
   if (warp == kConsumerWarps) {
     if (lane == 0)
       produce(g, scores, smem, full, empty, info, blockIdx.x, ntiles, gridDim.x,
-              PosCopy{rot.pos, scores, w, smem, g.H, g.block_size});
+              PosCopy{rot.pos, scores, w, smem, g.H, g.block_size, rot.qpos});
     return;
   }
 
@@ -209,7 +211,7 @@ score_pos_kernel(const __grid_constant__ Geom g, const __grid_constant__ Rot rot
     const TileInfo T = info[s];
     const bool live = r < T.rows && tok < (paged ? T.tvalid : T.rows);
     if (T.rows > 0) {
-      const int32_t t_b = rot.qpos[T.b];
+      const int32_t t_b = T.tq;
       const int32_t* sp = reinterpret_cast<const int32_t*>(smem + kPosOffset + s * kPosStageBytes);
       const int32_t p_i = !live ? t_b : rot.pos ? sp[paged ? h * g.block_size + tok : r] : T.i0 + tok;
       const Dist d = distance(t_b, p_i);

@@ -83,6 +83,7 @@ score_pos_tma_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUt
       int64_t src;
       bool ok;
       decode(g, t, scores, &T, &src, &ok);     // CONTIG / RAGGED: always ok
+      T.tq = rot.qpos[T.b];
       info[s] = T;
       unsigned char* stage = smem + static_cast<size_t>(s) * kTileBytes;
       // a tiled copy always lands (and counts) the whole box; rows past the
@@ -109,7 +110,7 @@ score_pos_tma_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUt
     if (!mbar_wait_bounded(&full[s], n & 1)) break;
     const TileInfo T = info[s];
     const bool live = r < T.rows;
-    const int32_t t_b = rot.qpos[T.b];
+    const int32_t t_b = T.tq;
     const int32_t* sp = reinterpret_cast<const int32_t*>(smem + kPtPosOffset + s * kPosStageBytes);
     const int32_t p_i = !live ? t_b : rot.pos ? sp[r] : T.i0 + r;
     const Dist d = distance(t_b, p_i);
