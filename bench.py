@@ -76,7 +76,8 @@ def measured_hbm_peak():
 SCORE_KERNELS = {
     "mean": ("score_kernel", ("common.cuh", "score.cuh"), "score_keys_traffic.txt"),
     "max": ("score_max_kernel", ("common.cuh", "score.cuh", "score_max.cuh"), "score_max_traffic.txt"),
-    "pos": ("score_pos_kernel", ("common.cuh", "score.cuh", "score_pos.cuh"), "score_pos_traffic.txt"),
+    "pos": ("score_pos_tma_kernel", ("common.cuh", "score.cuh", "score_max.cuh", "score_pos.cuh",
+                                     "score_pos_tma.cuh"), "score_pos_traffic.txt"),
 }
 POS_SPREAD = 4             # pre-RoPE variant: keys keep 1 in 4 of the original positions
 
