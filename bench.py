@@ -211,29 +211,30 @@ def run_ours(args):
         positions, qpos = gen.key_positions(cache, seed=rank_seed(args.seed, rank), stride=stride,
                                             spread=POS_SPREAD)
 
-    def step(ev=None):
+    def step(ev=None, st=None):
+        st = st or stream
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record(st)
         if args.variant == "max":
-            tri.fold_offset_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+            tri.fold_offset_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=st)
         else:
-            tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+            tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=st)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(st)
         if args.variant == "max":
-            tri.score_keys_max(d, w, scores, stream=stream)
+            tri.score_keys_max(d, w, scores, stream=st)
         elif args.variant == "pos":
-            tri.score_keys_at_positions(d, w, wl.theta, qpos, positions, tri.PAIRING_HALF, scores, stream=stream)
+            tri.score_keys_at_positions(d, w, wl.theta, qpos, positions, tri.PAIRING_HALF, scores, stream=st)
         else:
-            tri.score_keys(d, w, scores, stream=stream)
+            tri.score_keys(d, w, scores, stream=st)
         if ev is not None:
-            ev[2].record(stream)
-        tri.select_topk(d, scores, B, kept, cnt, stream=stream)
+            ev[2].record(st)
+        tri.select_topk(d, scores, B, kept, cnt, stream=st)
         if ev is not None:
-            ev[3].record(stream)
-        tri.compact_kv(d, kept, cnt, B, tri.COMPACT_OUT_OF_PLACE, k_out, v_out, stream=stream)
+            ev[3].record(st)
+        tri.compact_kv(d, kept, cnt, B, tri.COMPACT_OUT_OF_PLACE, k_out, v_out, stream=st)
         if ev is not None:
-            ev[4].record(stream)
+            ev[4].record(st)
 
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
@@ -245,7 +246,19 @@ def run_ours(args):
     if st:
         raise RuntimeError(f"device status {st:#x} after warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # The timed steps replay the step as one CUDA graph (its launches issued
+    # with no host work in between); --eager times plain launches instead.
+    graph = None
+    launches_per_step = 4
+    if not args.eager:
+        graph = torch.cuda.CUDAGraph()
+        before = tri.kernel_launches()
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+            step(st=torch.cuda.current_stream(dev))
+        launches_per_step = tri.kernel_launches() - before
+        graph.replay()
+        torch.cuda.synchronize()
+
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if ws > 1:
         torch.distributed.barrier()
@@ -254,16 +267,28 @@ def run_ours(args):
     t0 = time.time()
     start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
     end.record(stream)
     torch.cuda.synchronize()
     t1 = time.time()
     if ws > 1:
         torch.distributed.barrier()
-    launches = tri.kernel_launches() - launches0
+    launches = launches_per_step * args.steps if graph is not None else tri.kernel_launches() - launches0
     ms = start.elapsed_time(end)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
+
+    # Per-kernel times: plain launches with events between the kernels, queued
+    # behind a GPU sleep so that the host is far ahead when they run.
+    nb = min(args.steps, 100)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nb)]
+    torch.cuda._sleep(int(4e7 + nb * 4e5))
+    for i in range(nb):
+        step(evs[i])
+    torch.cuda.synchronize()
     per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])   # ms: fold, score, select, compact
     st = tri.read_device_status()
     if st:
@@ -308,6 +333,8 @@ def run_ours(args):
                          "traffic": traffic, "algorithmic_bytes_per_launch": score_bytes},
             "clocks": clocks,
             "gpu_launches": int(launches),
+            "timing": ("CUDA graph of the step, replayed" if graph is not None else "plain launches") +
+                      "; step_breakdown_ms from plain launches queued ahead of the GPU",
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
@@ -474,6 +501,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time plain launches instead of a CUDA graph of the step")
     ap.add_argument("--variant", default="mean", choices=["mean", "max", "pos"],
                     help="mean: the folded offset average (default); max: the max over the offsets; "
                          "pos: the offset average at per-key distances (pre-RoPE cache with positions)")

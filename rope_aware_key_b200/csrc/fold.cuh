@@ -26,6 +26,11 @@ namespace fold {
 constexpr int kThreads = 256;
 constexpr int kBands = kD / 2;
 
+// The schedule travels in the kernel parameters; short schedules (the usual
+// case) use a small parameter block, which launches faster than the largest.
+constexpr int kSmallOffsets = 64;
+
+template <int MAX_OFFSETS>
 struct Args {
   const float* q;     // [n_centers][128]
   float* w;           // [n_centers][128]
@@ -34,14 +39,16 @@ struct Args {
   double theta;
   double delta0;
   int n_offsets;
-  double offsets[TRI_MAX_OFFSETS];
+  double omega[kBands];            // theta^(-2f/128), computed on the host in fp64
+  double offsets[MAX_OFFSETS];
 };
 
-__global__ void __launch_bounds__(kThreads) fold_kernel(const __grid_constant__ Args a) {
+template <int N>
+__global__ void __launch_bounds__(kThreads) fold_kernel(const __grid_constant__ Args<N> a) {
   __shared__ double s_c[kThreads / 32], s_s[kThreads / 32];
   const int f = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const double omega = pow(a.theta, -2.0 * f / kD);
+  const double omega = a.omega[f];
 
   // W_f = mean over the schedule of e^{i omega delta}
   double c = 0.0, s = 0.0;
@@ -101,9 +108,10 @@ __global__ void __launch_bounds__(kThreads) fold_kernel(const __grid_constant__ 
 // Per-offset weights for the max-over-offsets score (no averaging):
 //   a_{f,t} = E[q_f] e^{i w_f (delta0 + delta_t)},  w[c][t][re(f)] = Re, w[c][t][im(f)] = Im.
 // Grid: (band f, block of kThreads (center, offset) pairs); fp64, fp32 out.
-__global__ void __launch_bounds__(kThreads) fold_offsets_kernel(const __grid_constant__ Args a) {
+template <int N>
+__global__ void __launch_bounds__(kThreads) fold_offsets_kernel(const __grid_constant__ Args<N> a) {
   const int f = blockIdx.x;
-  const double omega = pow(a.theta, -2.0 * f / kD);
+  const double omega = a.omega[f];
   if (f == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     bool finite = isfinite(a.theta) && isfinite(a.delta0);
     for (int t = 0; t < a.n_offsets; ++t) finite = finite && isfinite(a.offsets[t]);

@@ -290,8 +290,32 @@ tri_status check_compact_args(const tri_cache_desc* desc, const int32_t* kept, c
 }
 
 
+// Fill the parameter block and launch one of the fold kernels.
+template <int N>
+void launch_fold_n(const tri_fold_params* p, const float* q_center, int n_centers, float* w_out, cudaStream_t s,
+                   bool per_offset) {
+  static tri::fold::Args<N> a;   // parameter block: built in static storage (under the caller's lock)
+  a.q = q_center;
+  a.w = w_out;
+  a.n_centers = n_centers;
+  a.pairing = p->pairing;
+  a.theta = p->theta;
+  a.delta0 = p->delta0;
+  a.n_offsets = p->n_offsets;
+  for (int f = 0; f < tri::fold::kBands; ++f) a.omega[f] = std::pow(p->theta, -2.0 * f / TRI_HEAD_DIM);
+  std::memcpy(a.offsets, p->offsets, sizeof(double) * p->n_offsets);
+  if (per_offset) {
+    const int pairs = n_centers * p->n_offsets;
+    const dim3 grid(tri::fold::kBands, (pairs + tri::fold::kThreads - 1) / tri::fold::kThreads);
+    tri::fold::fold_offsets_kernel<N><<<grid, tri::fold::kThreads, 0, s>>>(a);
+  } else {
+    const dim3 grid(tri::fold::kBands, (n_centers + tri::fold::kThreads - 1) / tri::fold::kThreads);
+    tri::fold::fold_kernel<N><<<grid, tri::fold::kThreads, 0, s>>>(a);
+  }
+}
+
 // Shared by the two fold calls: checks, then one launch with the schedule in
-// the kernel parameters (built in static storage under a lock).
+// the kernel parameters.
 tri_status launch_fold(const tri_fold_params* p, const float* q_center, int n_centers, float* w_out,
                        tri_stream_t stream, bool per_offset) {
   if (!p || !q_center || !w_out || n_centers < 1) return TRI_ERR_INVALID_ARG;
@@ -307,26 +331,13 @@ tri_status launch_fold(const tri_fold_params* p, const float* q_center, int n_ce
   int dev;
   tri_status st = use_device_of(q_center, &dev);
   if (st != TRI_OK) return st;
-  static tri::fold::Args a;   // large parameter block: built in static storage, copied by the launch
   static std::mutex m;
   std::lock_guard<std::mutex> lock(m);
-  a.q = q_center;
-  a.w = w_out;
-  a.n_centers = n_centers;
-  a.pairing = p->pairing;
-  a.theta = p->theta;
-  a.delta0 = p->delta0;
-  a.n_offsets = p->n_offsets;
-  std::memcpy(a.offsets, p->offsets, sizeof(double) * p->n_offsets);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (per_offset) {
-    const int pairs = n_centers * p->n_offsets;
-    const dim3 grid(tri::fold::kBands, (pairs + tri::fold::kThreads - 1) / tri::fold::kThreads);
-    tri::fold::fold_offsets_kernel<<<grid, tri::fold::kThreads, 0, s>>>(a);
-  } else {
-    const dim3 grid(tri::fold::kBands, (n_centers + tri::fold::kThreads - 1) / tri::fold::kThreads);
-    tri::fold::fold_kernel<<<grid, tri::fold::kThreads, 0, s>>>(a);
-  }
+  if (p->n_offsets <= tri::fold::kSmallOffsets)
+    launch_fold_n<tri::fold::kSmallOffsets>(p, q_center, n_centers, w_out, s, per_offset);
+  else
+    launch_fold_n<TRI_MAX_OFFSETS>(p, q_center, n_centers, w_out, s, per_offset);
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
   return TRI_OK;
