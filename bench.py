@@ -206,6 +206,10 @@ def run_ours(args):
     k_out = torch.empty((d.units, B, wl.head_dim), dtype=torch.bfloat16, device=dev)
     v_out = torch.empty_like(k_out)
     stream = torch.cuda.current_stream(dev)
+    ws_buf = None
+    if args.path == "compress":
+        assert args.variant == "mean", "--path compress runs the folded score"
+        ws_buf = torch.empty(tri.workspace_size(d, B), dtype=torch.uint8, device=dev)
     positions = qpos = None
     if args.variant == "pos":
         positions, qpos = gen.key_positions(cache, seed=rank_seed(args.seed, rank), stride=stride,
@@ -221,6 +225,13 @@ def run_ours(args):
             tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=st)
         if ev is not None:
             ev[1].record(st)
+        if args.path == "compress":
+            # one call: the single-kernel step when the units fit one wave of clusters, else three kernels
+            tri.compress(d, w, B, tri.COMPACT_OUT_OF_PLACE, kept, cnt, k_out, v_out, ws_buf, stream=st)
+            if ev is not None:
+                for e in ev[2:]:
+                    e.record(st)
+            return
         if args.variant == "max":
             tri.score_keys_max(d, w, scores, stream=st)
         elif args.variant == "pos":
@@ -298,10 +309,12 @@ def run_ours(args):
     ms_step = ms_max / args.steps
     value = keys * ws * args.steps / (ms_max / 1e3)
 
-    # roofline of the dominant kernel (scoring) and of the whole step
+    # roofline of the dominant kernel (scoring; or the one-call step) and of the whole step
     peak, peak_kind = measured_hbm_peak()
     score_ms = float(per[:, 1].mean())
     score_bytes = keys * (KEY_BYTES + (4 if args.variant == "pos" else 0))   # + the positions read
+    if args.path == "compress":
+        score_bytes = keys * KEY_BYTES + moved * MOVE_BYTES
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     step_bytes = keys * KEY_BYTES + moved * MOVE_BYTES
     step_gbs = step_bytes / (ms_step / 1e3) / 1e9
@@ -324,13 +337,17 @@ def run_ours(args):
                        "keys_per_gpu": keys, "budget": B, "parallelism": f"independent caches x{ws}",
                        "l2": "inputs larger than L2 (K and V of %.2f GB each vs 126 MB); no flush"
                              % (keys * KEY_BYTES / 1e9)},
-            "step_breakdown_ms": {"fold": float(per[:, 0].mean()), "score": score_ms,
-                                  "select": float(per[:, 2].mean()), "compact": float(per[:, 3].mean())},
+            "step_breakdown_ms": ({"fold": float(per[:, 0].mean()), "score": score_ms,
+                                   "select": float(per[:, 2].mean()), "compact": float(per[:, 3].mean())}
+                                  if args.path == "calls" else
+                                  {"fold": float(per[:, 0].mean()), "compress": score_ms}),
             "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_gbs,
                     "frac_of_measured": step_gbs / peak, "frac_of_8tbps_spec": step_gbs / SPEC_HBM_GBS},
-            "roofline": {"kernel": SCORE_KERNELS[args.variant][0], "bound": "hbm", "achieved": achieved, "peak": peak,
+            "roofline": {"kernel": (SCORE_KERNELS[args.variant][0] if args.path == "calls" else
+                                    f"tri_compress ({launches_per_step - 1} kernel(s))"), "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": traffic, "algorithmic_bytes_per_launch": score_bytes},
+                         "traffic": traffic if args.path == "calls" else None,
+                         "algorithmic_bytes_per_launch": score_bytes},
             "clocks": clocks,
             "gpu_launches": int(launches),
             "timing": ("CUDA graph of the step, replayed" if graph is not None else "plain launches") +
@@ -359,6 +376,8 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
     hpos = positions.cpu().pin_memory() if positions is not None else None
     B = kept.shape[1]
     scores = torch.empty((d.units, tri.score_row_stride(d)), dtype=torch.float32, device=qc.device)
+    ws_e2e = torch.empty(tri.workspace_size(d, B), dtype=torch.uint8, device=qc.device) \
+        if args.path == "compress" else None
 
     def one():
         cache.k.copy_(hk, non_blocking=True)
@@ -366,7 +385,10 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
         qc.copy_(hq, non_blocking=True)
         if hpos is not None:
             positions.copy_(hpos, non_blocking=True)
-        if args.variant == "max":
+        if args.path == "compress":
+            tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+            tri.compress(d, w, B, tri.COMPACT_OUT_OF_PLACE, kept, cnt, k_out, v_out, ws_e2e, stream=stream)
+        elif args.variant == "max":
             tri.fold_offset_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
             tri.score_keys_max(d, w, scores, stream=stream)
         elif args.variant == "pos":
@@ -502,6 +524,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time plain launches instead of a CUDA graph of the step")
+    ap.add_argument("--path", default="calls", choices=["calls", "compress"],
+                    help="calls: fold, score, select, compact as four calls (default); compress: fold + tri_compress")
     ap.add_argument("--variant", default="mean", choices=["mean", "max", "pos"],
                     help="mean: the folded offset average (default); max: the max over the offsets; "
                          "pos: the offset average at per-key distances (pre-RoPE cache with positions)")

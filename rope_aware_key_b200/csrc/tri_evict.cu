@@ -21,6 +21,7 @@
 #include "score_max.cuh"
 #include "score_pos.cuh"
 #include "score_pos_tma.cuh"
+#include "fused.cuh"
 
 namespace {
 
@@ -37,6 +38,7 @@ struct DeviceInfo {
   int smax_blocks_per_sm = 0;
   int pos_blocks_per_sm = 0;
   int pt_blocks_per_sm = 0;
+  int fused_cluster = 0;        // cluster size of the single-kernel step (0: unavailable)
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -104,6 +106,34 @@ tri_status use_device_of(const void* ptr, int* dev_out) {
     TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.smax_blocks_per_sm, tri::smax::score_max_kernel,
                                                            tri::smax::kThreads, tri::smax::kSmemBytes));
     if (d.smax_blocks_per_sm < 1) return TRI_ERR_UNSUPPORTED;
+    // the single-kernel step: clusters of 16 CTAs if the device can hold one, else 8
+    TRI_CUDA(cudaFuncSetAttribute(tri::fused::fused_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tri::fused::kSmemBytes)));
+    TRI_CUDA(cudaFuncSetAttribute(tri::fused::fused_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    TRI_CUDA(cudaFuncSetAttribute(tri::fused::fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tri::fused::kSmemBytes)));
+    for (int cs : {16, 8}) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = cs;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.gridDim = dim3(cs);
+      cfg.blockDim = dim3(tri::fused::kThreads);
+      cfg.dynamicSmemBytes = tri::fused::kSmemBytes;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      const cudaError_t e = cs == 16
+          ? cudaOccupancyMaxActiveClusters(&clusters, tri::fused::fused_kernel<16>, &cfg)
+          : cudaOccupancyMaxActiveClusters(&clusters, tri::fused::fused_kernel<8>, &cfg);
+      if (e == cudaSuccess && clusters > 0) {
+        d.fused_cluster = cs;
+        break;
+      }
+      (void)cudaGetLastError();
+    }
     const int fill_smem = ((tri::compact::kMaxFillBudget + 31) / 32 + tri::compact::kMaxFillBudget) * 4;
     TRI_CUDA(cudaFuncSetAttribute(tri::compact::holefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   fill_smem));
@@ -270,6 +300,43 @@ tri_status launch_compact(const Geom& g, const int32_t* kept, const int32_t* kep
         g, kept, B, const_cast<uint16_t*>(g.k), const_cast<uint16_t*>(g.v));
   }
   ++g_launches;
+  TRI_CUDA(cudaGetLastError());
+  return TRI_OK;
+}
+
+// The single-kernel step (fused.cuh), when it applies: out-of-place
+// compaction of a CONTIG or RAGGED cache whose units fill at most one wave of
+// clusters and whose longest row fits the cluster's slices.  Returns
+// TRI_ERR_UNSUPPORTED when it does not apply (the caller then runs the three
+// kernels).
+tri_status launch_fused(const Geom& g, const float* w, float* scores, int B, int32_t* kept, int32_t* kept_count,
+                        void* k_out, void* v_out, int dev, cudaStream_t s) {
+  const int C = g_dev[dev].fused_cluster;
+  if (C == 0 || g.layout == TRI_LAYOUT_PAGED) return TRI_ERR_UNSUPPORTED;
+  const int64_t units = int64_t{g.L} * g.H * g.batch;
+  if (units * C > g_dev[dev].sms) return TRI_ERR_UNSUPPORTED;
+  int max_len = 0;
+  for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
+  const int per = ((max_len + C - 1) / C + tri::score::kTileRows - 1) / tri::score::kTileRows * tri::score::kTileRows;
+  if (per > tri::fused::kMaxSlice) return TRI_ERR_UNSUPPORTED;
+  tri::fused::Args a{w, scores, kept, kept_count, static_cast<uint16_t*>(k_out), static_cast<uint16_t*>(v_out), B,
+                     per > 0 ? per : tri::score::kTileRows};
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = C;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(units * C));
+  cfg.blockDim = dim3(tri::fused::kThreads);
+  cfg.dynamicSmemBytes = tri::fused::kSmemBytes;
+  cfg.stream = s;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = C == 16 ? cudaLaunchKernelEx(&cfg, tri::fused::fused_kernel<16>, g, a)
+                                : cudaLaunchKernelEx(&cfg, tri::fused::fused_kernel<8>, g, a);
+  ++g_launches;
+  if (e != cudaSuccess) return cuda_fail(e);
   TRI_CUDA(cudaGetLastError());
   return TRI_OK;
 }
@@ -573,6 +640,10 @@ tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B, tri_c
   if (st != TRI_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* scores = static_cast<float*>(workspace);
+  if (mode == TRI_COMPACT_OUT_OF_PLACE) {
+    st = launch_fused(g, w, scores, B, kept, kept_count, k_out, v_out, dev, s);
+    if (st != TRI_ERR_UNSUPPORTED) return st;
+  }
   st = launch_score(g, w, scores, dev, s);
   if (st != TRI_OK) return st;
   st = launch_select(g, scores, B, kept, kept_count, s);
@@ -604,6 +675,10 @@ tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int 
     scores = g_noalloc_ptr[dev];
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (mode == TRI_COMPACT_OUT_OF_PLACE) {
+    st = launch_fused(g, w, scores, B, kept, kept_count, k_out, v_out, dev, s);
+    if (st != TRI_ERR_UNSUPPORTED) return st;
+  }
   st = launch_score(g, w, scores, dev, s);
   if (st != TRI_OK) return st;
   st = launch_select(g, scores, B, kept, kept_count, s);
