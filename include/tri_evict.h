@@ -248,9 +248,15 @@ tri_status tri_compact_kv(const tri_cache_desc* desc, const int32_t* kept,
 /* Bytes of workspace tri_compress needs for `desc` (the score matrix). */
 tri_status tri_workspace_size(const tri_cache_desc* desc, int B, size_t* bytes);
 
-/* score -> select -> compact in one call (three kernels, no host sync).
- * Same arguments as the three calls; the scores live in `workspace`
- * (device, >= tri_workspace_size bytes, 256-byte aligned). */
+/* score -> select -> compact in one call (no host sync).  Same arguments and
+ * results as the three calls; the scores live in `workspace` (device,
+ * >= tri_workspace_size bytes, 256-byte aligned).
+ * A CONTIG or RAGGED cache compacted OUT_OF_PLACE whose units fit one wave of
+ * thread-block clusters (units x 16 CTAs <= the SM count, rows of at most
+ * 65536 keys) runs as ONE kernel: a cluster per unit scores its keys into
+ * shared memory, selects across the cluster and copies the kept rows; its
+ * scores, kept indices and compacted rows are identical, bit for bit, to the
+ * three-kernel path's, which every other case takes. */
 tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B,
                         tri_compact_mode mode, int32_t* kept, int32_t* kept_count,
                         void* k_out, void* v_out, void* workspace, size_t workspace_bytes,
