@@ -140,8 +140,10 @@ typedef struct tri_cache_desc {
  *     a_f = E[q_f] * W_f * e^{i omega_f delta0},   E[q_f] = q[re] + i q[im]
  *     w[c][re(f)] = Re a_f,   w[c][im(f)] = Im a_f
  * so that for a key k, Re sum_f a_f conj(k_f) = sum_j w[j] k[j] is the
- * offset-averaged trigonometric score.  Computed on the device in fp64,
- * stored as fp32.
+ * offset-averaged trigonometric score.  The per-band factor
+ * W_f e^{i omega_f delta0} depends only on (theta, D, delta0): it is summed on
+ * the host in fp64, in schedule order; the device maps every center in fp64
+ * and stores fp32.
  *
  * q_center: device fp32 [n_centers][128]; w_out: device fp32 [n_centers][128].
  * Centers are indexed (l * num_kv_heads + h) by the other calls.

@@ -12,10 +12,8 @@
 //     a_f = E[q_f] W_f e^{i w_f delta0},   w[re(f)] = Re a_f,  w[im(f)] = Im a_f,
 // and Re sum_f a_f conj(k_f) = sum_j w[j] k[j].
 //
-// Grid: one CTA per (band f, block of kThreads centers).  Each CTA sums W_f
-// over the schedule with a fixed-order fp64 tree, then maps its centers'
-// band f.  fp64 throughout (w_f * delta reaches 2^16 rad for the default
-// schedule, far beyond what fp32 phases can hold); fp32 output.
+// fp64 throughout (w_f * delta reaches 2^16 rad for the default schedule, far
+// beyond what fp32 phases can hold); fp32 output.
 #pragma once
 
 #include "common.cuh"
@@ -43,66 +41,32 @@ struct Args {
   double offsets[MAX_OFFSETS];
 };
 
-template <int N>
-__global__ void __launch_bounds__(kThreads) fold_kernel(const __grid_constant__ Args<N> a) {
-  __shared__ double s_c[kThreads / 32], s_s[kThreads / 32];
-  const int f = blockIdx.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const double omega = a.omega[f];
+// The averaged fold.  The offset mean and the kept distance depend only on
+// (theta, D, delta0), so the host sums them in fp64 into one complex factor
+// per band, A_f = W_f e^{i w_f delta0}; the kernel maps every center:
+// a_f = E[q_f] A_f (fp64), stored as fp32.
+struct FoldArgs {
+  const float* q;     // [n_centers][128]
+  float* w;           // [n_centers][128]
+  int n_centers;
+  int pairing;
+  double a_re[kBands], a_im[kBands];
+};
 
-  // W_f = mean over the schedule of e^{i omega delta}
-  double c = 0.0, s = 0.0;
-  for (int t = threadIdx.x; t < a.n_offsets; t += kThreads) {
-    double sn, cs;
-    sincos(omega * a.offsets[t], &sn, &cs);
-    c += cs;
-    s += sn;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    c += __shfl_xor_sync(0xffffffffu, c, o);
-    s += __shfl_xor_sync(0xffffffffu, s, o);
-  }
-  if (lane == 0) {
-    s_c[warp] = c;
-    s_s[warp] = s;
-  }
-  __syncthreads();
-  double wre = 0.0, wim = 0.0;
-  for (int i = 0; i < kThreads / 32; ++i) {
-    wre += s_c[i];
-    wim += s_s[i];
-  }
-  wre /= a.n_offsets;
-  wim /= a.n_offsets;
-
-  if (f == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    bool finite = isfinite(a.theta) && isfinite(a.delta0);
-    for (int t = 0; t < a.n_offsets; ++t) finite = finite && isfinite(a.offsets[t]);
-    if (!finite) flag(TRI_DEVFLAG_NONFINITE);
-  }
-
-  const int ci = blockIdx.y * kThreads + threadIdx.x;
-  if (ci >= a.n_centers) return;
+__global__ void __launch_bounds__(kThreads) fold_kernel(const __grid_constant__ FoldArgs a) {
+  const int ci = blockIdx.x * kThreads + threadIdx.x;
+  if (ci >= a.n_centers * kBands) return;
+  const int c = ci / kBands, f = ci - c * kBands;
   const int re = a.pairing == TRI_PAIRING_HALF ? f : 2 * f;
   const int im = a.pairing == TRI_PAIRING_HALF ? f + kBands : 2 * f + 1;
-  const float* q = a.q + static_cast<int64_t>(ci) * kD;
+  const float* q = a.q + static_cast<int64_t>(c) * kD;
   const float qr_f = q[re], qi_f = q[im];
   if (!isfinite(qr_f) || !isfinite(qi_f)) flag(TRI_DEVFLAG_NONFINITE);
   const double qr = qr_f, qi = qi_f;
-  // mu'_f = E[q_f] W_f
-  const double mr = wre * qr - wim * qi;
-  const double mi = wim * qr + wre * qi;
-  double ar = mr, ai = mi;
-  if (a.delta0 != 0.0) {
-    double sn, cs;
-    sincos(omega * a.delta0, &sn, &cs);
-    ar = cs * mr - sn * mi;
-    ai = sn * mr + cs * mi;
-  }
-  float* w = a.w + static_cast<int64_t>(ci) * kD;
-  w[re] = static_cast<float>(ar);
-  w[im] = static_cast<float>(ai);
+  const double ar = a.a_re[f], ai = a.a_im[f];
+  float* w = a.w + static_cast<int64_t>(c) * kD;
+  w[re] = static_cast<float>(ar * qr - ai * qi);
+  w[im] = static_cast<float>(ai * qr + ar * qi);
 }
 
 // Per-offset weights for the max-over-offsets score (no averaging):

@@ -357,10 +357,36 @@ tri_status check_compact_args(const tri_cache_desc* desc, const int32_t* kept, c
 }
 
 
-// Fill the parameter block and launch one of the fold kernels.
+// The averaged fold: A_f = (1/|D|) sum_delta e^{i w_f delta} * e^{i w_f delta0}
+// summed here in fp64 (in schedule order), then one launch maps the centers.
+void launch_fold_mean(const tri_fold_params* p, const float* q_center, int n_centers, float* w_out, cudaStream_t s) {
+  tri::fold::FoldArgs a;
+  a.q = q_center;
+  a.w = w_out;
+  a.n_centers = n_centers;
+  a.pairing = p->pairing;
+  for (int f = 0; f < tri::fold::kBands; ++f) {
+    const double omega = std::pow(p->theta, -2.0 * f / TRI_HEAD_DIM);
+    double c = 0.0, sn = 0.0;
+    for (int t = 0; t < p->n_offsets; ++t) {
+      c += std::cos(omega * p->offsets[t]);
+      sn += std::sin(omega * p->offsets[t]);
+    }
+    c /= p->n_offsets;
+    sn /= p->n_offsets;
+    const double rc = std::cos(omega * p->delta0), rs = std::sin(omega * p->delta0);
+    a.a_re[f] = c * rc - sn * rs;
+    a.a_im[f] = sn * rc + c * rs;
+  }
+  const int total = n_centers * tri::fold::kBands;
+  tri::fold::fold_kernel<<<(total + tri::fold::kThreads - 1) / tri::fold::kThreads, tri::fold::kThreads, 0, s>>>(a);
+}
+
+// The per-offset fold: the schedule in the kernel parameters (a small block
+// for short schedules, which launches faster than the largest).
 template <int N>
-void launch_fold_n(const tri_fold_params* p, const float* q_center, int n_centers, float* w_out, cudaStream_t s,
-                   bool per_offset) {
+void launch_fold_offsets(const tri_fold_params* p, const float* q_center, int n_centers, float* w_out,
+                         cudaStream_t s) {
   static tri::fold::Args<N> a;   // parameter block: built in static storage (under the caller's lock)
   a.q = q_center;
   a.w = w_out;
@@ -371,14 +397,9 @@ void launch_fold_n(const tri_fold_params* p, const float* q_center, int n_center
   a.n_offsets = p->n_offsets;
   for (int f = 0; f < tri::fold::kBands; ++f) a.omega[f] = std::pow(p->theta, -2.0 * f / TRI_HEAD_DIM);
   std::memcpy(a.offsets, p->offsets, sizeof(double) * p->n_offsets);
-  if (per_offset) {
-    const int pairs = n_centers * p->n_offsets;
-    const dim3 grid(tri::fold::kBands, (pairs + tri::fold::kThreads - 1) / tri::fold::kThreads);
-    tri::fold::fold_offsets_kernel<N><<<grid, tri::fold::kThreads, 0, s>>>(a);
-  } else {
-    const dim3 grid(tri::fold::kBands, (n_centers + tri::fold::kThreads - 1) / tri::fold::kThreads);
-    tri::fold::fold_kernel<N><<<grid, tri::fold::kThreads, 0, s>>>(a);
-  }
+  const int pairs = n_centers * p->n_offsets;
+  const dim3 grid(tri::fold::kBands, (pairs + tri::fold::kThreads - 1) / tri::fold::kThreads);
+  tri::fold::fold_offsets_kernel<N><<<grid, tri::fold::kThreads, 0, s>>>(a);
 }
 
 // Shared by the two fold calls: checks, then one launch with the schedule in
@@ -395,16 +416,19 @@ tri_status launch_fold(const tri_fold_params* p, const float* q_center, int n_ce
     if (!std::isfinite(p->offsets[t])) return TRI_ERR_INVALID_ARG;
   if (!aligned16(q_center) || !aligned16(w_out)) return TRI_ERR_INVALID_ARG;
   if (per_offset && int64_t{n_centers} * p->n_offsets > INT32_MAX / 2) return TRI_ERR_UNSUPPORTED;
+  if (int64_t{n_centers} * TRI_HEAD_DIM > INT32_MAX / 2) return TRI_ERR_UNSUPPORTED;
   int dev;
   tri_status st = use_device_of(q_center, &dev);
   if (st != TRI_OK) return st;
   static std::mutex m;
   std::lock_guard<std::mutex> lock(m);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (p->n_offsets <= tri::fold::kSmallOffsets)
-    launch_fold_n<tri::fold::kSmallOffsets>(p, q_center, n_centers, w_out, s, per_offset);
+  if (!per_offset)
+    launch_fold_mean(p, q_center, n_centers, w_out, s);
+  else if (p->n_offsets <= tri::fold::kSmallOffsets)
+    launch_fold_offsets<tri::fold::kSmallOffsets>(p, q_center, n_centers, w_out, s);
   else
-    launch_fold_n<TRI_MAX_OFFSETS>(p, q_center, n_centers, w_out, s, per_offset);
+    launch_fold_offsets<TRI_MAX_OFFSETS>(p, q_center, n_centers, w_out, s);
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
   return TRI_OK;
