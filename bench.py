@@ -132,6 +132,13 @@ class ClockSampler:
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    def wait_first(self, limit_s=5.0):
+        """Wait (bounded) for the first sample: nvidia-smi's start-up then lies
+        outside the timed region."""
+        t = time.time()
+        while self.proc is not None and not self.samples and time.time() - t < limit_s:
+            time.sleep(0.02)
+
     def _read(self):
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
@@ -271,6 +278,7 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.wait_first()
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
