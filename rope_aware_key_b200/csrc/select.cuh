@@ -539,7 +539,9 @@ __device__ __forceinline__ bool sampled_path(const float* row, int n, int B, int
     L = S.bounds[0];
   }
   // list every key >= L: U float4 loads in flight per thread, one
-  // warp-aggregated reservation per warp and pass step
+  // warp-aggregated reservation per warp and pass step.  Only the indices go
+  // into the list here (walking the set bits of a lane's flags, with no
+  // per-element work); the keys are read back from the row afterwards.
   if (G::tid() == 0) S.count = 0;
   G::sync();
   // key >= L as a float comparison: L = 0 takes every key (NaN included);
@@ -547,26 +549,34 @@ __device__ __forceinline__ bool sampled_path(const float* row, int n, int B, int
   // when score >= value(L) (-0 and +0 compare equal, NaN compares false).
   const bool take_all = L == 0u;
   const float Lv = L <= kKeyNegInf ? -INFINITY : key_value(L);
-  float lmaxf = -INFINITY;
   for (int w0 = warp * 32 * 4 * U; w0 < n; w0 += G::NT * 4 * U) {
     float4 v[U];
-#pragma unroll
-    for (int e = 0; e < U; ++e) {
-      const int i = w0 + (e * 32 + lane) * 4;
-      if (i + 3 < n) v[e] = __ldcg(reinterpret_cast<const float4*>(row + i));
-      else v[e] = make_float4(i < n ? __ldcg(row + i) : 0.f, i + 1 < n ? __ldcg(row + i + 1) : 0.f,
-                              i + 2 < n ? __ldcg(row + i + 2) : 0.f, 0.f);
-    }
     uint32_t flags = 0u;       // bit 4e+q: key w0 + (32e + lane)*4 + q is >= L
+    if (w0 + 32 * 4 * U <= n) {                    // warp-uniform: a full step
 #pragma unroll
-    for (int e = 0; e < U; ++e) {
-      const int i = w0 + (e * 32 + lane) * 4;
-      const float t[4] = {v[e].x, v[e].y, v[e].z, v[e].w};
+      for (int e = 0; e < U; ++e) v[e] = __ldcg(reinterpret_cast<const float4*>(row + w0 + (e * 32 + lane) * 4));
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const bool f = i + q < n && (take_all || t[q] >= Lv);
-        flags |= static_cast<uint32_t>(f) << (4 * e + q);
-        lmaxf = fmaxf(lmaxf, f ? t[q] : -INFINITY);
+      for (int e = 0; e < U; ++e) {
+        flags |= static_cast<uint32_t>(take_all || v[e].x >= Lv) << (4 * e);
+        flags |= static_cast<uint32_t>(take_all || v[e].y >= Lv) << (4 * e + 1);
+        flags |= static_cast<uint32_t>(take_all || v[e].z >= Lv) << (4 * e + 2);
+        flags |= static_cast<uint32_t>(take_all || v[e].w >= Lv) << (4 * e + 3);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < U; ++e) {
+        const int i = w0 + (e * 32 + lane) * 4;
+        if (i + 3 < n) v[e] = __ldcg(reinterpret_cast<const float4*>(row + i));
+        else v[e] = make_float4(i < n ? __ldcg(row + i) : 0.f, i + 1 < n ? __ldcg(row + i + 1) : 0.f,
+                                i + 2 < n ? __ldcg(row + i + 2) : 0.f, 0.f);
+      }
+#pragma unroll
+      for (int e = 0; e < U; ++e) {
+        const int i = w0 + (e * 32 + lane) * 4;
+        const float t[4] = {v[e].x, v[e].y, v[e].z, v[e].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          flags |= static_cast<uint32_t>(i + q < n && (take_all || t[q] >= Lv)) << (4 * e + q);
       }
     }
     const uint32_t cnt = __popc(flags);
@@ -580,26 +590,25 @@ __device__ __forceinline__ bool sampled_path(const float* row, int n, int B, int
     uint32_t base = 0u;
     if (lane == 0 && total) base = atomicAdd(&S.count, total);
     uint32_t pos = __shfl_sync(0xffffffffu, base, 0) + incl - cnt;
-#pragma unroll
-    for (int e = 0; e < U; ++e) {
-      const float t[4] = {v[e].x, v[e].y, v[e].z, v[e].w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (flags & (1u << (4 * e + q))) {
-          if (pos < static_cast<uint32_t>(lcap)) {
-            m.list_key[pos] = order_key(t[q]);
-            m.list_idx[pos] = w0 + (e * 32 + lane) * 4 + q;
-          }
-          ++pos;
-        }
-      }
+    while (flags) {
+      const int bit = __ffs(flags) - 1;
+      flags &= flags - 1u;
+      if (pos < static_cast<uint32_t>(lcap)) m.list_idx[pos] = w0 + ((bit >> 2) * 32 + lane) * 4 + (bit & 3);
+      ++pos;
     }
   }
-  // the largest listed key (NaN keys are 0, below every bound)
-  const uint32_t lmax = __reduce_max_sync(0xffffffffu, max(order_key(lmaxf), L));
+  G::sync();                                       // the list's indices and its count are complete
+  const uint32_t c = S.count;
+  // the listed keys, and the largest of them (NaN keys are 0, below every bound)
+  uint32_t lmax = L;
+  for (int jj = G::tid(); jj < min(static_cast<int>(c), lcap); jj += G::NT) {
+    const uint32_t k = order_key(__ldcg(row + m.list_idx[jj]));
+    m.list_key[jj] = k;
+    lmax = max(lmax, k);
+  }
+  lmax = __reduce_max_sync(0xffffffffu, lmax);
   if (lane == 0) S.red[1][warp] = lmax;
   G::sync();
-  const uint32_t c = S.count;
   uint32_t hi = 0u;
   for (int w = 0; w < G::NW; ++w) hi = max(hi, S.red[1][w]);
   const bool ok = c >= static_cast<uint32_t>(B) && c <= static_cast<uint32_t>(lcap);
