@@ -254,8 +254,8 @@ tri_status tri_workspace_size(const tri_cache_desc* desc, int B, size_t* bytes);
  * results as the three calls; the scores live in `workspace` (device,
  * >= tri_workspace_size bytes, 256-byte aligned).
  * A CONTIG or RAGGED cache compacted OUT_OF_PLACE whose units fit one wave of
- * thread-block clusters (units x 16 CTAs <= the SM count, rows of at most
- * 65536 keys) runs as ONE kernel: a cluster per unit scores its keys into
+ * thread-block clusters (units x 16 CTAs <= the SM count) and whose rows hold
+ * at most 8192 keys runs as ONE kernel: a cluster per unit scores its keys into
  * shared memory, selects across the cluster and copies the kept rows; its
  * scores, kept indices and compacted rows are identical, bit for bit, to the
  * three-kernel path's, which every other case takes. */

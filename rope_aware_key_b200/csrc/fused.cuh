@@ -41,6 +41,7 @@ namespace cg = cooperative_groups;
 constexpr int kThreads = score::kThreads;           // 8 consumer warps + 1 producer warp during scoring
 constexpr int kStages = 2;                          // two CTAs fit an SM, so a wave holds every cluster
 constexpr int kMaxSlice = 4096;                     // keys per CTA
+constexpr int kMaxRow = 8192;                       // longest row the host sends here
 constexpr int kBins = 2048;
 constexpr size_t kStageBytes = score::kTileBytes;
 constexpr size_t kKeysOffset = kStages * kStageBytes;                      // uint32 [kMaxSlice]

@@ -54,8 +54,8 @@ def assert_same(cache, fused, split, B):
 
 
 def test_single_kernel_step_8_units():
-    """One layer of the Qwen3 cache (8 KV heads x 32768 keys): 8 clusters."""
-    wl = gen.WORKLOADS["qwen3_layer"]
+    """One layer of a Qwen3-shaped cache (8 KV heads x 8192 keys): 8 clusters."""
+    wl = gen.scaled(gen.WORKLOADS["qwen3_layer"], seq_len=8192)
     cache = gen.make_cache(wl, seed=51, device=DEV)
     fused, split = both_paths(cache, wl.budget)
     assert_same(cache, fused, split, wl.budget)
@@ -66,7 +66,7 @@ def test_single_kernel_step_8_units():
 
 
 def test_single_kernel_step_ragged_edges():
-    lens = [0, 1, 127, 2048, 2049, 3000, 40000, 65536]
+    lens = [0, 1, 127, 2048, 2049, 3000, 5000, 8192]
     wl = gen.scaled(gen.WORKLOADS["qwen3_ragged"], num_layers=1, num_kv_heads=1, batch=len(lens))
     cache = gen.make_cache(wl, seed=52, device=DEV, lens=lens)
     fused, split = both_paths(cache, wl.budget)
@@ -80,8 +80,9 @@ def test_single_kernel_step_ties_across_slices():
     """Two distinct keys, one at 1000 random places and the other everywhere
     else: with B = 3000 one of the two fills the budget only in part, so the
     kept set ends in a run of equal scores whose lowest indices win, and that
-    run spreads over several CTAs' slices.  NaN and +/-inf keys take part too."""
-    wl = gen.scaled(gen.WORKLOADS["qwen3_layer"], num_kv_heads=2, seq_len=20000)
+    run spreads over several CTAs' slices (500 keys each).  NaN and +/-inf
+    keys take part too."""
+    wl = gen.scaled(gen.WORKLOADS["qwen3_layer"], num_kv_heads=2, seq_len=8000)
     cache = gen.make_cache(wl, seed=53, device=DEV)
     rng = np.random.default_rng(53)
     qc = cache.query_center.reshape(-1, 128)
@@ -90,22 +91,36 @@ def test_single_kernel_step_ties_across_slices():
         lo = (-qc[h].sign()).to(torch.bfloat16)
         rows = cache.k[0, h, 0]
         rows[:] = lo.to(DEV)
-        pick = torch.from_numpy(rng.choice(20000, size=1000, replace=False)).to(DEV)
+        pick = torch.from_numpy(rng.choice(8000, size=1000, replace=False)).to(DEV)
         rows[pick] = hi.to(DEV)
         rows[17] = float("nan")
         rows[18] = float("inf")
-        rows[19000] = -float("inf")
+        rows[7000] = -float("inf")
     B = 3000
     fused, split = both_paths(cache, B)
     assert_same(cache, fused, split, B)
     for h in range(2):
-        s = fused.scores[h, :20000].cpu().numpy()
+        s = fused.scores[h, :8000].cpu().numpy()
         np.testing.assert_array_equal(fused.kept[h].cpu().numpy(), oracle.select(s, B))
 
 
-@pytest.mark.parametrize("n,B", [(5000, 4999), (5000, 5000), (5000, 5001), (4096, 1), (300, 2048)])
+@pytest.mark.parametrize("n,B", [(5000, 4999), (5000, 5000), (5000, 5001), (4096, 1), (300, 2048), (8192, 3000)])
 def test_single_kernel_step_budget_edges(n, B):
     wl = gen.scaled(gen.WORKLOADS["tiny"], num_kv_heads=3, seq_len=n)
     cache = gen.make_cache(wl, seed=54, device=DEV)
     fused, split = both_paths(cache, B)
     assert_same(cache, fused, split, B)
+
+
+def test_single_kernel_step_is_taken_for_short_rows_only():
+    import rope_aware_key_b200 as tri
+    short = gen.make_cache(gen.scaled(gen.WORKLOADS["qwen3_layer"], num_kv_heads=2, seq_len=8192), seed=55,
+                           device=DEV, with_values=True)
+    n0 = tri.kernel_launches()
+    parity.run_gpu(short, fused=True)
+    assert tri.kernel_launches() - n0 == 2           # fold + one cluster kernel
+    long = gen.make_cache(gen.scaled(gen.WORKLOADS["qwen3_layer"], num_kv_heads=2, seq_len=8193), seed=55,
+                          device=DEV, with_values=True)
+    n0 = tri.kernel_launches()
+    parity.run_gpu(long, fused=True)
+    assert tri.kernel_launches() - n0 == 4           # fold + score, select, compact
