@@ -117,8 +117,6 @@ struct Args {
   int B;
   int cap;          // >= every row length, a multiple of 4: sizes the shared-memory bitmaps
   int lcap;         // capacity of the shared-memory key list
-  uint16_t* k_out;  // the compacting variant: out-of-place K and V, [units][B][128]
-  uint16_t* v_out;
 };
 
 // A group of NT threads that selects one row: the whole CTA (BAR == 0,
@@ -671,43 +669,7 @@ __device__ __forceinline__ void select_row(const float* row, int n, int B, int l
   G::sync();                                       // the shared arrays may be reused next
 }
 
-// The unit's kept rows of K and V, copied to their compacted places (the
-// out-of-place layout of compact.cuh): 16 threads per 256-byte row, 4 rows in
-// flight per thread.  `kept` holds m ascending indices written by this CTA.
 template <int NT>
-__device__ __forceinline__ void copy_kept_rows(const Geom& g, int u, const int32_t* kept, int m, int B,
-                                               uint16_t* k_out, uint16_t* v_out) {
-  const int b = u % g.batch, lh = u / g.batch;
-  const int l = lh / g.H, h = lh - l * g.H;
-  const int sub = threadIdx.x & 15;
-  constexpr int kRows = NT / 16;
-  const int64_t out0 = static_cast<int64_t>(u) * B;
-  for (int j0 = threadIdx.x >> 4; j0 < m; j0 += 4 * kRows) {
-    uint4 kv[4], vv[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = j0 + q * kRows;
-      if (j < m) {
-        bool ok = true;
-        const int64_t e = row_elem(g, l, h, b, __ldcg(kept + j), &ok);
-        kv[q] = ld_nc_v4(g.k + e + sub * 8);
-        vv[q] = ld_nc_v4(g.v + e + sub * 8);
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = j0 + q * kRows;
-      if (j < m) {
-        reinterpret_cast<uint4*>(k_out + (out0 + j) * kD)[sub] = kv[q];
-        reinterpret_cast<uint4*>(v_out + (out0 + j) * kD)[sub] = vv[q];
-      }
-    }
-  }
-}
-
-// COMPACT: also copy the kept rows (tri_compress, out of place, CONTIG or
-// RAGGED): each unit's compaction starts as soon as its own selection is done.
-template <int NT, bool COMPACT = false>
 __global__ void __launch_bounds__(NT, 1024 / NT) select_kernel(const __grid_constant__ Geom g, const Args a) {
   using G = Group<NT, 0, 0>;
   extern __shared__ uint4 select_dyn[];
@@ -722,14 +684,10 @@ __global__ void __launch_bounds__(NT, 1024 / NT) select_kernel(const __grid_cons
   if (threadIdx.x == 0) a.kept_count[u] = min(n, B);
   if (n <= B) {
     for (int i = threadIdx.x; i < n; i += NT) kept[i] = i;
-  } else {
-    const Smem m = carve(reinterpret_cast<uint32_t*>(select_dyn), a.cap, a.lcap);
-    select_row<G>(row, n, B, a.lcap, m, S, kept);
+    return;
   }
-  if constexpr (COMPACT) {
-    __syncthreads();                               // this CTA's kept indices are written
-    copy_kept_rows<NT>(g, u, kept, min(n, B), B, a.k_out, a.v_out);
-  }
+  const Smem m = carve(reinterpret_cast<uint32_t*>(select_dyn), a.cap, a.lcap);
+  select_row<G>(row, n, B, a.lcap, m, S, kept);
 }
 
 // Capacity of the key list for budget B on rows of at most `cap` keys.

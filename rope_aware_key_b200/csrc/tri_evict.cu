@@ -101,10 +101,6 @@ tri_status use_device_of(const void* ptr, int* dev_out) {
                                   tri::select::kMaxShared));
     TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   tri::select::kMaxShared));
-    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<512, true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, tri::select::kMaxShared));
-    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256, true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, tri::select::kMaxShared));
     TRI_CUDA(cudaFuncSetAttribute(tri::smax::score_max_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(tri::smax::kSmemBytes)));
     TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.smax_blocks_per_sm, tri::smax::score_max_kernel,
@@ -267,10 +263,8 @@ tri_status launch_score(const Geom& g0, const float* w, float* scores, int dev, 
   return TRI_OK;
 }
 
-// k_out / v_out non-null: the compacting variant (the kept rows are copied out
-// of place by the same CTAs; CONTIG and RAGGED only).
 tri_status launch_select(const Geom& g, const float* scores, int B, int32_t* kept, int32_t* kept_count,
-                         cudaStream_t s, void* k_out = nullptr, void* v_out = nullptr) {
+                         cudaStream_t s) {
   const int units = g.L * g.H * g.batch;
   int max_len = 0;
   for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
@@ -278,19 +272,11 @@ tri_status launch_select(const Geom& g, const float* scores, int B, int32_t* kep
   const int lcap = tri::select::list_capacity(B, cap);
   const size_t smem = tri::select::smem_bytes(cap, lcap);
   if (smem > static_cast<size_t>(tri::select::kMaxShared)) return TRI_ERR_UNSUPPORTED;
-  tri::select::Args a{scores, kept, kept_count, B, cap, lcap, static_cast<uint16_t*>(k_out),
-                      static_cast<uint16_t*>(v_out)};
-  const bool compact = k_out != nullptr;
+  tri::select::Args a{scores, kept, kept_count, B, cap, lcap};
   if (cap >= 8192) {
-    if (compact)
-      tri::select::select_kernel<512, true><<<units, 512, smem, s>>>(g, a);
-    else
-      tri::select::select_kernel<512><<<units, 512, smem, s>>>(g, a);
+    tri::select::select_kernel<512><<<units, 512, smem, s>>>(g, a);
   } else {
-    if (compact)
-      tri::select::select_kernel<256, true><<<units, 256, smem, s>>>(g, a);
-    else
-      tri::select::select_kernel<256><<<units, 256, smem, s>>>(g, a);
+    tri::select::select_kernel<256><<<units, 256, smem, s>>>(g, a);
   }
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
@@ -688,8 +674,6 @@ tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B, tri_c
   }
   st = launch_score(g, w, scores, dev, s);
   if (st != TRI_OK) return st;
-  if (mode == TRI_COMPACT_OUT_OF_PLACE && g.layout != TRI_LAYOUT_PAGED)
-    return launch_select(g, scores, B, kept, kept_count, s, k_out, v_out);   // selection + compaction
   st = launch_select(g, scores, B, kept, kept_count, s);
   if (st != TRI_OK) return st;
   return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, s);
@@ -725,8 +709,6 @@ tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int 
   }
   st = launch_score(g, w, scores, dev, s);
   if (st != TRI_OK) return st;
-  if (mode == TRI_COMPACT_OUT_OF_PLACE && g.layout != TRI_LAYOUT_PAGED)
-    return launch_select(g, scores, B, kept, kept_count, s, k_out, v_out);   // selection + compaction
   st = launch_select(g, scores, B, kept, kept_count, s);
   if (st != TRI_OK) return st;
   return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, s);

@@ -31,7 +31,7 @@ def fold64(cache):
 
 
 def both_paths(cache, B):
-    """(tri_compress: the single kernel for these shapes; the separate calls)."""
+    """(single kernel via tri_compress, three kernels via the separate calls)."""
     import rope_aware_key_b200 as tri
     fused = parity.run_gpu(cache, budget=B, fused=True)
     split = parity.run_gpu(cache, budget=B, fused=False)
@@ -123,4 +123,4 @@ def test_single_kernel_step_is_taken_for_short_rows_only():
                           device=DEV, with_values=True)
     n0 = tri.kernel_launches()
     parity.run_gpu(long, fused=True)
-    assert tri.kernel_launches() - n0 == 3           # fold + score, select with compaction
+    assert tri.kernel_launches() - n0 == 4           # fold + score, select, compact
