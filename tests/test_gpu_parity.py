@@ -322,3 +322,21 @@ def test_full_paged_incremental_rounds():
         after = snapshot(cache, units)
         check_sampled(cache, res, units, before=before, after=after)
         gen.release_tail_blocks(cache, [min(wl.budget, n) for n in cache.lens])
+
+
+def test_fold_follows_every_schedule_change():
+    """The host keeps the factors of the last schedule: alternating schedules,
+    offsets and kept distances must each give their own weights."""
+    t = tri()
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_kv_heads=3)
+    q = gen.make_cache(wl, seed=71, device=DEV, with_values=False).query_center.reshape(-1, 128)
+    qd = q.to(DEV).contiguous()
+    geo = [float(2 ** e) for e in range(17)]
+    cases = [(1e4, geo, 0.0), (1e6, geo, 0.0), (1e6, geo, 7.0), (1e6, geo[:-1] + [65537.0], 0.0),
+             (1e4, geo, 0.0), (5e5, [float(i) for i in range(1, 1025)], 0.0), (1e4, geo, 0.0)]
+    for theta, offs, d0 in cases:
+        for pairing in (0, 1):
+            w = t.fold_weights(qd, theta, offs, d0, pairing).cpu().numpy().astype(np.float64)
+            ref = oracle.fold_w(q, theta, offs, d0, pairing)
+            err = np.abs(w - ref)
+            assert np.all(err <= 2.0 ** -23 * np.abs(ref) + 1e-12 * np.abs(ref).max()), (theta, len(offs), d0)
