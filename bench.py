@@ -35,6 +35,8 @@ import gen  # noqa: E402
 KEY_BYTES = 256            # one bf16 key of head_dim 128, read once by the scorer
 MOVE_BYTES = 4 * 256       # a kept K row and V row, each read and written by the gather
 SPEC_HBM_GBS = 8000.0      # B200 HBM3e, nominal
+L2_BYTES = 126 * 2 ** 20   # B200 L2
+FLUSH_BYTES = 512 * 2 ** 20
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -277,7 +279,14 @@ def run_ours(args):
         graph.replay()
         torch.cuda.synchronize()
 
+    # Caches that L2 could hold a good part of are timed step by step with L2
+    # flushed in between (a 512 MB fill, outside the events); larger ones back to back.
+    kv_bytes = cache.k.numel() * 2 + cache.v.numel() * 2
+    flush = kv_bytes < 4 * L2_BYTES
+    flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)] if flush else None
     sampler.wait_first()
     if ws > 1:
         torch.distributed.barrier()
@@ -286,17 +295,22 @@ def run_ours(args):
     t0 = time.time()
     start.record(stream)
     for i in range(args.steps):
+        if flush:
+            flush_buf.fill_(i)
+            step_evs[i][0].record(stream)
         if graph is not None:
             graph.replay()
         else:
             step()
+        if flush:
+            step_evs[i][1].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
     t1 = time.time()
     if ws > 1:
         torch.distributed.barrier()
     launches = launches_per_step * args.steps if graph is not None else tri.kernel_launches() - launches0
-    ms = start.elapsed_time(end)
+    ms = start.elapsed_time(end) if not flush else sum(a.elapsed_time(b) for a, b in step_evs)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
 
@@ -306,6 +320,8 @@ def run_ours(args):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nb)]
     torch.cuda._sleep(int(4e7 + nb * 4e5))
     for i in range(nb):
+        if flush:
+            flush_buf.fill_(i)
         step(evs[i])
     torch.cuda.synchronize()
     per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])   # ms: fold, score, select, compact
@@ -343,7 +359,9 @@ def run_ours(args):
                                    f"{max(cache.lens)} keys, batch {wl.batch}, {wl.layout}, B={B}, "
                                    f"theta={wl.theta:g}, |D|={len(wl.offsets)}",
                        "keys_per_gpu": keys, "budget": B, "parallelism": f"independent caches x{ws}",
-                       "l2": "inputs larger than L2 (K and V of %.2f GB each vs 126 MB); no flush"
+                       "l2": ("K and V of %.3f GB each vs a 126 MB L2: L2 flushed (512 MB fill) before every "
+                              "timed step, each step timed alone" if flush else
+                              "inputs larger than L2 (K and V of %.2f GB each vs 126 MB); no flush")
                              % (keys * KEY_BYTES / 1e9)},
             "step_breakdown_ms": ({"fold": float(per[:, 0].mean()), "score": score_ms,
                                    "select": float(per[:, 2].mean()), "compact": float(per[:, 3].mean())}
