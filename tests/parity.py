@@ -1,7 +1,7 @@
 """Parity harness: run the CUDA path through the C ABI and compare it, unit by
 unit, with the CPU oracle on the same seeded inputs.
 
-Bars (BASELINE north star, restated):
+Bars:
 * scores: |s_gpu - s_ref| <= 1e-4 * sum_j |w_j k_j| per key, s_ref the
   oracle's literal per-offset average (or its folded form, pinned equal to
   it on the CPU, where the literal one is too slow);
