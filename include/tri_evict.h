@@ -13,8 +13,10 @@
  *    cache (the library launches on the device of desc->k, or of q_center for
  *    the fold); "host" pointers are ordinary CPU memory read during the call.
  *  - The caller allocates and owns every buffer.  The library never allocates
- *    or frees memory and never synchronises the stream, except
- *    tri_read_device_status, which reads a status word and waits for it.
+ *    or frees device memory at run time (tri_compress_noalloc uses a fixed
+ *    array of the module, allocated when the library loads) and never
+ *    synchronises the stream, except tri_read_device_status, which reads a
+ *    status word and waits for it.
  *  - Device calls are asynchronous on `stream` (NULL = legacy default stream).
  *    Pointers must stay valid until the stream reaches the work.
  *  - Arguments are checked on the host before anything is launched; a call
