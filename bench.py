@@ -182,7 +182,8 @@ def run_ours(args):
     import rope_aware_key_b200 as tri
     from rope_aware_key_b200 import build as tri_build
     if tri_build.needs_build():
-        raise RuntimeError("libtri_evict.so is missing or stale: run `python -m rope_aware_key_b200.build`")
+        log("building libtri_evict.so (missing or older than its sources)")
+        tri_build.build()
     ws, rank, local = dist_env()
     if ws > 1:
         import datetime
