@@ -19,6 +19,7 @@ struct Geom {
   int layout;                // tri_layout
   int L, H, batch;
   int block_size, max_blocks, num_blocks;
+  int pages_per_tile;        // PAGED: consecutive pages of a sequence scored as one tile
   int64_t sL, sH, sB;        // layer / head / (seq for CONTIG, page for PAGED) strides, elements
   int64_t score_stride;      // floats per score row
   const uint16_t* k;

@@ -48,7 +48,10 @@ struct TileInfo {
   int rows;          // rows held in the stage (0: nothing to do)
   int paged;         // rows interleave heads (PAGED)
   int lh;            // layer*H + head of row 0 (CONTIG / RAGGED), layer*H (PAGED)
-  int tvalid;        // PAGED: tokens of the page inside the sequence
+  int tvalid;        // PAGED: tokens of the tile inside the sequence
+  int page0;         // PAGED: the tile's first page (index in the sequence's block table)
+  int pages;         // PAGED: pages in the tile (their rows follow one another in the stage)
+  uint32_t page_ok;  // PAGED: bit p set when page p of the tile has a valid id (and was copied)
   int b;             // sequence
   int i0;            // index in the sequence of the tile's first key
   int tq;            // distance scorers: the query position of sequence b
@@ -61,7 +64,9 @@ constexpr size_t kInfoOffset = kBarOffset + 2 * kStages * sizeof(uint64_t);
 constexpr size_t kSmemBytes = kInfoOffset + kStages * sizeof(TileInfo);
 
 // Tiles are numbered layer-major: CONTIG / RAGGED per (layer, head) then
-// sequence then 128-key chunk; PAGED per layer then sequence then page.
+// sequence then 128-key chunk; PAGED per layer then sequence then group of
+// pages_per_tile consecutive pages (as many as fill 128 rows).  For PAGED,
+// *src is unused: the producer copies each page of the tile on its own.
 __device__ __forceinline__ void decode(const Geom& g, int t, float* scores, TileInfo* T, int64_t* src,
                                        bool* ok) {
   const int per = g.tile_prefix[g.batch];
@@ -73,21 +78,25 @@ __device__ __forceinline__ void decode(const Geom& g, int t, float* scores, Tile
   T->b = b;
   if (g.layout == TRI_LAYOUT_PAGED) {
     const int l = outer;
-    const int i0 = j * g.block_size;
+    const int P = g.pages_per_tile;
+    const int i0 = j * P * g.block_size;
+    const int seq_pages = (g.len[b] + g.block_size - 1) / g.block_size;
     T->i0 = i0;
-    T->rows = g.block_size * g.H;
+    T->page0 = j * P;
+    T->pages = min(P, seq_pages - j * P);
+    T->rows = T->pages * g.block_size * g.H;
     T->paged = 1;
     T->lh = l * g.H;
-    T->tvalid = min(g.block_size, g.len[b] - i0);
+    T->tvalid = min(P * g.block_size, g.len[b] - i0);
     T->head_step = static_cast<int64_t>(g.batch) * g.score_stride;
     T->out = scores + (static_cast<int64_t>(l) * g.H * g.batch + b) * g.score_stride + i0;
-    const int blk = g.block_table[static_cast<int64_t>(b) * g.max_blocks + j];
-    if (static_cast<unsigned>(blk) >= static_cast<unsigned>(g.num_blocks)) {
-      *ok = false;
-      *src = 0;
-    } else {
-      *src = l * g.sL + static_cast<int64_t>(blk) * g.sB;
+    T->page_ok = 0u;
+    for (int p = 0; p < T->pages; ++p) {
+      const int blk = g.block_table[static_cast<int64_t>(b) * g.max_blocks + j * P + p];
+      if (static_cast<unsigned>(blk) < static_cast<unsigned>(g.num_blocks)) T->page_ok |= 1u << p;
+      else *ok = false;
     }
+    *src = 0;
   } else {
     const int l = outer / g.H;
     const int h = outer - l * g.H;
@@ -95,6 +104,9 @@ __device__ __forceinline__ void decode(const Geom& g, int t, float* scores, Tile
     T->i0 = i0;
     T->rows = min(kTileRows, g.len[b] - i0);
     T->paged = 0;
+    T->page0 = 0;
+    T->pages = 0;
+    T->page_ok = 0u;
     T->lh = outer;
     T->tvalid = T->rows;
     T->head_step = 0;
@@ -155,16 +167,26 @@ __device__ __forceinline__ void produce(const Geom& g, float* scores, unsigned c
     int64_t src;
     bool ok;
     decode(g, t, scores, &T, &src, &ok);
-    if (!ok) {
-      T.rows = 0;
-      flag(TRI_DEVFLAG_BAD_PAGE);
-    }
+    if (!ok) flag(TRI_DEVFLAG_BAD_PAGE);           // the bad pages are skipped, the others scored
     side.annotate(T);
     info[s] = T;
     if (T.rows > 0) {
-      const uint32_t bytes = static_cast<uint32_t>(T.rows) * kRowBytes;
-      mbar_arrive_expect_tx(&full[s], bytes + side.bytes(T));
-      bulk_g2s(smem + static_cast<size_t>(s) * kTileBytes, g.k + src, bytes, &full[s], policy);
+      unsigned char* dst = smem + static_cast<size_t>(s) * kTileBytes;
+      if (!T.paged) {
+        const uint32_t bytes = static_cast<uint32_t>(T.rows) * kRowBytes;
+        mbar_arrive_expect_tx(&full[s], bytes + side.bytes(T));
+        bulk_g2s(dst, g.k + src, bytes, &full[s], policy);
+      } else {
+        const uint32_t page_bytes = static_cast<uint32_t>(g.block_size * g.H) * kRowBytes;
+        mbar_arrive_expect_tx(&full[s], page_bytes * __popc(T.page_ok) + side.bytes(T));
+        const int l = T.lh / g.H;
+        for (int p = 0; p < T.pages; ++p) {
+          if (!((T.page_ok >> p) & 1u)) continue;
+          const int blk = g.block_table[static_cast<int64_t>(T.b) * g.max_blocks + T.page0 + p];
+          bulk_g2s(dst + static_cast<size_t>(p) * page_bytes, g.k + l * g.sL + static_cast<int64_t>(blk) * g.sB,
+                   page_bytes, &full[s], policy);
+        }
+      }
       side.issue(T, s, &full[s], policy);
     } else {
       mbar_arrive(&full[s]);
@@ -253,7 +275,7 @@ score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float*
           if (c == 0 && r < T.rows) {
             if (T.paged) {
               const int tok = r / g.H;
-              if (tok < T.tvalid) T.out[h * T.head_step + tok] = a;
+              if (tok < T.tvalid && ((T.page_ok >> (tok / g.block_size)) & 1u)) T.out[h * T.head_step + tok] = a;
             } else {
               T.out[r] = a;
             }

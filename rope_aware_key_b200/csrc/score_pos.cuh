@@ -52,7 +52,7 @@ struct Rot {
 
 // Shared memory: the folded scorer's ring plus, per stage, the positions of
 // the tile's keys (CONTIG / RAGGED: key r at r; PAGED: head h, token j at
-// h * block_size + j) and the weight rows of its heads (one, or H for a
+// h * (tokens per tile) + j) and the weight rows of its heads (one, or H for a
 // page), and once per CTA the band constants: for each group j of 8 bands
 // {C_hi, C_lo} x 8 with a 16-byte pad, so that lanes reading eight different
 // groups hit eight different bank groups.
@@ -73,7 +73,7 @@ constexpr size_t kPosSmemBytes = kBandTabOffset + 8 * kBandTabStride;
 __device__ __forceinline__ uint32_t pos_row_bytes(const TileInfo& T) {
   return static_cast<uint32_t>((T.paged ? T.tvalid : T.rows) + 3) / 4 * 16;
 }
-__device__ __forceinline__ void copy_positions(const int32_t* pos, const float* scores, int H, int block_size,
+__device__ __forceinline__ void copy_positions(const int32_t* pos, const float* scores, int H, int tok_stride,
                                                const TileInfo& T, unsigned char* dst, uint64_t* bar,
                                                uint64_t policy) {
   const uint32_t nb = pos_row_bytes(T);
@@ -81,7 +81,7 @@ __device__ __forceinline__ void copy_positions(const int32_t* pos, const float* 
   if (!T.paged) {
     bulk_g2s(dst, src, nb, bar, policy);
   } else {
-    for (int h = 0; h < H; ++h) bulk_g2s(dst + h * block_size * 4, src + h * T.head_step, nb, bar, policy);
+    for (int h = 0; h < H; ++h) bulk_g2s(dst + h * tok_stride * 4, src + h * T.head_step, nb, bar, policy);
   }
 }
 
@@ -92,7 +92,7 @@ struct PosCopy {
   const float* scores;
   const float* w;
   unsigned char* smem;
-  int H, block_size;
+  int H, tok_stride;      // PAGED: positions per head in a stage (tokens per tile)
   const int32_t* qpos;
   __device__ __forceinline__ void annotate(TileInfo& T) const { T.tq = qpos[T.b]; }
   __device__ __forceinline__ uint32_t w_bytes(const TileInfo& T) const {
@@ -103,7 +103,7 @@ struct PosCopy {
   }
   __device__ __forceinline__ void issue(const TileInfo& T, int s, uint64_t* bar, uint64_t policy) const {
     bulk_g2s(smem + kWOffset + s * kWStageBytes, w + static_cast<int64_t>(T.lh) * kD, w_bytes(T), bar, policy);
-    if (pos) copy_positions(pos, scores, H, block_size, T, smem + kPosOffset + s * kPosStageBytes, bar, policy);
+    if (pos) copy_positions(pos, scores, H, tok_stride, T, smem + kPosOffset + s * kPosStageBytes, bar, policy);
   }
 };
 
@@ -189,7 +189,7 @@ score_pos_kernel(const __grid_constant__ Geom g, const __grid_constant__ Rot rot
   if (warp == kConsumerWarps) {
     if (lane == 0)
       produce(g, scores, smem, full, empty, info, blockIdx.x, ntiles, gridDim.x,
-              PosCopy{rot.pos, scores, w, smem, g.H, g.block_size, rot.qpos});
+              PosCopy{rot.pos, scores, w, smem, g.H, g.block_size * g.pages_per_tile, rot.qpos});
     return;
   }
 
@@ -204,16 +204,18 @@ score_pos_kernel(const __grid_constant__ Geom g, const __grid_constant__ Rot rot
   const bool paged = g.layout == TRI_LAYOUT_PAGED;
   const int h = paged ? r % g.H : 0;               // PAGED rows interleave heads: row = token * H + head
   const int tok = paged ? r / g.H : r;
+  const int tok_stride = g.block_size * g.pages_per_tile;   // PAGED: positions per head in a stage
   int k = 0;
   for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
     const int s = k % kStages, n = k / kStages;
     if (!mbar_wait_bounded(&full[s], n & 1)) break;
     const TileInfo T = info[s];
-    const bool live = r < T.rows && tok < (paged ? T.tvalid : T.rows);
+    const bool live = r < T.rows && tok < (paged ? T.tvalid : T.rows) &&
+                      (!paged || ((T.page_ok >> (tok / g.block_size)) & 1u));
     if (T.rows > 0) {
       const int32_t t_b = T.tq;
       const int32_t* sp = reinterpret_cast<const int32_t*>(smem + kPosOffset + s * kPosStageBytes);
-      const int32_t p_i = !live ? t_b : rot.pos ? sp[paged ? h * g.block_size + tok : r] : T.i0 + tok;
+      const int32_t p_i = !live ? t_b : rot.pos ? sp[paged ? h * tok_stride + tok : r] : T.i0 + tok;
       const Dist d = distance(t_b, p_i);
       const unsigned char* row = smem + static_cast<size_t>(s) * kTileBytes + (live ? r : 0) * kRowBytes;
       const float* wr = reinterpret_cast<const float*>(smem + kWOffset + s * kWStageBytes) + h * kD;

@@ -220,6 +220,8 @@ tri_status make_geom(const tri_cache_desc* c, bool need_v, Geom* g) {
         if (n > max_len) max_len = n;
       }
       g->block_size = c->block_size;
+      // as many consecutive pages per score tile as fill its 128 rows (at most 32)
+      g->pages_per_tile = static_cast<int>(std::min<int64_t>(32, tri::score::kTileRows / (int64_t{c->block_size} * H)));
       g->max_blocks = c->max_blocks_per_seq;
       g->num_blocks = c->num_blocks;
       g->sB = c->stride_block;
@@ -238,12 +240,13 @@ tri_status make_geom(const tri_cache_desc* c, bool need_v, Geom* g) {
   return TRI_OK;
 }
 
-// Score tiles: per sequence, 128-key chunks (CONTIG / RAGGED) or pages (PAGED).
+// Score tiles: per sequence, 128-key chunks (CONTIG / RAGGED) or groups of
+// pages_per_tile pages (PAGED).
 int64_t fill_tile_prefix(Geom* g) {
   int32_t acc = 0;
   for (int b = 0; b < g->batch; ++b) {
     g->tile_prefix[b] = acc;
-    const int per = g->layout == TRI_LAYOUT_PAGED ? g->block_size : tri::score::kTileRows;
+    const int per = g->layout == TRI_LAYOUT_PAGED ? g->block_size * g->pages_per_tile : tri::score::kTileRows;
     acc += (g->len[b] + per - 1) / per;
   }
   g->tile_prefix[g->batch] = acc;
