@@ -484,39 +484,43 @@ __device__ __forceinline__ bool sampled_path(const float* row, int n, int B, int
   // 32-byte sectors, so the sample costs 1/8 of a pass over the row)
   const int chunks = min((n + 7) / 8, kSamples / 8);
   const int ms = n < 8 * chunks ? n : 8 * chunks;
-  uint32_t mm[4] = {0xffffffffu, 0u, 0xffffffffu, 0u};
-  for (int q = G::tid(); q < chunks; q += G::NT) {
-    const int i0 = n <= 8 * chunks ? 8 * q : static_cast<int>(static_cast<int64_t>(q) * (n / 8) / chunks) * 8;
-    float v[8];
-    if (i0 + 7 < n) {
-      const float4 a = __ldcg(reinterpret_cast<const float4*>(row + i0));
-      const float4 b = __ldcg(reinterpret_cast<const float4*>(row + i0 + 4));
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = 0.f;
-      for (int e = 0; i0 + e < n && e < 8; ++e) v[e] = __ldcg(row + i0 + e);
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int j = 8 * q + e;
-      if (j < ms) {
-        const uint32_t k = order_key(v[e]);
-        m.samples[j] = k;
-        if (k > kKeyNegInf && k < kKeyPosInf) {
-          mm[2] = min(mm[2], k);
-          mm[3] = max(mm[3], k);
-        }
-      }
-    }
-  }
+  const float qm = static_cast<float>(B) * static_cast<float>(ms) / static_cast<float>(n);
+  const int r = static_cast<int>(ceilf(qm + 5.f * sqrtf(qm) + 20.f));
   for (int w = G::tid(); w < words; w += G::NT) {
     m.keepmap[w] = 0u;
     m.tiemap[w] = 0u;
   }
-  group_minmax4<G>(mm, S);
-  const float qm = static_cast<float>(B) * static_cast<float>(ms) / static_cast<float>(n);
-  const int r = static_cast<int>(ceilf(qm + 5.f * sqrtf(qm) + 20.f));
+  // r >= ms: every key will be listed, whatever the samples say (rows only a
+  // little longer than B), so they are not drawn
+  uint32_t mm[4] = {0xffffffffu, 0u, 0xffffffffu, 0u};
+  if (r < ms) {
+    for (int q = G::tid(); q < chunks; q += G::NT) {
+      const int i0 = n <= 8 * chunks ? 8 * q : static_cast<int>(static_cast<int64_t>(q) * (n / 8) / chunks) * 8;
+      float v[8];
+      if (i0 + 7 < n) {
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(row + i0));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(row + i0 + 4));
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+        for (int e = 0; i0 + e < n && e < 8; ++e) v[e] = __ldcg(row + i0 + e);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int j = 8 * q + e;
+        if (j < ms) {
+          const uint32_t k = order_key(v[e]);
+          m.samples[j] = k;
+          if (k > kKeyNegInf && k < kKeyPosInf) {
+            mm[2] = min(mm[2], k);
+            mm[3] = max(mm[3], k);
+          }
+        }
+      }
+    }
+    group_minmax4<G>(mm, S);
+  }
   uint32_t L = 0u;                                 // r >= ms: every key is listed
   if (r < ms) {
     if (!(mm[2] < mm[3])) return false;            // no spread among the samples
