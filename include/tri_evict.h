@@ -210,6 +210,9 @@ tri_status tri_score_keys_at_positions(const tri_cache_desc* desc, const float* 
  * the mean; it is not linear, so it does not fold):
  *     scores[u][i] = max_{t < n_offsets} sum_j w[l*H + h][t][j] * float(K_u[i][j])
  * with w from tri_fold_offset_weights (device fp32 [L*H][n_offsets][128]).
+ * More generally it is the max over any set of at most TRI_MAX_SCORE_OFFSETS
+ * weight vectors per head: e.g. the offset-averaged weights of the query heads
+ * of a grouped-query-attention group (n_offsets = the group size).
  * Runs on the tensor cores (bf16 keys; each fp32 weight split into two bf16
  * parts whose products accumulate in fp32, so the result keeps fp32-level
  * accuracy).  Layouts: CONTIG and RAGGED caches whose units are packed back

@@ -119,3 +119,43 @@ def test_score_max_full_qwen3_sampled():
         check_unit_max(cache, scores, w64, l, h, 0, GEO17, 0.0, 0, subset=2048)
     # every key of every unit was written
     assert not torch.isnan(scores).any()
+
+
+@pytest.mark.parametrize("group", [2, 4, 8])
+def test_gqa_group_aggregation(group):
+    """Grouped-query attention: several query heads share a KV head.  The
+    pages leave their aggregation open; the two plain readings run on the
+    existing calls.  Max over the group's query heads: each head's offset
+    average folded on its own, then the max scorer over the group's weight
+    vectors.  Mean over the group: the fold is linear in the center, so it is
+    the folded score of the mean center."""
+    import rope_aware_key_b200 as tri
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=2, num_kv_heads=2, seq_len=900, theta=1e6)
+    cache = gen.make_cache(wl, seed=81, device=DEV, with_values=False)
+    rng = np.random.default_rng(81)
+    LH = wl.num_layers * wl.num_kv_heads
+    centers = rng.standard_normal((LH, group, 128)).astype(np.float32)      # one center per query head
+    cd = torch.from_numpy(centers).to(DEV).reshape(LH * group, 128).contiguous()
+    w_group = tri.fold_weights(cd, wl.theta, wl.offsets).reshape(LH, group, 128).contiguous()
+    d = parity.make_desc(cache)
+    s_max = torch.full((d.units, tri.score_row_stride(d)), float("nan"), device=DEV)
+    tri.score_keys_max(d, w_group, s_max)
+    mean_c = torch.from_numpy(centers.mean(axis=1)).to(DEV).contiguous()
+    w_mean = tri.fold_weights(mean_c, wl.theta, wl.offsets)
+    s_mean = tri.score_keys(d, w_mean)
+    assert tri.read_device_status() == 0
+    torch.cuda.synchronize()
+    for l in range(wl.num_layers):
+        for h in range(wl.num_kv_heads):
+            lh = l * wl.num_kv_heads + h
+            u = parity.unit_id(wl, l, h, 0)
+            keys = parity.bits16(gen.unit_rows(cache, cache.k, l, h, 0))
+            per_head = np.stack([oracle.score_literal(keys, centers[lh, i], wl.theta, wl.offsets) for i in range(group)])
+            w64 = np.stack([oracle.fold_w(centers[lh, i][None, :], wl.theta, wl.offsets)[0] for i in range(group)])
+            scale = np.max(np.stack([oracle.abs_dot(keys, w64[i]) for i in range(group)]), axis=0)
+            got = s_max[u, :900].cpu().numpy().astype(np.float64)
+            assert np.all(np.abs(got - per_head.max(axis=0)) <= parity.SCORE_TOL * scale)
+            got_mean = s_mean[u, :900].cpu().numpy().astype(np.float64)
+            wm = oracle.fold_w(centers[lh].mean(axis=0)[None, :].astype(np.float32), wl.theta, wl.offsets)[0]
+            assert np.all(np.abs(got_mean - per_head.mean(axis=0)) <= parity.SCORE_TOL * oracle.abs_dot(keys, wm)
+                          + 1e-9 * scale)
