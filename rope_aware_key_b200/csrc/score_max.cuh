@@ -39,6 +39,19 @@
 #endif
 
 namespace tri {
+
+// `raw` (a __shared__ array) advanced to the next multiple of kAlign bytes
+// of the shared window, as the 128-byte swizzle of the TMA tiles needs.  The
+// offset is added to the array pointer itself, so the compiler still sees a
+// shared-memory pointer and emits shared loads; a round trip through an
+// integer would leave a generic (64-bit) pointer, whose loads take the
+// slower generic path and whose address arithmetic costs registers.
+template <uint32_t kAlign>
+__device__ __forceinline__ unsigned char* align_shared(unsigned char* raw) {
+  static_assert((kAlign & (kAlign - 1)) == 0, "power of two");
+  return raw + ((kAlign - (smem_addr(raw) & (kAlign - 1))) & (kAlign - 1));
+}
+
 namespace smax {
 
 constexpr int kTileRows = score::kTileRows;     // 128 keys: the MMA's M
@@ -148,7 +161,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int n, int k, int n_cols) {
 __global__ void __launch_bounds__(kThreads, TRI_SMAX_CTAS_PER_SM)
 score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtensorMap kmap, const Args a) {
   extern __shared__ unsigned char smax_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smax_raw) + 1023) & ~uintptr_t{1023});
+  unsigned char* smem = align_shared<1024>(smax_raw);
   unsigned char* bhi = smem + kBOffset;
   unsigned char* blo = bhi + a.n_cols * kRowBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);

@@ -55,8 +55,7 @@ score_pos_tma_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUt
                      const __grid_constant__ Rot rot, const float* __restrict__ w, float* __restrict__ scores,
                      int ntiles) {
   extern __shared__ unsigned char pt_raw[];
-  unsigned char* smem =
-      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(pt_raw) + 1023) & ~uintptr_t{1023});
+  unsigned char* smem = align_shared<1024>(pt_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPtBarOffset);
   uint64_t* empty = full + kPtStages;
   TileInfo* info = reinterpret_cast<TileInfo*>(smem + kPtInfoOffset);
