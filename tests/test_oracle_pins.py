@@ -432,3 +432,27 @@ def test_per_key_distance_constant_positions(orc):
     got = orc.score_at_positions(bits, q, 1e6, D, np.full(40, 1000), 4321)
     ref = orc.score_literal(bits, q, 1e6, D, delta0=3321.0)
     np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-10)
+
+
+def test_abs_dot_is_the_absolute_term_sum(orc):
+    """The parity bar's scale sum_j |w_j k_j|: at least |sum_j w_j k_j|
+    (triangle inequality) and equal to it when every term has one sign;
+    blind to the signs of the key and of the weights; linear in |w|; and on a
+    one-hot weight it is the one key element's magnitude."""
+    bits, vals, _ = rand_case(257, 128, seed=41)
+    rng = np.random.default_rng(42)
+    w = rng.standard_normal(128)
+    a = orc.abs_dot(bits, w)
+    s = orc.score_realdot(bits, w)
+    assert a.shape == (257,)
+    assert np.all(a >= np.abs(s) * (1 - 1e-12))
+    assert np.all(a > np.abs(s) * (1 + 1e-6))          # mixed signs: strictly larger here
+    pos_bits = bits & np.uint16(0x7FFF)                 # |k| (bf16 sign bit cleared)
+    np.testing.assert_allclose(orc.abs_dot(pos_bits, np.abs(w)), orc.score_realdot(pos_bits, np.abs(w)),
+                               rtol=1e-13)
+    np.testing.assert_array_equal(orc.abs_dot(bits ^ np.uint16(0x8000), -w), a)
+    np.testing.assert_array_equal(orc.abs_dot(bits, 2.0 * w), 2.0 * a)
+    for j in (0, 63, 64, 127):
+        e = np.zeros(128)
+        e[j] = -3.0
+        np.testing.assert_array_equal(orc.abs_dot(bits, e), 3.0 * np.abs(vals[:, j]))
