@@ -102,7 +102,8 @@ def lib() -> ctypes.CDLL:
     L.tri_kernel_launches.restype = ctypes.c_uint64
     L.tri_version.restype = ctypes.c_char_p
     for name in ("tri_fold_weights", "tri_fold_offset_weights", "tri_score_keys_max", "tri_score_keys",
-                 "tri_select_topk", "tri_compact_kv", "tri_workspace_size", "tri_compress", "tri_read_device_status"):
+                 "tri_score_keys_at_positions", "tri_select_topk", "tri_compact_kv", "tri_workspace_size",
+                 "tri_compress", "tri_read_device_status"):
         getattr(L, name).restype = I
     _lib = L
     return L
@@ -113,9 +114,11 @@ def _check(st: int, call: str) -> None:
         raise TriError(st, call)
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _stream(stream, device=None) -> ctypes.c_void_p:
+    """The given stream, or the current stream of `device` (the device that
+    holds the call's tensors: the library launches there)."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     if isinstance(stream, torch.cuda.Stream):
         return ctypes.c_void_p(stream.cuda_stream)
     return ctypes.c_void_p(int(stream))
@@ -123,6 +126,17 @@ def _stream(stream) -> ctypes.c_void_p:
 
 def _ptr(t: Optional[torch.Tensor]):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _need(t: Optional[torch.Tensor], dtype: torch.dtype, numel: int, name: str) -> None:
+    """The library takes plain pointers and cannot see a buffer's size, so the
+    binding checks each tensor it passes: device memory of the right type,
+    contiguous, and at least as many elements as the call touches."""
+    if t is None:
+        return
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous() and t.numel() >= numel):
+        raise ValueError(f"{name}: need a contiguous {dtype} cuda tensor of >= {numel} elements, got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}" + ("" if t.is_contiguous() else " (strided)"))
 
 
 class Desc:
@@ -212,14 +226,15 @@ def fold_weights(q_center: torch.Tensor, theta: float, offsets: Sequence[float],
                  pairing: int = PAIRING_HALF, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Fold the offset average into fp32 weights [n][128] (on the device)."""
     q = q_center.reshape(-1, HEAD_DIM)
-    assert q.dtype == torch.float32 and q.is_cuda and q.is_contiguous()
+    _need(q, torch.float32, q.numel(), "q_center")
     if out is None:
         out = torch.empty_like(q)
+    _need(out, torch.float32, q.numel(), "out")
     offs = [float(x) for x in offsets]
     arr = (ctypes.c_double * len(offs))(*offs)
     p = _FoldParams(head_dim=HEAD_DIM, theta=float(theta), offsets=arr, n_offsets=len(offs),
                     delta0=float(delta0), pairing=int(pairing))
-    _check(lib().tri_fold_weights(ctypes.byref(p), _ptr(q), q.shape[0], _ptr(out), _stream(stream)),
+    _check(lib().tri_fold_weights(ctypes.byref(p), _ptr(q), q.shape[0], _ptr(out), _stream(stream, q.device)),
            "tri_fold_weights")
     return out
 
@@ -229,14 +244,16 @@ def fold_offset_weights(q_center: torch.Tensor, theta: float, offsets: Sequence[
                         stream=None) -> torch.Tensor:
     """Per-offset (unaveraged) weights, fp32 [n][len(offsets)][128] on the device."""
     q = q_center.reshape(-1, HEAD_DIM)
-    assert q.dtype == torch.float32 and q.is_cuda and q.is_contiguous()
+    _need(q, torch.float32, q.numel(), "q_center")
     offs = [float(x) for x in offsets]
     if out is None:
         out = torch.empty((q.shape[0], len(offs), HEAD_DIM), dtype=torch.float32, device=q.device)
+    _need(out, torch.float32, q.numel() * len(offs), "out")
     arr = (ctypes.c_double * len(offs))(*offs)
     p = _FoldParams(head_dim=HEAD_DIM, theta=float(theta), offsets=arr, n_offsets=len(offs),
                     delta0=float(delta0), pairing=int(pairing))
-    _check(lib().tri_fold_offset_weights(ctypes.byref(p), _ptr(q), q.shape[0], _ptr(out), _stream(stream)),
+    _check(lib().tri_fold_offset_weights(ctypes.byref(p), _ptr(q), q.shape[0], _ptr(out),
+                                         _stream(stream, q.device)),
            "tri_fold_offset_weights")
     return out
 
@@ -245,9 +262,12 @@ def score_keys_max(d: Desc, w_offsets: torch.Tensor, scores: Optional[torch.Tens
                    stream=None) -> torch.Tensor:
     """Max over the offsets of the per-offset scores (tensor cores)."""
     n_off = w_offsets.shape[-2]
+    _need(w_offsets, torch.float32, d.num_layers * d.num_kv_heads * n_off * HEAD_DIM, "w_offsets")
     if scores is None:
         scores = torch.empty((d.units, score_row_stride(d)), dtype=torch.float32, device=w_offsets.device)
-    _check(lib().tri_score_keys_max(d.ref, _ptr(w_offsets), int(n_off), _ptr(scores), _stream(stream)),
+    _need(scores, torch.float32, d.units * score_row_stride(d), "scores")
+    _check(lib().tri_score_keys_max(d.ref, _ptr(w_offsets), int(n_off), _ptr(scores),
+                                    _stream(stream, w_offsets.device)),
            "tri_score_keys_max")
     return scores
 
@@ -260,9 +280,11 @@ def score_row_stride(d: Desc) -> int:
 
 
 def score_keys(d: Desc, w: torch.Tensor, scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _need(w, torch.float32, d.num_layers * d.num_kv_heads * HEAD_DIM, "w")
     if scores is None:
         scores = torch.empty((d.units, score_row_stride(d)), dtype=torch.float32, device=w.device)
-    _check(lib().tri_score_keys(d.ref, _ptr(w), _ptr(scores), _stream(stream)), "tri_score_keys")
+    _need(scores, torch.float32, d.units * score_row_stride(d), "scores")
+    _check(lib().tri_score_keys(d.ref, _ptr(w), _ptr(scores), _stream(stream, w.device)), "tri_score_keys")
     return scores
 
 
@@ -272,24 +294,33 @@ def score_keys_at_positions(d: Desc, w: torch.Tensor, theta: float, query_pos: S
     """Offset-averaged score of a pre-RoPE cache at each key's own distance
     t_b - p_i.  positions: device int32 laid out like the scores, or None for
     p_i = i; query_pos: one position per sequence."""
+    stride = score_row_stride(d)
+    _need(w, torch.float32, d.num_layers * d.num_kv_heads * HEAD_DIM, "w")
     if scores is None:
-        scores = torch.empty((d.units, score_row_stride(d)), dtype=torch.float32, device=w.device)
-    if positions is not None:
-        assert positions.dtype == torch.int32 and positions.is_contiguous()
+        scores = torch.empty((d.units, stride), dtype=torch.float32, device=w.device)
+    _need(scores, torch.float32, d.units * stride, "scores")
+    _need(positions, torch.int32, d.units * stride, "positions")
+    if len(query_pos) < d.batch:
+        raise ValueError(f"query_pos: need one position per sequence ({d.batch}), got {len(query_pos)}")
     qp = (ctypes.c_int64 * max(1, len(query_pos)))(*[int(t) for t in query_pos])
     _check(lib().tri_score_keys_at_positions(d.ref, _ptr(w), float(theta), int(pairing), _ptr(positions),
-                                             ctypes.cast(qp, ctypes.c_void_p), _ptr(scores), _stream(stream)),
+                                             ctypes.cast(qp, ctypes.c_void_p), _ptr(scores),
+                                             _stream(stream, w.device)),
            "tri_score_keys_at_positions")
     return scores
 
 
 def select_topk(d: Desc, scores: torch.Tensor, budget: int, kept: Optional[torch.Tensor] = None,
                 kept_count: Optional[torch.Tensor] = None, stream=None):
+    _need(scores, torch.float32, d.units * score_row_stride(d), "scores")
     if kept is None:
         kept = torch.empty((d.units, budget), dtype=torch.int32, device=scores.device)
     if kept_count is None:
         kept_count = torch.empty((d.units,), dtype=torch.int32, device=scores.device)
-    _check(lib().tri_select_topk(d.ref, _ptr(scores), int(budget), _ptr(kept), _ptr(kept_count), _stream(stream)),
+    _need(kept, torch.int32, d.units * max(int(budget), 0), "kept")
+    _need(kept_count, torch.int32, d.units, "kept_count")
+    _check(lib().tri_select_topk(d.ref, _ptr(scores), int(budget), _ptr(kept), _ptr(kept_count),
+                                 _stream(stream, scores.device)),
            "tri_select_topk")
     return kept, kept_count
 
@@ -297,8 +328,12 @@ def select_topk(d: Desc, scores: torch.Tensor, budget: int, kept: Optional[torch
 def compact_kv(d: Desc, kept: torch.Tensor, kept_count: torch.Tensor, budget: int,
                mode: int = COMPACT_OUT_OF_PLACE, k_out: Optional[torch.Tensor] = None,
                v_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    _need(kept, torch.int32, d.units * max(int(budget), 0), "kept")
+    _need(kept_count, torch.int32, d.units, "kept_count")
+    _need(k_out, torch.bfloat16, d.units * max(int(budget), 0) * HEAD_DIM, "k_out")
+    _need(v_out, torch.bfloat16, d.units * max(int(budget), 0) * HEAD_DIM, "v_out")
     _check(lib().tri_compact_kv(d.ref, _ptr(kept), _ptr(kept_count), int(budget), int(mode), _ptr(k_out),
-                                _ptr(v_out), _stream(stream)), "tri_compact_kv")
+                                _ptr(v_out), _stream(stream, kept.device)), "tri_compact_kv")
 
 
 def workspace_size(d: Desc, budget: int) -> int:
@@ -319,8 +354,16 @@ def compress(d: Desc, w: torch.Tensor, budget: int, mode: int = COMPACT_OUT_OF_P
         kept_count = torch.empty((d.units,), dtype=torch.int32, device=dev)
     if workspace is None:
         workspace = torch.empty(workspace_size(d, budget), dtype=torch.uint8, device=dev)
+    nb = d.units * max(int(budget), 0)
+    _need(w, torch.float32, d.num_layers * d.num_kv_heads * HEAD_DIM, "w")
+    _need(kept, torch.int32, nb, "kept")
+    _need(kept_count, torch.int32, d.units, "kept_count")
+    _need(k_out, torch.bfloat16, nb * HEAD_DIM, "k_out")
+    _need(v_out, torch.bfloat16, nb * HEAD_DIM, "v_out")
+    _need(workspace, torch.uint8, 0, "workspace")      # its size goes to the library, which checks it
     _check(lib().tri_compress(d.ref, _ptr(w), int(budget), int(mode), _ptr(kept), _ptr(kept_count), _ptr(k_out),
-                              _ptr(v_out), _ptr(workspace), workspace.numel(), _stream(stream)), "tri_compress")
+                              _ptr(v_out), _ptr(workspace), workspace.numel(), _stream(stream, dev)),
+           "tri_compress")
     return kept, kept_count
 
 

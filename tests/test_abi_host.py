@@ -212,3 +212,16 @@ def test_score_positions_checks(L):
         qb = (ctypes.c_int64 * 1)(bad)
         assert fn(ctypes.byref(d), P(FAKE), 1e4, 0, None, ctypes.cast(qb, P), P(FAKE), None) == 1
     assert fn(ctypes.byref(contig(head_dim=64)), P(FAKE), 1e4, 0, None, q, P(FAKE), None) == 2
+
+
+def test_binding_checks_buffers_before_the_library():
+    """The C ABI takes plain pointers and cannot see a buffer's size: the
+    binding checks each tensor before it calls the library; here a host tensor
+    and a wrong dtype (short device buffers: test_gpu_parity)."""
+    import torch
+    k = torch.zeros((2, 3, 1, 16, 128), dtype=torch.bfloat16)
+    d = tri.desc_contig(k, k)
+    with pytest.raises(ValueError, match="w: need"):
+        tri.score_keys(d, torch.zeros((6, 128)))                       # host memory
+    with pytest.raises(ValueError, match="q_center: need"):
+        tri.fold_weights(torch.zeros((6, 128), dtype=torch.float64), 1e4, [1.0])

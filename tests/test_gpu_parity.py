@@ -340,3 +340,43 @@ def test_fold_follows_every_schedule_change():
             ref = oracle.fold_w(q, theta, offs, d0, pairing)
             err = np.abs(w - ref)
             assert np.all(err <= 2.0 ** -23 * np.abs(ref) + 1e-12 * np.abs(ref).max()), (theta, len(offs), d0)
+
+
+def test_binding_refuses_short_or_mistyped_buffers():
+    """A device buffer one row short, of the wrong dtype or strided is refused
+    on the host, before any launch; the right sizes go through."""
+    import rope_aware_key_b200 as tri
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=2, num_kv_heads=2, seq_len=300, budget=64)
+    cache = gen.make_cache(wl, seed=51, device=DEV)
+    d = parity.make_desc(cache)
+    qc = cache.query_center.reshape(-1, wl.head_dim).to(DEV).contiguous()
+    w = tri.fold_weights(qc, wl.theta, wl.offsets)
+    stride = tri.score_row_stride(d)
+    B = wl.budget
+    launches = tri.kernel_launches()
+    with pytest.raises(ValueError, match="w: need"):
+        tri.score_keys(d, w[:-1])
+    with pytest.raises(ValueError, match="scores: need"):
+        tri.score_keys(d, w, torch.empty((d.units, stride - 4), device=DEV))
+    with pytest.raises(ValueError, match="scores: need"):
+        tri.score_keys(d, w, torch.empty((stride, d.units), device=DEV).t())
+    scores = tri.score_keys(d, w)
+    with pytest.raises(ValueError, match="kept: need"):
+        tri.select_topk(d, scores, B, torch.empty((d.units, B - 1), dtype=torch.int32, device=DEV))
+    with pytest.raises(ValueError, match="kept_count: need"):
+        tri.select_topk(d, scores, B, None, torch.empty((d.units,), dtype=torch.int64, device=DEV))
+    kept, cnt = tri.select_topk(d, scores, B)
+    short = torch.empty((d.units, B - 1, wl.head_dim), dtype=torch.bfloat16, device=DEV)
+    full = torch.empty((d.units, B, wl.head_dim), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ValueError, match="k_out: need"):
+        tri.compact_kv(d, kept, cnt, B, tri.COMPACT_OUT_OF_PLACE, short, full)
+    with pytest.raises(ValueError, match="v_out: need"):
+        tri.compact_kv(d, kept, cnt, B, tri.COMPACT_OUT_OF_PLACE, full, full.float())
+    with pytest.raises(ValueError, match="positions: need"):
+        tri.score_keys_at_positions(d, w, wl.theta, [300], torch.zeros((d.units, stride - 4), dtype=torch.int32,
+                                                                        device=DEV))
+    with pytest.raises(ValueError, match="query_pos: need one position per sequence"):
+        tri.score_keys_at_positions(d, w, wl.theta, [])
+    assert tri.kernel_launches() == launches + 2          # the two calls that went through
+    tri.compact_kv(d, kept, cnt, B, tri.COMPACT_OUT_OF_PLACE, full, torch.empty_like(full))
+    assert tri.read_device_status() == 0
