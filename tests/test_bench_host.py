@@ -1,0 +1,87 @@
+"""Host-side pieces of the bench, on CPU: the clock summary taken during the
+timed region (median SM clock, throttle reasons) and the ncu traffic record,
+which is reported only for the workload it was taken on and only while the
+scorer's sources are the ones it was captured from."""
+import json
+import os
+import shutil
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _sampler(rows):
+    s = bench.ClockSampler.__new__(bench.ClockSampler)   # no nvidia-smi process
+    s.samples = rows
+    s.proc = None
+    return s
+
+
+def _row(sm, power, hw="Not Active", hw_thermal="Not Active", sw_thermal="Not Active", power_cap="Not Active"):
+    return ["2026/01/01 00:00:00.000", "0", str(sm), "1965", str(power), "0x0", hw, hw_thermal, sw_thermal, power_cap]
+
+
+def test_clock_summary_inside_the_window():
+    rows = [(1.0, _row(1800, 500.5, power_cap="Active")),
+            (1.1, _row(1900, 600.0)),
+            (1.2, _row(1950, 610.0, hw_thermal="Active")),
+            (5.0, _row(500, 100.0, hw="Active"))]          # after the timed region: ignored
+    d = _sampler(rows).summary(0.9, 1.3)
+    assert d["samples"] == 3
+    assert d["sm_mhz"] == 1900.0 and d["sm_max_mhz"] == 1965.0
+    assert d["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert d["power_w_max"] == 610.0
+
+
+def test_clock_summary_unparsable_fields_and_no_samples():
+    rows = [(1.0, _row("[N/A]", "[N/A]")), (1.1, _row(1700, 400.0))]
+    d = _sampler(rows).summary(0.0, 2.0)
+    assert d["sm_mhz"] == 1700.0 and d["power_w_max"] == 400.0 and d["reasons"] == []
+    d = _sampler([]).summary(0.0, 1.0)
+    assert d["samples"] == 0 and d["sm_mhz"] is None and d["reasons"] == ["nvidia-smi unavailable"]
+
+
+def _tree(tmp_path):
+    """A copy of the scorer sources and an empty profiles folder."""
+    src = os.path.join(ROOT, "rope_aware_key_b200", "csrc")
+    dst = tmp_path / "rope_aware_key_b200" / "csrc"
+    shutil.copytree(src, dst)
+    (tmp_path / "profiles").mkdir()
+    return dst
+
+
+def _record(tmp_path, variant, workload, fingerprint, nbytes):
+    name = bench.SCORE_KERNELS[variant][2]
+    with open(tmp_path / "profiles" / name, "w") as f:
+        json.dump({"workload": workload, "kernel_sources": fingerprint, "dram_bytes_per_launch": nbytes}, f)
+
+
+def test_traffic_record_follows_the_sources(tmp_path, monkeypatch):
+    csrc = _tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.ncu_traffic("qwen3_full", "mean") is None              # no record
+    fp = bench.score_kernel_fingerprint("mean")
+    _record(tmp_path, "mean", "qwen3_full", fp, 12345)
+    assert bench.ncu_traffic("qwen3_full", "mean") == 12345
+    assert bench.ncu_traffic("qwen3_layer", "mean") is None             # another workload
+    # a source the scorer is built from changes: the record no longer applies
+    with open(csrc / "score.cuh", "a") as f:
+        f.write("\n")
+    assert bench.score_kernel_fingerprint("mean") != fp
+    assert bench.ncu_traffic("qwen3_full", "mean") is None
+
+
+def test_fingerprints_cover_each_scorers_sources(tmp_path, monkeypatch):
+    csrc = _tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    before = {v: bench.score_kernel_fingerprint(v) for v in ("mean", "max", "pos")}
+    with open(csrc / "score_pos_tma.cuh", "a") as f:      # only the distance scorer is built from it
+        f.write("\n")
+    after = {v: bench.score_kernel_fingerprint(v) for v in ("mean", "max", "pos")}
+    assert after["mean"] == before["mean"] and after["max"] == before["max"]
+    assert after["pos"] != before["pos"]
+    with open(csrc / "common.cuh", "a") as f:             # every scorer includes it
+        f.write("\n")
+    assert all(bench.score_kernel_fingerprint(v) != after[v] for v in ("mean", "max", "pos"))
