@@ -456,3 +456,26 @@ def test_abs_dot_is_the_absolute_term_sum(orc):
         e = np.zeros(128)
         e[j] = -3.0
         np.testing.assert_array_equal(orc.abs_dot(bits, e), 3.0 * np.abs(vals[:, j]))
+
+
+def test_threads_do_not_change_results(orc):
+    """Keys are split across host threads; each key's sum runs in one thread
+    in a fixed order, so any thread count gives the same bits."""
+    bits, _, q = rand_case(203, 128, seed=61)          # 203 keys: uneven chunks for 7 threads
+    D = [1.0, 3.0, 17.5, 1024.0]
+    rng = np.random.default_rng(62)
+    pos = np.sort(rng.choice(4 * 203, size=203, replace=False)).astype(np.int32)
+    w = orc.fold_w(q[None, :], 1e4, D, 0.0, 0)[0]
+    for pairing in (0, 1):
+        calls = [
+            lambda t: orc.score_cosine(bits, q, 1e4, D, 2.0, pairing, threads=t),
+            lambda t: orc.score_literal(bits, q, 1e4, D, 2.0, pairing, threads=t),
+            lambda t: orc.score_max_literal(bits, q, 1e4, D, 2.0, pairing, threads=t),
+            lambda t: orc.score_folded(bits, q, 1e4, D, 2.0, pairing, threads=t),
+            lambda t: orc.score_polar(bits, q, 1e4, D, 2.0, pairing, threads=t),
+            lambda t: orc.score_at_positions(bits, q, 1e4, D, pos, 4 * 203, pairing, threads=t),
+        ]
+        for fn in calls:
+            np.testing.assert_array_equal(fn(1), fn(7))
+    np.testing.assert_array_equal(orc.score_realdot(bits, w, threads=1), orc.score_realdot(bits, w, threads=7))
+    np.testing.assert_array_equal(orc.abs_dot(bits, w, threads=1), orc.abs_dot(bits, w, threads=7))
