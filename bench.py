@@ -563,6 +563,22 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def relaunch_per_gpu(n: int) -> int:
+    """Run this same command under torch.distributed.run with n processes on
+    this node (rendezvous on 127.0.0.1, a free port); returns its exit code."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    log("launching " + " ".join(cmd[2:]))
+    try:
+        return subprocess.call(cmd, timeout=3600)      # last bound; the process group times out first
+    except subprocess.TimeoutExpired:
+        return 124
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -583,6 +599,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    ws = dist_env()[0]
+    if args.impl == "ours" and args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # started by hand with --gpus N: one process per GPU, the launch torchrun gives
+        raise SystemExit(relaunch_per_gpu(args.gpus))
+    if args.impl == "ours" and ws != args.gpus:
+        log(f"--gpus {args.gpus} but {ws} rank(s) were launched: reporting {ws}")
     res = run_reference(args) if args.impl == "reference" else run_ours(args)
     if res is not None:
         print(json.dumps(res), flush=True)

@@ -85,3 +85,26 @@ def test_fingerprints_cover_each_scorers_sources(tmp_path, monkeypatch):
     with open(csrc / "common.cuh", "a") as f:             # every scorer includes it
         f.write("\n")
     assert all(bench.score_kernel_fingerprint(v) != after[v] for v in ("mean", "max", "pos"))
+
+
+def test_gpus_flag_relaunches_one_process_per_gpu(monkeypatch):
+    """`bench.py --gpus N` started by hand runs itself under torch.distributed.run
+    with N processes and a loopback rendezvous, passing its own arguments on."""
+    seen = {}
+
+    def fake_call(cmd, timeout=None):
+        seen["cmd"], seen["timeout"] = cmd, timeout
+        return 0
+
+    monkeypatch.setattr(bench.subprocess, "call", fake_call)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "4", "--steps", "7", "--warmup", "3"])
+    try:
+        bench.main()
+    except SystemExit as e:
+        assert e.code == 0
+    cmd = seen["cmd"]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-6:] == ["--gpus", "4", "--steps", "7", "--warmup", "3"]
+    assert cmd[-7].endswith("bench.py") and seen["timeout"] > 0
