@@ -1,6 +1,13 @@
 // Compaction of K and V to the kept keys (bit copies, 16 bytes per lane,
 // a half-warp per 256-byte row).
 //
+// Page "The future-offset average in TriAttention can be precomputed",
+// opening section: once the keys are scored, the cache keeps the highest
+// within its budget and evicts the rest.  The pages do not say how the
+// survivors are laid out; the two forms below are this library's reading
+// (ascending order out of place; a hole fill that moves the fewest rows in
+// place, which attention does not notice since K and V rows move together).
+//
 //  * gather (out of place): out[u][j] = cache row kept[u][j] of unit u, for
 //    j < kept_count[u]; the output is [units][B][128] for K and for V.
 //  * hole fill (in place): in a unit with n > B keys the kept keys below B

@@ -1,5 +1,9 @@
 // One kernel for the whole step of a cache with few units (score, keep the
 // top B, compact K and V), for CONTIG and RAGGED caches compacted out of place.
+// The step is the one of the page "The future-offset average in TriAttention
+// can be precomputed": the folded score of its section "The averaging step -
+// the one we improve" (one dot product per key with the folded weights), then
+// the opening section's keep-the-highest-within-budget and evict-the-rest.
 //
 // With few units, the three-kernel path is latency-bound: selection runs one
 // CTA per unit, so a handful of SMs work while the rest idle.  Here each unit
