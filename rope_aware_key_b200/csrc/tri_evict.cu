@@ -197,9 +197,10 @@ tri_status make_geom(const tri_cache_desc* c, bool need_v, Geom* g) {
       if (c->stride_head < 0 || (c->stride_head % 8)) return TRI_ERR_INVALID_ARG;
       if (H > 1 && c->stride_head == 0) return TRI_ERR_INVALID_ARG;
       for (int b = 0; b < c->batch; ++b) {
-        const int32_t n = c->cu_seqlens[b + 1] - c->cu_seqlens[b];
-        if (n < 0) return TRI_ERR_INVALID_ARG;
-        g->len[b] = n;
+        // in 64 bits: the int32 difference of hostile offsets could wrap
+        const int64_t n = int64_t{c->cu_seqlens[b + 1]} - c->cu_seqlens[b];
+        if (n < 0 || n > INT32_MAX) return TRI_ERR_INVALID_ARG;
+        g->len[b] = static_cast<int32_t>(n);
         g->start[b] = c->cu_seqlens[b];
         if (n > max_len) max_len = n;
       }

@@ -96,6 +96,12 @@ def test_ragged_checks(L):
     cu3 = (ctypes.c_int32 * 4)(0, 10, 15, 21)
     d.cu_seqlens = ctypes.cast(cu3, ctypes.POINTER(ctypes.c_int32))
     assert L.tri_score_row_stride(ctypes.byref(d)) == 12
+    # offsets whose int32 difference wraps: the third length would come out as
+    # 11, starting below the buffer; it must be refused
+    cu4 = (ctypes.c_int32 * 4)(0, 1 << 30, (1 << 31) - 1, -(1 << 31) + 10)
+    d.cu_seqlens = ctypes.cast(cu4, ctypes.POINTER(ctypes.c_int32))
+    assert L.tri_score_row_stride(ctypes.byref(d)) == -1
+    assert L.tri_score_keys(ctypes.byref(d), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), None) == 1
 
 
 def paged(**kw):
