@@ -210,7 +210,7 @@ tri_status make_geom(const tri_cache_desc* c, bool need_v, Geom* g) {
     case TRI_LAYOUT_PAGED: {
       if (!c->seq_lens || !c->block_table) return TRI_ERR_INVALID_ARG;
       if (c->block_size < 1 || c->max_blocks_per_seq < 1 || c->num_blocks < 1) return TRI_ERR_INVALID_ARG;
-      if (8 % c->num_kv_heads != 0 || c->block_size * c->num_kv_heads > tri::score::kTileRows)
+      if (8 % c->num_kv_heads != 0 || int64_t{c->block_size} * c->num_kv_heads > tri::score::kTileRows)
         return TRI_ERR_UNSUPPORTED;
       const int64_t page = int64_t{c->block_size} * c->num_kv_heads * TRI_HEAD_DIM;
       if (c->stride_block < page || (c->stride_block % 8)) return TRI_ERR_INVALID_ARG;

@@ -120,6 +120,7 @@ def paged(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(num_kv_heads=3, stride_block=16 * 3 * 128, stride_layer=100 * 16 * 3 * 128), 2),   # H must divide 8
     (dict(block_size=64), 2),                     # block_size * H > 128
+    (dict(num_kv_heads=8, block_size=1 << 29, stride_block=1 << 39, stride_layer=1 << 40), 2),   # product wraps int32
     (dict(stride_block=16 * 4 * 128 - 8), 1),     # pages overlap
     (dict(lens=(65, 1)), 1),                      # longer than max_blocks * block_size
     (dict(block_table=None), 1),
