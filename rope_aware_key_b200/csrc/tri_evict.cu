@@ -243,16 +243,20 @@ tri_status make_geom(const tri_cache_desc* c, bool need_v, Geom* g) {
 
 // Score tiles: per sequence, 128-key chunks (CONTIG / RAGGED) or groups of
 // pages_per_tile pages (PAGED).
+// Returns the tile count, or INT64_MAX when the per-sequence prefix would not
+// fit the int32 table the kernels search (callers reject counts > INT32_MAX).
 int64_t fill_tile_prefix(Geom* g) {
-  int32_t acc = 0;
+  int64_t acc = 0;
   for (int b = 0; b < g->batch; ++b) {
-    g->tile_prefix[b] = acc;
-    const int per = g->layout == TRI_LAYOUT_PAGED ? g->block_size * g->pages_per_tile : tri::score::kTileRows;
+    g->tile_prefix[b] = static_cast<int32_t>(acc);
+    const int64_t per = g->layout == TRI_LAYOUT_PAGED ? int64_t{g->block_size} * g->pages_per_tile
+                                                      : int64_t{tri::score::kTileRows};
     acc += (g->len[b] + per - 1) / per;
+    if (acc > INT32_MAX) return INT64_MAX;
   }
-  g->tile_prefix[g->batch] = acc;
+  g->tile_prefix[g->batch] = static_cast<int32_t>(acc);
   const int64_t outer = g->layout == TRI_LAYOUT_PAGED ? g->L : int64_t{g->L} * g->H;
-  return outer * acc;
+  return outer * acc;                                  // < 2^31 * 2^31
 }
 
 tri_status launch_score(const Geom& g0, const float* w, float* scores, int dev, cudaStream_t s) {
@@ -487,20 +491,26 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // Rows of the key cache as one 2-D bf16 tensor [rows][128] (256-byte rows),
 // when the layout packs the units back to back (CONTIG or RAGGED); 0 otherwise.
+// (Sizes are checked first, so the stride products below stay in range; the
+// descriptor has already passed make_geom.)
 int64_t packed_rows(const tri_cache_desc* c) {
   const int64_t H = c->num_kv_heads, L = c->num_layers, Bt = c->batch;
   if (c->layout == TRI_LAYOUT_CONTIG) {
     const int64_t n = c->seq_len;
+    const int64_t rows = L * H * Bt * n;               // < 2^31 * 2^30
+    if (rows > INT32_MAX) return 0;
     if (Bt > 1 && c->stride_seq != n * TRI_HEAD_DIM) return 0;
     if (H > 1 && c->stride_head != Bt * n * TRI_HEAD_DIM) return 0;
     if (L > 1 && c->stride_layer != H * Bt * n * TRI_HEAD_DIM) return 0;
-    return L * H * Bt * n;
+    return rows;
   }
   if (c->layout == TRI_LAYOUT_RAGGED) {
     const int64_t T = c->cu_seqlens[c->batch];
+    const int64_t rows = L * H * T;                    // < 2^31 * 2^31
+    if (T < 0 || rows > INT32_MAX) return 0;
     if (H > 1 && c->stride_head != T * TRI_HEAD_DIM) return 0;
     if (L > 1 && c->stride_layer != H * T * TRI_HEAD_DIM) return 0;
-    return L * H * T;
+    return rows;
   }
   return 0;
 }
