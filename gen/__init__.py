@@ -27,7 +27,6 @@ both sides, so that never matters for parity.
 from __future__ import annotations
 
 import dataclasses
-import math
 from typing import Dict, List, Optional, Sequence
 
 import torch

@@ -15,7 +15,7 @@ Bars:
 from __future__ import annotations
 
 import dataclasses
-from typing import Dict, List, Optional, Sequence
+from typing import Optional
 
 import numpy as np
 import torch
