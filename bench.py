@@ -8,6 +8,14 @@ selection per (layer, head, sequence) and the out-of-place compaction of K
 and V (four C-ABI calls, four kernels).  Default workload: a Qwen3-8B-shaped
 cache of 36 layers x 8 KV heads x 32768 keys (batch 1, contiguous), B = 2048.
 
+The paged workload (--workload qwen25_paged: 28 layers x 4 KV heads, 64
+sequences of 8192..32768 tokens in 16-token pages) is a serving cache that is
+pruned once per window of generated tokens: one initial event (every
+sequence down to B in place), then steady rounds, each appending 128 tokens
+per sequence (untimed, as a decoder would) and re-compressing every
+2176-key row down to B in place.  A step there is one steady round (default
+8 timed rounds); the initial event is reported beside it.
+
 Prints one JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun);
 every rank compresses its own cache (independent problems, no collective on
 the data path), time = max over ranks.
@@ -82,6 +90,8 @@ SCORE_KERNELS = {
                                      "score_pos_tma.cuh"), "score_pos_traffic.txt"),
 }
 POS_SPREAD = 4             # pre-RoPE variant: keys keep 1 in 4 of the original positions
+PAGED_ROUNDS = 8           # timed steady rounds of the paged workload
+PAGED_APPEND = 128         # tokens a sequence generates between two pruning events
 
 METRICS = {
     "mean": "keys scored+selected/s (fold + score + top-B select + K/V compaction)",
@@ -115,31 +125,79 @@ def ncu_traffic(workload, variant="mean"):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 100 ms in the background."""
+    """SM clock, power and throttle reasons sampled in the background while
+    the timed region runs: through NVML every 2 ms (so that even a timed
+    region of a few milliseconds gets a dozen samples), or, without NVML,
+    nvidia-smi every 100 ms.  Each sample is a row
+    [time, index, sm MHz, max sm MHz, power W, reasons, hw_slowdown,
+     hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap]."""
 
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, uuid: str = None, period_s: float = 0.002):
         self.samples = []
         self.proc = None
+        self.source = None
+        self.period_s = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = None
+            if uuid:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self._nvml, self._h, self._index = pynvml, h, gpu_index
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
                  "-i", str(gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi"
+            self.period_s = 0.1
         except Exception:
             self.proc = None
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    def _poll(self):
+        nv, h = self._nvml, self._h
+        try:
+            smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception:
+            smax = "[N/A]"
+        bits = (nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap)
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                row = ["", str(self._index), str(sm), str(smax), f"{pw:.1f}", hex(r)] + \
+                      ["Active" if r & b else "Not Active" for b in bits]
+                self.samples.append((time.time(), row))
+            except Exception:
+                pass
+            self._stop.wait(self.period_s)
+
     def wait_first(self, limit_s=5.0):
-        """Wait (bounded) for the first sample: nvidia-smi's start-up then lies
+        """Wait (bounded) for the first sample: the sampler's start-up then lies
         outside the timed region."""
         t = time.time()
-        while self.proc is not None and not self.samples and time.time() - t < limit_s:
-            time.sleep(0.02)
+        while self.source is not None and not self.samples and time.time() - t < limit_s:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -148,6 +206,9 @@ class ClockSampler:
                 self.samples.append((time.time(), parts))
 
     def stop(self):
+        ev = getattr(self, "_stop", None)
+        if ev is not None:
+            ev.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -157,6 +218,7 @@ class ClockSampler:
 
     def summary(self, t0, t1):
         rows = [p for (t, p) in self.samples if t0 <= t <= t1]
+        inside = len(rows)
         if not rows:
             rows = [p for (_, p) in self.samples[-5:]]
         if not rows:
@@ -172,8 +234,27 @@ class ClockSampler:
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         reasons = sorted({n for r in rows for n, v in zip(names, r[6:10]) if v.strip().lower() == "active"})
         pw = [num(r[4]) for r in rows if num(r[4]) is not None]
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+               "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+        if getattr(self, "source", None):
+            out["source"] = f"{self.source}, every {self.period_s * 1e3:g} ms"
+        if inside == 0:
+            out["note"] = "no sample inside the timed region: the last samples before it"
+        return out
+
+
+def gpu_identity(dev, local):
+    """(NVML index guess, NVML uuid) of the torch device `dev`."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    try:
+        index = int(vis.split(",")[local]) if vis else local
+    except ValueError:
+        index = local
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    return index, uuid
 
 
 # ---------------------------------------------------------------- our arm
@@ -193,16 +274,34 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     wl = gen.WORKLOADS[args.workload]
-    assert wl.layout in ("contig", "ragged"), "the bench compresses contiguous or ragged caches out of place"
+    if wl.layout == "paged":
+        return run_paged(args, tri, dev, rank, ws)
     B = wl.budget
 
     t = time.time()
-    cache = gen.make_cache(wl, seed=rank_seed(args.seed, rank), device=dev)
+    if args.shard == "layers":
+        # one cache split by whole layers (every KV head and sequence of a
+        # layer on one rank): each rank draws only its own layers
+        from rope_aware_key_b200.shard import layer_ranges
+        whole = wl
+        l0, l1 = layer_ranges(whole.num_layers, ws)[rank]
+        if l1 == l0:
+            raise SystemExit(f"--shard layers: {ws} ranks for {whole.num_layers} layers leaves rank {rank} empty")
+        cache = gen.make_cache(whole, seed=args.seed, device=dev, layer_range=(l0, l1))
+        wl = cache.wl
+        job_keys = sum(cache.lens) * whole.num_layers * whole.num_kv_heads
+        parallelism = f"one cache split by layers over {ws} ranks (layers {l0}..{l1 - 1} on rank {rank})"
+    else:
+        cache = gen.make_cache(wl, seed=rank_seed(args.seed, rank), device=dev)
+        job_keys = None
+        parallelism = f"independent caches x{ws}"
     torch.cuda.synchronize()
     log(f"[rank {rank}] generated {args.workload} in {time.time() - t:.1f}s")
     d = (tri.desc_contig(cache.k, cache.v) if wl.layout == "contig"
          else tri.desc_ragged(cache.k, cache.v, cache.cu_seqlens.cpu().tolist()))
     keys = sum(cache.lens) * wl.num_layers * wl.num_kv_heads
+    if job_keys is None:
+        job_keys = keys * ws                       # every rank its own cache of the same shape
     moved = sum(min(B, n) for n in cache.lens) * wl.num_layers * wl.num_kv_heads
     qc = cache.query_center.reshape(-1, wl.head_dim).to(dev).contiguous()
     if args.variant == "max":
@@ -257,9 +356,7 @@ def run_ours(args):
         if ev is not None:
             ev[4].record(st)
 
-    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
-        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
-    sampler = ClockSampler(gpu_index)
+    sampler = ClockSampler(*gpu_identity(dev, local))
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -332,7 +429,7 @@ def run_ours(args):
 
     ms_max = max_over_ranks(ms, ws, dev)
     ms_step = ms_max / args.steps
-    value = keys * ws * args.steps / (ms_max / 1e3)
+    value = job_keys * args.steps / (ms_max / 1e3)
 
     # roofline of the dominant kernel (scoring; or the one-call step) and of the whole step
     peak, peak_kind = measured_hbm_peak()
@@ -346,7 +443,7 @@ def run_ours(args):
     traffic = ncu_traffic(args.workload, args.variant)
 
     # end to end through the C ABI with host buffers (pinned), copies inside the timed region
-    e2e = run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, keys, ws, positions, qpos)
+    e2e = run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, job_keys, ws, positions, qpos)
 
     result = None
     if rank == 0:
@@ -354,12 +451,14 @@ def run_ours(args):
         result = {
             "metric": METRICS[args.variant],
             "value": value, "unit": "keys/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong" if args.shard == "layers" else "weak", "vs_baseline": None,
             "dtype": "bf16 keys/values, fp32 scores (fp64 fold)", "data": "synthetic (seeded generator)",
-            "config": {"workload": f"{args.workload}: {wl.num_layers} layers x {wl.num_kv_heads} KV heads x "
+            "config": {"workload": f"{args.workload}: {gen.WORKLOADS[args.workload].num_layers} layers x "
+                                   f"{wl.num_kv_heads} KV heads x "
                                    f"{max(cache.lens)} keys, batch {wl.batch}, {wl.layout}, B={B}, "
                                    f"theta={wl.theta:g}, |D|={len(wl.offsets)}",
-                       "keys_per_gpu": keys, "budget": B, "parallelism": f"independent caches x{ws}",
+                       "keys_per_gpu": keys, "budget": B, "parallelism": parallelism,
                        "l2": ("K and V of %.3f GB each vs a 126 MB L2: L2 flushed (512 MB fill) before every "
                               "timed step, each step timed alone" if flush else
                               "inputs larger than L2 (K and V of %.2f GB each vs 126 MB); no flush")
@@ -387,7 +486,244 @@ def run_ours(args):
     return result
 
 
-def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, keys, ws, positions=None, qpos=None):
+def run_paged(args, tri, dev, rank, ws):
+    """The paged serving cache: an initial pruning event, then steady rounds
+    (append PAGED_APPEND tokens per sequence, untimed; re-compress in place).
+    Each event is fold + score + select + in-place hole fill (four calls),
+    queued behind a GPU sleep so that the launches are all waiting when the
+    first one runs, and timed with CUDA events on the launching stream; L2 is
+    flushed (a 512 MB fill) before every event."""
+    _, _, local = dist_env()
+    if args.shard != "replicas":
+        raise SystemExit("the paged workload runs as replicas (one cache per rank)")
+    wl = gen.WORKLOADS[args.workload]
+    B = wl.budget
+    L, H = wl.num_layers, wl.num_kv_heads
+    seed = rank_seed(args.seed, rank)
+    t = time.time()
+    cache = gen.make_cache(wl, seed=seed, device=dev)
+    torch.cuda.synchronize()
+    log(f"[rank {rank}] generated {args.workload} in {time.time() - t:.1f}s "
+        f"({sum(cache.lens) * L * H / 1e6:.1f} M keys)")
+    units = wl.units
+    qc = cache.query_center.reshape(-1, wl.head_dim).to(dev).contiguous()
+    w = torch.empty_like(qc)
+    kept = torch.empty((units, B), dtype=torch.int32, device=dev)
+    cnt = torch.empty((units,), dtype=torch.int32, device=dev)
+    flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    col = torch.arange(B, device=dev)[None, :]
+
+    def event(d, scores, evs=None):
+        def rec(i):
+            if evs is not None:
+                evs[i].record(stream)
+        rec(0)
+        tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+        rec(1)
+        tri.score_keys(d, w, scores, stream=stream)
+        rec(2)
+        tri.select_topk(d, scores, B, kept, cnt, stream=stream)
+        rec(3)
+        tri.compact_kv(d, kept, cnt, B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None, stream=stream)
+        rec(4)
+
+    def timed_event(d, scores):
+        flush_buf.fill_(1)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        torch.cuda.synchronize()
+        torch.cuda._sleep(int(2e6))
+        event(d, scores, evs)
+        torch.cuda.synchronize()
+        per = [evs[i].elapsed_time(evs[i + 1]) for i in range(4)]
+        moved = int(((kept >= B) & (col < cnt[:, None])).sum())     # rows the hole fill moved
+        return per, moved
+
+    # initial event: warm-up with the non-destructive stages, then the event once
+    d0 = tri.desc_paged(cache.k, cache.v, cache.block_table, cache.lens)
+    scores0 = torch.empty((units, tri.score_row_stride(d0)), dtype=torch.float32, device=dev)
+    keys0 = sum(cache.lens) * L * H
+    for _ in range(args.warmup):
+        tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+        tri.score_keys(d0, w, scores0, stream=stream)
+        tri.select_topk(d0, scores0, B, kept, cnt, stream=stream)
+    per0, moved0 = timed_event(d0, scores0)
+    gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
+    del scores0
+    torch.cuda.empty_cache()
+    st = tri.read_device_status()
+    if st:
+        raise RuntimeError(f"device status {st:#x} after the initial event")
+
+    # steady rounds
+    sampler = ClockSampler(*gpu_identity(dev, local), period_s=0.001)
+    sampler.wait_first()
+    scores = None
+    rounds = []
+    launches0 = tri.kernel_launches()
+    t0 = None
+    for i in range(args.warmup + args.steps):
+        gen.append_tokens(cache, PAGED_APPEND, step=1 + i)
+        d = tri.desc_paged(cache.k, cache.v, cache.block_table, cache.lens)
+        if scores is None:
+            scores = torch.empty((units, tri.score_row_stride(d)), dtype=torch.float32, device=dev)
+        if i == args.warmup:
+            if ws > 1:
+                torch.distributed.barrier()
+            t0 = time.time()
+            launches0 = tri.kernel_launches()
+        per, moved = timed_event(d, scores)
+        if i >= args.warmup:
+            rounds.append((per, moved, sum(cache.lens) * L * H))
+        gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
+    t1 = time.time()
+    launches = tri.kernel_launches() - launches0
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+    clocks["window"] = "the steady rounds, appends between them included"
+    st = tri.read_device_status()
+    if st:
+        raise RuntimeError(f"device status {st:#x} after the steady rounds")
+
+    per = np.array([r[0] for r in rounds])                       # ms: fold, score, select, hole fill
+    ms_rounds = float(per.sum())
+    ms_max = max_over_ranks(ms_rounds, ws, dev)
+    keys_round = rounds[0][2]
+    moved = float(np.mean([r[1] for r in rounds]))
+    value = keys_round * len(rounds) * ws / (ms_max / 1e3)
+    ms_step = ms_max / len(rounds)
+    peak, peak_kind = measured_hbm_peak()
+    score_ms = float(per[:, 1].mean())
+    score_bytes = keys_round * KEY_BYTES
+    achieved = score_bytes / (score_ms / 1e3) / 1e9
+    step_bytes = keys_round * KEY_BYTES + moved * MOVE_BYTES
+    step_gbs = step_bytes / (ms_step / 1e3) / 1e9
+    init_ms = float(sum(per0))
+    init_bytes = keys0 * KEY_BYTES + moved0 * MOVE_BYTES
+
+    e2e = run_paged_e2e(args, tri, cache, wl, qc, w, kept, cnt, stream, ws)
+
+    result = None
+    if rank == 0:
+        cpu = cpu_baseline(wl, args) if ws == 1 and not args.no_cpu_baseline else None
+        result = {
+            "metric": METRICS["mean"] + ", paged cache, in place",
+            "value": value, "unit": "keys/s", "n_gpus": ws, "steps": len(rounds), "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 keys/values, fp32 scores (fp64 fold)", "data": "synthetic (seeded generator)",
+            "config": {"workload": f"{args.workload}: {L} layers x {H} KV heads, {wl.batch} sequences of "
+                                   f"{wl.len_lo}..{wl.len_hi} tokens in {wl.block_size}-token pages, B={B}, "
+                                   f"theta={wl.theta:g}, |D|={len(wl.offsets)}; a step is one steady round: "
+                                   f"{PAGED_APPEND} tokens appended per sequence (untimed), every row of "
+                                   f"{B + PAGED_APPEND} keys re-compressed to {B} in place",
+                       "keys_per_gpu": keys_round, "budget": B, "parallelism": f"independent caches x{ws}",
+                       "l2": "L2 flushed (512 MB fill) before every pruning event, outside the events"},
+            "step_breakdown_ms": {"fold": float(per[:, 0].mean()), "score": score_ms,
+                                  "select": float(per[:, 2].mean()), "holefill": float(per[:, 3].mean())},
+            "rows_moved_per_step": moved,
+            "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_gbs,
+                    "frac_of_measured": step_gbs / peak, "frac_of_8tbps_spec": step_gbs / SPEC_HBM_GBS},
+            "initial_event": {"ms": init_ms, "keys": keys0, "rows_moved": moved0,
+                              "breakdown_ms": dict(zip(("fold", "score", "select", "holefill"), per0)),
+                              "keys_per_s": keys0 / (init_ms / 1e3),
+                              "achieved_gbs": init_bytes / (init_ms / 1e3) / 1e9,
+                              "frac_of_8tbps_spec": init_bytes / (init_ms / 1e3) / 1e9 / SPEC_HBM_GBS,
+                              "timing": "one event (it compacts the cache in place), after warm-up passes of "
+                                        "the fold, score and select"},
+            "roofline": {"kernel": "score_kernel (paged)", "bound": "hbm", "achieved": achieved, "peak": peak,
+                         "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": ncu_traffic(args.workload, "mean"),
+                         "algorithmic_bytes_per_launch": score_bytes},
+            "clocks": clocks,
+            "gpu_launches": int(launches),
+            "timing": "each round: plain launches queued behind a GPU sleep, CUDA events around the four calls",
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+    return result
+
+
+def run_paged_e2e(args, tri, cache, wl, qc, w, kept, cnt, stream, ws):
+    """A steady round end to end from host memory: the round's new tokens
+    (K and V of PAGED_APPEND tokens per sequence, pinned) are copied to the
+    device and written into fresh pages, the block table follows, the four
+    calls run, and the kept indices and counts come back to the host.  The
+    cache itself stays resident, as a serving cache does."""
+    steps = max(1, min(args.steps, args.e2e_steps))
+    B, L, H, bs, d = wl.budget, wl.num_layers, wl.num_kv_heads, wl.block_size, wl.head_dim
+    per_seq = PAGED_APPEND // bs
+    assert PAGED_APPEND % bs == 0 and all(n % bs == 0 for n in cache.lens)
+    g = torch.Generator().manual_seed(gen.sub_seed(args.seed, "append_K", 1 << 20, 0))
+    shape = (L, wl.batch * per_seq, bs * H * d)
+    hk = torch.randn(shape, generator=g).to(torch.bfloat16).pin_memory()
+    hv = torch.randn(shape, generator=g).to(torch.bfloat16).pin_memory()
+    sk, sv = torch.empty(shape, dtype=torch.bfloat16, device=qc.device), \
+        torch.empty(shape, dtype=torch.bfloat16, device=qc.device)
+    hkept = torch.empty(kept.shape, dtype=kept.dtype, pin_memory=True)
+    hcnt = torch.empty(cnt.shape, dtype=cnt.dtype, pin_memory=True)
+    nb = cache.k.shape[1]
+    kpool, vpool = cache.k.view(L, nb, -1), cache.v.view(L, nb, -1)
+    table = cache.block_table.cpu()
+    htable = torch.empty(table.shape, dtype=torch.int32, pin_memory=True)
+    scores = None
+    times = []
+    for i in range(steps + 1):                     # the first round is a warm-up
+        # host bookkeeping of the append: fresh pages for every sequence
+        pages = []
+        for b in range(wl.batch):
+            n0 = cache.lens[b] // bs
+            for j in range(per_seq):
+                p = cache.free_blocks.pop()
+                table[b, n0 + j] = p
+                pages.append(p)
+            cache.lens[b] += PAGED_APPEND
+        htable.copy_(table)
+        idx = torch.tensor(pages, dtype=torch.int64).pin_memory()
+        dt = tri.desc_paged(cache.k, cache.v, cache.block_table, cache.lens)
+        if scores is None:
+            scores = torch.empty((wl.units, tri.score_row_stride(dt)), dtype=torch.float32, device=qc.device)
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record(stream)
+        cache.block_table.copy_(htable, non_blocking=True)
+        di = idx.to(qc.device, non_blocking=True)
+        sk.copy_(hk, non_blocking=True)
+        sv.copy_(hv, non_blocking=True)
+        kpool[:, di] = sk                          # the new tokens into their pages
+        vpool[:, di] = sv
+        tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+        tri.score_keys(dt, w, scores, stream=stream)
+        tri.select_topk(dt, scores, B, kept, cnt, stream=stream)
+        tri.compact_kv(dt, kept, cnt, B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None, stream=stream)
+        hkept.copy_(kept, non_blocking=True)
+        hcnt.copy_(cnt, non_blocking=True)
+        end.record(stream)
+        torch.cuda.synchronize()
+        if i > 0:
+            times.append(start.elapsed_time(end))
+        # shrink every sequence back to B and free its tail pages (host)
+        for b in range(wl.batch):
+            keep = (B + bs - 1) // bs
+            for j in range(keep, cache.lens[b] // bs):
+                cache.free_blocks.append(int(table[b, j]))
+                table[b, j] = 0
+            cache.lens[b] = min(B, cache.lens[b])
+        cache.block_table.copy_(table.to(qc.device))
+    ms = max_over_ranks(float(np.sum(times)), ws, qc.device)
+    keys = wl.units * (B + PAGED_APPEND)
+    h2d = hk.numel() * 2 + hv.numel() * 2 + htable.numel() * 4 + len(pages) * 8
+    d2h = hkept.numel() * 4 + hcnt.numel() * 4
+    return {"value": keys * ws * steps / (ms / 1e3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps, "host_memory": "pinned",
+            "what": "per round: the new tokens' K and V and the block table in, written into fresh pages, "
+                    "fold + score + select + in-place hole fill, kept indices and counts out; the cache stays "
+                    "resident"}
+
+
+def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, job_keys, ws, positions=None,
+            qpos=None):
     """Same step with the cache in pinned host memory: H2D of K and V, the four
     calls, D2H of the kept indices, counts and compacted K/V, every step.
 
@@ -467,7 +803,7 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
     ms = max_over_ranks(start.elapsed_time(end), ws, qc.device)
     h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 4 + (hpos.numel() * 4 if hpos is not None else 0)
     d2h = hkept.numel() * 4 + hcnt.numel() * 4 + hko.numel() * 2 + hvo.numel() * 2
-    return {"value": keys * ws * steps / (ms / 1e3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
+    return {"value": job_keys * steps / (ms / 1e3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps,
             "host_memory": "pinned",
             "overlap": "results of step i copied back on a second stream while step i+1's inputs are copied in"}
@@ -477,7 +813,8 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, key
 
 def oracle_unit_pipeline(orc, keys_bits, vals_bits, qc, wl, B, threads, variant="mean"):
     """The oracle's own path for one unit: literal per-offset average (or
-    maximum), keep-highest, gather."""
+    maximum), keep-highest, then a gather (or, for a paged cache, the
+    in-place hole fill)."""
     if variant == "pos":
         # a compacted pre-RoPE unit: sorted distinct positions in [0, POS_SPREAD * n), query at POS_SPREAD * n
         n = keys_bits.shape[0]
@@ -488,8 +825,12 @@ def oracle_unit_pipeline(orc, keys_bits, vals_bits, qc, wl, B, threads, variant=
         score = orc.score_max_literal if variant == "max" else orc.score_literal
         s = score(keys_bits, qc, wl.theta, wl.offsets, wl.delta0, 0, threads)
     kept = orc.select(s, B)
-    orc.gather_rows(keys_bits, kept)
-    orc.gather_rows(vals_bits, kept)
+    if wl.layout == "paged":
+        orc.holefill(keys_bits, kept, B)
+        orc.holefill(vals_bits, kept, B)
+    else:
+        orc.gather_rows(keys_bits, kept)
+        orc.gather_rows(vals_bits, kept)
     return len(s)
 
 
@@ -507,7 +848,8 @@ def cpu_baseline(wl, args, budget_s=None):
     orc.build()
     threads = orc.default_threads()
     budget_s = args.cpu_seconds if budget_s is None else budget_s
-    n = min(max(wl.seq_len, wl.len_hi, 4096), 32768)
+    # a paged cache is timed in its steady rounds: rows of B + PAGED_APPEND keys
+    n = wl.budget + PAGED_APPEND if wl.layout == "paged" else min(max(wl.seq_len, wl.len_hi, 4096), 32768)
     kb, vb, qc = cpu_sample(wl, n, args.seed)
     B = min(wl.budget, n)
     done = 0
@@ -523,7 +865,8 @@ def cpu_baseline(wl, args, budget_s=None):
             "sample": f"{reps} x one unit of {n} keys (literal {'max' if args.variant == 'max' else 'average'} "
                       f"{'at per-key distances ' if args.variant == 'pos' else ''}over "
                       f"|D|={len(wl.offsets)} offsets, "
-                      f"select B={B}, gather K and V), fp64, {dt:.1f}s"}
+                      f"select B={B}, {'hole fill' if wl.layout == 'paged' else 'gather'} K and V), fp64, "
+                      f"{dt:.1f}s"}
 
 
 def run_reference(args):
@@ -582,7 +925,8 @@ def relaunch_per_gpu(n: int) -> int:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 1000; 8 steady rounds for the paged workload)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="qwen3_full", choices=sorted(gen.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -593,10 +937,15 @@ def main():
     ap.add_argument("--eager", action="store_true", help="time plain launches instead of a CUDA graph of the step")
     ap.add_argument("--path", default="calls", choices=["calls", "compress"],
                     help="calls: fold, score, select, compact as four calls (default); compress: fold + tri_compress")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "layers"],
+                    help="N > 1: replicas (default): every rank compresses its own cache (weak scaling); "
+                         "layers: one cache split by whole layers over the ranks (strong scaling)")
     ap.add_argument("--variant", default="mean", choices=["mean", "max", "pos"],
                     help="mean: the folded offset average (default); max: the max over the offsets; "
                          "pos: the offset average at per-key distances (pre-RoPE cache with positions)")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = PAGED_ROUNDS if gen.WORKLOADS[args.workload].layout == "paged" else 1000
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     ws = dist_env()[0]

@@ -188,6 +188,7 @@ class Cache:
     block_table: Optional[torch.Tensor] = None   # paged, int32 [batch][max_blocks]
     seq_lens: Optional[torch.Tensor] = None      # paged, int32 [batch]
     free_blocks: Optional[List[int]] = None      # paged, unused physical pages
+    layer0: int = 0                              # first layer of the full cache that this one holds
 
     @property
     def max_len(self) -> int:
@@ -195,17 +196,27 @@ class Cache:
 
 
 def make_cache(wl: Workload, seed: int, device="cpu", with_values: bool = True,
-               lens: Optional[Sequence[int]] = None) -> Cache:
+               lens: Optional[Sequence[int]] = None, layer_range: Optional[Sequence[int]] = None) -> Cache:
     """Draw a full cache for ``wl`` in its layout.
 
     contig: K, V bf16 [L][H][batch][N][d]
     ragged: K, V bf16 [L][H][T][d] with cu_seqlens (int32, prefix sums of lens)
     paged:  K, V bf16 [L][num_blocks][block_size][H][d] with an int32 block table
+
+    ``layer_range`` = (l0, l1) draws only layers l0 .. l1-1 of that cache --
+    the very same numbers, since every layer has its own generator seeds --
+    as a cache of l1 - l0 layers (its workload's num_layers cut to match).
     """
-    L, H, d = wl.num_layers, wl.num_kv_heads, wl.head_dim
+    l0, l1 = (0, wl.num_layers) if layer_range is None else (int(layer_range[0]), int(layer_range[1]))
+    assert 0 <= l0 <= l1 <= wl.num_layers
+    H, d = wl.num_kv_heads, wl.head_dim
     lens = list(lens) if lens is not None else seq_lengths(wl, seed)
     kc, qc = centers(wl, seed)
-    c = Cache(wl, seed, lens, kc, qc, None, None)
+    kc, qc = kc[l0:l1].contiguous(), qc[l0:l1].contiguous()
+    if layer_range is not None:
+        wl = scaled(wl, num_layers=l1 - l0)
+    L = wl.num_layers
+    c = Cache(wl, seed, lens, kc, qc, None, None, layer0=l0)
 
     if wl.layout == "contig":
         N = wl.seq_len if lens is None else max(lens)
@@ -214,9 +225,9 @@ def make_cache(wl: Workload, seed: int, device="cpu", with_values: bool = True,
         c.v = torch.empty_like(c.k) if with_values else None
         for l in range(L):
             for b in range(wl.batch):
-                c.k[l, :, b] = draw_keys(wl, seed, l, b, N, kc[l], device)
+                c.k[l, :, b] = draw_keys(wl, seed, l0 + l, b, N, kc[l], device)
                 if with_values:
-                    c.v[l, :, b] = draw_values(wl, seed, l, b, N, device)
+                    c.v[l, :, b] = draw_values(wl, seed, l0 + l, b, N, device)
     elif wl.layout == "ragged":
         cu = [0]
         for n in lens:
@@ -226,9 +237,9 @@ def make_cache(wl: Workload, seed: int, device="cpu", with_values: bool = True,
         c.v = torch.empty_like(c.k) if with_values else None
         for l in range(L):
             for b, n in enumerate(lens):
-                c.k[l, :, cu[b]:cu[b + 1]] = draw_keys(wl, seed, l, b, n, kc[l], device)
+                c.k[l, :, cu[b]:cu[b + 1]] = draw_keys(wl, seed, l0 + l, b, n, kc[l], device)
                 if with_values:
-                    c.v[l, :, cu[b]:cu[b + 1]] = draw_values(wl, seed, l, b, n, device)
+                    c.v[l, :, cu[b]:cu[b + 1]] = draw_values(wl, seed, l0 + l, b, n, device)
         c.cu_seqlens = torch.tensor(cu, dtype=torch.int32, device=device)
     elif wl.layout == "paged":
         bs = wl.block_size
@@ -251,10 +262,10 @@ def make_cache(wl: Workload, seed: int, device="cpu", with_values: bool = True,
             for b, n in enumerate(lens):
                 slots = paged_slots(table[b], n, bs).to(device)
                 kf = c.k[l].view(num_blocks * bs, H, d)
-                kf[slots] = draw_keys(wl, seed, l, b, n, kc[l], device).permute(1, 0, 2)
+                kf[slots] = draw_keys(wl, seed, l0 + l, b, n, kc[l], device).permute(1, 0, 2)
                 if with_values:
                     vf = c.v[l].view(num_blocks * bs, H, d)
-                    vf[slots] = draw_values(wl, seed, l, b, n, device).permute(1, 0, 2)
+                    vf[slots] = draw_values(wl, seed, l0 + l, b, n, device).permute(1, 0, 2)
     else:
         raise ValueError(f"unknown layout {wl.layout!r}")
     return c
@@ -275,7 +286,7 @@ def key_positions(c: Cache, seed: int, stride: int, spread: int = 4, device=None
             for b, n in enumerate(c.lens):
                 if n == 0:
                     continue
-                g = _gen(device, sub_seed(seed, "positions", l, h, b))
+                g = _gen(device, sub_seed(seed, "positions", c.layer0 + l, h, b))
                 pick = torch.randperm(spread * n, generator=g, device=device)[:n]
                 u = (l * wl.num_kv_heads + h) * wl.batch + b
                 pos[u, :n] = torch.sort(pick).values.to(torch.int32)
@@ -327,11 +338,11 @@ def append_tokens(c: Cache, n_new: int, step: int) -> None:
         slots = slots_all[n0:n1].to(dev)
         for l in range(wl.num_layers):
             kf = c.k[l].view(-1, H, d)
-            kf[slots] = draw_keys(wl, c.seed, l, (step << 16) | b, n_new,
+            kf[slots] = draw_keys(wl, c.seed, c.layer0 + l, (step << 16) | b, n_new,
                                   c.key_center[l], dev, tag="append_K").permute(1, 0, 2)
             if c.v is not None:
                 vf = c.v[l].view(-1, H, d)
-                vf[slots] = draw_values(wl, c.seed, l, (step << 16) | b, n_new, dev,
+                vf[slots] = draw_values(wl, c.seed, c.layer0 + l, (step << 16) | b, n_new, dev,
                                         tag="append_V").permute(1, 0, 2)
         c.lens[b] = n1
     c.block_table = table.to(dev)

@@ -11,7 +11,9 @@
  * Conventions used by every call:
  *  - "device" pointers are CUDA global memory of the device that owns the
  *    cache (the library launches on the device of desc->k, or of q_center for
- *    the fold); "host" pointers are ordinary CPU memory read during the call.
+ *    the fold, making it current during the call only: the calling thread's
+ *    current device and context are the same on return); "host" pointers are
+ *    ordinary CPU memory read during the call.
  *  - The caller allocates and owns every buffer.  The library never allocates
  *    or frees device memory at run time (tri_compress_noalloc uses a fixed
  *    array of the module, allocated when the library loads) and never
@@ -234,14 +236,23 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
  * kept_count[u] = min(B, n).  Entries past kept_count are not written.
  * scores: device fp32 [units][tri_score_row_stride(desc)].
  * kept: device int32 [units][B]; kept_count: device int32 [units].
- * B >= 1.  Needs no workspace. */
+ * B >= 1.  Needs no workspace.  Rows of at most 4096 keys (a cache
+ * re-compressed every window of generated tokens holds rows of B + the
+ * window) are selected by one warp each, longer rows by one CTA each; both
+ * give the same result.  A row too long for the CTA's shared memory (more
+ * than about 655,000 keys at B = 2048) is TRI_ERR_UNSUPPORTED. */
 tri_status tri_select_topk(const tri_cache_desc* desc, const float* scores, int B,
                            int32_t* kept, int32_t* kept_count, tri_stream_t stream);
 
 /* ---------------------------------------------------------------- compact */
 
-/* Compact K and V to the kept keys (bit copies).  See tri_compact_mode for
- * the two layouts.  kept / kept_count as written by tri_select_topk with the
+/* Compact K and V to the kept keys (bit copies): after scoring, the cache
+ * keeps its highest-scoring keys and evicts the rest (page "The future-offset
+ * average in TriAttention can be precomputed", opening section).  The page
+ * does not say where the survivors go; the two layouts of tri_compact_mode
+ * are this library's reading: ascending order out of place, and a hole fill
+ * in place that moves the fewest rows (attention does not depend on the slot
+ * order when a key's K and V rows move together).  kept / kept_count as written by tri_select_topk with the
  * same desc and B.  OUT_OF_PLACE: k_out, v_out device bf16 [units][B][128]
  * (16-byte aligned).  IN_PLACE_HOLEFILL: k_out and v_out must be NULL; the
  * cache (desc->k, desc->v) is modified, so they must point to writable
@@ -255,9 +266,14 @@ tri_status tri_compact_kv(const tri_cache_desc* desc, const int32_t* kept,
 /* Bytes of workspace tri_compress needs for `desc` (the score matrix). */
 tri_status tri_workspace_size(const tri_cache_desc* desc, int B, size_t* bytes);
 
-/* score -> select -> compact in one call (no host sync).  Same arguments and
- * results as the three calls; the scores live in `workspace` (device,
- * >= tri_workspace_size bytes, 256-byte aligned).
+/* score -> select -> compact in one call (no host sync): one pruning event of
+ * the page above -- every cached key scored with the folded weights ("The
+ * averaging step - the one we improve"), the highest-scoring keys within the
+ * budget kept and the rest evicted (opening section) -- with the survivors
+ * laid out as tri_compact_mode describes.  Same arguments and results as the
+ * three calls; the scores live in `workspace` (device, >= tri_workspace_size
+ * bytes, 256-byte aligned).  Every check of the three stages is made before
+ * the first launch.
  * A CONTIG or RAGGED cache compacted OUT_OF_PLACE whose units fit one wave of
  * thread-block clusters (units x 16 CTAs <= the SM count) and whose rows hold
  * at most 8192 keys runs as ONE kernel: a cluster per unit scores its keys into
@@ -292,7 +308,12 @@ tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B,
  *    before anything is launched (split the cache, e.g. by layers).
  *  - Set-up: the first call on a device looks up the scratch array's device
  *    address (cudaGetSymbolAddress) with that device current; make that
- *    first call before any stream capture.
+ *    first call before any stream capture.  The array belongs to the
+ *    library's module, which the CUDA runtime loads on a device the first
+ *    time any tri_* call uses that device (lazy module loading, the default);
+ *    a caller that will hand nearly all free memory to its own pool should
+ *    make its first library call on each device (for instance this one, on a
+ *    small cache) before it takes that memory, or the module load can fail.
  *  - Sharing: every call on a device uses the same scratch array, and it
  *    keeps the last call's contents (nothing in it needs to start at zero).
  *    Calls that overlap on the GPU -- on different streams, or from several
@@ -309,6 +330,9 @@ tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int 
 #define TRI_DEVFLAG_TIMEOUT       0x4u  /* a bounded wait inside a kernel gave up */
 #define TRI_DEVFLAG_BAD_KEPT      0x8u  /* compaction met a kept index outside [0, n) */
 #define TRI_DEVFLAG_BAD_POSITION  0x10u /* a key's distance t - p fell outside (-2^31, 2^31); its score is NaN */
+#define TRI_DEVFLAG_INVARIANT     0x20u /* only in a library built with -DTRI_CHECKED: a selection or compaction
+                                           invariant failed (a unit's kept count is not min(B, n), a histogram
+                                           does not total the row, holes and movers of a hole fill differ) */
 
 /* Wait for `stream`, then read the status word of the device that owns
  * `stream` (the current device for NULL) into *flags, and zero it if `clear`.

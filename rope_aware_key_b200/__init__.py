@@ -24,7 +24,8 @@ __all__ = [
     "score_row_stride", "read_device_status",
     "kernel_launches", "LAYOUT_CONTIG", "LAYOUT_RAGGED", "LAYOUT_PAGED", "PAIRING_HALF",
     "PAIRING_INTERLEAVED", "COMPACT_OUT_OF_PLACE", "COMPACT_IN_PLACE_HOLEFILL", "DEVFLAG_BAD_PAGE",
-    "DEVFLAG_NONFINITE", "DEVFLAG_TIMEOUT", "DEVFLAG_BAD_KEPT", "DEVFLAG_BAD_POSITION",
+    "DEVFLAG_NONFINITE", "DEVFLAG_TIMEOUT", "DEVFLAG_BAD_KEPT", "DEVFLAG_BAD_POSITION", "DEVFLAG_INVARIANT",
+    "load",
     "score_keys_at_positions",
 ]
 
@@ -36,6 +37,7 @@ PAIRING_HALF, PAIRING_INTERLEAVED = 0, 1
 COMPACT_OUT_OF_PLACE, COMPACT_IN_PLACE_HOLEFILL = 0, 1
 DEVFLAG_BAD_PAGE, DEVFLAG_NONFINITE, DEVFLAG_TIMEOUT, DEVFLAG_BAD_KEPT = 0x1, 0x2, 0x4, 0x8
 DEVFLAG_BAD_POSITION = 0x10
+DEVFLAG_INVARIANT = 0x20          # set only by a build with -DTRI_CHECKED
 MAX_OFFSETS, MAX_BATCH, HEAD_DIM = 2048, 256, 128
 
 _STATUS = {0: "TRI_OK", 1: "TRI_ERR_INVALID_ARG", 2: "TRI_ERR_UNSUPPORTED", 3: "TRI_ERR_WORKSPACE",
@@ -81,7 +83,14 @@ def lib() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: run `python -m rope_aware_key_b200.build` "
                           "(there is no fallback implementation)")
-    L = ctypes.CDLL(LIB_PATH)
+    _lib = load(LIB_PATH)
+    return _lib
+
+
+def load(path: str) -> ctypes.CDLL:
+    """A build of the library at `path` with the call signatures set (the
+    product library, or one of the test-only builds of the same sources)."""
+    L = ctypes.CDLL(path)
     P, I, I64, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     D = ctypes.POINTER(_CacheDesc)
     L.tri_fold_weights.argtypes = [ctypes.POINTER(_FoldParams), P, I, P, P]
@@ -105,7 +114,6 @@ def lib() -> ctypes.CDLL:
                  "tri_score_keys_at_positions", "tri_select_topk", "tri_compact_kv", "tri_workspace_size",
                  "tri_compress", "tri_read_device_status"):
         getattr(L, name).restype = I
-    _lib = L
     return L
 
 

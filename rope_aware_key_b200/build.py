@@ -1,6 +1,7 @@
 """Build libtri_evict.so in-tree with nvcc for sm_100a.
 
     python -m rope_aware_key_b200.build [--force] [-D NAME=VALUE ...]
+    python -m rope_aware_key_b200.build --variants     # the test-only builds, in _build/
 
 One translation unit (csrc/tri_evict.cu includes the kernel headers), static
 CUDA runtime, -lineinfo.  ptxas resource usage goes to _build/ptxas.txt.
@@ -50,8 +51,30 @@ def needs_build(out: str = LIB) -> bool:
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
+# Test-only builds of the same sources, each to its own file (never the
+# product library): name -> preprocessor definitions.
+VARIANTS = {
+    # bounded waits of 1 ms and a hook that makes the score producer leave a
+    # tile out, so that a test can make a wait run out
+    "hooks": ("TRI_TEST_HOOKS", "TRI_WAIT_LIMIT_NS=1000000ull"),
+    # device-side invariant checks of the selection and compaction
+    "checked": ("TRI_CHECKED",),
+}
+
+
+def variant_path(name: str) -> str:
+    return os.path.join(ROOT, "_build", f"libtri_evict_{name}.so")
+
+
+def build_variant(name: str) -> str:
+    """Build (if missing or older than the sources) a test-only variant."""
+    return build(defines=VARIANTS[name], out=variant_path(name))
+
+
 def build(force: bool = False, defines=(), out: str = LIB, verbose: bool = False) -> str:
-    if not force and not defines and not needs_build(out):
+    """Compile the sources with `defines` into `out`, unless `out` is newer
+    than every source (callers give each set of definitions its own file)."""
+    if not force and not needs_build(out):
         return out
     os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
     tmp = out + f".tmp{os.getpid()}"
@@ -73,5 +96,9 @@ def build(force: bool = False, defines=(), out: str = LIB, verbose: bool = False
 
 if __name__ == "__main__":
     args = sys.argv[1:]
+    if "--variants" in args:
+        for name in VARIANTS:
+            print(build_variant(name))
+        sys.exit(0)
     defs = [args[i + 1] for i, a in enumerate(args) if a == "-D"]
     build(force="--force" in args or bool(defs), defines=defs, verbose=True)

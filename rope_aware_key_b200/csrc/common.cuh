@@ -28,12 +28,30 @@ struct Geom {
   int32_t len[TRI_MAX_BATCH];         // keys per sequence
   int32_t start[TRI_MAX_BATCH];       // RAGGED: first token of the sequence
   int32_t tile_prefix[TRI_MAX_BATCH + 1];  // score tiles before sequence b (per layer-head or layer)
+#ifdef TRI_TEST_HOOKS
+  int test_skip_tile;        // test builds only: the score producer issues nothing for this tile (-1: none)
+#endif
 };
 
 // Per-device status word; kernels OR TRI_DEVFLAG_* bits into it.
 __device__ unsigned int g_status;
 
 __device__ __forceinline__ void flag(unsigned int bits) { atomicOr(&g_status, bits); }
+
+// Invariants of the selection and compaction (kept counts, histogram
+// totals, holes against movers), checked on the device in a library built
+// with -DTRI_CHECKED; a violation sets TRI_DEVFLAG_INVARIANT and the kernel
+// carries on.  The product build compiles them out.
+#ifdef TRI_CHECKED
+#define TRI_CHECK(cond)                                   \
+  do {                                                    \
+    if (!(cond)) ::tri::flag(TRI_DEVFLAG_INVARIANT);      \
+  } while (0)
+#else
+#define TRI_CHECK(cond) \
+  do {                  \
+  } while (0)
+#endif
 
 // Element offset of row i of unit (l, h, b).  For PAGED, *ok is cleared (and
 // 0 returned) when the page id is outside the pool.
@@ -104,8 +122,12 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Wait for the phase with the given parity to complete, for at most about
-// two seconds; on timeout set TRI_DEVFLAG_TIMEOUT and return false.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// two seconds (a test build may set a shorter limit); on timeout set
+// TRI_DEVFLAG_TIMEOUT and return false.
+#ifndef TRI_WAIT_LIMIT_NS
+#define TRI_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = TRI_WAIT_LIMIT_NS;
 
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;

@@ -9,7 +9,8 @@
 // place, which attention does not notice since K and V rows move together).
 //
 //  * gather (out of place): out[u][j] = cache row kept[u][j] of unit u, for
-//    j < kept_count[u]; the output is [units][B][128] for K and for V.
+//    j < kept_count[u]; the output is [units][B][128] for K and for V.  A
+//    warp copies a chunk of 32 consecutive kept rows of one unit.
 //  * hole fill (in place): in a unit with n > B keys the kept keys below B
 //    stay, and the evicted positions below B, ascending, receive the kept keys
 //    at or above B, ascending.  Sources (>= B) and destinations (< B) are
@@ -22,16 +23,17 @@
 namespace tri {
 namespace compact {
 
-#ifndef TRI_GATHER_ROWS
-#define TRI_GATHER_ROWS 2
+#ifndef TRI_GATHER_UNROLL
+#define TRI_GATHER_UNROLL 4
 #endif
 #ifndef TRI_GATHER_BLOCKS_PER_SM
-#define TRI_GATHER_BLOCKS_PER_SM 16
+#define TRI_GATHER_BLOCKS_PER_SM 4
 #endif
 
 constexpr int kGatherThreads = 256;
-constexpr int kGatherRows = TRI_GATHER_ROWS;
+constexpr int kGatherUnroll = TRI_GATHER_UNROLL;     // rows in flight per half-warp
 constexpr int kGatherBlocksPerSm = TRI_GATHER_BLOCKS_PER_SM;
+constexpr int kChunkRows = 32;                      // kept rows of one unit per warp and step
 constexpr int kFillThreads = 256;
 constexpr int kMaxFillBudget = 16384;
 
@@ -42,50 +44,72 @@ __device__ __forceinline__ void unit_coords(const Geom& g, int u, int* l, int* h
   *h = lh - *l * g.H;
 }
 
-// Each half-warp copies kGatherRows rows per step (all loads issued before
-// the stores, so 2 x kGatherRows x 16 bytes per lane are in flight).
+// A warp takes a chunk of kChunkRows consecutive kept rows of one unit: the
+// unit, its base address and its kept indices (one coalesced load, then
+// shuffles) are found once per chunk, and each half-warp copies rows with
+// 2 x kGatherUnroll 16-byte loads in flight per lane before its stores.
 __global__ void __launch_bounds__(kGatherThreads)
 gather_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept,
               const int32_t* __restrict__ kept_count, int B, uint16_t* __restrict__ kout,
-              uint16_t* __restrict__ vout, int total_rows) {
-  // total_rows = units * B < 2^31 (checked on the host)
-  const int l16 = threadIdx.x & 15;
-  const int hw = (blockIdx.x * kGatherThreads + threadIdx.x) >> 4;
-  const int nhw = (gridDim.x * kGatherThreads) >> 4;
-  for (int base = hw; base < total_rows; base += nhw * kGatherRows) {
-    uint4 kx[kGatherRows], vx[kGatherRows];
-    bool live[kGatherRows];
-#pragma unroll
-    for (int r = 0; r < kGatherRows; ++r) {
-      const int row = base + r * nhw;
-      live[r] = false;
-      if (row >= total_rows) continue;
-      const int u = row / B;
-      const int j = row - u * B;
-      if (j >= __ldg(kept_count + u)) continue;
-      const int i = __ldg(kept + row);
-      int l, h, b;
-      unit_coords(g, u, &l, &h, &b);
-      if (static_cast<unsigned>(i) >= static_cast<unsigned>(g.len[b])) {
-        if (l16 == 0) flag(TRI_DEVFLAG_BAD_KEPT);
-        continue;
-      }
-      bool ok = true;
-      const int64_t e = row_elem(g, l, h, b, i, &ok);
-      if (!ok) {
-        if (l16 == 0) flag(TRI_DEVFLAG_BAD_PAGE);
-        continue;
-      }
-      kx[r] = ld_nc_v4(g.k + e + l16 * 8);
-      vx[r] = ld_nc_v4(g.v + e + l16 * 8);
-      live[r] = true;
+              uint16_t* __restrict__ vout, int chunks_per_unit, int total_chunks) {
+  const int lane = threadIdx.x & 31;
+  const int l16 = lane & 15, hw = lane >> 4;
+  const int warp0 = (blockIdx.x * kGatherThreads + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * kGatherThreads) >> 5;
+  const bool packed = g.layout != TRI_LAYOUT_PAGED;
+  for (int c = warp0; c < total_chunks; c += nwarps) {
+    const int u = c / chunks_per_unit;
+    const int j0 = (c - u * chunks_per_unit) * kChunkRows;
+    const int cnt = __ldg(kept_count + u);
+#ifdef TRI_CHECKED
+    if (j0 == 0 && lane == 0) {
+      int l_, h_, b_;
+      unit_coords(g, u, &l_, &h_, &b_);
+      TRI_CHECK(cnt == min(B, g.len[b_]));         // the selection kept min(B, n)
     }
+#endif
+    const int rows = min(kChunkRows, cnt - j0);     // warp-uniform
+    if (rows <= 0) continue;
+    int l, h, b;
+    unit_coords(g, u, &l, &h, &b);
+    const int n = g.len[b];
+    const int my_i = lane < rows ? __ldg(kept + static_cast<int64_t>(u) * B + j0 + lane) : 0;
+    bool ok0 = true;
+    const int64_t base = packed ? row_elem(g, l, h, b, 0, &ok0) : 0;
+    const int64_t out0 = static_cast<int64_t>(u) * B + j0;
+    for (int r0 = 0; r0 < rows; r0 += 2 * kGatherUnroll) {
+      uint4 kx[kGatherUnroll], vx[kGatherUnroll];
+      bool live[kGatherUnroll];
 #pragma unroll
-    for (int r = 0; r < kGatherRows; ++r) {
-      if (!live[r]) continue;
-      const int64_t row = base + r * nhw;
-      reinterpret_cast<uint4*>(kout + row * kD)[l16] = kx[r];
-      reinterpret_cast<uint4*>(vout + row * kD)[l16] = vx[r];
+      for (int q = 0; q < kGatherUnroll; ++q) {
+        const int r = r0 + 2 * q + hw;
+        const int i = __shfl_sync(0xffffffffu, my_i, r & (kChunkRows - 1));
+        live[q] = false;
+        if (r >= rows) continue;
+        if (static_cast<unsigned>(i) >= static_cast<unsigned>(n)) {
+          if (l16 == 0) flag(TRI_DEVFLAG_BAD_KEPT);
+          continue;
+        }
+        int64_t e = base + static_cast<int64_t>(i) * kD;
+        if (!packed) {
+          bool ok = true;
+          e = row_elem(g, l, h, b, i, &ok);
+          if (!ok) {
+            if (l16 == 0) flag(TRI_DEVFLAG_BAD_PAGE);
+            continue;
+          }
+        }
+        kx[q] = ld_nc_v4(g.k + e + l16 * 8);
+        vx[q] = ld_nc_v4(g.v + e + l16 * 8);
+        live[q] = true;
+      }
+#pragma unroll
+      for (int q = 0; q < kGatherUnroll; ++q) {
+        if (!live[q]) continue;
+        const int64_t row = out0 + r0 + 2 * q + hw;
+        reinterpret_cast<uint4*>(kout + row * kD)[l16] = kx[q];
+        reinterpret_cast<uint4*>(vout + row * kD)[l16] = vx[q];
+      }
     }
   }
 }
@@ -137,10 +161,13 @@ holefill_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept
 
   const int nh = static_cast<int>(base);
   const int first_mover = B - nh;         // kept[first_mover..B) are >= B
+  // ascending kept indices: the last one below B sits just before the movers
+  if (threadIdx.x == 0) TRI_CHECK(first_mover == 0 || ku[first_mover - 1] < B);
   const int l16 = threadIdx.x & 15;
   for (int r = threadIdx.x >> 4; r < nh; r += kFillThreads / 16) {
     const int src_i = ku[first_mover + r];
     const int dst_i = holes[r];
+    if (l16 == 0 && r > 0) TRI_CHECK(ku[first_mover + r - 1] < src_i);    // movers ascending
     if (src_i < B || src_i >= n) {
       if (l16 == 0) flag(TRI_DEVFLAG_BAD_KEPT);
       continue;

@@ -402,6 +402,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_kernel(const __grid_constan
     }
   }
   if (rank == 0 && threadIdx.x == 0) a.kept_count[u] = M;
+  // the last slice's kept keys end the unit's list at exactly M
+  if (rank == C - 1 && threadIdx.x == 0 && !misc[kAbort]) TRI_CHECK(out_off + kept_base == static_cast<uint32_t>(M));
   if (threadIdx.x == 0 && misc[kAbort]) flag(TRI_DEVFLAG_TIMEOUT);
   cluster.sync();                                       // peers are done with this CTA's shared memory
 }

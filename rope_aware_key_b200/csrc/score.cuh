@@ -7,12 +7,14 @@
 // stream of the key cache through shared memory.
 //
 // Design (persistent, TRI_SCORE_CTAS_PER_SM CTAs per SM):
-//  * a producer thread decodes each tile once -- up to 128 consecutive keys
-//    of one unit (CONTIG, RAGGED) or one page of all heads (PAGED) -- writes
-//    its metadata next to the stage and issues one 1-D bulk copy
-//    (cp.async.bulk, no multicast, L2 evict-first) into a ring of
-//    TRI_SCORE_STAGES 32 KB shared-memory stages guarded by full/empty
-//    mbarriers;
+//  * a producer warp decodes the CTA's next kPreTiles tiles at once, one
+//    lane per tile -- up to 128 consecutive keys of one unit (CONTIG,
+//    RAGGED) or consecutive pages of all heads (PAGED), whose page ids come
+//    from the block table in global memory, so the lookups of a batch
+//    overlap -- then one lane writes each tile's metadata next to its stage
+//    and issues its 1-D bulk copies (cp.async.bulk, no multicast, L2
+//    evict-first) into a ring of TRI_SCORE_STAGES 32 KB shared-memory stages
+//    guarded by full/empty mbarriers;
 //  * 8 consumer warps read a stage with 16-byte shared loads, four lanes per
 //    key (32 bf16 each).  The two keys of a quarter-warp read opposite halves
 //    of the 128-byte bank window at every load (the odd key's chunk order is
@@ -59,16 +61,29 @@ struct TileInfo {
   int64_t head_step; // PAGED: floats between the score rows of consecutive heads
 };
 
+// Tiles decoded ahead by the producer warp (one lane each), with the first
+// kPrePages page ids of a PAGED tile.
+constexpr int kPreTiles = 16;
+constexpr int kPrePages = 8;
+struct PreTile {
+  TileInfo T;
+  int64_t src;
+  int32_t blk[kPrePages];
+  int ok;
+};
+
 constexpr size_t kBarOffset = static_cast<size_t>(kStages) * kTileBytes;
 constexpr size_t kInfoOffset = kBarOffset + 2 * kStages * sizeof(uint64_t);
-constexpr size_t kSmemBytes = kInfoOffset + kStages * sizeof(TileInfo);
+constexpr size_t kPreOffset = (kInfoOffset + kStages * sizeof(TileInfo) + 15) & ~size_t{15};
+constexpr size_t kSmemBytes = kPreOffset + kPreTiles * sizeof(PreTile);
 
 // Tiles are numbered layer-major: CONTIG / RAGGED per (layer, head) then
 // sequence then 128-key chunk; PAGED per layer then sequence then group of
 // pages_per_tile consecutive pages (as many as fill 128 rows).  For PAGED,
-// *src is unused: the producer copies each page of the tile on its own.
+// *src is unused: the producer copies each page of the tile on its own, and
+// the first kPrePages page ids go to blk when it is given.
 __device__ __forceinline__ void decode(const Geom& g, int t, float* scores, TileInfo* T, int64_t* src,
-                                       bool* ok) {
+                                       bool* ok, int32_t* blk_out = nullptr) {
   const int per = g.tile_prefix[g.batch];
   const int outer = t / per;
   const int r = t - outer * per;
@@ -95,6 +110,7 @@ __device__ __forceinline__ void decode(const Geom& g, int t, float* scores, Tile
       const int blk = g.block_table[static_cast<int64_t>(b) * g.max_blocks + j * P + p];
       if (static_cast<unsigned>(blk) < static_cast<unsigned>(g.num_blocks)) T->page_ok |= 1u << p;
       else *ok = false;
+      if (blk_out && p < kPrePages) blk_out[p] = blk;
     }
     *src = 0;
   } else {
@@ -148,53 +164,87 @@ struct NoSideCopy {
   __device__ __forceinline__ void issue(const TileInfo&, int, uint64_t*, uint64_t) const {}
 };
 
-// The producer thread: decodes this CTA's tiles in order, writes each one's
-// metadata next to its stage and issues its bulk copy (plus the side copies
-// of `side`, on the same barrier).  Before returning it waits (bounded) for
-// the last copy into every stage, so that no copy is in flight into the
-// shared memory of an exiting CTA.
-// The tiles a CTA takes are t_begin, t_begin + t_step, ... < t_end.
+// The producer warp (all 32 lanes call this).  The tiles a CTA takes are
+// t_begin, t_begin + t_step, ... < t_end.  Per batch of kPreTiles of them,
+// lane j decodes the j-th (page lookups included) into shared memory; then
+// lane 0, in order, waits for each tile's stage to be free, writes the
+// tile's metadata next to the stage and issues its bulk copy (plus the side
+// copies of `side`, on the same barrier).  Before returning, lane 0 waits
+// (bounded) for the last copy into every stage, so that no copy is in flight
+// into the shared memory of an exiting CTA.
 template <class Side = NoSideCopy>
 __device__ __forceinline__ void produce(const Geom& g, float* scores, unsigned char* smem, uint64_t* full,
                                         uint64_t* empty, TileInfo* info, int t_begin, int t_end, int t_step,
                                         const Side& side = Side()) {
+  const int lane = threadIdx.x & 31;
+  PreTile* pre = reinterpret_cast<PreTile*>(smem + kPreOffset);
   const uint64_t policy = policy_evict_first();
-  int k = 0;
-  for (int t = t_begin; t < t_end; t += t_step, ++k) {
-    const int s = k % kStages, n = k / kStages;
-    if (n > 0 && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) break;
-    TileInfo T;
-    int64_t src;
-    bool ok;
-    decode(g, t, scores, &T, &src, &ok);
-    if (!ok) flag(TRI_DEVFLAG_BAD_PAGE);           // the bad pages are skipped, the others scored
-    side.annotate(T);
-    info[s] = T;
-    if (T.rows > 0) {
-      unsigned char* dst = smem + static_cast<size_t>(s) * kTileBytes;
-      if (!T.paged) {
-        const uint32_t bytes = static_cast<uint32_t>(T.rows) * kRowBytes;
-        mbar_arrive_expect_tx(&full[s], bytes + side.bytes(T));
-        bulk_g2s(dst, g.k + src, bytes, &full[s], policy);
-      } else {
-        const uint32_t page_bytes = static_cast<uint32_t>(g.block_size * g.H) * kRowBytes;
-        mbar_arrive_expect_tx(&full[s], page_bytes * __popc(T.page_ok) + side.bytes(T));
-        const int l = T.lh / g.H;
-        for (int p = 0; p < T.pages; ++p) {
-          if (!((T.page_ok >> p) & 1u)) continue;
-          const int blk = g.block_table[static_cast<int64_t>(T.b) * g.max_blocks + T.page0 + p];
-          bulk_g2s(dst + static_cast<size_t>(p) * page_bytes, g.k + l * g.sL + static_cast<int64_t>(blk) * g.sB,
-                   page_bytes, &full[s], policy);
-        }
+  int k = 0;                                     // tiles issued (lane 0's count, shared after each batch)
+  bool stop = false;
+  for (int64_t t0 = t_begin; t0 < t_end && !stop; t0 += int64_t{kPreTiles} * t_step) {
+    if (lane < kPreTiles) {
+      const int64_t t = t0 + int64_t{lane} * t_step;
+      if (t < t_end) {
+        PreTile& P = pre[lane];
+        bool ok;
+        decode(g, static_cast<int>(t), scores, &P.T, &P.src, &ok, P.blk);
+        if (!ok) flag(TRI_DEVFLAG_BAD_PAGE);       // the bad pages are skipped, the others scored
+        side.annotate(P.T);
       }
-      side.issue(T, s, &full[s], policy);
-    } else {
-      mbar_arrive(&full[s]);
     }
+    __syncwarp();
+    if (lane == 0) {
+      for (int j = 0; j < kPreTiles; ++j) {
+        const int64_t t = t0 + int64_t{j} * t_step;
+        if (t >= t_end) break;
+        const int s = k % kStages, n = k / kStages;
+#ifdef TRI_TEST_HOOKS
+        if (t == g.test_skip_tile) {               // test builds: no copy and no arrival for this tile
+          ++k;
+          continue;
+        }
+#endif
+        if (n > 0 && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) {
+          stop = true;
+          break;
+        }
+        const PreTile& P = pre[j];
+        const TileInfo T = P.T;
+        info[s] = T;
+        if (T.rows > 0) {
+          unsigned char* dst = smem + static_cast<size_t>(s) * kTileBytes;
+          if (!T.paged) {
+            const uint32_t bytes = static_cast<uint32_t>(T.rows) * kRowBytes;
+            mbar_arrive_expect_tx(&full[s], bytes + side.bytes(T));
+            bulk_g2s(dst, g.k + P.src, bytes, &full[s], policy);
+          } else {
+            const uint32_t page_bytes = static_cast<uint32_t>(g.block_size * g.H) * kRowBytes;
+            mbar_arrive_expect_tx(&full[s], page_bytes * __popc(T.page_ok) + side.bytes(T));
+            const int l = T.lh / g.H;
+            for (int p = 0; p < T.pages; ++p) {
+              if (!((T.page_ok >> p) & 1u)) continue;
+              const int blk = p < kPrePages
+                  ? P.blk[p]
+                  : g.block_table[static_cast<int64_t>(T.b) * g.max_blocks + T.page0 + p];
+              bulk_g2s(dst + static_cast<size_t>(p) * page_bytes,
+                       g.k + l * g.sL + static_cast<int64_t>(blk) * g.sB, page_bytes, &full[s], policy);
+            }
+          }
+          side.issue(T, s, &full[s], policy);
+        } else {
+          mbar_arrive(&full[s]);
+        }
+        ++k;
+      }
+    }
+    stop = __shfl_sync(0xffffffffu, stop, 0);
+    __syncwarp();                                  // the batch's slots may be rewritten
   }
-  for (int s = 0; s < kStages && s < k; ++s) {
-    const int last = (k - 1 - s) / kStages;   // issues on stage s: s, s+S, ... < k
-    mbar_wait_bounded(&full[s], last & 1);
+  if (lane == 0) {
+    for (int s = 0; s < kStages && s < k; ++s) {
+      const int last = (k - 1 - s) / kStages;      // issues on stage s: s, s+S, ... < k
+      mbar_wait_bounded(&full[s], last & 1);
+    }
   }
 }
 
@@ -222,7 +272,7 @@ score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float*
   init_ring(full, empty);
 
   if (warp == kConsumerWarps) {
-    if (lane == 0) produce(g, scores, smem, full, empty, info, blockIdx.x, ntiles, gridDim.x);
+    produce(g, scores, smem, full, empty, info, blockIdx.x, ntiles, gridDim.x);
     return;
   }
 

@@ -10,7 +10,7 @@
 // kept distance taken per key instead of one scalar per pruning event.
 //
 // The keys stream through the same shared-memory ring as the folded scorer
-// (score.cuh: one producer thread, bulk copies, full/empty barriers); the
+// (score.cuh: one producer warp, bulk copies, full/empty barriers); the
 // tile's positions and its heads' weight rows ride along on the same barrier,
 // so no consumer waits on a global load.  This kernel takes every layout;
 // score_pos_tma.cuh has a faster one for caches whose units are packed back
@@ -187,9 +187,8 @@ score_pos_kernel(const __grid_constant__ Geom g, const __grid_constant__ Rot rot
   }
   init_ring(full, empty);   // its barrier also publishes the table
   if (warp == kConsumerWarps) {
-    if (lane == 0)
-      produce(g, scores, smem, full, empty, info, blockIdx.x, ntiles, gridDim.x,
-              PosCopy{rot.pos, scores, w, smem, g.H, g.block_size * g.pages_per_tile, rot.qpos});
+    produce(g, scores, smem, full, empty, info, blockIdx.x, ntiles, gridDim.x,
+            PosCopy{rot.pos, scores, w, smem, g.H, g.block_size * g.pages_per_tile, rot.qpos});
     return;
   }
 

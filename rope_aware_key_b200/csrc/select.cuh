@@ -173,6 +173,11 @@ __device__ __forceinline__ Smem carve(uint32_t* base, int cap, int lcap) {
 // by other SMs during the same launch.
 __device__ __forceinline__ uint32_t key_at(const float* row, int i) { return order_key(__ldcg(row + i)); }
 
+// In a TRI_CHECKED build: the first `nbins` bins of hist total `want`
+// (every listed key landed in exactly one bin).  Call from the whole group.
+template <class G>
+__device__ __forceinline__ void check_hist_total(const uint32_t* hist, int nbins, uint32_t want, uint32_t* scan);
+
 // Exclusive sum of v over the group; *total gets the group's sum.
 template <class G>
 __device__ __forceinline__ uint32_t group_exclusive_sum(uint32_t v, uint32_t* sh, uint32_t* total) {
@@ -199,6 +204,18 @@ __device__ __forceinline__ uint32_t group_exclusive_sum(uint32_t v, uint32_t* sh
   *total = sh[G::NW - 1];
   G::sync();
   return before + x - v;
+}
+
+template <class G>
+__device__ __forceinline__ void check_hist_total(const uint32_t* hist, int nbins, uint32_t want, uint32_t* scan) {
+#ifdef TRI_CHECKED
+  uint32_t part = 0, total = 0;
+  for (int i = G::tid(); i < nbins; i += G::NT) part += hist[i];
+  group_exclusive_sum<G>(part, scan, &total);
+  if (G::tid() == 0) TRI_CHECK(total == want);
+#else
+  (void)hist, (void)nbins, (void)want, (void)scan;
+#endif
 }
 
 // The digit d with (count above d) < need <= (count above d) + hist[d],
@@ -332,6 +349,7 @@ __device__ __forceinline__ uint32_t exact_path(const float* row, int n, int B, i
     G::sync();
     for (int i = G::tid(); i < n; i += G::NT) atomicAdd(&S.hist[value_bin(key_at(row, i), scale, lo_s)], 1u);
     G::sync();
+    check_hist_total<G>(S.hist, kBins, static_cast<uint32_t>(n), S.scan);
     uint32_t above;
     const int bin = find_digit<G>(S.hist, kBins, need, S, &above);
     need -= above;
@@ -428,6 +446,7 @@ __device__ __forceinline__ uint32_t list_threshold(const Smem& m, int nc, uint32
   G::sync();
   for (int j = G::tid(); j < nc; j += G::NT) atomicAdd(&S.hist[value_bin(m.list_key[j], scale, lo_s)], 1u);
   G::sync();
+  check_hist_total<G>(S.hist, kBins, static_cast<uint32_t>(nc), S.scan);
   uint32_t above;
   const int bin = find_digit<G>(S.hist, kBins, *need, S, &above);
   *need -= above;
@@ -662,6 +681,7 @@ __device__ __forceinline__ void select_row(const float* row, int n, int B, int l
   cnt = 0;
   for (int w = w0; w < w1; ++w) cnt += __popc(m.keepmap[w]);
   uint32_t slot = group_exclusive_sum<G>(cnt, S.scan, &total);
+  if (G::tid() == 0) TRI_CHECK(total == static_cast<uint32_t>(B));     // exactly B kept
   for (int w = w0; w < w1; ++w) {
     uint32_t bits = m.keepmap[w];
     while (bits) {

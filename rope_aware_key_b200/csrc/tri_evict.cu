@@ -19,6 +19,7 @@
 #include "fold.cuh"
 #include "score.cuh"
 #include "select.cuh"
+#include "select_warp.cuh"
 #include "compact.cuh"
 #include "score_max.cuh"
 #include "score_pos.cuh"
@@ -56,9 +57,68 @@ tri_status cuda_fail(cudaError_t e) {
     if (e_ != cudaSuccess) return cuda_fail(e_);     \
   } while (0)
 
-// Make the device that owns `ptr` current (the library's runtime keeps its
-// own notion of the current device), and set up per-device state once.
-tri_status use_device_of(const void* ptr, int* dev_out) {
+// The driver's current-context calls, looked up once through the runtime
+// (the library links the runtime statically and does not link libcuda).
+struct CtxCalls {
+  PFN_cuCtxGetCurrent_v4000 get = nullptr;
+  PFN_cuCtxSetCurrent_v4000 set = nullptr;
+};
+const CtxCalls& ctx_calls() {
+  static CtxCalls c;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      c.get = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxSetCurrent", &p, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      c.set = reinterpret_cast<PFN_cuCtxSetCurrent_v4000>(p);
+  });
+  return c;
+}
+
+// The device a call works on is made current for the length of the call
+// only: the runtime's current device belongs to the caller's host thread,
+// so the caller's own context (possibly none) is put back when the scope
+// ends.  Nothing is switched when the caller is already on that device.
+class DeviceScope {
+ public:
+  DeviceScope() = default;
+  DeviceScope(const DeviceScope&) = delete;
+  DeviceScope& operator=(const DeviceScope&) = delete;
+  ~DeviceScope() {
+    if (!switched_) return;
+    const CtxCalls& c = ctx_calls();
+    if (c.set) c.set(saved_ctx_);
+    else if (saved_dev_ >= 0) cudaSetDevice(saved_dev_);
+  }
+  // Make `dev` current (remembering what was current before).
+  cudaError_t enter(int dev) {
+    int cur = -1;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return e;
+    if (cur == dev) return cudaSuccess;
+    const CtxCalls& c = ctx_calls();
+    saved_ctx_ = nullptr;
+    if (c.get) c.get(&saved_ctx_);
+    saved_dev_ = cur;
+    e = cudaSetDevice(dev);
+    if (e == cudaSuccess) switched_ = true;
+    return e;
+  }
+
+ private:
+  bool switched_ = false;
+  CUcontext saved_ctx_ = nullptr;
+  int saved_dev_ = -1;
+};
+
+// Make the device that owns `ptr` current for the scope's lifetime, and set
+// up per-device state once.
+tri_status use_device_of(const void* ptr, int* dev_out, DeviceScope* scope) {
   int dev = -1;
   cudaPointerAttributes attr;
   cudaError_t e = cudaPointerGetAttributes(&attr, ptr);
@@ -66,9 +126,7 @@ tri_status use_device_of(const void* ptr, int* dev_out) {
   if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return TRI_ERR_INVALID_ARG;
   dev = attr.device;
   if (dev < 0 || dev >= kMaxDevices) return TRI_ERR_UNSUPPORTED;
-  int cur = -1;
-  TRI_CUDA(cudaGetDevice(&cur));
-  if (cur != dev) TRI_CUDA(cudaSetDevice(dev));
+  TRI_CUDA(scope->enter(dev));
   std::lock_guard<std::mutex> lock(g_dev_mutex);
   DeviceInfo& d = g_dev[dev];
   if (!d.ready) {
@@ -259,8 +317,16 @@ int64_t fill_tile_prefix(Geom* g) {
   return outer * acc;                                  // < 2^31 * 2^31
 }
 
+#ifdef TRI_TEST_HOOKS
+// Test builds only: the score tile whose copy the producer leaves out (-1: none).
+std::atomic<int> g_test_skip_tile{-1};
+#endif
+
 tri_status launch_score(const Geom& g0, const float* w, float* scores, int dev, cudaStream_t s) {
   Geom g = g0;
+#ifdef TRI_TEST_HOOKS
+  g.test_skip_tile = g_test_skip_tile.load();
+#endif
   const int64_t ntiles = fill_tile_prefix(&g);
   if (ntiles == 0) return TRI_OK;
   if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
@@ -273,37 +339,85 @@ tri_status launch_score(const Geom& g0, const float* w, float* scores, int dev, 
   return TRI_OK;
 }
 
-tri_status launch_select(const Geom& g, const float* scores, int B, int32_t* kept, int32_t* kept_count,
-                         cudaStream_t s) {
-  const int units = g.L * g.H * g.batch;
+// How one selection launch is shaped, decided (and checked) on the host
+// before anything is launched: a warp per row when every row holds at most
+// kWarpMaxRow keys, else a CTA per row with its working set in shared memory.
+struct SelectPlan {
+  int warp_chunks = 0;   // > 0: the warp kernel, rows of at most 128 * warp_chunks keys
+  int cap = 0, lcap = 0;
+  size_t smem = 0;
+};
+
+// Chunk counts the warp kernel is built for (rows of 512 .. 4096 keys).
+constexpr int kWarpChunkSizes[] = {4, 8, 12, 16, 20, 24, 28, 32};
+
+tri_status plan_select(const Geom& g, int B, SelectPlan* p) {
   int max_len = 0;
   for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
-  const int cap = (max_len + 3) & ~3;
-  const int lcap = tri::select::list_capacity(B, cap);
-  const size_t smem = tri::select::smem_bytes(cap, lcap);
-  if (smem > static_cast<size_t>(tri::select::kMaxShared)) return TRI_ERR_UNSUPPORTED;
-  tri::select::Args a{scores, kept, kept_count, B, cap, lcap};
-  if (cap >= 8192) {
-    tri::select::select_kernel<512><<<units, 512, smem, s>>>(g, a);
-  } else {
-    tri::select::select_kernel<256><<<units, 256, smem, s>>>(g, a);
+  *p = SelectPlan();
+  if (max_len <= tri::select::kWarpMaxRow) {
+    for (int c : kWarpChunkSizes)
+      if (128 * c >= max_len) {
+        p->warp_chunks = c;
+        return TRI_OK;
+      }
+  }
+  p->cap = (max_len + 3) & ~3;
+  p->lcap = tri::select::list_capacity(B, p->cap);
+  p->smem = tri::select::smem_bytes(p->cap, p->lcap);
+  if (p->smem > static_cast<size_t>(tri::select::kMaxShared)) return TRI_ERR_UNSUPPORTED;
+  return TRI_OK;
+}
+
+template <int J>
+void launch_select_warp(const Geom& g, const tri::select::Args& a, int units, cudaStream_t s) {
+  const int grid = (units + tri::select::kWarpRowsPerCta - 1) / tri::select::kWarpRowsPerCta;
+  tri::select::select_warp_kernel<J><<<grid, tri::select::kWarpThreads, 0, s>>>(g, a, units);
+}
+
+tri_status launch_select(const Geom& g, const SelectPlan& p, const float* scores, int B, int32_t* kept,
+                         int32_t* kept_count, cudaStream_t s) {
+  const int units = g.L * g.H * g.batch;
+  tri::select::Args a{scores, kept, kept_count, B, p.cap, p.lcap};
+  switch (p.warp_chunks) {
+    case 0:
+      if (p.cap >= 8192) tri::select::select_kernel<512><<<units, 512, p.smem, s>>>(g, a);
+      else tri::select::select_kernel<256><<<units, 256, p.smem, s>>>(g, a);
+      break;
+    case 4: launch_select_warp<4>(g, a, units, s); break;
+    case 8: launch_select_warp<8>(g, a, units, s); break;
+    case 12: launch_select_warp<12>(g, a, units, s); break;
+    case 16: launch_select_warp<16>(g, a, units, s); break;
+    case 20: launch_select_warp<20>(g, a, units, s); break;
+    case 24: launch_select_warp<24>(g, a, units, s); break;
+    case 28: launch_select_warp<28>(g, a, units, s); break;
+    default: launch_select_warp<32>(g, a, units, s); break;
   }
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
   return TRI_OK;
 }
 
+// Host checks of a compaction launch (everything launch_compact would refuse).
+tri_status check_compact_launch(const Geom& g, int B, tri_compact_mode mode) {
+  if (mode == TRI_COMPACT_OUT_OF_PLACE && int64_t{g.L} * g.H * g.batch * B > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  return TRI_OK;
+}
+
 tri_status launch_compact(const Geom& g, const int32_t* kept, const int32_t* kept_count, int B,
                           tri_compact_mode mode, void* k_out, void* v_out, int dev, cudaStream_t s) {
   const int units = g.L * g.H * g.batch;
+  if (check_compact_launch(g, B, mode) != TRI_OK) return TRI_ERR_UNSUPPORTED;
   if (mode == TRI_COMPACT_OUT_OF_PLACE) {
-    const int64_t rows = int64_t{units} * B;
-    if (rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
-    const int64_t want = (rows * 16 + tri::compact::kGatherThreads - 1) / tri::compact::kGatherThreads;
+    const int chunks_per_unit = (B + tri::compact::kChunkRows - 1) / tri::compact::kChunkRows;
+    const int64_t chunks = int64_t{units} * chunks_per_unit;          // <= units * B <= INT32_MAX
+    constexpr int kWarps = tri::compact::kGatherThreads / 32;
+    const int64_t want = (chunks + kWarps - 1) / kWarps;
     const int64_t cap = int64_t{g_dev[dev].sms} * tri::compact::kGatherBlocksPerSm;
     const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
     tri::compact::gather_kernel<<<grid, tri::compact::kGatherThreads, 0, s>>>(
-        g, kept, kept_count, B, static_cast<uint16_t*>(k_out), static_cast<uint16_t*>(v_out), rows);
+        g, kept, kept_count, B, static_cast<uint16_t*>(k_out), static_cast<uint16_t*>(v_out), chunks_per_unit,
+        static_cast<int>(chunks));
   } else {
     const size_t smem = static_cast<size_t>((B + 31) / 32 + B) * 4;
     tri::compact::holefill_kernel<<<units, tri::compact::kFillThreads, smem, s>>>(
@@ -370,6 +484,33 @@ tri_status check_compact_args(const tri_cache_desc* desc, const int32_t* kept, c
   return TRI_OK;
 }
 
+
+// Everything the three stages of a compress call would refuse, checked on
+// the host before the first launch (so an error return has launched nothing).
+tri_status compress_checks(const Geom& g0, int B, tri_compact_mode mode, SelectPlan* plan) {
+  Geom g = g0;
+  if (fill_tile_prefix(&g) > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  tri_status st = plan_select(g0, B, plan);
+  if (st != TRI_OK) return st;
+  return check_compact_launch(g0, B, mode);
+}
+
+// The stages of tri_compress / tri_compress_noalloc once their checks have
+// passed: the single-kernel step where it applies, else score, select, compact.
+tri_status run_compress(const Geom& g, const SelectPlan& plan, const float* w, int B, tri_compact_mode mode,
+                        int32_t* kept, int32_t* kept_count, void* k_out, void* v_out, float* scores, int dev,
+                        cudaStream_t s) {
+  tri_status st;
+  if (mode == TRI_COMPACT_OUT_OF_PLACE) {
+    st = launch_fused(g, w, scores, B, kept, kept_count, k_out, v_out, dev, s);
+    if (st != TRI_ERR_UNSUPPORTED) return st;
+  }
+  st = launch_score(g, w, scores, dev, s);
+  if (st != TRI_OK) return st;
+  st = launch_select(g, plan, scores, B, kept, kept_count, s);
+  if (st != TRI_OK) return st;
+  return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, s);
+}
 
 // The averaged fold: A_f = (1/|D|) sum_delta e^{i w_f delta} * e^{i w_f delta0}
 // summed here in fp64 (in schedule order), then one launch maps the centers.
@@ -458,8 +599,9 @@ tri_status launch_fold(const tri_fold_params* p, const float* q_center, int n_ce
   if (!aligned16(q_center) || !aligned16(w_out)) return TRI_ERR_INVALID_ARG;
   if (per_offset && int64_t{n_centers} * p->n_offsets > INT32_MAX / 2) return TRI_ERR_UNSUPPORTED;
   if (int64_t{n_centers} * TRI_HEAD_DIM > INT32_MAX / 2) return TRI_ERR_UNSUPPORTED;
+  DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
-  tri_status st = use_device_of(q_center, &dev);
+  tri_status st = use_device_of(q_center, &dev, &scope);
   if (st != TRI_OK) return st;
   static std::mutex m;
   std::lock_guard<std::mutex> lock(m);
@@ -553,8 +695,9 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   if (n_offsets > tri::smax::kMaxOffsets) return TRI_ERR_UNSUPPORTED;
   const int64_t rows = packed_rows(desc);
   if (rows <= 0 || rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
-  st = use_device_of(desc->k, &dev);
+  st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
   CUtensorMap map;
   st = encode_key_map(desc, rows, &map);
@@ -602,8 +745,9 @@ tri_status tri_score_keys_at_positions(const tri_cache_desc* desc, const float* 
     rot.c_hi[f] = static_cast<uint32_t>(c >> 32);
     rot.c_lo[f] = static_cast<uint32_t>(c);
   }
+  DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
-  st = use_device_of(desc->k, &dev);
+  st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
   const int64_t ntiles = fill_tile_prefix(&g);
   if (ntiles == 0) return TRI_OK;
@@ -651,8 +795,9 @@ tri_status tri_score_keys(const tri_cache_desc* desc, const float* w, float* sco
   tri_status st = make_geom(desc, false, &g);
   if (st != TRI_OK) return st;
   if (!w || !scores || !aligned16(w) || !aligned16(scores)) return TRI_ERR_INVALID_ARG;
+  DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
-  st = use_device_of(desc->k, &dev);
+  st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
   return launch_score(g, w, scores, dev, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -663,10 +808,14 @@ tri_status tri_select_topk(const tri_cache_desc* desc, const float* scores, int 
   tri_status st = make_geom(desc, false, &g);
   if (st != TRI_OK) return st;
   if (!scores || !aligned16(scores) || !kept || !kept_count || B < 1) return TRI_ERR_INVALID_ARG;
+  DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
-  st = use_device_of(desc->k, &dev);
+  SelectPlan plan;
+  st = plan_select(g, B, &plan);
   if (st != TRI_OK) return st;
-  return launch_select(g, scores, B, kept, kept_count, reinterpret_cast<cudaStream_t>(stream));
+  st = use_device_of(desc->k, &dev, &scope);
+  if (st != TRI_OK) return st;
+  return launch_select(g, plan, scores, B, kept, kept_count, reinterpret_cast<cudaStream_t>(stream));
 }
 
 tri_status tri_compact_kv(const tri_cache_desc* desc, const int32_t* kept, const int32_t* kept_count, int B,
@@ -676,8 +825,9 @@ tri_status tri_compact_kv(const tri_cache_desc* desc, const int32_t* kept, const
   if (st != TRI_OK) return st;
   st = check_compact_args(desc, kept, kept_count, B, mode, k_out, v_out);
   if (st != TRI_OK) return st;
+  DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
-  st = use_device_of(desc->k, &dev);
+  st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
   return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -706,20 +856,15 @@ tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B, tri_c
   if (st != TRI_OK) return st;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return TRI_ERR_INVALID_ARG;
   if (workspace_bytes < need) return TRI_ERR_WORKSPACE;
+  SelectPlan plan;
+  st = compress_checks(g, B, mode, &plan);
+  if (st != TRI_OK) return st;
+  DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
-  st = use_device_of(desc->k, &dev);
+  st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  float* scores = static_cast<float*>(workspace);
-  if (mode == TRI_COMPACT_OUT_OF_PLACE) {
-    st = launch_fused(g, w, scores, B, kept, kept_count, k_out, v_out, dev, s);
-    if (st != TRI_ERR_UNSUPPORTED) return st;
-  }
-  st = launch_score(g, w, scores, dev, s);
-  if (st != TRI_OK) return st;
-  st = launch_select(g, scores, B, kept, kept_count, s);
-  if (st != TRI_OK) return st;
-  return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, s);
+  return run_compress(g, plan, w, B, mode, kept, kept_count, k_out, v_out, static_cast<float*>(workspace), dev,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int B, tri_compact_mode mode,
@@ -732,8 +877,12 @@ tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int 
   if (st != TRI_OK) return st;
   const int64_t units = int64_t{g.L} * g.H * g.batch;
   if (units * g.score_stride > int64_t{TRI_NOALLOC_MAX_SCORES}) return TRI_ERR_WORKSPACE;
+  SelectPlan plan;
+  st = compress_checks(g, B, mode, &plan);
+  if (st != TRI_OK) return st;
+  DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
-  st = use_device_of(desc->k, &dev);   // makes the cache's device current
+  st = use_device_of(desc->k, &dev, &scope);   // makes the cache's device current
   if (st != TRI_OK) return st;
   float* scores = nullptr;
   {
@@ -745,27 +894,18 @@ tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int 
     }
     scores = g_noalloc_ptr[dev];
   }
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (mode == TRI_COMPACT_OUT_OF_PLACE) {
-    st = launch_fused(g, w, scores, B, kept, kept_count, k_out, v_out, dev, s);
-    if (st != TRI_ERR_UNSUPPORTED) return st;
-  }
-  st = launch_score(g, w, scores, dev, s);
-  if (st != TRI_OK) return st;
-  st = launch_select(g, scores, B, kept, kept_count, s);
-  if (st != TRI_OK) return st;
-  return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, s);
+  return run_compress(g, plan, w, B, mode, kept, kept_count, k_out, v_out, scores, dev,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 tri_status tri_read_device_status(tri_stream_t stream, uint32_t* flags, int clear) {
   if (!flags) return TRI_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeviceScope scope;   // the caller's current device comes back when the call returns
   if (s) {
     int dev = -1;
     TRI_CUDA(cudaStreamGetDevice(s, &dev));
-    int cur = -1;
-    TRI_CUDA(cudaGetDevice(&cur));
-    if (cur != dev) TRI_CUDA(cudaSetDevice(dev));
+    TRI_CUDA(scope.enter(dev));
   }
   unsigned int v = 0;
   TRI_CUDA(cudaMemcpyFromSymbolAsync(&v, tri::g_status, sizeof(v), 0, cudaMemcpyDeviceToHost, s));
@@ -799,5 +939,12 @@ int tri_last_cuda_error(void) { return g_last_cuda_error; }
 uint64_t tri_kernel_launches(void) { return g_launches.load(); }
 
 const char* tri_version(void) { return "0.1.0"; }
+
+#ifdef TRI_TEST_HOOKS
+// Test builds only (not part of the product library or its header): make the
+// score producer leave out one tile, so that the consumers' bounded waits run
+// out and the kernel reports TRI_DEVFLAG_TIMEOUT.  -1 turns it off.
+void tri_test_skip_tile(int tile) { g_test_skip_tile.store(tile); }
+#endif
 
 }  // extern "C"

@@ -127,23 +127,31 @@ def test_contig_in_place_holefill():
     check_every_unit(cache, res, before=before, after=after)
 
 
-@pytest.mark.parametrize("B", [1, 2, 999, 1000, 1005])
-def test_budget_edges(B):
-    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=1000, budget=B)
+# Rows of at most 4096 keys are selected by one warp each, longer rows by one
+# CTA each: the selection edge cases below run at a length of each kind.
+WARP_ROW, CTA_ROW = 1000, 5000
+
+
+@pytest.mark.parametrize("n", [WARP_ROW, CTA_ROW])
+@pytest.mark.parametrize("budget", ["1", "2", "n-1", "n", "n+5"])
+def test_budget_edges(n, budget):
+    B = {"1": 1, "2": 2, "n-1": n - 1, "n": n, "n+5": n + 5}[budget]
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=n, budget=B)
     cache = gen.make_cache(wl, seed=6, device=DEV)
     res = parity.run_gpu(cache)
     check_every_unit(cache, res)
 
 
-def test_exact_ties_go_to_lower_index():
-    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=3000, budget=700)
+@pytest.mark.parametrize("n", [3000, 6000])
+def test_exact_ties_go_to_lower_index(n):
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=n, budget=700 * n // 3000)
     cache = gen.make_cache(wl, seed=7, device=DEV)
-    # 37 distinct rows repeated: every score appears ~81 times, exactly
+    # 37 distinct rows repeated: every score appears n / 37 times, exactly
     base = cache.k[0, 0, 0, :37].clone()
-    cache.k[0, 0, 0] = base.repeat(82, 1)[:3000]
+    cache.k[0, 0, 0] = base.repeat(n // 37 + 1, 1)[:n]
     res = parity.run_gpu(cache)
     check_every_unit(cache, res)
-    s = res.scores[0, :3000].cpu().numpy()
+    s = res.scores[0, :n].cpu().numpy()
     kept = res.kept[0].cpu().numpy()
     t = s[kept].min()
     eq = np.flatnonzero(s == t)
@@ -151,10 +159,11 @@ def test_exact_ties_go_to_lower_index():
     assert len(kept_eq) < len(eq) and np.array_equal(kept_eq, eq[: len(kept_eq)])
 
 
-def test_all_scores_equal():
-    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=4100, budget=333)
+@pytest.mark.parametrize("n", [4096, 4100])
+def test_all_scores_equal(n):
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=n, budget=333)
     cache = gen.make_cache(wl, seed=8, device=DEV)
-    cache.k[0, 0, 0] = cache.k[0, 0, 0, :1].expand(4100, -1)
+    cache.k[0, 0, 0] = cache.k[0, 0, 0, :1].expand(n, -1)
     res = parity.run_gpu(cache)
     check_every_unit(cache, res)
     assert np.array_equal(res.kept[0].cpu().numpy(), np.arange(333))
@@ -169,36 +178,39 @@ def test_long_rows_select_without_shared_cache():
     check_every_unit(cache, res, literal=False)
 
 
-def test_heavy_duplicates_overflow_path():
-    """Three distinct scores over 10000 keys: the threshold's bin holds more
-    keys than the candidate list, so the selection takes its fallback path."""
-    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=10000, budget=4100)
+@pytest.mark.parametrize("n,B", [(10000, 4100), (4096, 1700)])
+def test_heavy_duplicates_overflow_path(n, B):
+    """Three distinct scores: the threshold's bin holds more keys than the
+    candidate list, so the selection takes its fallback path."""
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=n, budget=B)
     cache = gen.make_cache(wl, seed=13, device=DEV)
     for h in range(2):
         base = cache.k[0, h, 0, :3].clone()
-        cache.k[0, h, 0] = base.repeat(3334, 1)[:10000]
+        cache.k[0, h, 0] = base.repeat(n // 3 + 1, 1)[:n]
     res = parity.run_gpu(cache)
     check_every_unit(cache, res)
 
 
-def test_single_finite_value_with_infinities():
+@pytest.mark.parametrize("n", [3000, 5000])
+def test_single_finite_value_with_infinities(n):
     """One finite score value plus +/-inf keys: no finite range to bin."""
-    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=3000, budget=1500)
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=n, budget=1500)
     cache = gen.make_cache(wl, seed=14, device=DEV)
     k = cache.k[0, 0, 0]
     k[:] = k[:1].clone()
     k[100, :] = float("inf")
     k[200, :] = float("-inf")
     res = parity.run_gpu(cache)
-    s = res.scores[0, :3000].cpu().numpy()
+    s = res.scores[0, :n].cpu().numpy()
     kept = res.kept[0, :1500].cpu().numpy()
     np.testing.assert_array_equal(kept, oracle.select(s, 1500))
     assert res.status == 0
 
 
-def test_nonfinite_keys_rank_lowest():
+@pytest.mark.parametrize("n", [600, 4600])
+def test_nonfinite_keys_rank_lowest(n):
     """NaN scores rank lowest; +/-inf keys give +/-inf or NaN scores."""
-    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=600, budget=590)
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=n, budget=n - 10)
     cache = gen.make_cache(wl, seed=9, device=DEV)
     k = cache.k[0, 0, 0]
     k[10] = float("nan")
@@ -206,10 +218,10 @@ def test_nonfinite_keys_rank_lowest():
     k[30, 7] = float("-inf")
     k[40] = 0.0
     res = parity.run_gpu(cache)
-    s = res.scores[0, :600].cpu().numpy()
+    s = res.scores[0, :n].cpu().numpy()
     assert np.isnan(s[10])
-    kept = res.kept[0, :590].cpu().numpy()
-    np.testing.assert_array_equal(kept, oracle.select(s, 590))
+    kept = res.kept[0, :n - 10].cpu().numpy()
+    np.testing.assert_array_equal(kept, oracle.select(s, n - 10))
     assert 10 not in set(kept.tolist())
     # finite keys: scores within tolerance of the oracle
     w64 = parity.check_fold(res, cache)
@@ -217,6 +229,37 @@ def test_nonfinite_keys_rank_lowest():
     fin = np.all(np.isfinite(k.float().cpu().numpy()), axis=1)
     ref = oracle.score_literal(keys[fin], cache.query_center[0, 0].numpy(), wl.theta, wl.offsets)
     parity.check_scores(keys[fin], s[fin], ref, w64[0])
+
+
+@pytest.mark.parametrize("n,B,nans", [(1000, 900, 200), (4000, 3990, 64), (5000, 4900, 300)])
+def test_fewer_numbers_than_budget_keeps_lowest_nans(n, B, nans):
+    """More NaN scores than n - B: the threshold is NaN itself, and the
+    lowest-index NaN keys fill the budget."""
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=1, batch=1, seq_len=n, budget=B)
+    cache = gen.make_cache(wl, seed=17, device=DEV)
+    rng = np.random.default_rng(n)
+    bad = np.sort(rng.choice(n, size=nans, replace=False))
+    cache.k[0, 0, 0, torch.as_tensor(bad, device=DEV)] = float("nan")
+    res = parity.run_gpu(cache)
+    s = res.scores[0, :n].cpu().numpy()
+    assert np.isnan(s[bad]).all()
+    kept = res.kept[0, :B].cpu().numpy()
+    np.testing.assert_array_equal(kept, oracle.select(s, B))
+    assert int(res.kept_count[0]) == B
+
+
+def test_steady_round_shape_every_unit():
+    """The shape of a paged cache re-compressed every 128 generated tokens:
+    rows of B + 128 keys (and shorter ones), 16-token pages of 4 KV heads,
+    compacted in place; every key of every unit against the oracle."""
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=4, batch=6, budget=2048,
+                    spare_blocks_per_seq=1)
+    cache = gen.make_cache(wl, seed=18, device=DEV, lens=[2176, 2176, 2048, 2175, 2049, 4096])
+    units = all_units(wl)
+    before = snapshot(cache, units)
+    res = parity.run_gpu(cache, mode=tri().COMPACT_IN_PLACE_HOLEFILL)
+    after = snapshot(cache, units)
+    check_every_unit(cache, res, literal=False, before=before, after=after)
 
 
 def test_score_row_padding():

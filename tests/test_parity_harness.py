@@ -134,3 +134,33 @@ def test_key_positions_recipe():
     again, _ = gen.key_positions(c, seed=5, stride=304, spread=3)
     assert torch.equal(pos, again)
     assert not torch.equal(pos[2], pos[5])           # units draw independently
+
+
+@pytest.mark.parametrize("layout", ["contig", "ragged", "paged"])
+def test_generator_layer_range_is_a_slice_of_the_whole(layout):
+    """A rank that holds layers l0..l1-1 of a cache draws exactly those layers
+    of the whole cache (keys, values, centers, appended tokens)."""
+    base = {"contig": gen.scaled(gen.WORKLOADS["tiny"], num_layers=5, num_kv_heads=2, batch=2, seq_len=40),
+            "ragged": gen.scaled(gen.WORKLOADS["qwen3_ragged"], num_layers=5, num_kv_heads=2, batch=3),
+            "paged": gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=5, num_kv_heads=2, batch=3,
+                                spare_blocks_per_seq=2)}[layout]
+    lens = None if layout == "contig" else [30, 17, 64]
+    whole = gen.make_cache(base, seed=3, device="cpu", lens=lens)
+    part = gen.make_cache(base, seed=3, device="cpu", lens=lens, layer_range=(2, 4))
+    assert part.wl.num_layers == 2 and part.layer0 == 2
+    assert torch.equal(part.key_center, whole.key_center[2:4])
+    assert torch.equal(part.query_center, whole.query_center[2:4])
+    for l in range(2):
+        for h in range(base.num_kv_heads):
+            for b in range(base.batch):
+                for t in ("k", "v"):
+                    a = gen.unit_rows(part, getattr(part, t), l, h, b)
+                    w = gen.unit_rows(whole, getattr(whole, t), 2 + l, h, b)
+                    assert torch.equal(a.view(torch.int16), w.view(torch.int16))
+    if layout == "paged":
+        gen.append_tokens(whole, 16, step=1)
+        gen.append_tokens(part, 16, step=1)
+        for b in range(base.batch):
+            a = gen.unit_rows(part, part.k, 1, 0, b)[-16:]
+            w = gen.unit_rows(whole, whole.k, 3, 0, b)[-16:]
+            assert torch.equal(a.view(torch.int16), w.view(torch.int16))

@@ -28,47 +28,71 @@ def _noalloc(lib):
     return fn
 
 
+def _call_noalloc(fn, tri, d, w, B, mode, kept, cnt, ko, vo):
+    P = ctypes.c_void_p
+    st = fn(d.ref, P(w.data_ptr()), B, mode, P(kept.data_ptr()), P(cnt.data_ptr()),
+            P(ko.data_ptr() if ko is not None else 0), P(vo.data_ptr() if vo is not None else 0),
+            P(torch.cuda.current_stream().cuda_stream))
+    assert st == 0, tri.TriError(st, "tri_compress_noalloc")
+
+
 def test_noalloc_matches_compress_on_two_calls():
     import rope_aware_key_b200 as tri
     lib = tri.lib()
     fn = _noalloc(lib)
     dev = torch.device("cuda:0")
-    # first call: a full 8-head layer; second call: a smaller ragged cache,
-    # which must not be affected by the scores the first call left behind
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    # in a row: a full 8-head layer (three kernels); a smaller ragged cache,
+    # which must not be affected by the scores the first call left behind; a
+    # cache of 4 units x 4096 keys, which takes the single-kernel step (one
+    # cluster per unit, scores in the shared array); and a paged cache
+    # compacted in place (three kernels, hole fill)
     cases = [
-        (gen.WORKLOADS["qwen3_layer"], None, 1),
-        (gen.scaled(gen.WORKLOADS["qwen3_ragged"], num_layers=2, num_kv_heads=4, batch=3, budget=300), [900, 4000, 77], 2),
+        (gen.WORKLOADS["qwen3_layer"], None, 1, tri.COMPACT_OUT_OF_PLACE, 3),
+        (gen.scaled(gen.WORKLOADS["qwen3_ragged"], num_layers=2, num_kv_heads=4, batch=3, budget=300),
+         [900, 4000, 77], 2, tri.COMPACT_OUT_OF_PLACE, 3),
+        (gen.scaled(gen.WORKLOADS["qwen3_layer"], num_kv_heads=4, seq_len=4096, budget=512), None, 3,
+         tri.COMPACT_OUT_OF_PLACE, 1 if 4 * 16 <= sms else 3),
+        (gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=4, batch=3, budget=2048,
+                    spare_blocks_per_seq=1), [2176, 5000, 300], 4, tri.COMPACT_IN_PLACE_HOLEFILL, 3),
     ]
-    for wl, lens, seed in cases:
+    for wl, lens, seed, mode, launches in cases:
+        in_place = mode == tri.COMPACT_IN_PLACE_HOLEFILL
         cache = gen.make_cache(wl, seed=seed, device=dev, lens=lens)
-        d = parity.make_desc(cache)
+        twin = gen.make_cache(wl, seed=seed, device=dev, lens=lens) if in_place else cache
+        d, d2 = parity.make_desc(cache), parity.make_desc(twin)
         qc = cache.query_center.reshape(-1, wl.head_dim).to(dev).contiguous()
         w = tri.fold_weights(qc, wl.theta, wl.offsets)
         B = wl.budget
         assert d.units * tri.score_row_stride(d) <= 4 * 1024 * 1024
 
         def outputs():
+            ko = vo = None
+            if not in_place:
+                ko = torch.zeros((d.units, B, wl.head_dim), dtype=torch.bfloat16, device=dev)
+                vo = torch.zeros((d.units, B, wl.head_dim), dtype=torch.bfloat16, device=dev)
             return (torch.full((d.units, B), -1, dtype=torch.int32, device=dev),
-                    torch.full((d.units,), -1, dtype=torch.int32, device=dev),
-                    torch.zeros((d.units, B, wl.head_dim), dtype=torch.bfloat16, device=dev),
-                    torch.zeros((d.units, B, wl.head_dim), dtype=torch.bfloat16, device=dev))
+                    torch.full((d.units,), -1, dtype=torch.int32, device=dev), ko, vo)
 
         kept, cnt, ko, vo = outputs()
-        tri.compress(d, w, B, tri.COMPACT_OUT_OF_PLACE, kept, cnt, ko, vo)
+        ws = torch.empty(tri.workspace_size(d, B), dtype=torch.uint8, device=dev)
+        tri.compress(d, w, B, mode, kept, cnt, ko, vo, ws)
         kept2, cnt2, ko2, vo2 = outputs()
-        st = fn(d.ref, ctypes.c_void_p(w.data_ptr()), B, tri.COMPACT_OUT_OF_PLACE,
-                ctypes.c_void_p(kept2.data_ptr()), ctypes.c_void_p(cnt2.data_ptr()),
-                ctypes.c_void_p(ko2.data_ptr()), ctypes.c_void_p(vo2.data_ptr()),
-                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
-        assert st == 0, tri.TriError(st, "tri_compress_noalloc")
+        n0 = tri.kernel_launches()
+        _call_noalloc(fn, tri, d2, w, B, mode, kept2, cnt2, ko2, vo2)
+        assert tri.kernel_launches() - n0 == launches
         assert tri.read_device_status() == 0
         torch.cuda.synchronize()
         assert torch.equal(cnt2, cnt)
         valid = torch.arange(B, device=dev)[None, :] < cnt[:, None]
         assert torch.equal(torch.where(valid, kept2, 0), torch.where(valid, kept, 0))
-        v3 = valid[:, :, None]
-        assert torch.equal(torch.where(v3, ko2.view(torch.int16), 0), torch.where(v3, ko.view(torch.int16), 0))
-        assert torch.equal(torch.where(v3, vo2.view(torch.int16), 0), torch.where(v3, vo.view(torch.int16), 0))
+        if in_place:
+            assert torch.equal(twin.k.view(torch.int16), cache.k.view(torch.int16))
+            assert torch.equal(twin.v.view(torch.int16), cache.v.view(torch.int16))
+        else:
+            v3 = valid[:, :, None]
+            assert torch.equal(torch.where(v3, ko2.view(torch.int16), 0), torch.where(v3, ko.view(torch.int16), 0))
+            assert torch.equal(torch.where(v3, vo2.view(torch.int16), 0), torch.where(v3, vo.view(torch.int16), 0))
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch():
