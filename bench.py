@@ -111,9 +111,16 @@ def score_kernel_fingerprint(variant="mean"):
     return h.hexdigest()[:16]
 
 
+def traffic_record(workload, variant="mean"):
+    """The committed ncu traffic record of a variant's scorer on a workload."""
+    if gen.WORKLOADS[workload].layout == "paged":
+        return f"score_keys_paged_{workload}_traffic.txt"
+    return SCORE_KERNELS[variant][2]
+
+
 def ncu_traffic(workload, variant="mean"):
     """Per-launch DRAM bytes of the scoring kernel from the committed ncu summary, if current."""
-    p = os.path.join(ROOT, "profiles", SCORE_KERNELS[variant][2])
+    p = os.path.join(ROOT, "profiles", traffic_record(workload, variant))
     try:
         with open(p) as f:
             d = json.load(f)

@@ -124,6 +124,10 @@ WORKLOADS: Dict[str, Workload] = {
     "qwen25_paged": Workload("qwen25_paged", 28, 4, 128, 1e6, _GEO17, 2048,
                              "paged", batch=64, len_lo=8192, len_hi=32768,
                              block_size=16, spare_blocks_per_seq=8),
+    # 1 of those 28 layers: a smaller case of the same shape (profiling)
+    "qwen25_paged_1layer": Workload("qwen25_paged_1layer", 1, 4, 128, 1e6, _GEO17, 2048,
+                                    "paged", batch=64, len_lo=8192, len_hi=32768,
+                                    block_size=16, spare_blocks_per_seq=8),
 }
 
 

@@ -256,7 +256,7 @@ tri_status tri_select_topk(const tri_cache_desc* desc, const float* scores, int 
  * same desc and B.  OUT_OF_PLACE: k_out, v_out device bf16 [units][B][128]
  * (16-byte aligned).  IN_PLACE_HOLEFILL: k_out and v_out must be NULL; the
  * cache (desc->k, desc->v) is modified, so they must point to writable
- * memory; B <= 16384.  desc->v must be non-NULL. */
+ * memory.  desc->v must be non-NULL. */
 tri_status tri_compact_kv(const tri_cache_desc* desc, const int32_t* kept,
                           const int32_t* kept_count, int B, tri_compact_mode mode,
                           void* k_out, void* v_out, tri_stream_t stream);

@@ -15,7 +15,8 @@
 //    stay, and the evicted positions below B, ascending, receive the kept keys
 //    at or above B, ascending.  Sources (>= B) and destinations (< B) are
 //    disjoint, so one pass without any ordering between rows is race-free,
-//    and only the rows that must move are touched.
+//    and only the rows that must move are touched.  A warp per unit finds
+//    every mover's hole by a search over the kept indices (no barrier).
 #pragma once
 
 #include "common.cuh"
@@ -24,18 +25,16 @@ namespace tri {
 namespace compact {
 
 #ifndef TRI_GATHER_UNROLL
-#define TRI_GATHER_UNROLL 4
+#define TRI_GATHER_UNROLL 2
 #endif
 #ifndef TRI_GATHER_BLOCKS_PER_SM
-#define TRI_GATHER_BLOCKS_PER_SM 4
+#define TRI_GATHER_BLOCKS_PER_SM 6
 #endif
 
 constexpr int kGatherThreads = 256;
 constexpr int kGatherUnroll = TRI_GATHER_UNROLL;     // rows in flight per half-warp
 constexpr int kGatherBlocksPerSm = TRI_GATHER_BLOCKS_PER_SM;
 constexpr int kChunkRows = 32;                      // kept rows of one unit per warp and step
-constexpr int kFillThreads = 256;
-constexpr int kMaxFillBudget = 16384;
 
 __device__ __forceinline__ void unit_coords(const Geom& g, int u, int* l, int* h, int* b) {
   *b = u % g.batch;
@@ -114,75 +113,74 @@ gather_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept,
   }
 }
 
-// One CTA per unit.  Dynamic shared memory: bitmap of the kept positions
-// below B (ceil(B/32) words) followed by the list of holes (B ints).
-__global__ void __launch_bounds__(kFillThreads)
-holefill_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept, int B,
-                uint16_t* k, uint16_t* v) {
-  extern __shared__ uint32_t fill_smem[];
-  __shared__ uint32_t scan_sh[kFillThreads / 32];
-  const int u = blockIdx.x;
+// Hole fill, one warp per unit (units [blockIdx.x * kFillWarps, ...)).  With
+// the kept indices ascending, let f be the first kept index >= B: the m = B - f
+// movers are kept[f .. B), and the r-th hole (the r-th position below B that
+// is not kept) is at r + #{i < f : kept[i] - i <= r} -- z_i = kept[i] - i,
+// the number of holes before kept[i], never decreases, so an upper bound
+// search over it places every mover.  Each lane places one mover per step;
+// then the movers' K and V rows are copied by half-warps (16 bytes a lane).
+constexpr int kFillWarps = 8;
+constexpr int kFillThreadsWarp = kFillWarps * 32;
+
+__global__ void __launch_bounds__(kFillThreadsWarp)
+holefill_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept, int B, uint16_t* k, uint16_t* v,
+                int units) {
+  const int lane = threadIdx.x & 31, l16 = lane & 15, hw = lane >> 4;
+  const int u = blockIdx.x * kFillWarps + (threadIdx.x >> 5);
+  if (u >= units) return;                          // whole warps
   int l, h, b;
   unit_coords(g, u, &l, &h, &b);
   const int n = g.len[b];
   if (n <= B) return;
   const int32_t* __restrict__ ku = kept + static_cast<int64_t>(u) * B;
-  const int words = (B + 31) >> 5;
-  uint32_t* bitmap = fill_smem;
-  int32_t* holes = reinterpret_cast<int32_t*>(fill_smem + words);
-
-  for (int w = threadIdx.x; w < words; w += kFillThreads) bitmap[w] = 0u;
-  __syncthreads();
-  for (int j = threadIdx.x; j < B; j += kFillThreads) {
-    const int i = ku[j];
-    if (i >= 0 && i < B) atomicOr(&bitmap[i >> 5], 1u << (i & 31));
+  // f: the first kept index >= B (every lane searches the same range)
+  int lo = 0, hi = B;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(ku + mid) >= B) hi = mid;
+    else lo = mid + 1;
   }
-  __syncthreads();
-
-  // holes in ascending order
-  uint32_t base = 0;
-  for (int w0 = 0; w0 < words; w0 += kFillThreads) {
-    const int w = w0 + threadIdx.x;
-    uint32_t m = 0u;
-    if (w < words) {
-      const uint32_t valid = (w == words - 1 && (B & 31)) ? ((1u << (B & 31)) - 1u) : 0xffffffffu;
-      m = ~bitmap[w] & valid;
-    }
-    uint32_t total;
-    uint32_t pos = base + block_exclusive_sum<kFillThreads>(__popc(m), scan_sh, &total);
-    while (m) {
-      const int bit = __ffs(m) - 1;
-      holes[pos++] = w * 32 + bit;
-      m &= m - 1u;
-    }
-    base += total;
-  }
-  __syncthreads();
-
-  const int nh = static_cast<int>(base);
-  const int first_mover = B - nh;         // kept[first_mover..B) are >= B
+  const int f = lo;
+  const int m = B - f;                             // movers = holes below B
   // ascending kept indices: the last one below B sits just before the movers
-  if (threadIdx.x == 0) TRI_CHECK(first_mover == 0 || ku[first_mover - 1] < B);
-  const int l16 = threadIdx.x & 15;
-  for (int r = threadIdx.x >> 4; r < nh; r += kFillThreads / 16) {
-    const int src_i = ku[first_mover + r];
-    const int dst_i = holes[r];
-    if (l16 == 0 && r > 0) TRI_CHECK(ku[first_mover + r - 1] < src_i);    // movers ascending
-    if (src_i < B || src_i >= n) {
-      if (l16 == 0) flag(TRI_DEVFLAG_BAD_KEPT);
-      continue;
+  if (lane == 0) TRI_CHECK(f == 0 || __ldg(ku + f - 1) < B);
+  for (int r0 = 0; r0 < m; r0 += 32) {
+    const int r = r0 + lane;
+    int src = -1, dst = -1;
+    if (r < m) {
+      src = __ldg(ku + f + r);
+      // upper bound of r in z_i = kept[i] - i, i < f
+      int a = 0, c = f;
+      while (a < c) {
+        const int mid = (a + c) >> 1;
+        if (__ldg(ku + mid) - mid <= r) a = mid + 1;
+        else c = mid;
+      }
+      dst = r + a;
+      if (src < B || src >= n || dst >= B) {       // not ascending, or out of the row
+        flag(TRI_DEVFLAG_BAD_KEPT);
+        src = -1;
+      }
+      if (r > 0) TRI_CHECK(__ldg(ku + f + r - 1) < src || src < 0);    // movers ascending
     }
-    bool ok = true;
-    const int64_t es = row_elem(g, l, h, b, src_i, &ok);
-    const int64_t ed = row_elem(g, l, h, b, dst_i, &ok);
-    if (!ok) {
-      if (l16 == 0) flag(TRI_DEVFLAG_BAD_PAGE);
-      continue;
+    const int cnt = min(32, m - r0);
+    for (int q = 0; q < cnt; q += 2) {             // half-warp hw copies pair q + hw
+      const int s_i = __shfl_sync(0xffffffffu, src, (q + hw) & 31);
+      const int d_i = __shfl_sync(0xffffffffu, dst, (q + hw) & 31);
+      if (q + hw >= cnt || s_i < 0) continue;
+      bool ok = true;
+      const int64_t es = row_elem(g, l, h, b, s_i, &ok);
+      const int64_t ed = row_elem(g, l, h, b, d_i, &ok);
+      if (!ok) {
+        if (l16 == 0) flag(TRI_DEVFLAG_BAD_PAGE);
+        continue;
+      }
+      const uint4 kx = ld_nc_v4(k + es + l16 * 8);
+      const uint4 vx = ld_nc_v4(v + es + l16 * 8);
+      reinterpret_cast<uint4*>(k + ed)[l16] = kx;
+      reinterpret_cast<uint4*>(v + ed)[l16] = vx;
     }
-    const uint4 kx = ld_nc_v4(k + es + l16 * 8);
-    const uint4 vx = ld_nc_v4(v + es + l16 * 8);
-    reinterpret_cast<uint4*>(k + ed)[l16] = kx;
-    reinterpret_cast<uint4*>(v + ed)[l16] = vx;
   }
 }
 

@@ -20,6 +20,7 @@
 #include "score.cuh"
 #include "select.cuh"
 #include "select_warp.cuh"
+#include "select_block.cuh"
 #include "compact.cuh"
 #include "score_max.cuh"
 #include "score_pos.cuh"
@@ -161,6 +162,10 @@ tri_status use_device_of(const void* ptr, int* dev_out, DeviceScope* scope) {
                                   tri::select::kMaxShared));
     TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   tri::select::kMaxShared));
+    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(sizeof(tri::select::BlkScratch))));
+    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tri::select::kWarpSmemBytes)));
     TRI_CUDA(cudaFuncSetAttribute(tri::smax::score_max_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(tri::smax::kSmemBytes)));
     TRI_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.smax_blocks_per_sm, tri::smax::score_max_kernel,
@@ -194,9 +199,6 @@ tri_status use_device_of(const void* ptr, int* dev_out, DeviceScope* scope) {
       }
       (void)cudaGetLastError();
     }
-    const int fill_smem = ((tri::compact::kMaxFillBudget + 31) / 32 + tri::compact::kMaxFillBudget) * 4;
-    TRI_CUDA(cudaFuncSetAttribute(tri::compact::holefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  fill_smem));
     d.ready = true;
   }
   *dev_out = dev;
@@ -343,25 +345,25 @@ tri_status launch_score(const Geom& g0, const float* w, float* scores, int dev, 
 // before anything is launched: a warp per row when every row holds at most
 // kWarpMaxRow keys, else a CTA per row with its working set in shared memory.
 struct SelectPlan {
-  int warp_chunks = 0;   // > 0: the warp kernel, rows of at most 128 * warp_chunks keys
+  bool warp = false;     // the warp kernel (rows of at most kWarpMaxRow keys)
+  bool block = false;    // the block kernel (longer rows)
   int cap = 0, lcap = 0;
   size_t smem = 0;
 };
-
-// Chunk counts the warp kernel is built for (rows of 512 .. 4096 keys).
-constexpr int kWarpChunkSizes[] = {4, 8, 12, 16, 20, 24, 28, 32};
 
 tri_status plan_select(const Geom& g, int B, SelectPlan* p) {
   int max_len = 0;
   for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
   *p = SelectPlan();
   if (max_len <= tri::select::kWarpMaxRow) {
-    for (int c : kWarpChunkSizes)
-      if (128 * c >= max_len) {
-        p->warp_chunks = c;
-        return TRI_OK;
-      }
+    p->warp = true;
+    p->smem = tri::select::kWarpSmemBytes;
+    return TRI_OK;
   }
+#ifndef TRI_SELECT_LIST
+  p->block = true;
+  return TRI_OK;
+#endif
   p->cap = (max_len + 3) & ~3;
   p->lcap = tri::select::list_capacity(B, p->cap);
   p->smem = tri::select::smem_bytes(p->cap, p->lcap);
@@ -369,29 +371,19 @@ tri_status plan_select(const Geom& g, int B, SelectPlan* p) {
   return TRI_OK;
 }
 
-template <int J>
-void launch_select_warp(const Geom& g, const tri::select::Args& a, int units, cudaStream_t s) {
-  const int grid = (units + tri::select::kWarpRowsPerCta - 1) / tri::select::kWarpRowsPerCta;
-  tri::select::select_warp_kernel<J><<<grid, tri::select::kWarpThreads, 0, s>>>(g, a, units);
-}
-
 tri_status launch_select(const Geom& g, const SelectPlan& p, const float* scores, int B, int32_t* kept,
                          int32_t* kept_count, cudaStream_t s) {
   const int units = g.L * g.H * g.batch;
   tri::select::Args a{scores, kept, kept_count, B, p.cap, p.lcap};
-  switch (p.warp_chunks) {
-    case 0:
-      if (p.cap >= 8192) tri::select::select_kernel<512><<<units, 512, p.smem, s>>>(g, a);
-      else tri::select::select_kernel<256><<<units, 256, p.smem, s>>>(g, a);
-      break;
-    case 4: launch_select_warp<4>(g, a, units, s); break;
-    case 8: launch_select_warp<8>(g, a, units, s); break;
-    case 12: launch_select_warp<12>(g, a, units, s); break;
-    case 16: launch_select_warp<16>(g, a, units, s); break;
-    case 20: launch_select_warp<20>(g, a, units, s); break;
-    case 24: launch_select_warp<24>(g, a, units, s); break;
-    case 28: launch_select_warp<28>(g, a, units, s); break;
-    default: launch_select_warp<32>(g, a, units, s); break;
+  if (p.warp) {
+    const int grid = (units + tri::select::kWarpRows - 1) / tri::select::kWarpRows;
+    tri::select::select_warp_kernel<<<grid, tri::select::kWarpThreads, p.smem, s>>>(g, a, units);
+  } else if (p.block) {
+    tri::select::select_block_kernel<<<units, tri::select::kBlkThreads, sizeof(tri::select::BlkScratch), s>>>(g, a);
+  } else if (p.cap >= 8192) {
+    tri::select::select_kernel<512><<<units, 512, p.smem, s>>>(g, a);
+  } else {
+    tri::select::select_kernel<256><<<units, 256, p.smem, s>>>(g, a);
   }
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
@@ -419,9 +411,9 @@ tri_status launch_compact(const Geom& g, const int32_t* kept, const int32_t* kep
         g, kept, kept_count, B, static_cast<uint16_t*>(k_out), static_cast<uint16_t*>(v_out), chunks_per_unit,
         static_cast<int>(chunks));
   } else {
-    const size_t smem = static_cast<size_t>((B + 31) / 32 + B) * 4;
-    tri::compact::holefill_kernel<<<units, tri::compact::kFillThreads, smem, s>>>(
-        g, kept, B, const_cast<uint16_t*>(g.k), const_cast<uint16_t*>(g.v));
+    const int grid = (units + tri::compact::kFillWarps - 1) / tri::compact::kFillWarps;
+    tri::compact::holefill_kernel<<<grid, tri::compact::kFillThreadsWarp, 0, s>>>(
+        g, kept, B, const_cast<uint16_t*>(g.k), const_cast<uint16_t*>(g.v), units);
   }
   ++g_launches;
   TRI_CUDA(cudaGetLastError());
@@ -476,7 +468,6 @@ tri_status check_compact_args(const tri_cache_desc* desc, const int32_t* kept, c
     if (!k_out || !v_out || !aligned16(k_out) || !aligned16(v_out)) return TRI_ERR_INVALID_ARG;
   } else if (mode == TRI_COMPACT_IN_PLACE_HOLEFILL) {
     if (k_out || v_out) return TRI_ERR_INVALID_ARG;
-    if (B > tri::compact::kMaxFillBudget) return TRI_ERR_UNSUPPORTED;
   } else {
     return TRI_ERR_INVALID_ARG;
   }

@@ -138,7 +138,6 @@ def test_select_and_compact_args(L):
     assert L.tri_select_topk(ctypes.byref(d), P(FAKE), 8, None, P(FAKE), None) == 1
     assert L.tri_compact_kv(ctypes.byref(d), P(FAKE), P(FAKE), 8, 0, None, P(FAKE), None) == 1   # no k_out
     assert L.tri_compact_kv(ctypes.byref(d), P(FAKE), P(FAKE), 8, 1, P(FAKE), None, None) == 1   # in place + out
-    assert L.tri_compact_kv(ctypes.byref(d), P(FAKE), P(FAKE), 20000, 1, None, None, None) == 2  # budget cap
     assert L.tri_compact_kv(ctypes.byref(d), P(FAKE), P(FAKE), 8, 5, P(FAKE), P(FAKE), None) == 1
     dv = contig(v=None)
     assert L.tri_compact_kv(ctypes.byref(dv), P(FAKE), P(FAKE), 8, 0, P(FAKE), P(FAKE), None) == 1

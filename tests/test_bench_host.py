@@ -53,7 +53,7 @@ def _tree(tmp_path):
 
 
 def _record(tmp_path, variant, workload, fingerprint, nbytes):
-    name = bench.SCORE_KERNELS[variant][2]
+    name = bench.traffic_record(workload, variant)
     with open(tmp_path / "profiles" / name, "w") as f:
         json.dump({"workload": workload, "kernel_sources": fingerprint, "dram_bytes_per_launch": nbytes}, f)
 

@@ -262,6 +262,36 @@ def test_steady_round_shape_every_unit():
     check_every_unit(cache, res, literal=False, before=before, after=after)
 
 
+def test_in_place_budget_above_16384():
+    """The hole fill has no budget limit of its own."""
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=20000, budget=17000)
+    cache = gen.make_cache(wl, seed=20, device=DEV)
+    units = all_units(wl)
+    before = snapshot(cache, units)
+    res = parity.run_gpu(cache, mode=tri().COMPACT_IN_PLACE_HOLEFILL)
+    after = snapshot(cache, units)
+    check_every_unit(cache, res, literal=False, before=before, after=after)
+
+
+def test_second_round_rows_crowd_at_the_threshold():
+    """After one pruning event every row holds the survivors, which all sit
+    just above the old threshold; 128 new tokens later the new threshold lies
+    among them, in a crowded value range (the warp selection bins that range
+    again).  Two events on a paged cache, every unit against the oracle."""
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=4, batch=3, budget=2048,
+                    spare_blocks_per_seq=8)
+    cache = gen.make_cache(wl, seed=19, device=DEV, lens=[20000, 32768, 9000])
+    t = tri()
+    parity.run_gpu(cache, mode=t.COMPACT_IN_PLACE_HOLEFILL)
+    gen.release_tail_blocks(cache, [min(wl.budget, n) for n in cache.lens])
+    gen.append_tokens(cache, 128, step=1)
+    units = all_units(wl)
+    before = snapshot(cache, units)
+    res = parity.run_gpu(cache, mode=t.COMPACT_IN_PLACE_HOLEFILL)
+    after = snapshot(cache, units)
+    check_every_unit(cache, res, literal=False, before=before, after=after)
+
+
 def test_score_row_padding():
     wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=513, budget=64)
     cache = gen.make_cache(wl, seed=11, device=DEV)
