@@ -686,6 +686,9 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   if (n_offsets > tri::smax::kMaxOffsets) return TRI_ERR_UNSUPPORTED;
   const int64_t rows = packed_rows(desc);
   if (rows <= 0 || rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  const int64_t ntiles = fill_tile_prefix(&g);
+  if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  if (ntiles == 0) return TRI_OK;
   DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
   st = use_device_of(desc->k, &dev, &scope);
@@ -693,9 +696,6 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   CUtensorMap map;
   st = encode_key_map(desc, rows, &map);
   if (st != TRI_OK) return st;
-  const int64_t ntiles = fill_tile_prefix(&g);
-  if (ntiles == 0) return TRI_OK;
-  if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
   tri::smax::Args a{w, scores, static_cast<int>(ntiles), n_offsets, (n_offsets + 15) & ~15};
   const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].smax_blocks_per_sm;
   const int grid = static_cast<int>(ntiles < resident ? ntiles : resident);
@@ -736,13 +736,13 @@ tri_status tri_score_keys_at_positions(const tri_cache_desc* desc, const float* 
     rot.c_hi[f] = static_cast<uint32_t>(c >> 32);
     rot.c_lo[f] = static_cast<uint32_t>(c);
   }
+  const int64_t ntiles = fill_tile_prefix(&g);
+  if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  if (ntiles == 0) return TRI_OK;
   DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
   st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
-  const int64_t ntiles = fill_tile_prefix(&g);
-  if (ntiles == 0) return TRI_OK;
-  if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // units packed back to back: one lane per key over 2-D swizzled tiles
   const int64_t rows = desc->layout == TRI_LAYOUT_PAGED ? 0 : packed_rows(desc);
@@ -786,6 +786,10 @@ tri_status tri_score_keys(const tri_cache_desc* desc, const float* w, float* sco
   tri_status st = make_geom(desc, false, &g);
   if (st != TRI_OK) return st;
   if (!w || !scores || !aligned16(w) || !aligned16(scores)) return TRI_ERR_INVALID_ARG;
+  {
+    Geom gt = g;
+    if (fill_tile_prefix(&gt) > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  }
   DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
   st = use_device_of(desc->k, &dev, &scope);

@@ -157,23 +157,21 @@ def test_compress_workspace_checked_on_host(L):
 
 
 def test_compress_refuses_before_any_launch(L):
-    """A row too long for the selection's shared memory (2^20 keys at B = 2048)
-    is refused by both compress calls before the scorer runs: the status is
+    """More score tiles than an int32 counts (65536 heads x 2^24 keys) is
+    refused by both compress calls before the scorer runs: the status is
     TRI_ERR_UNSUPPORTED and no kernel was launched (no CUDA call is made
     either, which is why this runs without a GPU)."""
-    n = 1 << 20
-    d = contig(num_layers=1, num_kv_heads=1, seq_len=n, stride_layer=n * 128, stride_head=n * 128,
+    n, H = 1 << 24, 1 << 16
+    d = contig(num_layers=1, num_kv_heads=H, seq_len=n, stride_layer=H * n * 128, stride_head=n * 128,
                stride_seq=n * 128)
     P = ctypes.c_void_p
     need = ctypes.c_size_t(0)
     assert L.tri_workspace_size(ctypes.byref(d), 2048, ctypes.byref(need)) == 0
     n0 = L.tri_kernel_launches()
-    assert L.tri_select_topk(ctypes.byref(d), P(FAKE), 2048, P(FAKE), P(FAKE), None) == 2
+    assert L.tri_score_keys(ctypes.byref(d), P(FAKE), P(FAKE), None) == 2
     for mode, ko in ((0, FAKE), (1, None)):
         st = L.tri_compress(ctypes.byref(d), P(FAKE), 2048, mode, P(FAKE), P(FAKE), P(ko), P(ko), P(FAKE),
                             need.value, None)
-        assert st == 2
-        st = L.tri_compress_noalloc(ctypes.byref(d), P(FAKE), 2048, mode, P(FAKE), P(FAKE), P(ko), P(ko), None)
         assert st == 2
     assert L.tri_kernel_launches() == n0
 
