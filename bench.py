@@ -521,26 +521,52 @@ def run_paged(args, tri, dev, rank, ws):
     stream = torch.cuda.current_stream(dev)
     col = torch.arange(B, device=dev)[None, :]
 
-    def event(d, scores, evs=None):
+    side = torch.cuda.Stream(device=dev)
+
+    def event(d, scores, evs=None, pipeline=1):
+        """One pruning event: the fold, then the score, select and in-place
+        hole fill of every unit.  pipeline > 1: the layers in that many chunks
+        (whole layers each: every unit is independent); each chunk is scored
+        on `stream`, then selected and compacted on `side`, while the next
+        chunk is scored.  evs: fold, scoring, selection (+ hole fill) ends."""
         def rec(i):
             if evs is not None:
                 evs[i].record(stream)
         rec(0)
         tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
         rec(1)
-        tri.score_keys(d, w, scores, stream=stream)
+        if pipeline <= 1:
+            tri.score_keys(d, w, scores, stream=stream)
+            rec(2)
+            tri.select_topk(d, scores, B, kept, cnt, stream=stream)
+            rec(3)
+            tri.compact_kv(d, kept, cnt, B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None, stream=stream)
+            rec(4)
+            return
+        from rope_aware_key_b200.shard import shard_layers
+        for c in range(pipeline):
+            sh = shard_layers(d, c, pipeline)
+            if sh.desc is None:
+                continue
+            (u0, u1), (r0, r1) = sh.units, sh.weight_rows
+            tri.score_keys(sh.desc, w[r0:r1], scores[u0:u1], stream=stream)
+            scored = torch.cuda.Event()
+            scored.record(stream)
+            side.wait_event(scored)
+            tri.select_topk(sh.desc, scores[u0:u1], B, kept[u0:u1], cnt[u0:u1], stream=side)
+            tri.compact_kv(sh.desc, kept[u0:u1], cnt[u0:u1], B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None,
+                           stream=side)
         rec(2)
-        tri.select_topk(d, scores, B, kept, cnt, stream=stream)
+        stream.wait_stream(side)
         rec(3)
-        tri.compact_kv(d, kept, cnt, B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None, stream=stream)
         rec(4)
 
-    def timed_event(d, scores):
+    def timed_event(d, scores, pipeline=1):
         flush_buf.fill_(1)
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
         torch.cuda.synchronize()
         torch.cuda._sleep(int(2e6))
-        event(d, scores, evs)
+        event(d, scores, evs, pipeline)
         torch.cuda.synchronize()
         per = [evs[i].elapsed_time(evs[i + 1]) for i in range(4)]
         moved = int(((kept >= B) & (col < cnt[:, None])).sum())     # rows the hole fill moved
@@ -579,7 +605,7 @@ def run_paged(args, tri, dev, rank, ws):
                 torch.distributed.barrier()
             t0 = time.time()
             launches0 = tri.kernel_launches()
-        per, moved = timed_event(d, scores)
+        per, moved = timed_event(d, scores, args.pipeline)
         if i >= args.warmup:
             rounds.append((per, moved, sum(cache.lens) * L * H))
         gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
@@ -588,11 +614,16 @@ def run_paged(args, tri, dev, rank, ws):
     sampler.stop()
     clocks = sampler.summary(t0, t1)
     clocks["window"] = "the steady rounds, appends between them included"
+    # one more round, unpipelined, for the per-kernel times
+    gen.append_tokens(cache, PAGED_APPEND, step=1 + args.warmup + args.steps)
+    d = tri.desc_paged(cache.k, cache.v, cache.block_table, cache.lens)
+    per1, _ = timed_event(d, scores, 1)
+    gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
     st = tri.read_device_status()
     if st:
         raise RuntimeError(f"device status {st:#x} after the steady rounds")
 
-    per = np.array([r[0] for r in rounds])                       # ms: fold, score, select, hole fill
+    per = np.array([r[0] for r in rounds])       # ms: fold, score, select, hole fill (pipelined: fold, scoring, tail, 0)
     ms_rounds = float(per.sum())
     ms_max = max_over_ranks(ms_rounds, ws, dev)
     keys_round = rounds[0][2]
@@ -608,7 +639,8 @@ def run_paged(args, tri, dev, rank, ws):
     init_ms = float(sum(per0))
     init_bytes = keys0 * KEY_BYTES + moved0 * MOVE_BYTES
 
-    e2e = run_paged_e2e(args, tri, cache, wl, qc, w, kept, cnt, stream, ws)
+    e2e = run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws,
+                        lambda dd, ss: event(dd, ss, None, args.pipeline))
 
     result = None
     if rank == 0:
@@ -625,8 +657,14 @@ def run_paged(args, tri, dev, rank, ws):
                                    f"{B + PAGED_APPEND} keys re-compressed to {B} in place",
                        "keys_per_gpu": keys_round, "budget": B, "parallelism": f"independent caches x{ws}",
                        "l2": "L2 flushed (512 MB fill) before every pruning event, outside the events"},
-            "step_breakdown_ms": {"fold": float(per[:, 0].mean()), "score": score_ms,
-                                  "select": float(per[:, 2].mean()), "holefill": float(per[:, 3].mean())},
+            "step_breakdown_ms": ({"fold": float(per[:, 0].mean()), "score": score_ms,
+                                   "select": float(per[:, 2].mean()), "holefill": float(per[:, 3].mean())}
+                                  if args.pipeline <= 1 else
+                                  {"fold": float(per[:, 0].mean()), "scoring (all chunks)": score_ms,
+                                   "tail (last chunk's select + hole fill)": float(per[:, 2].mean())}),
+            "unpipelined_round_ms": dict(zip(("fold", "score", "select", "holefill"), per1)),
+            "pipeline": (f"{args.pipeline} chunks of whole layers: chunk c+1 scored while chunk c is selected and "
+                         f"compacted on a second stream" if args.pipeline > 1 else "one stream"),
             "rows_moved_per_step": moved,
             "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_gbs,
                     "frac_of_measured": step_gbs / peak, "frac_of_8tbps_spec": step_gbs / SPEC_HBM_GBS},
@@ -652,7 +690,7 @@ def run_paged(args, tri, dev, rank, ws):
     return result
 
 
-def run_paged_e2e(args, tri, cache, wl, qc, w, kept, cnt, stream, ws):
+def run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws, do_round):
     """A steady round end to end from host memory: the round's new tokens
     (K and V of PAGED_APPEND tokens per sequence, pinned) are copied to the
     device and written into fresh pages, the block table follows, the four
@@ -700,10 +738,7 @@ def run_paged_e2e(args, tri, cache, wl, qc, w, kept, cnt, stream, ws):
         sv.copy_(hv, non_blocking=True)
         kpool[:, di] = sk                          # the new tokens into their pages
         vpool[:, di] = sv
-        tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
-        tri.score_keys(dt, w, scores, stream=stream)
-        tri.select_topk(dt, scores, B, kept, cnt, stream=stream)
-        tri.compact_kv(dt, kept, cnt, B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None, stream=stream)
+        do_round(dt, scores)                       # fold, score, select, hole fill
         hkept.copy_(kept, non_blocking=True)
         hcnt.copy_(cnt, non_blocking=True)
         end.record(stream)
@@ -944,6 +979,9 @@ def main():
     ap.add_argument("--eager", action="store_true", help="time plain launches instead of a CUDA graph of the step")
     ap.add_argument("--path", default="calls", choices=["calls", "compress"],
                     help="calls: fold, score, select, compact as four calls (default); compress: fold + tri_compress")
+    ap.add_argument("--pipeline", type=int, default=4,
+                    help="paged workload: chunks of layers whose selection and hole fill overlap the scoring of "
+                         "the next chunk (1: one stream)")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "layers"],
                     help="N > 1: replicas (default): every rank compresses its own cache (weak scaling); "
                          "layers: one cache split by whole layers over the ranks (strong scaling)")

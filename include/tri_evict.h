@@ -239,7 +239,8 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
  * B >= 1.  Needs no workspace.  Rows of at most 4096 keys (a cache
  * re-compressed every window of generated tokens holds rows of B + the
  * window) are selected by one warp each, longer rows by one CTA each; both
- * give the same result. */
+ * give the same result.  A row too long for the CTA's shared memory (more
+ * than about 655,000 keys at B = 2048) is TRI_ERR_UNSUPPORTED. */
 tri_status tri_select_topk(const tri_cache_desc* desc, const float* scores, int B,
                            int32_t* kept, int32_t* kept_count, tri_stream_t stream);
 

@@ -15,8 +15,10 @@
 //    stay, and the evicted positions below B, ascending, receive the kept keys
 //    at or above B, ascending.  Sources (>= B) and destinations (< B) are
 //    disjoint, so one pass without any ordering between rows is race-free,
-//    and only the rows that must move are touched.  A warp per unit finds
-//    every mover's hole by a search over the kept indices (no barrier).
+//    and only the rows that must move are touched.  Units that move few rows
+//    take a warp each, which finds every mover's hole by a search over the
+//    kept indices (no barrier); units that move many take a CTA each, which
+//    lists the holes with a shared bitmap.
 #pragma once
 
 #include "common.cuh"
@@ -113,18 +115,20 @@ gather_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept,
   }
 }
 
-// Hole fill, one warp per unit (units [blockIdx.x * kFillWarps, ...)).  With
+// Hole fill, one warp per unit (units [blockIdx.x * kFillWarps, ...)), for
+// units that move few rows (a row of B + a window of new tokens).  With
 // the kept indices ascending, let f be the first kept index >= B: the m = B - f
 // movers are kept[f .. B), and the r-th hole (the r-th position below B that
 // is not kept) is at r + #{i < f : kept[i] - i <= r} -- z_i = kept[i] - i,
 // the number of holes before kept[i], never decreases, so an upper bound
 // search over it places every mover.  Each lane places one mover per step;
 // then the movers' K and V rows are copied by half-warps (16 bytes a lane).
-constexpr int kFillWarps = 8;
+constexpr int kFillWarps = 4;
 constexpr int kFillThreadsWarp = kFillWarps * 32;
+constexpr int kFillWarpMovers = 512;               // rows moved per unit up to which a warp per unit is used
 
 __global__ void __launch_bounds__(kFillThreadsWarp)
-holefill_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept, int B, uint16_t* k, uint16_t* v,
+holefill_warp_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept, int B, uint16_t* k, uint16_t* v,
                 int units) {
   const int lane = threadIdx.x & 31, l16 = lane & 15, hw = lane >> 4;
   const int u = blockIdx.x * kFillWarps + (threadIdx.x >> 5);
@@ -181,6 +185,82 @@ holefill_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept
       reinterpret_cast<uint4*>(k + ed)[l16] = kx;
       reinterpret_cast<uint4*>(v + ed)[l16] = vx;
     }
+  }
+}
+
+// Hole fill, one CTA per unit, for units that move many rows (a long row
+// pruned to B for the first time): a shared bitmap of the kept positions
+// below B, the holes listed in order by a block scan, then 16 rows in flight
+// per CTA.  Dynamic shared memory: ceil(B/32) + B words.
+constexpr int kFillThreads = 256;
+constexpr int kMaxFillCta = 16384;                 // largest B the CTA form's shared memory takes
+
+__global__ void __launch_bounds__(kFillThreads)
+holefill_cta_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept, int B, uint16_t* k,
+                    uint16_t* v) {
+  extern __shared__ uint32_t fill_smem[];
+  __shared__ uint32_t scan_sh[kFillThreads / 32];
+  const int u = blockIdx.x;
+  int l, h, b;
+  unit_coords(g, u, &l, &h, &b);
+  const int n = g.len[b];
+  if (n <= B) return;
+  const int32_t* __restrict__ ku = kept + static_cast<int64_t>(u) * B;
+  const int words = (B + 31) >> 5;
+  uint32_t* bitmap = fill_smem;
+  int32_t* holes = reinterpret_cast<int32_t*>(fill_smem + words);
+
+  for (int w = threadIdx.x; w < words; w += kFillThreads) bitmap[w] = 0u;
+  __syncthreads();
+  for (int j = threadIdx.x; j < B; j += kFillThreads) {
+    const int i = ku[j];
+    if (i >= 0 && i < B) atomicOr(&bitmap[i >> 5], 1u << (i & 31));
+  }
+  __syncthreads();
+
+  // holes in ascending order
+  uint32_t base = 0;
+  for (int w0 = 0; w0 < words; w0 += kFillThreads) {
+    const int w = w0 + threadIdx.x;
+    uint32_t m = 0u;
+    if (w < words) {
+      const uint32_t valid = (w == words - 1 && (B & 31)) ? ((1u << (B & 31)) - 1u) : 0xffffffffu;
+      m = ~bitmap[w] & valid;
+    }
+    uint32_t total;
+    uint32_t pos = base + block_exclusive_sum<kFillThreads>(__popc(m), scan_sh, &total);
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      holes[pos++] = w * 32 + bit;
+      m &= m - 1u;
+    }
+    base += total;
+  }
+  __syncthreads();
+
+  const int nh = static_cast<int>(base);
+  const int first_mover = B - nh;                  // kept[first_mover..B) are >= B
+  if (threadIdx.x == 0) TRI_CHECK(first_mover == 0 || ku[first_mover - 1] < B);
+  const int l16 = threadIdx.x & 15;
+  for (int r = threadIdx.x >> 4; r < nh; r += kFillThreads / 16) {
+    const int src_i = ku[first_mover + r];
+    const int dst_i = holes[r];
+    if (src_i < B || src_i >= n) {
+      if (l16 == 0) flag(TRI_DEVFLAG_BAD_KEPT);
+      continue;
+    }
+    if (l16 == 0 && r > 0) TRI_CHECK(ku[first_mover + r - 1] < src_i);    // movers ascending
+    bool ok = true;
+    const int64_t es = row_elem(g, l, h, b, src_i, &ok);
+    const int64_t ed = row_elem(g, l, h, b, dst_i, &ok);
+    if (!ok) {
+      if (l16 == 0) flag(TRI_DEVFLAG_BAD_PAGE);
+      continue;
+    }
+    const uint4 kx = ld_nc_v4(k + es + l16 * 8);
+    const uint4 vx = ld_nc_v4(v + es + l16 * 8);
+    reinterpret_cast<uint4*>(k + ed)[l16] = kx;
+    reinterpret_cast<uint4*>(v + ed)[l16] = vx;
   }
 }
 

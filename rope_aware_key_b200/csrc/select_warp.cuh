@@ -10,26 +10,31 @@
 // (same page, "What it saves, and what it does not") holds rows only a little
 // longer than the budget (B + the window, e.g. 2048 + 128), and there are
 // thousands of them (layers x KV heads x sequences).  A CTA per row spends
-// its time in a chain of block barriers; a warp per row needs none, and a
-// few kilobytes of shared memory per warp let 32 or more rows run on an SM.
-// Lane l owns keys 128 j + 4 l + q (one 16-byte load per 128-key chunk).
-//  1. 256 evenly spaced scores of the row are binned into kWarpBins
-//     equal-width value bins over their finite range (scores outside it
-//     clamp to the end bins); a suffix scan of the bins over the lanes finds
-//     the bins that hold the sample's ranks B/n * 256 -/+ (3 sigma + 4) from
-//     the top: b_hi and b_lo.
-//  2. One pass over the row counts the scores in bins above b_hi (all kept)
-//     and gathers the scores in bins b_lo..b_hi, as order-preserving integer
-//     keys, into a candidate buffer.  Binning is monotone in the score (NaN
-//     in the lowest bin), so if the B-th largest lies among the candidates --
-//     checked: above < B <= above + candidates -- a bitwise search over them
-//     gives it exactly: T, and `need`, how many keys equal to T are kept.
-//  3. The emit walks the row in index order: per chunk, ballots give each
-//     kept key its output slot and each key equal to T its tie rank, so the
-//     `need` lowest-index ties are kept.  These comparisons are made on the
-//     floats themselves (-0 == +0; NaN, the lowest, compared apart).
-// If the check fails (a pathological order, heavy duplication, no finite
-// spread among the samples), a bitwise search over the whole row finds T.
+// its time in a chain of block barriers; a warp per row needs none, and with
+// 5 KB of shared memory per warp a CTA of 4 rows fits beside the scorer's
+// CTAs on an SM, so the selection of some layers can run while later layers
+// are scored.  Every decision is made on order-preserving integer keys of the
+// fp32 scores (NaN lowest), so the result is exact:
+//  1. 256 evenly spaced scores of the row are sorted (a bitonic network in
+//     registers, 8 per lane); their ranks B/n * 256 -/+ (3 sigma + 4) from
+//     the top give two keys U >= L that bracket the B-th largest key for any
+//     but a pathological order of the scores;
+//  2. one pass over the row counts the keys above U (all kept) and gathers
+//     the keys in [L, U] into a candidate buffer.  When L would fall below
+//     the sample (rows that evict few keys), every key up to U is a
+//     candidate and is gathered with its index, in index order;
+//  3. if the B-th largest lies among the candidates (above < B <= above +
+//     candidates), a radix search over them (8-bit digits, a shared histogram
+//     per digit) gives it exactly: T, and `need`, how many keys equal to T
+//     are kept (the lowest-index ones);
+//  4. rows that evict few keys: the evicted indices (candidates below T, and
+//     ties past the first `need`) are listed in order, and the kept index of
+//     slot j is j + #{t : ev[t] - t <= j}, written four slots per lane, the
+//     lanes' groups interleaved so that every store covers 512 consecutive
+//     bytes.  Other rows: a second pass emits the kept keys in index order
+//     (ballots per 128-key chunk).
+// If the check fails (a pathological order, heavy duplication, NaN where the
+// bracket lies), a bitwise search over the whole row finds T instead.
 #pragma once
 
 #include "common.cuh"
@@ -38,26 +43,18 @@
 namespace tri {
 namespace select {
 
-constexpr int kWarpRows = 8;                       // rows (warps) per CTA
+constexpr int kWarpRows = 4;                       // rows (warps) per CTA
 constexpr int kWarpThreads = kWarpRows * 32;
-constexpr int kWarpBins = 256;
 constexpr int kWarpSamples = 256;                  // 8 per lane
-constexpr int kWarpCand = 768;
+constexpr int kWarpCand = 512;
 constexpr int kWarpMaxRow = 4096;
 
 struct __align__(16) WarpScratch {
-  uint32_t hist[kWarpBins];
+  uint32_t hist[256];                              // the sorted samples, then the radix digits
   uint32_t cand[kWarpCand];                        // candidate keys (later: the evicted indices)
   int32_t cidx[kWarpCand];                         // their indices (rows that evict few keys)
 };
-
-// Value bin of a score: clamp(trunc(v * scale - lo_s), 0, kWarpBins - 1).
-// The multiply-add and the saturating conversion are monotone; NaN converts
-// to 0, scores below or above the binned range saturate to the end bins.
-__device__ __forceinline__ int bin_of(float v, float scale, float lo_s) {
-  const int t = __float2int_rz(fmaf(v, scale, -lo_s));
-  return min(max(t, 0), kWarpBins - 1);
-}
+constexpr size_t kWarpSmemBytes = kWarpRows * sizeof(WarpScratch);
 
 // Chunk j of a row (4 scores per lane); positions past the row read as 0.
 __device__ __forceinline__ float4 row_chunk(const float* __restrict__ row, int n, int full, int j, int lane) {
@@ -71,19 +68,102 @@ __device__ __forceinline__ float4 row_chunk(const float* __restrict__ row, int n
   return x;
 }
 
-// The largest t with #{x : x >= t} >= need, over the values each lane passes
-// through `each` (need >= 1 and at most that many values).  Bits above
-// those that all values in [lo, hi] share are fixed at once.
+// Ascending bitonic sort of 256 keys, lane l holding elements 8 l .. 8 l + 7.
+__device__ __forceinline__ void warp_sort256(uint32_t (&x)[8]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 256; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 8) {                                // the partner sits in lane ^ (j / 8), same slot
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int idx = 8 * lane + e;
+          const uint32_t y = __shfl_xor_sync(0xffffffffu, x[e], j >> 3);
+          const bool ascending = (idx & k) == 0, lower = (idx & j) == 0;
+          x[e] = lower == ascending ? min(x[e], y) : max(x[e], y);
+        }
+      } else {                                     // both elements in this lane
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (e & j) continue;
+          const bool ascending = ((8 * lane + e) & k) == 0;
+          const uint32_t a = x[e], b = x[e ^ j];
+          x[e] = ascending ? min(a, b) : max(a, b);
+          x[e ^ j] = ascending ? max(a, b) : min(a, b);
+        }
+      }
+    }
+  }
+}
+
+// The need-th largest (need >= 1) of the keys in [lo, hi] among keys[0 .. nc)
+// (at least `need` of them are >= lo, and none in [lo, hi] is missing), by
+// 8-bit digits of key - lo, most significant first: each digit's histogram
+// (hist, 256 words) picks the bin that holds the rank.  *need becomes the
+// rank of the result among the keys equal to it.
+__device__ __forceinline__ uint32_t warp_radix_kth(const uint32_t* keys, int nc, uint32_t lo, uint32_t hi,
+                                                   uint32_t* need, uint32_t* hist) {
+  const int lane = threadIdx.x & 31;
+  while (lo < hi) {
+    const int bits = 32 - __clz(hi - lo);
+    const int shift = bits > 8 ? bits - 8 : 0;
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) hist[32 * e + lane] = 0u;
+    __syncwarp();
+    for (int m = lane; m < nc; m += 32) {
+      const uint32_t k = keys[m];
+      if (k >= lo && k <= hi) atomicAdd(&hist[(k - lo) >> shift], 1u);
+    }
+    __syncwarp();
+    // lane l owns digits [8 l, 8 l + 8); counts above a lane's digits by a suffix scan
+    const uint4 h0 = reinterpret_cast<const uint4*>(hist)[2 * lane];
+    const uint4 h1 = reinterpret_cast<const uint4*>(hist)[2 * lane + 1];
+    const uint32_t h[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+    uint32_t mine = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mine += h[e];
+    uint32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += y;
+    }
+    const uint32_t above_lane = incl - mine;
+    int d = -1;
+    uint32_t above = 0;
+    if (above_lane < *need && incl >= *need) {
+      uint32_t acc = above_lane;
+#pragma unroll
+      for (int e = 7; e >= 0; --e) {
+        if (d < 0 && acc + h[e] >= *need) {
+          d = 8 * lane + e;
+          above = acc;
+        }
+        if (d < 0) acc += h[e];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, d >= 0)) - 1;
+    d = __shfl_sync(0xffffffffu, d, src);
+    *need -= __shfl_sync(0xffffffffu, above, src);
+    lo += static_cast<uint32_t>(d) << shift;
+    const uint64_t top = static_cast<uint64_t>(lo) + ((uint64_t{1} << shift) - 1u);   // no wrap near 2^32
+    hi = top < hi ? static_cast<uint32_t>(top) : hi;
+  }
+  return lo;
+}
+
+// The largest t with #{x : x >= t} >= need over the keys each lane passes
+// through `each` (the whole-row fallback).
 template <typename Each>
-__device__ __forceinline__ uint32_t warp_kth_largest(Each each, uint32_t lo, uint32_t hi, uint32_t need) {
-  const int fixed = lo == hi ? 32 : __clz(lo ^ hi);
-  uint32_t prefix = fixed == 32 ? hi : (fixed ? (hi & (0xffffffffu << (32 - fixed))) : 0u);
-  for (int bit = 31 - fixed; bit >= 0; --bit) {
+__device__ __forceinline__ uint32_t warp_bitwise_kth(Each each, uint32_t need) {
+  uint32_t prefix = 0u;
+  for (int bit = 31; bit >= 0; --bit) {
     const uint32_t t = prefix | (1u << bit);
     uint32_t c = 0;
     each([&](uint32_t x) { c += x >= t; });
-    c = __reduce_add_sync(0xffffffffu, c);
-    if (c >= need) prefix = t;
+    if (__reduce_add_sync(0xffffffffu, c) >= need) prefix = t;
   }
   return prefix;
 }
@@ -97,241 +177,124 @@ __device__ __forceinline__ void warp_select_row(const float* __restrict__ row, i
   const uint32_t lt = (1u << lane) - 1u;
   auto valid = [&](int j, int q) { return j < full || 128 * j + 4 * lane + q < n; };
 
-  // 1. samples: positions (p n) / 256, p = lane + 32 e
-  float sv[kWarpSamples / 32];
-  float mn = INFINITY, mx = -INFINITY;
+  // 1. the bracket from the sorted sample
+  uint32_t x[8];
 #pragma unroll
-  for (int e = 0; e < kWarpSamples / 32; ++e) {
-    sv[e] = __ldg(row + (((lane + 32 * e) * n) >> 8));
-    const float f = fabsf(sv[e]) <= 3.402823466e38f ? sv[e] : NAN;    // finite only
-    mn = fminf(mn, f);
-    mx = fmaxf(mx, f);
-  }
-  const uint32_t kmin = __reduce_min_sync(0xffffffffu, order_key(mn));
-  const uint32_t kmax = __reduce_max_sync(0xffffffffu, order_key(mx));
-  float scale = 0.f, lo_s = 0.f;
-  bool ok = false;
-  if (kmin < kmax) {
-    const float lo = key_value(kmin);
-    const float width = key_value(kmax) - lo;
-    scale = static_cast<float>(kWarpBins) / width;
-    lo_s = lo * scale;
-    ok = width > 0.f && isfinite(width) && isfinite(scale) && scale > 0.f && isfinite(lo_s);
-  }
-  uint32_t need = static_cast<uint32_t>(B);
-  uint32_t T = 0u;
-  if (ok) {
-    for (int b = lane; b < kWarpBins; b += 32) S.hist[b] = 0u;
-    __syncwarp();
-#pragma unroll
-    for (int e = 0; e < kWarpSamples / 32; ++e) atomicAdd(&S.hist[bin_of(sv[e], scale, lo_s)], 1u);
-    __syncwarp();
-    // lane l owns bins [8 l, 8 l + 8); sample counts above them by a suffix scan
-    constexpr int kPer = kWarpBins / 32;
-    static_assert(kPer == 8, "two 16-byte reads per lane");
-    uint32_t h[kPer], mine = 0;
-    const uint4 h0 = reinterpret_cast<const uint4*>(S.hist)[2 * lane];
-    const uint4 h1 = reinterpret_cast<const uint4*>(S.hist)[2 * lane + 1];
-    h[0] = h0.x; h[1] = h0.y; h[2] = h0.z; h[3] = h0.w;
-    h[4] = h1.x; h[5] = h1.y; h[6] = h1.z; h[7] = h1.w;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) mine += h[e];
-    uint32_t incl = mine;                          // samples in bins of lanes >= this one
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
-      if (lane + o < 32) incl += y;
-    }
-    const uint32_t above_lane = incl - mine;
-    // the bin of the R-th largest sample (R from 1); R < 1: the top bin, R > 256: bin 0
-    auto bin_of_rank = [&](int R) {
-      if (R < 1) return kWarpBins - 1;
-      if (R > kWarpSamples) return 0;
-      int d = -1;
-      if (above_lane < static_cast<uint32_t>(R) && incl >= static_cast<uint32_t>(R)) {
-        uint32_t acc = above_lane;
-#pragma unroll
-        for (int e = kPer - 1; e >= 0; --e) {
-          if (d < 0 && acc + h[e] >= static_cast<uint32_t>(R)) d = kPer * lane + e;
-          if (d < 0) acc += h[e];
-        }
-      }
-      const uint32_t owner = __ballot_sync(0xffffffffu, d >= 0);
-      return __shfl_sync(0xffffffffu, d, __ffs(owner) - 1);
-    };
-    const float r = static_cast<float>(B) * kWarpSamples / static_cast<float>(n);
-    const float delta = 3.f * sqrtf(r * (1.f - r / kWarpSamples)) + 4.f;
-    const int b_hi = bin_of_rank(static_cast<int>(floorf(r - delta)));
-    const int b_lo = bin_of_rank(static_cast<int>(ceilf(r + delta)));
+  for (int e = 0; e < 8; ++e) x[e] = order_key(__ldg(row + (((8 * lane + e) * n) >> 8)));
+  warp_sort256(x);
+  reinterpret_cast<uint4*>(S.hist)[2 * lane] = make_uint4(x[0], x[1], x[2], x[3]);
+  reinterpret_cast<uint4*>(S.hist)[2 * lane + 1] = make_uint4(x[4], x[5], x[6], x[7]);
+  __syncwarp();
+  const float r = static_cast<float>(B) * kWarpSamples / static_cast<float>(n);
+  const float delta = 3.f * sqrtf(r * (1.f - r / kWarpSamples)) + 4.f;
+  const int r_hi = static_cast<int>(floorf(r - delta)), r_lo = static_cast<int>(ceilf(r + delta));
+  const uint32_t U = r_hi >= 1 ? S.hist[kWarpSamples - r_hi] : 0xffffffffu;
+  const bool few = r_lo > kWarpSamples;            // rows that evict few keys: no lower bound
+  const uint32_t L = few ? 0u : S.hist[kWarpSamples - r_lo];
 
-    if (b_lo == 0) {
-      // Rows that evict few keys (B close to n): every key at or below bin
-      // b_hi -- NaN included -- is a candidate, kept with its index, so the
-      // evicted keys are all among the candidates.  One pass over the row;
-      // the output is then written from the sorted list of evicted indices.
-      const float U = b_hi >= kWarpBins - 1 ? INFINITY : (static_cast<float>(b_hi + 1) + lo_s) / scale;
-      uint32_t above = 0, base = 0, cmin = 0xffffffffu, cmax = 0u;
-      for (int j = 0; j < chunks; ++j) {
-        const float4 x = row_chunk(row, n, full, j, lane);
-        const float v[4] = {x.x, x.y, x.z, x.w};
-        bool in[4];
-        uint32_t before = 0, total = 0;
+  // 2. one pass: count the keys above U, gather those in [L, U]
+  uint32_t above = 0, base = 0, cmin = 0xffffffffu, cmax = 0u;
+  for (int j = 0; j < chunks; ++j) {
+    const float4 xv = row_chunk(row, n, full, j, lane);
+    const uint32_t k[4] = {order_key(xv.x), order_key(xv.y), order_key(xv.z), order_key(xv.w)};
+    bool in[4];
+    uint32_t before = 0, total = 0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const bool vq = valid(j, q);
-          const bool up = v[q] > U;                // NaN: not above, a candidate
-          above += vq && up;
-          in[q] = vq && !up;
-          const uint32_t m = __ballot_sync(0xffffffffu, in[q]);
-          before += __popc(m & lt);
-          total += __popc(m);
-        }
-        // index order: lanes, then q within a lane
-        uint32_t pos = base + before;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (in[q]) {
-            if (pos < static_cast<uint32_t>(kWarpCand)) {
-              const uint32_t key = order_key(v[q]);
-              S.cand[pos] = key;
-              S.cidx[pos] = 128 * j + 4 * lane + q;
-              cmin = min(cmin, key);
-              cmax = max(cmax, key);
-            }
-            ++pos;
-          }
-        base += total;
-      }
-      above = __reduce_add_sync(0xffffffffu, above);
-      if (above < static_cast<uint32_t>(B) && base <= static_cast<uint32_t>(kWarpCand) &&
-          static_cast<uint32_t>(B) <= above + base) {
-        __syncwarp();
-        cmin = __reduce_min_sync(0xffffffffu, cmin);
-        cmax = __reduce_max_sync(0xffffffffu, cmax);
-        const int nc = static_cast<int>(base);
-        const uint32_t need_c = static_cast<uint32_t>(B) - above;   // 1 <= need_c <= nc
-        const uint32_t Tc = warp_kth_largest(
-            [&](auto fn) {
-              for (int m = lane; m < nc; m += 32) fn(S.cand[m]);
-            },
-            cmin, cmax, need_c);
-        uint32_t gt = 0;
-        for (int m = lane; m < nc; m += 32) gt += S.cand[m] > Tc;
-        const uint32_t need_t = need_c - __reduce_add_sync(0xffffffffu, gt);   // ties to keep
-        // the evicted indices, ascending: candidates below T, and ties past the
-        // first need_t (written over the candidate keys already read)
-        uint32_t ev = 0, ties = 0;
-        for (int m0 = 0; m0 < nc; m0 += 32) {
-          const int m = m0 + lane;
-          const uint32_t k = m < nc ? S.cand[m] : 0xffffffffu;
-          const int32_t i = m < nc ? S.cidx[m] : 0;
-          const bool tie = m < nc && k == Tc;
-          const uint32_t tm = __ballot_sync(0xffffffffu, tie);
-          const bool out = m < nc && (k < Tc || (tie && ties + __popc(tm & lt) >= need_t));
-          const uint32_t om = __ballot_sync(0xffffffffu, out);
-          __syncwarp();                            // every lane has read its entry
-          if (out) S.cand[ev + __popc(om & lt)] = static_cast<uint32_t>(i);
-          ev += __popc(om);
-          ties += __popc(tm);
-        }
-        __syncwarp();
-        const int E = static_cast<int>(ev);
-        if (lane == 0) TRI_CHECK(E == n - B);                     // exactly B kept
-        const int32_t* evi = reinterpret_cast<const int32_t*>(S.cand);
-        // kept[j] = j + #{t : ev[t] - t <= j} (ev[t] - t: the kept keys below
-        // ev[t], non-decreasing); each lane writes a contiguous run of slots
-        const int per = (((B + 31) >> 5) + 3) & ~3;
-        const int jb = min(B, lane * per), je = min(B, jb + per);
-        int a = 0, c = E;                          // first t with ev[t] - t > jb
-        while (a < c) {
-          const int mid = (a + c) >> 1;
-          if (evi[mid] - mid <= jb) a = mid + 1;
-          else c = mid;
-        }
-        int e = a;
-        const bool vec = ((reinterpret_cast<uintptr_t>(kept + jb) & 15u) == 0) && ((je - jb) & 3) == 0;
-        if (vec) {
-          for (int j = jb; j < je; j += 4) {
-            int o[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              while (e < E && evi[e] - e <= j + q) ++e;
-              o[q] = j + q + e;
-            }
-            *reinterpret_cast<int4*>(kept + j) = make_int4(o[0], o[1], o[2], o[3]);
-          }
-        } else {
-          for (int j = jb; j < je; ++j) {
-            while (e < E && evi[e] - e <= j) ++e;
-            kept[j] = j + e;
-          }
-        }
-        return;
-      }
-      ok = false;                                  // the whole-row search below
-    } else {
-      // 2. one pass: count the scores above b_hi, gather those in [b_lo, b_hi]
-      uint32_t above = 0, base = 0, cmin = 0xffffffffu, cmax = 0u;
-      for (int j = 0; j < chunks; ++j) {
-        const float4 x = row_chunk(row, n, full, j, lane);
-        const float v[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int bq = bin_of(v[q], scale, lo_s);
-          const bool vq = valid(j, q);
-          above += vq && bq > b_hi;
-          const bool in = vq && bq >= b_lo && bq <= b_hi;
-          const uint32_t m = __ballot_sync(0xffffffffu, in);
-          const uint32_t pos = base + __popc(m & lt);
-          if (in && pos < static_cast<uint32_t>(kWarpCand)) {
-            const uint32_t key = order_key(v[q]);
-            S.cand[pos] = key;
-            cmin = min(cmin, key);
-            cmax = max(cmax, key);
-          }
-          base += __popc(m);
-        }
-      }
-      above = __reduce_add_sync(0xffffffffu, above);
-      ok = above < static_cast<uint32_t>(B) && static_cast<uint32_t>(B) <= above + base &&
-           base <= static_cast<uint32_t>(kWarpCand);
-      if (ok) {
-        __syncwarp();
-        cmin = __reduce_min_sync(0xffffffffu, cmin);
-        cmax = __reduce_max_sync(0xffffffffu, cmax);
-        need -= above;                               // 1 <= need <= candidates
-        const int nc = static_cast<int>(base);
-        T = warp_kth_largest(
-            [&](auto fn) {
-              for (int m = lane; m < nc; m += 32) fn(S.cand[m]);
-            },
-            cmin, cmax, need);
-        uint32_t gt = 0;
-        for (int m = lane; m < nc; m += 32) gt += S.cand[m] > T;
-        need -= __reduce_add_sync(0xffffffffu, gt);
-      }
+    for (int q = 0; q < 4; ++q) {
+      const bool vq = valid(j, q);
+      above += vq && k[q] > U;
+      in[q] = vq && k[q] >= L && k[q] <= U;
+      const uint32_t m = __ballot_sync(0xffffffffu, in[q]);
+      before += __popc(m & lt);
+      total += __popc(m);
     }
+    uint32_t pos = base + before;                  // index order: lanes, then q within a lane
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (in[q]) {
+        if (pos < static_cast<uint32_t>(kWarpCand)) {
+          S.cand[pos] = k[q];
+          if (few) S.cidx[pos] = 128 * j + 4 * lane + q;
+          cmin = min(cmin, k[q]);
+          cmax = max(cmax, k[q]);
+        }
+        ++pos;
+      }
+    base += total;
   }
-  if (!ok) {
+  above = __reduce_add_sync(0xffffffffu, above);
+  const bool ok = above < static_cast<uint32_t>(B) && static_cast<uint32_t>(B) <= above + base &&
+                  base <= static_cast<uint32_t>(kWarpCand);
+  uint32_t T, need;
+  if (ok) {
+    __syncwarp();
+    cmin = __reduce_min_sync(0xffffffffu, cmin);
+    cmax = __reduce_max_sync(0xffffffffu, cmax);
+    need = static_cast<uint32_t>(B) - above;       // 1 <= need <= base
+    // 3. the exact threshold among the candidates; need becomes the ties to keep
+    T = warp_radix_kth(S.cand, static_cast<int>(base), cmin, cmax, &need, S.hist);
+    if (few) {
+      // 4. the evicted indices, ascending, written over the candidate keys
+      // already read: candidates below T, and ties past the first `need`
+      const int nc = static_cast<int>(base);
+      uint32_t ev = 0, ties = 0;
+      for (int m0 = 0; m0 < nc; m0 += 32) {
+        const int m = m0 + lane;
+        const uint32_t k = m < nc ? S.cand[m] : 0xffffffffu;
+        const int32_t i = m < nc ? S.cidx[m] : 0;
+        const bool tie = m < nc && k == T;
+        const uint32_t tm = __ballot_sync(0xffffffffu, tie);
+        const bool out = m < nc && (k < T || (tie && ties + __popc(tm & lt) >= need));
+        const uint32_t om = __ballot_sync(0xffffffffu, out);
+        __syncwarp();                              // every lane has read its entry
+        if (out) S.cand[ev + __popc(om & lt)] = static_cast<uint32_t>(i);
+        ev += __popc(om);
+        ties += __popc(tm);
+      }
+      __syncwarp();
+      const int E = static_cast<int>(ev);
+      if (lane == 0) TRI_CHECK(E == n - B);        // exactly B kept
+      const int32_t* evi = reinterpret_cast<const int32_t*>(S.cand);
+      // kept[j] = j + #{t : ev[t] - t <= j}: ev[t] - t, the kept keys below
+      // ev[t], never decreases, so each lane walks its slots in order
+      int e = 0;
+      if ((reinterpret_cast<uintptr_t>(kept) & 15u) == 0 && (B & 3) == 0) {
+        for (int j = 4 * lane; j < B; j += 128) {  // groups of 4 slots, lanes interleaved
+          int o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            while (e < E && evi[e] - e <= j + q) ++e;
+            o[q] = j + q + e;
+          }
+          *reinterpret_cast<int4*>(kept + j) = make_int4(o[0], o[1], o[2], o[3]);
+        }
+      } else {
+        for (int j = lane; j < B; j += 32) {
+          while (e < E && evi[e] - e <= j) ++e;
+          kept[j] = j + e;
+        }
+      }
+      return;
+    }
+  } else {
     // whole-row search: every key of the row counts (NaN keys are 0, below
     // every t >= 1 the search tests)
     auto each_key = [&](auto fn) {
       for (int j = 0; j < chunks; ++j) {
-        const float4 x = row_chunk(row, n, full, j, lane);
-        const float v[4] = {x.x, x.y, x.z, x.w};
+        const float4 xv = row_chunk(row, n, full, j, lane);
+        const float v[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           if (valid(j, q)) fn(order_key(v[q]));
       }
     };
-    need = static_cast<uint32_t>(B);
-    T = warp_kth_largest(each_key, 0u, 0xffffffffu, need);
+    T = warp_bitwise_kth(each_key, static_cast<uint32_t>(B));
     uint32_t gt = 0;
-    each_key([&](uint32_t x) { gt += x > T; });
-    need -= __reduce_add_sync(0xffffffffu, gt);
+    each_key([&](uint32_t k) { gt += k > T; });
+    need = static_cast<uint32_t>(B) - __reduce_add_sync(0xffffffffu, gt);
   }
 
-  // 3. T is the B-th largest key; keep every key above it and the `need`
+  // 4'. T is the B-th largest key; keep every key above it and the `need`
   // lowest-index keys equal to it.  Emit in index order, comparing floats:
   // above T means a greater float (every number, if T is NaN's key), equal
   // to T a float that compares equal (NaN, if T is NaN's key).
@@ -339,8 +302,8 @@ __device__ __forceinline__ void warp_select_row(const float* __restrict__ row, i
   const float tf = key_value(T);
   uint32_t slot = 0, ties = 0;
   for (int j = 0; j < chunks; ++j) {
-    const float4 x = row_chunk(row, n, full, j, lane);
-    const float v[4] = {x.x, x.y, x.z, x.w};
+    const float4 xv = row_chunk(row, n, full, j, lane);
+    const float v[4] = {xv.x, xv.y, xv.z, xv.w};
     bool keep[4], tie[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -381,8 +344,6 @@ __device__ __forceinline__ void warp_select_row(const float* __restrict__ row, i
   }
   if (lane == 0) TRI_CHECK(slot == static_cast<uint32_t>(B));         // exactly B kept
 }
-
-constexpr size_t kWarpSmemBytes = kWarpRows * sizeof(WarpScratch);
 
 // One warp per unit, units [blockIdx.x * kWarpRows, ...): rows of at most
 // kWarpMaxRow keys.  Dynamic shared memory: kWarpSmemBytes.

@@ -20,7 +20,6 @@
 #include "score.cuh"
 #include "select.cuh"
 #include "select_warp.cuh"
-#include "select_block.cuh"
 #include "compact.cuh"
 #include "score_max.cuh"
 #include "score_pos.cuh"
@@ -162,8 +161,18 @@ tri_status use_device_of(const void* ptr, int* dev_out, DeviceScope* scope) {
                                   tri::select::kMaxShared));
     TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   tri::select::kMaxShared));
-    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(sizeof(tri::select::BlkScratch))));
+    // The warp selection and the warp hole fill are small enough to run beside
+    // the scorer's CTAs (a caller may select one group of layers while the
+    // next is scored); that needs the same split of on-chip memory between L1
+    // and shared memory as the scorer, so every one of them asks for the
+    // largest shared-memory carveout.
+    for (const void* fn : {reinterpret_cast<const void*>(tri::score::score_kernel),
+                           reinterpret_cast<const void*>(tri::select::select_warp_kernel),
+                           reinterpret_cast<const void*>(tri::compact::holefill_warp_kernel)})
+      TRI_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    cudaSharedmemCarveoutMaxShared));
+    TRI_CUDA(cudaFuncSetAttribute(tri::compact::holefill_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  ((tri::compact::kMaxFillCta + 31) / 32 + tri::compact::kMaxFillCta) * 4));
     TRI_CUDA(cudaFuncSetAttribute(tri::select::select_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(tri::select::kWarpSmemBytes)));
     TRI_CUDA(cudaFuncSetAttribute(tri::smax::score_max_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -346,7 +355,6 @@ tri_status launch_score(const Geom& g0, const float* w, float* scores, int dev, 
 // kWarpMaxRow keys, else a CTA per row with its working set in shared memory.
 struct SelectPlan {
   bool warp = false;     // the warp kernel (rows of at most kWarpMaxRow keys)
-  bool block = false;    // the block kernel (longer rows)
   int cap = 0, lcap = 0;
   size_t smem = 0;
 };
@@ -360,10 +368,6 @@ tri_status plan_select(const Geom& g, int B, SelectPlan* p) {
     p->smem = tri::select::kWarpSmemBytes;
     return TRI_OK;
   }
-#ifndef TRI_SELECT_LIST
-  p->block = true;
-  return TRI_OK;
-#endif
   p->cap = (max_len + 3) & ~3;
   p->lcap = tri::select::list_capacity(B, p->cap);
   p->smem = tri::select::smem_bytes(p->cap, p->lcap);
@@ -378,8 +382,6 @@ tri_status launch_select(const Geom& g, const SelectPlan& p, const float* scores
   if (p.warp) {
     const int grid = (units + tri::select::kWarpRows - 1) / tri::select::kWarpRows;
     tri::select::select_warp_kernel<<<grid, tri::select::kWarpThreads, p.smem, s>>>(g, a, units);
-  } else if (p.block) {
-    tri::select::select_block_kernel<<<units, tri::select::kBlkThreads, sizeof(tri::select::BlkScratch), s>>>(g, a);
   } else if (p.cap >= 8192) {
     tri::select::select_kernel<512><<<units, 512, p.smem, s>>>(g, a);
   } else {
@@ -411,9 +413,18 @@ tri_status launch_compact(const Geom& g, const int32_t* kept, const int32_t* kep
         g, kept, kept_count, B, static_cast<uint16_t*>(k_out), static_cast<uint16_t*>(v_out), chunks_per_unit,
         static_cast<int>(chunks));
   } else {
-    const int grid = (units + tri::compact::kFillWarps - 1) / tri::compact::kFillWarps;
-    tri::compact::holefill_kernel<<<grid, tri::compact::kFillThreadsWarp, 0, s>>>(
-        g, kept, B, const_cast<uint16_t*>(g.k), const_cast<uint16_t*>(g.v), units);
+    // rows moved per unit: at most n - B; a warp per unit while that is small
+    int max_len = 0;
+    for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
+    if (max_len - B <= tri::compact::kFillWarpMovers || B > tri::compact::kMaxFillCta) {
+      const int grid = (units + tri::compact::kFillWarps - 1) / tri::compact::kFillWarps;
+      tri::compact::holefill_warp_kernel<<<grid, tri::compact::kFillThreadsWarp, 0, s>>>(
+          g, kept, B, const_cast<uint16_t*>(g.k), const_cast<uint16_t*>(g.v), units);
+    } else {
+      const size_t smem = static_cast<size_t>((B + 31) / 32 + B) * 4;
+      tri::compact::holefill_cta_kernel<<<units, tri::compact::kFillThreads, smem, s>>>(
+          g, kept, B, const_cast<uint16_t*>(g.k), const_cast<uint16_t*>(g.v));
+    }
   }
   ++g_launches;
   TRI_CUDA(cudaGetLastError());

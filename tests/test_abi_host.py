@@ -176,6 +176,27 @@ def test_compress_refuses_before_any_launch(L):
     assert L.tri_kernel_launches() == n0
 
 
+def test_compress_refuses_a_row_the_selection_cannot_hold(L):
+    """A row too long for the selection's shared memory (2^20 keys at
+    B = 2048) is refused by the selection and by both compress calls before
+    the scorer runs: TRI_ERR_UNSUPPORTED, and no kernel launched."""
+    n = 1 << 20
+    d = contig(num_layers=1, num_kv_heads=1, seq_len=n, stride_layer=n * 128, stride_head=n * 128,
+               stride_seq=n * 128)
+    P = ctypes.c_void_p
+    need = ctypes.c_size_t(0)
+    assert L.tri_workspace_size(ctypes.byref(d), 2048, ctypes.byref(need)) == 0
+    n0 = L.tri_kernel_launches()
+    assert L.tri_select_topk(ctypes.byref(d), P(FAKE), 2048, P(FAKE), P(FAKE), None) == 2
+    for mode, ko in ((0, FAKE), (1, None)):
+        st = L.tri_compress(ctypes.byref(d), P(FAKE), 2048, mode, P(FAKE), P(FAKE), P(ko), P(ko), P(FAKE),
+                            need.value, None)
+        assert st == 2
+        st = L.tri_compress_noalloc(ctypes.byref(d), P(FAKE), 2048, mode, P(FAKE), P(FAKE), P(ko), P(ko), None)
+        assert st == 2
+    assert L.tri_kernel_launches() == n0
+
+
 def test_compress_refuses_oversized_gather_before_any_launch(L):
     """units x B past int32 (the gather's row count) is refused on the host."""
     d = contig(num_layers=1, num_kv_heads=8, batch=256, seq_len=4, stride_layer=8 * 256 * 4 * 128,
