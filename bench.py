@@ -13,12 +13,14 @@ sequences of 8192..32768 tokens in 16-token pages) is a serving cache that is
 pruned once per window of generated tokens: one initial event (every
 sequence down to B in place), then steady rounds, each appending 128 tokens
 per sequence (untimed, as a decoder would) and re-compressing every
-2176-key row down to B in place.  A step there is one steady round (default
-8 timed rounds); the initial event is reported beside it.
+2176-key row down to B in place (the fold and one tri_compress call, whose
+selection kernel also fills each row's holes).  A step there is one steady
+round (default 8 timed rounds); the initial event is reported beside it.
 
 Prints one JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun);
-every rank compresses its own cache (independent problems, no collective on
-the data path), time = max over ranks.
+every rank compresses its own cache (--shard replicas, the default), or the
+ranks split one cache by whole layers (--shard layers); either way there is
+no collective on the data path, and time = max over ranks.
 """
 from __future__ import annotations
 
@@ -92,6 +94,7 @@ SCORE_KERNELS = {
 POS_SPREAD = 4             # pre-RoPE variant: keys keep 1 in 4 of the original positions
 PAGED_ROUNDS = 8           # timed steady rounds of the paged workload
 PAGED_APPEND = 128         # tokens a sequence generates between two pruning events
+PAGED_BREAKDOWN_ROUNDS = 3  # extra rounds that also time the scorer on its own
 
 METRICS = {
     "mean": "keys scored+selected/s (fold + score + top-B select + K/V compaction)",
@@ -440,7 +443,7 @@ def run_ours(args):
 
     # roofline of the dominant kernel (scoring; or the one-call step) and of the whole step
     peak, peak_kind = measured_hbm_peak()
-    score_ms = float(per[:, 1].mean())
+    score_ms = float(per1[:, 1].mean())
     score_bytes = keys * (KEY_BYTES + (4 if args.variant == "pos" else 0))   # + the positions read
     if args.path == "compress":
         score_bytes = keys * KEY_BYTES + moved * MOVE_BYTES
@@ -496,10 +499,11 @@ def run_ours(args):
 def run_paged(args, tri, dev, rank, ws):
     """The paged serving cache: an initial pruning event, then steady rounds
     (append PAGED_APPEND tokens per sequence, untimed; re-compress in place).
-    Each event is fold + score + select + in-place hole fill (four calls),
-    queued behind a GPU sleep so that the launches are all waiting when the
-    first one runs, and timed with CUDA events on the launching stream; L2 is
-    flushed (a 512 MB fill) before every event."""
+    The initial event is four calls (fold, score, select, in-place hole fill),
+    a steady round two (fold, tri_compress in place).  Every event is queued
+    behind a GPU sleep so that the launches are all waiting when the first one
+    runs, and timed with CUDA events on the launching stream; L2 is flushed
+    (a 512 MB fill) before every event."""
     _, _, local = dist_env()
     if args.shard != "replicas":
         raise SystemExit("the paged workload runs as replicas (one cache per rank)")
@@ -521,54 +525,55 @@ def run_paged(args, tri, dev, rank, ws):
     stream = torch.cuda.current_stream(dev)
     col = torch.arange(B, device=dev)[None, :]
 
-    side = torch.cuda.Stream(device=dev)
+    ws_buf = None                                  # tri_compress's workspace (the score matrix)
 
-    def event(d, scores, evs=None, pipeline=1):
-        """One pruning event: the fold, then the score, select and in-place
-        hole fill of every unit.  pipeline > 1: the layers in that many chunks
-        (whole layers each: every unit is independent); each chunk is scored
-        on `stream`, then selected and compacted on `side`, while the next
-        chunk is scored.  evs: fold, scoring, selection (+ hole fill) ends."""
+    def event(d, scores, evs=None):
+        """The initial pruning event, one call per stage: fold, score, select,
+        in-place hole fill.  evs: five events around the four calls."""
         def rec(i):
             if evs is not None:
                 evs[i].record(stream)
         rec(0)
         tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
         rec(1)
-        if pipeline <= 1:
-            tri.score_keys(d, w, scores, stream=stream)
-            rec(2)
-            tri.select_topk(d, scores, B, kept, cnt, stream=stream)
-            rec(3)
-            tri.compact_kv(d, kept, cnt, B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None, stream=stream)
-            rec(4)
-            return
-        from rope_aware_key_b200.shard import shard_layers
-        for c in range(pipeline):
-            sh = shard_layers(d, c, pipeline)
-            if sh.desc is None:
-                continue
-            (u0, u1), (r0, r1) = sh.units, sh.weight_rows
-            tri.score_keys(sh.desc, w[r0:r1], scores[u0:u1], stream=stream)
-            scored = torch.cuda.Event()
-            scored.record(stream)
-            side.wait_event(scored)
-            tri.select_topk(sh.desc, scores[u0:u1], B, kept[u0:u1], cnt[u0:u1], stream=side)
-            tri.compact_kv(sh.desc, kept[u0:u1], cnt[u0:u1], B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None,
-                           stream=side)
+        tri.score_keys(d, w, scores, stream=stream)
         rec(2)
-        stream.wait_stream(side)
+        tri.select_topk(d, scores, B, kept, cnt, stream=stream)
         rec(3)
+        tri.compact_kv(d, kept, cnt, B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None, stream=stream)
         rec(4)
 
-    def timed_event(d, scores, pipeline=1):
+    def steady(d, evs=None, score_alone=None):
+        """A steady round: the fold, then tri_compress in place (score, then a
+        warp per row that selects and fills the row's holes).  score_alone: a
+        score matrix; the scorer then runs once more on its own first, timed
+        (the breakdown round).  evs: events around each call."""
+        nonlocal ws_buf
+        need = tri.workspace_size(d, B)
+        if ws_buf is None or ws_buf.numel() < need:
+            ws_buf = torch.empty(need, dtype=torch.uint8, device=dev)
+        marks = iter(evs or [])
+
+        def rec():
+            if evs is not None:
+                next(marks).record(stream)
+        rec()
+        tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+        rec()
+        if score_alone is not None:
+            tri.score_keys(d, w, score_alone, stream=stream)
+            rec()
+        tri.compress(d, w, B, tri.COMPACT_IN_PLACE_HOLEFILL, kept, cnt, None, None, ws_buf, stream=stream)
+        rec()
+
+    def timed(fn, n_events):
         flush_buf.fill_(1)
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
         torch.cuda.synchronize()
         torch.cuda._sleep(int(2e6))
-        event(d, scores, evs, pipeline)
+        fn(evs)
         torch.cuda.synchronize()
-        per = [evs[i].elapsed_time(evs[i + 1]) for i in range(4)]
+        per = [evs[i].elapsed_time(evs[i + 1]) for i in range(n_events - 1)]
         moved = int(((kept >= B) & (col < cnt[:, None])).sum())     # rows the hole fill moved
         return per, moved
 
@@ -580,7 +585,7 @@ def run_paged(args, tri, dev, rank, ws):
         tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
         tri.score_keys(d0, w, scores0, stream=stream)
         tri.select_topk(d0, scores0, B, kept, cnt, stream=stream)
-    per0, moved0 = timed_event(d0, scores0)
+    per0, moved0 = timed(lambda evs: event(d0, scores0, evs), 5)
     gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
     del scores0
     torch.cuda.empty_cache()
@@ -605,7 +610,7 @@ def run_paged(args, tri, dev, rank, ws):
                 torch.distributed.barrier()
             t0 = time.time()
             launches0 = tri.kernel_launches()
-        per, moved = timed_event(d, scores, args.pipeline)
+        per, moved = timed(lambda evs: steady(d, evs), 3)
         if i >= args.warmup:
             rounds.append((per, moved, sum(cache.lens) * L * H))
         gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
@@ -614,16 +619,19 @@ def run_paged(args, tri, dev, rank, ws):
     sampler.stop()
     clocks = sampler.summary(t0, t1)
     clocks["window"] = "the steady rounds, appends between them included"
-    # one more round, unpipelined, for the per-kernel times
-    gen.append_tokens(cache, PAGED_APPEND, step=1 + args.warmup + args.steps)
-    d = tri.desc_paged(cache.k, cache.v, cache.block_table, cache.lens)
-    per1, _ = timed_event(d, scores, 1)
-    gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
+    # breakdown rounds: the scorer alone, then the same round
+    per1 = []
+    for j in range(PAGED_BREAKDOWN_ROUNDS):
+        gen.append_tokens(cache, PAGED_APPEND, step=1 + args.warmup + args.steps + j)
+        d = tri.desc_paged(cache.k, cache.v, cache.block_table, cache.lens)
+        per1.append(timed(lambda evs: steady(d, evs, score_alone=scores), 4)[0])
+        gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
+    per1 = np.array(per1)                          # ms: fold, score alone, compress
     st = tri.read_device_status()
     if st:
         raise RuntimeError(f"device status {st:#x} after the steady rounds")
 
-    per = np.array([r[0] for r in rounds])       # ms: fold, score, select, hole fill (pipelined: fold, scoring, tail, 0)
+    per = np.array([r[0] for r in rounds])       # ms: fold, compress
     ms_rounds = float(per.sum())
     ms_max = max_over_ranks(ms_rounds, ws, dev)
     keys_round = rounds[0][2]
@@ -631,7 +639,7 @@ def run_paged(args, tri, dev, rank, ws):
     value = keys_round * len(rounds) * ws / (ms_max / 1e3)
     ms_step = ms_max / len(rounds)
     peak, peak_kind = measured_hbm_peak()
-    score_ms = float(per[:, 1].mean())
+    score_ms = float(per1[:, 1].mean())
     score_bytes = keys_round * KEY_BYTES
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     step_bytes = keys_round * KEY_BYTES + moved * MOVE_BYTES
@@ -639,8 +647,7 @@ def run_paged(args, tri, dev, rank, ws):
     init_ms = float(sum(per0))
     init_bytes = keys0 * KEY_BYTES + moved0 * MOVE_BYTES
 
-    e2e = run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws,
-                        lambda dd, ss: event(dd, ss, None, args.pipeline))
+    e2e = run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws, lambda dd: steady(dd))
 
     result = None
     if rank == 0:
@@ -657,14 +664,12 @@ def run_paged(args, tri, dev, rank, ws):
                                    f"{B + PAGED_APPEND} keys re-compressed to {B} in place",
                        "keys_per_gpu": keys_round, "budget": B, "parallelism": f"independent caches x{ws}",
                        "l2": "L2 flushed (512 MB fill) before every pruning event, outside the events"},
-            "step_breakdown_ms": ({"fold": float(per[:, 0].mean()), "score": score_ms,
-                                   "select": float(per[:, 2].mean()), "holefill": float(per[:, 3].mean())}
-                                  if args.pipeline <= 1 else
-                                  {"fold": float(per[:, 0].mean()), "scoring (all chunks)": score_ms,
-                                   "tail (last chunk's select + hole fill)": float(per[:, 2].mean())}),
-            "unpipelined_round_ms": dict(zip(("fold", "score", "select", "holefill"), per1)),
-            "pipeline": (f"{args.pipeline} chunks of whole layers: chunk c+1 scored while chunk c is selected and "
-                         f"compacted on a second stream" if args.pipeline > 1 else "one stream"),
+            "step_breakdown_ms": {"fold": float(per[:, 0].mean()), "compress": float(per[:, 1].mean()),
+                                  "score (alone)": score_ms,
+                                  "select + hole fill (compress minus score alone)":
+                                      float(per1[:, 2].mean() - per1[:, 1].mean()),
+                                  "breakdown": f"{PAGED_BREAKDOWN_ROUNDS} more rounds, each with the scorer "
+                                               "run once on its own before the compress call"},
             "rows_moved_per_step": moved,
             "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_gbs,
                     "frac_of_measured": step_gbs / peak, "frac_of_8tbps_spec": step_gbs / SPEC_HBM_GBS},
@@ -681,7 +686,8 @@ def run_paged(args, tri, dev, rank, ws):
                          "algorithmic_bytes_per_launch": score_bytes},
             "clocks": clocks,
             "gpu_launches": int(launches),
-            "timing": "each round: plain launches queued behind a GPU sleep, CUDA events around the four calls",
+            "timing": "each round: plain launches queued behind a GPU sleep, CUDA events around the fold and "
+                      "the compress call",
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
@@ -712,7 +718,6 @@ def run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws, do_round):
     kpool, vpool = cache.k.view(L, nb, -1), cache.v.view(L, nb, -1)
     table = cache.block_table.cpu()
     htable = torch.empty(table.shape, dtype=torch.int32, pin_memory=True)
-    scores = None
     times = []
     for i in range(steps + 1):                     # the first round is a warm-up
         # host bookkeeping of the append: fresh pages for every sequence
@@ -727,8 +732,6 @@ def run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws, do_round):
         htable.copy_(table)
         idx = torch.tensor(pages, dtype=torch.int64).pin_memory()
         dt = tri.desc_paged(cache.k, cache.v, cache.block_table, cache.lens)
-        if scores is None:
-            scores = torch.empty((wl.units, tri.score_row_stride(dt)), dtype=torch.float32, device=qc.device)
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         start.record(stream)
@@ -738,7 +741,7 @@ def run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws, do_round):
         sv.copy_(hv, non_blocking=True)
         kpool[:, di] = sk                          # the new tokens into their pages
         vpool[:, di] = sv
-        do_round(dt, scores)                       # fold, score, select, hole fill
+        do_round(dt)                               # fold, compress in place
         hkept.copy_(kept, non_blocking=True)
         hcnt.copy_(cnt, non_blocking=True)
         end.record(stream)
@@ -760,8 +763,7 @@ def run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws, do_round):
     return {"value": keys * ws * steps / (ms / 1e3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps, "host_memory": "pinned",
             "what": "per round: the new tokens' K and V and the block table in, written into fresh pages, "
-                    "fold + score + select + in-place hole fill, kept indices and counts out; the cache stays "
-                    "resident"}
+                    "fold + compress in place, kept indices and counts out; the cache stays resident"}
 
 
 def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, job_keys, ws, positions=None,
@@ -979,9 +981,6 @@ def main():
     ap.add_argument("--eager", action="store_true", help="time plain launches instead of a CUDA graph of the step")
     ap.add_argument("--path", default="calls", choices=["calls", "compress"],
                     help="calls: fold, score, select, compact as four calls (default); compress: fold + tri_compress")
-    ap.add_argument("--pipeline", type=int, default=4,
-                    help="paged workload: chunks of layers whose selection and hole fill overlap the scoring of "
-                         "the next chunk (1: one stream)")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "layers"],
                     help="N > 1: replicas (default): every rank compresses its own cache (weak scaling); "
                          "layers: one cache split by whole layers over the ranks (strong scaling)")

@@ -32,11 +32,31 @@ namespace compact {
 #ifndef TRI_GATHER_BLOCKS_PER_SM
 #define TRI_GATHER_BLOCKS_PER_SM 6
 #endif
+// Stores of the gathered rows: 0 plain, 1 streaming (.cs), 2 with an L2
+// evict-first policy (the output is not read again by this step).
+#ifndef TRI_GATHER_STORE
+#define TRI_GATHER_STORE 0
+#endif
 
 constexpr int kGatherThreads = 256;
 constexpr int kGatherUnroll = TRI_GATHER_UNROLL;     // rows in flight per half-warp
 constexpr int kGatherBlocksPerSm = TRI_GATHER_BLOCKS_PER_SM;
 constexpr int kChunkRows = 32;                      // kept rows of one unit per warp and step
+
+__device__ __forceinline__ void st_out_v4(void* p, const uint4& x, uint64_t policy) {
+#if TRI_GATHER_STORE == 1
+  (void)policy;
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w)
+               : "memory");
+#elif TRI_GATHER_STORE == 2
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(x.x), "r"(x.y),
+               "r"(x.z), "r"(x.w), "l"(policy)
+               : "memory");
+#else
+  (void)policy;
+  *reinterpret_cast<uint4*>(p) = x;
+#endif
+}
 
 __device__ __forceinline__ void unit_coords(const Geom& g, int u, int* l, int* h, int* b) {
   *b = u % g.batch;
@@ -58,6 +78,11 @@ gather_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept,
   const int warp0 = (blockIdx.x * kGatherThreads + threadIdx.x) >> 5;
   const int nwarps = (gridDim.x * kGatherThreads) >> 5;
   const bool packed = g.layout != TRI_LAYOUT_PAGED;
+#if TRI_GATHER_STORE == 2
+  const uint64_t out_policy = policy_evict_first();
+#else
+  const uint64_t out_policy = 0;
+#endif
   for (int c = warp0; c < total_chunks; c += nwarps) {
     const int u = c / chunks_per_unit;
     const int j0 = (c - u * chunks_per_unit) * kChunkRows;
@@ -108,8 +133,8 @@ gather_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept,
       for (int q = 0; q < kGatherUnroll; ++q) {
         if (!live[q]) continue;
         const int64_t row = out0 + r0 + 2 * q + hw;
-        reinterpret_cast<uint4*>(kout + row * kD)[l16] = kx[q];
-        reinterpret_cast<uint4*>(vout + row * kD)[l16] = vx[q];
+        st_out_v4(kout + row * kD + l16 * 8, kx[q], out_policy);
+        st_out_v4(vout + row * kD + l16 * 8, vx[q], out_policy);
       }
     }
   }
@@ -127,38 +152,31 @@ constexpr int kFillWarps = 4;
 constexpr int kFillThreadsWarp = kFillWarps * 32;
 constexpr int kFillWarpMovers = 512;               // rows moved per unit up to which a warp per unit is used
 
-__global__ void __launch_bounds__(kFillThreadsWarp)
-holefill_warp_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept, int B, uint16_t* k, uint16_t* v,
-                int units) {
+// The hole fill of one unit (n > B keys, kept ascending), by one warp.
+__device__ __forceinline__ void holefill_unit_warp(const Geom& g, const int32_t* __restrict__ ku, int B, int n,
+                                                   int l, int h, int b, uint16_t* k, uint16_t* v) {
   const int lane = threadIdx.x & 31, l16 = lane & 15, hw = lane >> 4;
-  const int u = blockIdx.x * kFillWarps + (threadIdx.x >> 5);
-  if (u >= units) return;                          // whole warps
-  int l, h, b;
-  unit_coords(g, u, &l, &h, &b);
-  const int n = g.len[b];
-  if (n <= B) return;
-  const int32_t* __restrict__ ku = kept + static_cast<int64_t>(u) * B;
   // f: the first kept index >= B (every lane searches the same range)
   int lo = 0, hi = B;
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
-    if (__ldg(ku + mid) >= B) hi = mid;
+    if (ku[mid] >= B) hi = mid;
     else lo = mid + 1;
   }
   const int f = lo;
   const int m = B - f;                             // movers = holes below B
   // ascending kept indices: the last one below B sits just before the movers
-  if (lane == 0) TRI_CHECK(f == 0 || __ldg(ku + f - 1) < B);
+  if (lane == 0) TRI_CHECK(f == 0 || ku[f - 1] < B);
   for (int r0 = 0; r0 < m; r0 += 32) {
     const int r = r0 + lane;
     int src = -1, dst = -1;
     if (r < m) {
-      src = __ldg(ku + f + r);
+      src = ku[f + r];
       // upper bound of r in z_i = kept[i] - i, i < f
       int a = 0, c = f;
       while (a < c) {
         const int mid = (a + c) >> 1;
-        if (__ldg(ku + mid) - mid <= r) a = mid + 1;
+        if (ku[mid] - mid <= r) a = mid + 1;
         else c = mid;
       }
       dst = r + a;
@@ -166,7 +184,7 @@ holefill_warp_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__
         flag(TRI_DEVFLAG_BAD_KEPT);
         src = -1;
       }
-      if (r > 0) TRI_CHECK(__ldg(ku + f + r - 1) < src || src < 0);    // movers ascending
+      if (r > 0) TRI_CHECK(ku[f + r - 1] < src || src < 0);    // movers ascending
     }
     const int cnt = min(32, m - r0);
     for (int q = 0; q < cnt; q += 2) {             // half-warp hw copies pair q + hw
@@ -186,6 +204,18 @@ holefill_warp_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__
       reinterpret_cast<uint4*>(v + ed)[l16] = vx;
     }
   }
+}
+
+__global__ void __launch_bounds__(kFillThreadsWarp)
+holefill_warp_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept, int B, uint16_t* k,
+                     uint16_t* v, int units) {
+  const int u = blockIdx.x * kFillWarps + (threadIdx.x >> 5);
+  if (u >= units) return;                          // whole warps
+  int l, h, b;
+  unit_coords(g, u, &l, &h, &b);
+  const int n = g.len[b];
+  if (n <= B) return;
+  holefill_unit_warp(g, kept + static_cast<int64_t>(u) * B, B, n, l, h, b, k, v);
 }
 
 // Hole fill, one CTA per unit, for units that move many rows (a long row

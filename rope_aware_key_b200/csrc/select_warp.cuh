@@ -16,12 +16,13 @@
 // are scored.  Every decision is made on order-preserving integer keys of the
 // fp32 scores (NaN lowest), so the result is exact:
 //  1. 256 evenly spaced scores of the row are sorted (a bitonic network in
-//     registers, 8 per lane); their ranks B/n * 256 -/+ (3 sigma + 4) from
+//     registers, 8 per lane); their ranks B/n * 256 -/+ (4 sigma + 8) from
 //     the top give two keys U >= L that bracket the B-th largest key for any
 //     but a pathological order of the scores;
 //  2. one pass over the row counts the keys above U (all kept) and gathers
-//     the keys in [L, U] into a candidate buffer.  When L would fall below
-//     the sample (rows that evict few keys), every key up to U is a
+//     the keys in [L, U] into a candidate buffer (the comparisons are made
+//     on the floats; the candidates are stored as keys).  When L would fall
+//     below the sample (rows that evict few keys), every key up to U is a
 //     candidate and is gathered with its index, in index order;
 //  3. if the B-th largest lies among the candidates (above < B <= above +
 //     candidates), a radix search over them (8-bit digits, a shared histogram
@@ -33,11 +34,12 @@
 //     lanes' groups interleaved so that every store covers 512 consecutive
 //     bytes.  Other rows: a second pass emits the kept keys in index order
 //     (ballots per 128-key chunk).
-// If the check fails (a pathological order, heavy duplication, NaN where the
-// bracket lies), a bitwise search over the whole row finds T instead.
+// If the check fails (a pathological order, heavy duplication), the radix
+// search runs over the whole row instead (one pass per digit).
 #pragma once
 
 #include "common.cuh"
+#include "compact.cuh"
 #include "select.cuh"
 
 namespace tri {
@@ -48,6 +50,7 @@ constexpr int kWarpThreads = kWarpRows * 32;
 constexpr int kWarpSamples = 256;                  // 8 per lane
 constexpr int kWarpCand = 512;
 constexpr int kWarpMaxRow = 4096;
+constexpr int kWarpBatch = 4;                     // chunks whose loads are in flight together
 
 struct __align__(16) WarpScratch {
   uint32_t hist[256];                              // the sorted samples, then the radix digits
@@ -72,9 +75,11 @@ __device__ __forceinline__ float4 row_chunk(const float* __restrict__ row, int n
 __device__ __forceinline__ void warp_sort256(uint32_t (&x)[8]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int k = 2; k <= 256; k <<= 1) {
+  for (int kb = 1; kb <= 8; ++kb) {
+    const int k = 1 << kb;
 #pragma unroll
-    for (int j = k >> 1; j > 0; j >>= 1) {
+    for (int jb = kb - 1; jb >= 0; --jb) {
+      const int j = 1 << jb;
       if (j >= 8) {                                // the partner sits in lane ^ (j / 8), same slot
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -97,13 +102,14 @@ __device__ __forceinline__ void warp_sort256(uint32_t (&x)[8]) {
   }
 }
 
-// The need-th largest (need >= 1) of the keys in [lo, hi] among keys[0 .. nc)
-// (at least `need` of them are >= lo, and none in [lo, hi] is missing), by
+// The need-th largest (need >= 1) of the keys in [lo, hi] among the keys the
+// lanes pass through `each` (at least `need` of them lie in [lo, hi]), by
 // 8-bit digits of key - lo, most significant first: each digit's histogram
 // (hist, 256 words) picks the bin that holds the rank.  *need becomes the
 // rank of the result among the keys equal to it.
-__device__ __forceinline__ uint32_t warp_radix_kth(const uint32_t* keys, int nc, uint32_t lo, uint32_t hi,
-                                                   uint32_t* need, uint32_t* hist) {
+template <typename Each>
+__device__ __forceinline__ uint32_t warp_radix_kth(Each each, uint32_t lo, uint32_t hi, uint32_t* need,
+                                                   uint32_t* hist) {
   const int lane = threadIdx.x & 31;
   while (lo < hi) {
     const int bits = 32 - __clz(hi - lo);
@@ -112,10 +118,9 @@ __device__ __forceinline__ uint32_t warp_radix_kth(const uint32_t* keys, int nc,
 #pragma unroll
     for (int e = 0; e < 8; ++e) hist[32 * e + lane] = 0u;
     __syncwarp();
-    for (int m = lane; m < nc; m += 32) {
-      const uint32_t k = keys[m];
+    each([&](uint32_t k) {
       if (k >= lo && k <= hi) atomicAdd(&hist[(k - lo) >> shift], 1u);
-    }
+    });
     __syncwarp();
     // lane l owns digits [8 l, 8 l + 8); counts above a lane's digits by a suffix scan
     const uint4 h0 = reinterpret_cast<const uint4*>(hist)[2 * lane];
@@ -154,22 +159,10 @@ __device__ __forceinline__ uint32_t warp_radix_kth(const uint32_t* keys, int nc,
   return lo;
 }
 
-// The largest t with #{x : x >= t} >= need over the keys each lane passes
-// through `each` (the whole-row fallback).
-template <typename Each>
-__device__ __forceinline__ uint32_t warp_bitwise_kth(Each each, uint32_t need) {
-  uint32_t prefix = 0u;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t t = prefix | (1u << bit);
-    uint32_t c = 0;
-    each([&](uint32_t x) { c += x >= t; });
-    if (__reduce_add_sync(0xffffffffu, c) >= need) prefix = t;
-  }
-  return prefix;
-}
-
 // Select one row of n > B scores (n <= kWarpMaxRow); kept gets the B indices.
-__device__ __forceinline__ void warp_select_row(const float* __restrict__ row, int n, int B, WarpScratch& S,
+// Returns the number of evicted keys when their indices are left in S.cand
+// (ascending), else -1.
+__device__ __forceinline__ int warp_select_row(const float* __restrict__ row, int n, int B, WarpScratch& S,
                                                 int32_t* __restrict__ kept) {
   const int lane = threadIdx.x & 31;
   const int chunks = (n + 127) >> 7;               // warp-uniform
@@ -186,41 +179,57 @@ __device__ __forceinline__ void warp_select_row(const float* __restrict__ row, i
   reinterpret_cast<uint4*>(S.hist)[2 * lane + 1] = make_uint4(x[4], x[5], x[6], x[7]);
   __syncwarp();
   const float r = static_cast<float>(B) * kWarpSamples / static_cast<float>(n);
-  const float delta = 3.f * sqrtf(r * (1.f - r / kWarpSamples)) + 4.f;
+  const float delta = 4.f * sqrtf(r * (1.f - r / kWarpSamples)) + 8.f;
   const int r_hi = static_cast<int>(floorf(r - delta)), r_lo = static_cast<int>(ceilf(r + delta));
   const uint32_t U = r_hi >= 1 ? S.hist[kWarpSamples - r_hi] : 0xffffffffu;
-  const bool few = r_lo > kWarpSamples;            // rows that evict few keys: no lower bound
-  const uint32_t L = few ? 0u : S.hist[kWarpSamples - r_lo];
+  const uint32_t L0 = r_lo <= kWarpSamples ? S.hist[kWarpSamples - r_lo] : 0u;
+  // rows that evict few keys (no lower bound; also when the bound is NaN's key)
+  const bool few = L0 == 0u;
+  // the same bounds as floats: above U is v > uf (NaN never is), in [L, U] is
+  // !(v > uf) && v >= lf (every number when L is -inf's key)
+  const float uf = U == 0xffffffffu ? INFINITY : key_value(U);
+  const float lf = key_value(L0);
 
-  // 2. one pass: count the keys above U, gather those in [L, U]
+  // 2. one pass: count the keys above U, gather those in [L, U]; the loads of
+  // kWarpBatch chunks are issued before any of them is used
   uint32_t above = 0, base = 0, cmin = 0xffffffffu, cmax = 0u;
-  for (int j = 0; j < chunks; ++j) {
-    const float4 xv = row_chunk(row, n, full, j, lane);
-    const uint32_t k[4] = {order_key(xv.x), order_key(xv.y), order_key(xv.z), order_key(xv.w)};
-    bool in[4];
-    uint32_t before = 0, total = 0;
+  for (int j0 = 0; j0 < chunks; j0 += kWarpBatch) {
+    float4 xb[kWarpBatch];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const bool vq = valid(j, q);
-      above += vq && k[q] > U;
-      in[q] = vq && k[q] >= L && k[q] <= U;
-      const uint32_t m = __ballot_sync(0xffffffffu, in[q]);
-      before += __popc(m & lt);
-      total += __popc(m);
-    }
-    uint32_t pos = base + before;                  // index order: lanes, then q within a lane
+    for (int i = 0; i < kWarpBatch; ++i)
+      if (j0 + i < chunks) xb[i] = row_chunk(row, n, full, j0 + i, lane);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (in[q]) {
-        if (pos < static_cast<uint32_t>(kWarpCand)) {
-          S.cand[pos] = k[q];
-          if (few) S.cidx[pos] = 128 * j + 4 * lane + q;
-          cmin = min(cmin, k[q]);
-          cmax = max(cmax, k[q]);
-        }
-        ++pos;
+    for (int i = 0; i < kWarpBatch; ++i) {
+      const int j = j0 + i;
+      if (j >= chunks) break;                      // warp-uniform
+      const float v[4] = {xb[i].x, xb[i].y, xb[i].z, xb[i].w};
+      bool in[4];
+      uint32_t before = 0, total = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const bool vq = valid(j, q);
+        const bool up = v[q] > uf;
+        above += vq && up;
+        in[q] = vq && !up && (few || v[q] >= lf);
+        const uint32_t m = __ballot_sync(0xffffffffu, in[q]);
+        before += __popc(m & lt);
+        total += __popc(m);
       }
-    base += total;
+      uint32_t pos = base + before;                // index order: lanes, then q within a lane
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (in[q]) {
+          if (pos < static_cast<uint32_t>(kWarpCand)) {
+            const uint32_t k = order_key(v[q]);
+            S.cand[pos] = k;
+            if (few) S.cidx[pos] = 128 * j + 4 * lane + q;
+            cmin = min(cmin, k);
+            cmax = max(cmax, k);
+          }
+          ++pos;
+        }
+      base += total;
+    }
   }
   above = __reduce_add_sync(0xffffffffu, above);
   const bool ok = above < static_cast<uint32_t>(B) && static_cast<uint32_t>(B) <= above + base &&
@@ -232,11 +241,15 @@ __device__ __forceinline__ void warp_select_row(const float* __restrict__ row, i
     cmax = __reduce_max_sync(0xffffffffu, cmax);
     need = static_cast<uint32_t>(B) - above;       // 1 <= need <= base
     // 3. the exact threshold among the candidates; need becomes the ties to keep
-    T = warp_radix_kth(S.cand, static_cast<int>(base), cmin, cmax, &need, S.hist);
+    const int nc = static_cast<int>(base);
+    T = warp_radix_kth(
+        [&](auto fn) {
+          for (int m = lane; m < nc; m += 32) fn(S.cand[m]);
+        },
+        cmin, cmax, &need, S.hist);
     if (few) {
       // 4. the evicted indices, ascending, written over the candidate keys
       // already read: candidates below T, and ties past the first `need`
-      const int nc = static_cast<int>(base);
       uint32_t ev = 0, ties = 0;
       for (int m0 = 0; m0 < nc; m0 += 32) {
         const int m = m0 + lane;
@@ -258,23 +271,30 @@ __device__ __forceinline__ void warp_select_row(const float* __restrict__ row, i
       // kept[j] = j + #{t : ev[t] - t <= j}: ev[t] - t, the kept keys below
       // ev[t], never decreases, so each lane walks its slots in order
       int e = 0;
+      int z = E > 0 ? evi[0] : 0x7fffffff;       // ev[e] - e, or past every slot
+      auto advance = [&](int j) {
+        while (z <= j) {
+          ++e;
+          z = e < E ? evi[e] - e : 0x7fffffff;
+        }
+      };
       if ((reinterpret_cast<uintptr_t>(kept) & 15u) == 0 && (B & 3) == 0) {
         for (int j = 4 * lane; j < B; j += 128) {  // groups of 4 slots, lanes interleaved
           int o[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            while (e < E && evi[e] - e <= j + q) ++e;
+            advance(j + q);
             o[q] = j + q + e;
           }
           *reinterpret_cast<int4*>(kept + j) = make_int4(o[0], o[1], o[2], o[3]);
         }
       } else {
         for (int j = lane; j < B; j += 32) {
-          while (e < E && evi[e] - e <= j) ++e;
+          advance(j);
           kept[j] = j + e;
         }
       }
-      return;
+      return E;
     }
   } else {
     // whole-row search: every key of the row counts (NaN keys are 0, below
@@ -288,10 +308,8 @@ __device__ __forceinline__ void warp_select_row(const float* __restrict__ row, i
           if (valid(j, q)) fn(order_key(v[q]));
       }
     };
-    T = warp_bitwise_kth(each_key, static_cast<uint32_t>(B));
-    uint32_t gt = 0;
-    each_key([&](uint32_t k) { gt += k > T; });
-    need = static_cast<uint32_t>(B) - __reduce_add_sync(0xffffffffu, gt);
+    need = static_cast<uint32_t>(B);
+    T = warp_radix_kth(each_key, 0u, 0xffffffffu, &need, S.hist);
   }
 
   // 4'. T is the B-th largest key; keep every key above it and the `need`
@@ -343,12 +361,80 @@ __device__ __forceinline__ void warp_select_row(const float* __restrict__ row, i
     slot += total;
   }
   if (lane == 0) TRI_CHECK(slot == static_cast<uint32_t>(B));         // exactly B kept
+  return -1;
+}
+
+// The in-place hole fill of a row from its evicted indices ev[0 .. E)
+// (ascending, n = B + E): the evicted positions below B are the holes, the
+// kept positions at or above B the movers, and the r-th mover goes to the
+// r-th hole -- the same moves as compact::holefill_unit_warp, found without
+// reading the kept list back.  `tail` (ceil(E / 32) words of shared memory)
+// marks the evicted positions at or above B.  Half a warp copies K and the
+// other half V, four rows in flight.
+__device__ __forceinline__ void warp_fill_row(const Geom& g, int l, int h, int b, const int32_t* ev, int E, int B,
+                                              int n, uint32_t* tail, uint16_t* k, uint16_t* v) {
+  const int lane = threadIdx.x & 31, l16 = lane & 15, hw = lane >> 4;
+  const uint32_t lt = (1u << lane) - 1u;
+  if (E != n - B) {                                // not a list of n - B evictions
+    if (lane == 0) flag(TRI_DEVFLAG_BAD_KEPT);
+    return;
+  }
+  int m = 0;                                       // holes: evicted positions below B
+  for (int t0 = 0; t0 < E; t0 += 32) m += __popc(__ballot_sync(0xffffffffu, t0 + lane < E && ev[t0 + lane] < B));
+  const int tw = (E + 31) >> 5;
+  for (int w = lane; w < tw; w += 32) tail[w] = 0u;
+  __syncwarp();
+  for (int t = m + lane; t < E; t += 32) {
+    const int p = ev[t] - B;
+    atomicOr(&tail[p >> 5], 1u << (p & 31));
+  }
+  __syncwarp();
+  uint16_t* const src_base = hw ? v : k;
+  int r0 = 0;
+  for (int c0 = 0; c0 < E; c0 += 32) {             // tail positions B + c0 + lane
+    const bool mv = c0 + lane < E && !((tail[c0 >> 5] >> lane) & 1u);
+    const uint32_t mm = __ballot_sync(0xffffffffu, mv);
+    bool ok = true;
+    int64_t es = 0, ed = 0;
+    if (mv) {
+      const int r = r0 + __popc(mm & lt);          // r < m
+      es = row_elem(g, l, h, b, B + c0 + lane, &ok);
+      ed = row_elem(g, l, h, b, ev[r], &ok);
+      if (!ok) flag(TRI_DEVFLAG_BAD_PAGE);
+    }
+    uint32_t rem = __ballot_sync(0xffffffffu, mv && ok);
+    r0 += __popc(mm);
+    while (rem) {                                  // warp-uniform
+      int sl[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        sl[i] = rem ? __ffs(rem) - 1 : -1;
+        rem &= rem - 1u;
+      }
+      uint4 x[4];
+      int64_t d[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int from = sl[i] < 0 ? 0 : sl[i];
+        const int64_t s_i = __shfl_sync(0xffffffffu, es, from);
+        d[i] = __shfl_sync(0xffffffffu, ed, from);
+        if (sl[i] >= 0) x[i] = ld_nc_v4(src_base + s_i + l16 * 8);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (sl[i] >= 0) reinterpret_cast<uint4*>(src_base + d[i])[l16] = x[i];
+    }
+  }
+  if (lane == 0) TRI_CHECK(r0 == m);               // as many movers as holes
 }
 
 // One warp per unit, units [blockIdx.x * kWarpRows, ...): rows of at most
-// kWarpMaxRow keys.  Dynamic shared memory: kWarpSmemBytes.
+// kWarpMaxRow keys.  Dynamic shared memory: kWarpSmemBytes.  FILL: the
+// in-place hole fill of each row follows its selection in the same warp
+// (k, v: the cache), for launches whose rows move few keys.
+template <bool FILL>
 __global__ void __launch_bounds__(kWarpThreads) select_warp_kernel(const __grid_constant__ Geom g, const Args a,
-                                                                   int units) {
+                                                                   int units, uint16_t* k, uint16_t* v) {
   extern __shared__ float4 select_warp_dyn[];
   WarpScratch* scratch = reinterpret_cast<WarpScratch*>(select_warp_dyn);
   const int w = threadIdx.x >> 5;
@@ -364,7 +450,17 @@ __global__ void __launch_bounds__(kWarpThreads) select_warp_kernel(const __grid_
     for (int i = lane; i < n; i += 32) kept[i] = i;
     return;
   }
-  warp_select_row(a.scores + static_cast<int64_t>(u) * g.score_stride, n, B, scratch[w], kept);
+  const int E = warp_select_row(a.scores + static_cast<int64_t>(u) * g.score_stride, n, B, scratch[w], kept);
+  if constexpr (FILL) {
+    int l, h, b_;
+    compact::unit_coords(g, u, &l, &h, &b_);       // b_ == b
+    __syncwarp();                                  // the kept list (global) and the evicted list (shared)
+    if (E >= 0)
+      warp_fill_row(g, l, h, b, reinterpret_cast<const int32_t*>(scratch[w].cand), E, B, n, scratch[w].hist,
+                    k, v);
+    else
+      compact::holefill_unit_warp(g, kept, B, n, l, h, b, k, v);
+  }
 }
 
 }  // namespace select

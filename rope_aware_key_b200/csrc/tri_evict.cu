@@ -161,19 +161,11 @@ tri_status use_device_of(const void* ptr, int* dev_out, DeviceScope* scope) {
                                   tri::select::kMaxShared));
     TRI_CUDA(cudaFuncSetAttribute(tri::select::select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   tri::select::kMaxShared));
-    // The warp selection and the warp hole fill are small enough to run beside
-    // the scorer's CTAs (a caller may select one group of layers while the
-    // next is scored); that needs the same split of on-chip memory between L1
-    // and shared memory as the scorer, so every one of them asks for the
-    // largest shared-memory carveout.
-    for (const void* fn : {reinterpret_cast<const void*>(tri::score::score_kernel),
-                           reinterpret_cast<const void*>(tri::select::select_warp_kernel),
-                           reinterpret_cast<const void*>(tri::compact::holefill_warp_kernel)})
-      TRI_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                    cudaSharedmemCarveoutMaxShared));
     TRI_CUDA(cudaFuncSetAttribute(tri::compact::holefill_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   ((tri::compact::kMaxFillCta + 31) / 32 + tri::compact::kMaxFillCta) * 4));
-    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_warp_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(tri::select::kWarpSmemBytes)));
+    TRI_CUDA(cudaFuncSetAttribute(tri::select::select_warp_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(tri::select::kWarpSmemBytes)));
     TRI_CUDA(cudaFuncSetAttribute(tri::smax::score_max_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(tri::smax::kSmemBytes)));
@@ -350,6 +342,13 @@ tri_status launch_score(const Geom& g0, const float* w, float* scores, int dev, 
   return TRI_OK;
 }
 
+// Keys in the longest row.
+int max_row(const Geom& g) {
+  int max_len = 0;
+  for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
+  return max_len;
+}
+
 // How one selection launch is shaped, decided (and checked) on the host
 // before anything is launched: a warp per row when every row holds at most
 // kWarpMaxRow keys, else a CTA per row with its working set in shared memory.
@@ -360,8 +359,7 @@ struct SelectPlan {
 };
 
 tri_status plan_select(const Geom& g, int B, SelectPlan* p) {
-  int max_len = 0;
-  for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
+  const int max_len = max_row(g);
   *p = SelectPlan();
   if (max_len <= tri::select::kWarpMaxRow) {
     p->warp = true;
@@ -375,13 +373,20 @@ tri_status plan_select(const Geom& g, int B, SelectPlan* p) {
   return TRI_OK;
 }
 
+// fill: the in-place hole fill runs in the warp selection kernel, row by row
+// (only with p.warp; see fill_in_select).
 tri_status launch_select(const Geom& g, const SelectPlan& p, const float* scores, int B, int32_t* kept,
-                         int32_t* kept_count, cudaStream_t s) {
+                         int32_t* kept_count, cudaStream_t s, bool fill = false) {
   const int units = g.L * g.H * g.batch;
   tri::select::Args a{scores, kept, kept_count, B, p.cap, p.lcap};
   if (p.warp) {
     const int grid = (units + tri::select::kWarpRows - 1) / tri::select::kWarpRows;
-    tri::select::select_warp_kernel<<<grid, tri::select::kWarpThreads, p.smem, s>>>(g, a, units);
+    uint16_t* k = const_cast<uint16_t*>(g.k);
+    uint16_t* v = const_cast<uint16_t*>(g.v);
+    if (fill)
+      tri::select::select_warp_kernel<true><<<grid, tri::select::kWarpThreads, p.smem, s>>>(g, a, units, k, v);
+    else
+      tri::select::select_warp_kernel<false><<<grid, tri::select::kWarpThreads, p.smem, s>>>(g, a, units, k, v);
   } else if (p.cap >= 8192) {
     tri::select::select_kernel<512><<<units, 512, p.smem, s>>>(g, a);
   } else {
@@ -396,6 +401,13 @@ tri_status launch_select(const Geom& g, const SelectPlan& p, const float* scores
 tri_status check_compact_launch(const Geom& g, int B, tri_compact_mode mode) {
   if (mode == TRI_COMPACT_OUT_OF_PLACE && int64_t{g.L} * g.H * g.batch * B > INT32_MAX) return TRI_ERR_UNSUPPORTED;
   return TRI_OK;
+}
+
+// In-place compaction whose rows move few keys (at most kFillWarpMovers, the
+// bound the standalone kernels also use for a warp per unit): a warp per row
+// selects and then fills the row's holes in one kernel.
+bool fill_in_select(const Geom& g, const SelectPlan& p, int B, tri_compact_mode mode) {
+  return mode == TRI_COMPACT_IN_PLACE_HOLEFILL && p.warp && max_row(g) - B <= tri::compact::kFillWarpMovers;
 }
 
 tri_status launch_compact(const Geom& g, const int32_t* kept, const int32_t* kept_count, int B,
@@ -414,9 +426,7 @@ tri_status launch_compact(const Geom& g, const int32_t* kept, const int32_t* kep
         static_cast<int>(chunks));
   } else {
     // rows moved per unit: at most n - B; a warp per unit while that is small
-    int max_len = 0;
-    for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
-    if (max_len - B <= tri::compact::kFillWarpMovers || B > tri::compact::kMaxFillCta) {
+    if (max_row(g) - B <= tri::compact::kFillWarpMovers || B > tri::compact::kMaxFillCta) {
       const int grid = (units + tri::compact::kFillWarps - 1) / tri::compact::kFillWarps;
       tri::compact::holefill_warp_kernel<<<grid, tri::compact::kFillThreadsWarp, 0, s>>>(
           g, kept, B, const_cast<uint16_t*>(g.k), const_cast<uint16_t*>(g.v), units);
@@ -442,8 +452,7 @@ tri_status launch_fused(const Geom& g, const float* w, float* scores, int B, int
   if (C == 0 || g.layout == TRI_LAYOUT_PAGED) return TRI_ERR_UNSUPPORTED;
   const int64_t units = int64_t{g.L} * g.H * g.batch;
   if (units * C > g_dev[dev].sms) return TRI_ERR_UNSUPPORTED;
-  int max_len = 0;
-  for (int b = 0; b < g.batch; ++b) max_len = g.len[b] > max_len ? g.len[b] : max_len;
+  const int max_len = max_row(g);
   // Longer rows stream faster through the standalone scorer on every SM than
   // through one cluster per unit (measured: 1 x 4096 keys 20 vs 25 us per
   // step, 8 x 8192 even, 1 x 32768 33 vs 25 us).
@@ -498,7 +507,9 @@ tri_status compress_checks(const Geom& g0, int B, tri_compact_mode mode, SelectP
 }
 
 // The stages of tri_compress / tri_compress_noalloc once their checks have
-// passed: the single-kernel step where it applies, else score, select, compact.
+// passed: the single-kernel step where it applies, else score, select,
+// compact (in place with rows that move few keys: score, then the selection
+// with the hole fill in it).
 tri_status run_compress(const Geom& g, const SelectPlan& plan, const float* w, int B, tri_compact_mode mode,
                         int32_t* kept, int32_t* kept_count, void* k_out, void* v_out, float* scores, int dev,
                         cudaStream_t s) {
@@ -509,8 +520,9 @@ tri_status run_compress(const Geom& g, const SelectPlan& plan, const float* w, i
   }
   st = launch_score(g, w, scores, dev, s);
   if (st != TRI_OK) return st;
-  st = launch_select(g, plan, scores, B, kept, kept_count, s);
-  if (st != TRI_OK) return st;
+  const bool fill = fill_in_select(g, plan, B, mode);
+  st = launch_select(g, plan, scores, B, kept, kept_count, s, fill);
+  if (st != TRI_OK || fill) return st;
   return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, s);
 }
 

@@ -262,6 +262,45 @@ def test_steady_round_shape_every_unit():
     check_every_unit(cache, res, literal=False, before=before, after=after)
 
 
+@pytest.mark.parametrize("lens,B", [([2176, 2176, 2048, 2175, 2049, 2560], 2048),
+                                    ([4096, 3700, 4000, 100, 3601], 3600)])
+def test_compress_in_place_fills_holes_in_the_selection(lens, B):
+    """tri_compress in place on rows that move at most 512 keys: one warp per
+    row selects and then fills the row's holes, from its evicted list (rows
+    that evict few keys) or from its kept list (the others).  Three launches
+    (fold, score, the selection with the fill); every unit against the
+    oracle, K and V before and after."""
+    t = tri()
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=4, batch=len(lens), budget=B,
+                    spare_blocks_per_seq=1)
+    cache = gen.make_cache(wl, seed=21 + B, device=DEV, lens=lens)
+    units = all_units(wl)
+    before = snapshot(cache, units)
+    n0 = t.kernel_launches()
+    res = parity.run_gpu(cache, mode=t.COMPACT_IN_PLACE_HOLEFILL, fused=True)
+    assert t.kernel_launches() - n0 == 3
+    after = snapshot(cache, units)
+    check_every_unit(cache, res, literal=False, before=before, after=after)
+
+
+@pytest.mark.parametrize("dup", [1, 3])
+def test_compress_in_place_fill_after_the_whole_row_search(dup):
+    """Rows whose scores take one or three values: the selection's bracket
+    check fails and the whole-row search decides; the fill in the same kernel
+    then follows the kept list.  Contiguous cache, in place."""
+    n, B = 2400, 2000
+    wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=n, budget=B)
+    cache = gen.make_cache(wl, seed=22 + dup, device=DEV)
+    for h in range(2):
+        base = cache.k[0, h, 0, :dup].clone()
+        cache.k[0, h, 0] = base.repeat(n // dup + 1, 1)[:n]
+    units = all_units(wl)
+    before = snapshot(cache, units)
+    res = parity.run_gpu(cache, mode=tri().COMPACT_IN_PLACE_HOLEFILL, fused=True)
+    after = snapshot(cache, units)
+    check_every_unit(cache, res, before=before, after=after)
+
+
 def test_in_place_budget_above_16384():
     """The hole fill has no budget limit of its own."""
     wl = gen.scaled(gen.WORKLOADS["tiny"], num_layers=1, num_kv_heads=2, batch=1, seq_len=20000, budget=17000)

@@ -45,8 +45,9 @@ def test_noalloc_matches_compress_on_two_calls():
     # in a row: a full 8-head layer (three kernels); a smaller ragged cache,
     # which must not be affected by the scores the first call left behind; a
     # cache of 4 units x 4096 keys, which takes the single-kernel step (one
-    # cluster per unit, scores in the shared array); and a paged cache
-    # compacted in place (three kernels, hole fill)
+    # cluster per unit, scores in the shared array); a paged cache compacted
+    # in place (three kernels, hole fill); and a paged cache whose rows move
+    # few keys (two kernels: the score, then the selection with the fill)
     cases = [
         (gen.WORKLOADS["qwen3_layer"], None, 1, tri.COMPACT_OUT_OF_PLACE, 3),
         (gen.scaled(gen.WORKLOADS["qwen3_ragged"], num_layers=2, num_kv_heads=4, batch=3, budget=300),
@@ -55,6 +56,8 @@ def test_noalloc_matches_compress_on_two_calls():
          tri.COMPACT_OUT_OF_PLACE, 1 if 4 * 16 <= sms else 3),
         (gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=4, batch=3, budget=2048,
                     spare_blocks_per_seq=1), [2176, 5000, 300], 4, tri.COMPACT_IN_PLACE_HOLEFILL, 3),
+        (gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=4, batch=3, budget=2048,
+                    spare_blocks_per_seq=1), [2176, 2100, 300], 5, tri.COMPACT_IN_PLACE_HOLEFILL, 2),
     ]
     for wl, lens, seed, mode, launches in cases:
         in_place = mode == tri.COMPACT_IN_PLACE_HOLEFILL
