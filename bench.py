@@ -443,7 +443,7 @@ def run_ours(args):
 
     # roofline of the dominant kernel (scoring; or the one-call step) and of the whole step
     peak, peak_kind = measured_hbm_peak()
-    score_ms = float(per1[:, 1].mean())
+    score_ms = float(per[:, 1].mean())
     score_bytes = keys * (KEY_BYTES + (4 if args.variant == "pos" else 0))   # + the positions read
     if args.path == "compress":
         score_bytes = keys * KEY_BYTES + moved * MOVE_BYTES

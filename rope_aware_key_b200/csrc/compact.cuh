@@ -32,31 +32,11 @@ namespace compact {
 #ifndef TRI_GATHER_BLOCKS_PER_SM
 #define TRI_GATHER_BLOCKS_PER_SM 6
 #endif
-// Stores of the gathered rows: 0 plain, 1 streaming (.cs), 2 with an L2
-// evict-first policy (the output is not read again by this step).
-#ifndef TRI_GATHER_STORE
-#define TRI_GATHER_STORE 0
-#endif
 
 constexpr int kGatherThreads = 256;
 constexpr int kGatherUnroll = TRI_GATHER_UNROLL;     // rows in flight per half-warp
 constexpr int kGatherBlocksPerSm = TRI_GATHER_BLOCKS_PER_SM;
 constexpr int kChunkRows = 32;                      // kept rows of one unit per warp and step
-
-__device__ __forceinline__ void st_out_v4(void* p, const uint4& x, uint64_t policy) {
-#if TRI_GATHER_STORE == 1
-  (void)policy;
-  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w)
-               : "memory");
-#elif TRI_GATHER_STORE == 2
-  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(x.x), "r"(x.y),
-               "r"(x.z), "r"(x.w), "l"(policy)
-               : "memory");
-#else
-  (void)policy;
-  *reinterpret_cast<uint4*>(p) = x;
-#endif
-}
 
 __device__ __forceinline__ void unit_coords(const Geom& g, int u, int* l, int* h, int* b) {
   *b = u % g.batch;
@@ -78,11 +58,6 @@ gather_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept,
   const int warp0 = (blockIdx.x * kGatherThreads + threadIdx.x) >> 5;
   const int nwarps = (gridDim.x * kGatherThreads) >> 5;
   const bool packed = g.layout != TRI_LAYOUT_PAGED;
-#if TRI_GATHER_STORE == 2
-  const uint64_t out_policy = policy_evict_first();
-#else
-  const uint64_t out_policy = 0;
-#endif
   for (int c = warp0; c < total_chunks; c += nwarps) {
     const int u = c / chunks_per_unit;
     const int j0 = (c - u * chunks_per_unit) * kChunkRows;
@@ -133,8 +108,8 @@ gather_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept,
       for (int q = 0; q < kGatherUnroll; ++q) {
         if (!live[q]) continue;
         const int64_t row = out0 + r0 + 2 * q + hw;
-        st_out_v4(kout + row * kD + l16 * 8, kx[q], out_policy);
-        st_out_v4(vout + row * kD + l16 * 8, vx[q], out_policy);
+        reinterpret_cast<uint4*>(kout + row * kD)[l16] = kx[q];
+        reinterpret_cast<uint4*>(vout + row * kD)[l16] = vx[q];
       }
     }
   }

@@ -281,6 +281,21 @@ score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float*
   const int r8 = lane >> 2;               // key within the warp's group of 8
   const int p = r8 & 1;                   // chunk-order rotation of odd keys
   const int row0 = warp * kRowsPerWarpPass + r8;
+  // PAGED rows interleave heads: row r is head r % H, and every row this
+  // lane reads has the same r % H (kGroup and the warp offset are multiples
+  // of 8, H | 8).  The lane's head, and for each pass the token of its row
+  // and that token's page within the tile, are the same in every tile.
+  int hp = 0, tok_it[kIters], page_it[kIters];
+  int64_t hoff = 0;
+  if (g.layout == TRI_LAYOUT_PAGED) {
+    hp = row0 % g.H;
+    hoff = hp * (static_cast<int64_t>(g.batch) * g.score_stride);
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+      tok_it[it] = (it * kGroup + row0) / g.H;
+      page_it[it] = tok_it[it] / g.block_size;
+    }
+  }
   float wv[32];
   int cur_lh = -1;
   int k = 0;
@@ -289,9 +304,7 @@ score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float*
     if (!mbar_wait_bounded(&full[s], n & 1)) break;
     const TileInfo T = info[s];
     if (T.rows > 0) {
-      // PAGED rows interleave heads: row r is head r % H, and every row this
-      // lane reads has the same r % H (kGroup and the warp offset are multiples of 8, H | 8).
-      const int h = T.paged ? (row0 % g.H) : 0;
+      const int h = T.paged ? hp : 0;
       const int lh = T.lh + h;
       if (lh != cur_lh) {
         load_w(w, lh, c, p, wv);
@@ -324,8 +337,8 @@ score_kernel(const __grid_constant__ Geom g, const float* __restrict__ w, float*
           const int r = it * kGroup + row0;
           if (c == 0 && r < T.rows) {
             if (T.paged) {
-              const int tok = r / g.H;
-              if (tok < T.tvalid && ((T.page_ok >> (tok / g.block_size)) & 1u)) T.out[h * T.head_step + tok] = a;
+              const int tok = tok_it[it];
+              if (tok < T.tvalid && ((T.page_ok >> page_it[it]) & 1u)) T.out[hoff + tok] = a;
             } else {
               T.out[r] = a;
             }

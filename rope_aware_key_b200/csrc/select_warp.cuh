@@ -11,10 +11,9 @@
 // longer than the budget (B + the window, e.g. 2048 + 128), and there are
 // thousands of them (layers x KV heads x sequences).  A CTA per row spends
 // its time in a chain of block barriers; a warp per row needs none, and with
-// 5 KB of shared memory per warp a CTA of 4 rows fits beside the scorer's
-// CTAs on an SM, so the selection of some layers can run while later layers
-// are scored.  Every decision is made on order-preserving integer keys of the
-// fp32 scores (NaN lowest), so the result is exact:
+// 5 KB of shared memory per warp, CTAs of 4 rows fill an SM seven at a time.
+// Every decision is made on order-preserving integer keys of the fp32 scores
+// (NaN lowest), so the result is exact:
 //  1. 256 evenly spaced scores of the row are sorted (a bitonic network in
 //     registers, 8 per lane); their ranks B/n * 256 -/+ (4 sigma + 8) from
 //     the top give two keys U >= L that bracket the B-th largest key for any
@@ -28,12 +27,13 @@
 //     candidates), a radix search over them (8-bit digits, a shared histogram
 //     per digit) gives it exactly: T, and `need`, how many keys equal to T
 //     are kept (the lowest-index ones);
-//  4. rows that evict few keys: the evicted indices (candidates below T, and
-//     ties past the first `need`) are listed in order, and the kept index of
-//     slot j is j + #{t : ev[t] - t <= j}, written four slots per lane, the
-//     lanes' groups interleaved so that every store covers 512 consecutive
-//     bytes.  Other rows: a second pass emits the kept keys in index order
-//     (ballots per 128-key chunk).
+//  4. rows that evict few keys: the evicted positions (candidates below T,
+//     and ties past the first `need`) are marked in a bitmap of the row, and
+//     a scan of its words' counts gives, for every kept position p, its slot
+//     p - #{evicted before p}; the kept indices are written position chunk by
+//     position chunk, with no second pass over the scores.  Other rows: a
+//     second pass emits the kept keys in index order (ballots per 128-key
+//     chunk).
 // If the check fails (a pathological order, heavy duplication), the radix
 // search runs over the whole row instead (one pass per digit).
 #pragma once
@@ -160,9 +160,10 @@ __device__ __forceinline__ uint32_t warp_radix_kth(Each each, uint32_t lo, uint3
 }
 
 // Select one row of n > B scores (n <= kWarpMaxRow); kept gets the B indices.
-// Returns the number of evicted keys when their indices are left in S.cand
-// (ascending), else -1.
-__device__ __forceinline__ int warp_select_row(const float* __restrict__ row, int n, int B, WarpScratch& S,
+// Returns true when the evicted positions are left as a bitmap in S.hist
+// (word w: positions 32 w .. 32 w + 31) with, in S.cand, the count of
+// evicted positions before each word.
+__device__ __forceinline__ bool warp_select_row(const float* __restrict__ row, int n, int B, WarpScratch& S,
                                                 int32_t* __restrict__ kept) {
   const int lane = threadIdx.x & 31;
   const int chunks = (n + 127) >> 7;               // warp-uniform
@@ -248,53 +249,61 @@ __device__ __forceinline__ int warp_select_row(const float* __restrict__ row, in
         },
         cmin, cmax, &need, S.hist);
     if (few) {
-      // 4. the evicted indices, ascending, written over the candidate keys
-      // already read: candidates below T, and ties past the first `need`
-      uint32_t ev = 0, ties = 0;
+      // 4. the evicted positions as a bitmap over the row (hist, 128 words):
+      // candidates below T, and ties past the first `need`
+      uint32_t* evb = S.hist;
+      __syncwarp();                                // the radix search is done with hist
+      reinterpret_cast<uint4*>(evb)[lane] = make_uint4(0u, 0u, 0u, 0u);
+      __syncwarp();
+      uint32_t ties = 0;
       for (int m0 = 0; m0 < nc; m0 += 32) {
         const int m = m0 + lane;
         const uint32_t k = m < nc ? S.cand[m] : 0xffffffffu;
-        const int32_t i = m < nc ? S.cidx[m] : 0;
         const bool tie = m < nc && k == T;
         const uint32_t tm = __ballot_sync(0xffffffffu, tie);
-        const bool out = m < nc && (k < T || (tie && ties + __popc(tm & lt) >= need));
-        const uint32_t om = __ballot_sync(0xffffffffu, out);
-        __syncwarp();                              // every lane has read its entry
-        if (out) S.cand[ev + __popc(om & lt)] = static_cast<uint32_t>(i);
-        ev += __popc(om);
+        if (m < nc && (k < T || (tie && ties + __popc(tm & lt) >= need))) {
+          const int i = S.cidx[m];
+          atomicOr(&evb[i >> 5], 1u << (i & 31));
+        }
         ties += __popc(tm);
       }
       __syncwarp();
-      const int E = static_cast<int>(ev);
-      if (lane == 0) TRI_CHECK(E == n - B);        // exactly B kept
-      const int32_t* evi = reinterpret_cast<const int32_t*>(S.cand);
-      // kept[j] = j + #{t : ev[t] - t <= j}: ev[t] - t, the kept keys below
-      // ev[t], never decreases, so each lane walks its slots in order
-      int e = 0;
-      int z = E > 0 ? evi[0] : 0x7fffffff;       // ev[e] - e, or past every slot
-      auto advance = [&](int j) {
-        while (z <= j) {
-          ++e;
-          z = e < E ? evi[e] - e : 0x7fffffff;
-        }
-      };
-      if ((reinterpret_cast<uintptr_t>(kept) & 15u) == 0 && (B & 3) == 0) {
-        for (int j = 4 * lane; j < B; j += 128) {  // groups of 4 slots, lanes interleaved
-          int o[4];
+      // evicted positions before each word (lane l owns words 4 l .. 4 l + 3),
+      // written over the candidate keys
+      const uint4 wv = reinterpret_cast<const uint4*>(evb)[lane];
+      const uint32_t c0 = __popc(wv.x), c1 = __popc(wv.y), c2 = __popc(wv.z), c3 = __popc(wv.w);
+      const uint32_t mine = c0 + c1 + c2 + c3;
+      uint32_t incl = mine;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            advance(j + q);
-            o[q] = j + q + e;
-          }
-          *reinterpret_cast<int4*>(kept + j) = make_int4(o[0], o[1], o[2], o[3]);
-        }
-      } else {
-        for (int j = lane; j < B; j += 32) {
-          advance(j);
-          kept[j] = j + e;
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t ex = incl - mine;
+      __syncwarp();                                // every lane has read its candidates
+      reinterpret_cast<uint4*>(S.cand)[lane] = make_uint4(ex, ex + c0, ex + c0 + c1, ex + c0 + c1 + c2);
+      __syncwarp();
+      const uint32_t evicted = __shfl_sync(0xffffffffu, incl, 31);
+      if (lane == 0) TRI_CHECK(evicted == static_cast<uint32_t>(n - B));      // exactly B kept
+      (void)evicted;
+      // kept position p goes to slot p - #{evicted before p}: each lane takes
+      // 4 consecutive positions of a 128-position chunk (one bitmap word)
+      const uint32_t* ebw = S.cand;
+      const int sh = (4 * lane) & 31;
+      for (int j = 0; j < chunks; ++j) {
+        const int p0 = 128 * j + 4 * lane;
+        const int w = p0 >> 5;
+        const uint32_t bits = evb[w];
+        uint32_t e = ebw[w] + __popc(bits & ((1u << sh) - 1u));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t ev = (bits >> (sh + q)) & 1u;
+          const int slot = p0 + q - static_cast<int>(e);
+          if (!ev && p0 + q < n && slot < B) kept[slot] = p0 + q;     // slot < B unless the count is off
+          e += ev;
         }
       }
-      return E;
+      return true;
     }
   } else {
     // whole-row search: every key of the row counts (NaN keys are 0, below
@@ -361,49 +370,54 @@ __device__ __forceinline__ int warp_select_row(const float* __restrict__ row, in
     slot += total;
   }
   if (lane == 0) TRI_CHECK(slot == static_cast<uint32_t>(B));         // exactly B kept
-  return -1;
+  return false;
 }
 
-// The in-place hole fill of a row from its evicted indices ev[0 .. E)
-// (ascending, n = B + E): the evicted positions below B are the holes, the
-// kept positions at or above B the movers, and the r-th mover goes to the
-// r-th hole -- the same moves as compact::holefill_unit_warp, found without
-// reading the kept list back.  `tail` (ceil(E / 32) words of shared memory)
-// marks the evicted positions at or above B.  Half a warp copies K and the
-// other half V, four rows in flight.
-__device__ __forceinline__ void warp_fill_row(const Geom& g, int l, int h, int b, const int32_t* ev, int E, int B,
-                                              int n, uint32_t* tail, uint16_t* k, uint16_t* v) {
+// The in-place hole fill of a row from the bitmap of its evicted positions
+// (evb, with ebw[w] the evicted positions before word w; n - B of them):
+// the evicted positions below B are the holes, the kept positions at or
+// above B the movers, and the r-th mover goes to the r-th hole -- the same
+// moves as compact::holefill_unit_warp, found without reading the kept list
+// back.  The holes are listed in `holes` (n - B ints of shared memory), in
+// order.  Half a warp copies K and the other half V, four rows in flight.
+__device__ __forceinline__ void warp_fill_row(const Geom& g, int l, int h, int b, const uint32_t* evb,
+                                              const uint32_t* ebw, int B, int n, int32_t* holes, uint16_t* k,
+                                              uint16_t* v) {
   const int lane = threadIdx.x & 31, l16 = lane & 15, hw = lane >> 4;
-  const uint32_t lt = (1u << lane) - 1u;
-  if (E != n - B) {                                // not a list of n - B evictions
-    if (lane == 0) flag(TRI_DEVFLAG_BAD_KEPT);
-    return;
-  }
-  int m = 0;                                       // holes: evicted positions below B
-  for (int t0 = 0; t0 < E; t0 += 32) m += __popc(__ballot_sync(0xffffffffu, t0 + lane < E && ev[t0 + lane] < B));
-  const int tw = (E + 31) >> 5;
-  for (int w = lane; w < tw; w += 32) tail[w] = 0u;
-  __syncwarp();
-  for (int t = m + lane; t < E; t += 32) {
-    const int p = ev[t] - B;
-    atomicOr(&tail[p >> 5], 1u << (p & 31));
+  const int wb = B >> 5, sb = B & 31;
+  const int m = static_cast<int>(ebw[wb] + __popc(evb[wb] & ((1u << sb) - 1u)));   // holes below B
+  for (int w = lane; w < wb + (sb != 0); w += 32) {
+    uint32_t bits = evb[w];
+    if (w == wb) bits &= (1u << sb) - 1u;          // the word that straddles B
+    uint32_t idx = ebw[w];
+    while (bits) {
+      holes[idx++] = 32 * w + __ffs(bits) - 1;
+      bits &= bits - 1u;
+    }
   }
   __syncwarp();
-  uint16_t* const src_base = hw ? v : k;
-  int r0 = 0;
-  for (int c0 = 0; c0 < E; c0 += 32) {             // tail positions B + c0 + lane
-    const bool mv = c0 + lane < E && !((tail[c0 >> 5] >> lane) & 1u);
-    const uint32_t mm = __ballot_sync(0xffffffffu, mv);
+  uint16_t* const base = hw ? v : k;
+  int movers = 0;
+  for (int p0 = B; p0 < n; p0 += 32) {             // positions p0 + lane
+    const int p = p0 + lane;
+    bool mv = false;
+    int r = 0;
+    if (p < n) {
+      const uint32_t bits = evb[p >> 5];
+      const uint32_t below = bits & ((1u << (p & 31)) - 1u);
+      // kept positions in [B, p): (p - B) minus the evicted ones
+      r = (p - B) - (static_cast<int>(ebw[p >> 5] + __popc(below)) - m);
+      mv = ((bits >> (p & 31)) & 1u) == 0u && r < m;       // r < m unless the counts are off
+    }
     bool ok = true;
     int64_t es = 0, ed = 0;
     if (mv) {
-      const int r = r0 + __popc(mm & lt);          // r < m
-      es = row_elem(g, l, h, b, B + c0 + lane, &ok);
-      ed = row_elem(g, l, h, b, ev[r], &ok);
+      es = row_elem(g, l, h, b, p, &ok);
+      ed = row_elem(g, l, h, b, holes[r], &ok);    // r < m
       if (!ok) flag(TRI_DEVFLAG_BAD_PAGE);
     }
+    movers += __popc(__ballot_sync(0xffffffffu, mv));
     uint32_t rem = __ballot_sync(0xffffffffu, mv && ok);
-    r0 += __popc(mm);
     while (rem) {                                  // warp-uniform
       int sl[4];
 #pragma unroll
@@ -418,14 +432,14 @@ __device__ __forceinline__ void warp_fill_row(const Geom& g, int l, int h, int b
         const int from = sl[i] < 0 ? 0 : sl[i];
         const int64_t s_i = __shfl_sync(0xffffffffu, es, from);
         d[i] = __shfl_sync(0xffffffffu, ed, from);
-        if (sl[i] >= 0) x[i] = ld_nc_v4(src_base + s_i + l16 * 8);
+        if (sl[i] >= 0) x[i] = ld_nc_v4(base + s_i + l16 * 8);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        if (sl[i] >= 0) reinterpret_cast<uint4*>(src_base + d[i])[l16] = x[i];
+        if (sl[i] >= 0) reinterpret_cast<uint4*>(base + d[i])[l16] = x[i];
     }
   }
-  if (lane == 0) TRI_CHECK(r0 == m);               // as many movers as holes
+  if (lane == 0) TRI_CHECK(movers == m);           // as many movers as holes
 }
 
 // One warp per unit, units [blockIdx.x * kWarpRows, ...): rows of at most
@@ -450,14 +464,13 @@ __global__ void __launch_bounds__(kWarpThreads) select_warp_kernel(const __grid_
     for (int i = lane; i < n; i += 32) kept[i] = i;
     return;
   }
-  const int E = warp_select_row(a.scores + static_cast<int64_t>(u) * g.score_stride, n, B, scratch[w], kept);
+  const bool bitmap = warp_select_row(a.scores + static_cast<int64_t>(u) * g.score_stride, n, B, scratch[w], kept);
   if constexpr (FILL) {
     int l, h, b_;
     compact::unit_coords(g, u, &l, &h, &b_);       // b_ == b
-    __syncwarp();                                  // the kept list (global) and the evicted list (shared)
-    if (E >= 0)
-      warp_fill_row(g, l, h, b, reinterpret_cast<const int32_t*>(scratch[w].cand), E, B, n, scratch[w].hist,
-                    k, v);
+    __syncwarp();                                  // the kept list (global) and the bitmap (shared)
+    if (bitmap && n - B <= kWarpCand)
+      warp_fill_row(g, l, h, b, scratch[w].hist, scratch[w].cand, B, n, scratch[w].cidx, k, v);
     else
       compact::holefill_unit_warp(g, kept, B, n, l, h, b, k, v);
   }

@@ -108,3 +108,36 @@ def test_gpus_flag_relaunches_one_process_per_gpu(monkeypatch):
     assert "--nproc-per-node=4" in cmd and cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
     assert cmd[-6:] == ["--gpus", "4", "--steps", "7", "--warmup", "3"]
     assert cmd[-7].endswith("bench.py") and seen["timeout"] > 0
+
+
+def test_bench_functions_read_only_names_they_can_see():
+    """Every name a top-level function of bench.py reads is bound in it (or in
+    a function nested in it), at module level, or is a builtin: the GPU legs
+    cannot run here, so a stale name in one of them would only show on a GPU."""
+    import ast
+    import builtins
+    tree = ast.parse(open(os.path.join(ROOT, "bench.py")).read())
+    module = set(dir(builtins)) | {"__file__"}
+    for node in tree.body:
+        for n in ast.walk(node) if isinstance(node, (ast.Assign, ast.AnnAssign, ast.Import, ast.ImportFrom)) else []:
+            if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Store):
+                module.add(n.id)
+            elif isinstance(n, ast.alias):
+                module.add((n.asname or n.name).split(".")[0])
+        if isinstance(node, (ast.FunctionDef, ast.ClassDef)):
+            module.add(node.name)
+    missing = []
+    for fn in (n for n in tree.body if isinstance(n, ast.FunctionDef)):
+        seen = set(module)
+        for n in ast.walk(fn):
+            if isinstance(n, ast.Name) and not isinstance(n.ctx, ast.Load):
+                seen.add(n.id)
+            elif isinstance(n, (ast.arg, ast.FunctionDef)):
+                seen.add(n.arg if isinstance(n, ast.arg) else n.name)
+            elif isinstance(n, ast.alias):
+                seen.add((n.asname or n.name).split(".")[0])
+            elif isinstance(n, ast.ExceptHandler) and n.name:
+                seen.add(n.name)
+        missing += [(fn.name, n.lineno, n.id) for n in ast.walk(fn)
+                    if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Load) and n.id not in seen]
+    assert not missing, missing
