@@ -14,10 +14,11 @@
 // 5 KB of shared memory per warp, CTAs of 4 rows fill an SM seven at a time.
 // Every decision is made on order-preserving integer keys of the fp32 scores
 // (NaN lowest), so the result is exact:
-//  1. 256 evenly spaced scores of the row are sorted (a bitonic network in
-//     registers, 8 per lane); their ranks B/n * 256 -/+ (4 sigma + 8) from
-//     the top give two keys U >= L that bracket the B-th largest key for any
-//     but a pathological order of the scores;
+//  1. of 256 evenly spaced scores of the row (8 per lane), the ones at ranks
+//     B/n * 256 -/+ (4 sigma + 8) from the top give two keys U >= L that
+//     bracket the B-th largest key for any but a pathological order of the
+//     scores; each is found by a bitwise search over the samples' key range
+//     (a step counts the samples below a trial key: one warp reduction);
 //  2. one pass over the row counts the keys above U (all kept) and gathers
 //     the keys in [L, U] into a candidate buffer (the comparisons are made
 //     on the floats; the candidates are stored as keys).  When L would fall
@@ -38,6 +39,8 @@
 // search runs over the whole row instead (one pass per digit).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "compact.cuh"
 #include "select.cuh"
@@ -51,9 +54,10 @@ constexpr int kWarpSamples = 256;                  // 8 per lane
 constexpr int kWarpCand = 512;
 constexpr int kWarpMaxRow = 4096;
 constexpr int kWarpBatch = 4;                     // chunks whose loads are in flight together
+constexpr int kWarpCtasPerSm = 7;                 // register budget: 72 per thread
 
 struct __align__(16) WarpScratch {
-  uint32_t hist[256];                              // the sorted samples, then the radix digits
+  uint32_t hist[256];                              // the radix digits, then the evicted bitmap
   uint32_t cand[kWarpCand];                        // candidate keys (later: the evicted indices)
   int32_t cidx[kWarpCand];                         // their indices (rows that evict few keys)
 };
@@ -71,35 +75,21 @@ __device__ __forceinline__ float4 row_chunk(const float* __restrict__ row, int n
   return x;
 }
 
-// Ascending bitonic sort of 256 keys, lane l holding elements 8 l .. 8 l + 7.
-__device__ __forceinline__ void warp_sort256(uint32_t (&x)[8]) {
-  const int lane = threadIdx.x & 31;
+// The k-th smallest (1 <= k <= 256) of the 256 keys the lanes hold, 8 each,
+// whose range is [lo, hi]: the largest t in [lo, hi] with fewer than k keys
+// below it (the count never decreases with t), found bit by bit of t - lo.
+__device__ __forceinline__ uint32_t warp_kth_smallest(const uint32_t (&x)[8], uint32_t lo, uint32_t hi, uint32_t k) {
+  uint32_t t = lo;                                 // fewer than k keys below t
+  const uint32_t span = hi - lo;
+  for (int bit = span ? 31 - __clz(span) : -1; bit >= 0; --bit) {
+    const uint64_t trial = uint64_t{t} + (uint64_t{1} << bit);
+    if (trial > hi) continue;                      // warp-uniform
+    uint32_t c = 0;
 #pragma unroll
-  for (int kb = 1; kb <= 8; ++kb) {
-    const int k = 1 << kb;
-#pragma unroll
-    for (int jb = kb - 1; jb >= 0; --jb) {
-      const int j = 1 << jb;
-      if (j >= 8) {                                // the partner sits in lane ^ (j / 8), same slot
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int idx = 8 * lane + e;
-          const uint32_t y = __shfl_xor_sync(0xffffffffu, x[e], j >> 3);
-          const bool ascending = (idx & k) == 0, lower = (idx & j) == 0;
-          x[e] = lower == ascending ? min(x[e], y) : max(x[e], y);
-        }
-      } else {                                     // both elements in this lane
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (e & j) continue;
-          const bool ascending = ((8 * lane + e) & k) == 0;
-          const uint32_t a = x[e], b = x[e ^ j];
-          x[e] = ascending ? min(a, b) : max(a, b);
-          x[e ^ j] = ascending ? max(a, b) : min(a, b);
-        }
-      }
-    }
+    for (int e = 0; e < 8; ++e) c += x[e] < static_cast<uint32_t>(trial);
+    if (__reduce_add_sync(0xffffffffu, c) < k) t = static_cast<uint32_t>(trial);
   }
+  return t;
 }
 
 // The need-th largest (need >= 1) of the keys in [lo, hi] among the keys the
@@ -171,19 +161,24 @@ __device__ __forceinline__ bool warp_select_row(const float* __restrict__ row, i
   const uint32_t lt = (1u << lane) - 1u;
   auto valid = [&](int j, int q) { return j < full || 128 * j + 4 * lane + q < n; };
 
-  // 1. the bracket from the sorted sample
+  // 1. the bracket from the sample: two of its order statistics
   uint32_t x[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) x[e] = order_key(__ldg(row + (((8 * lane + e) * n) >> 8)));
-  warp_sort256(x);
-  reinterpret_cast<uint4*>(S.hist)[2 * lane] = make_uint4(x[0], x[1], x[2], x[3]);
-  reinterpret_cast<uint4*>(S.hist)[2 * lane + 1] = make_uint4(x[4], x[5], x[6], x[7]);
-  __syncwarp();
+  uint32_t kmin = x[0], kmax = x[0];
+#pragma unroll
+  for (int e = 1; e < 8; ++e) {
+    kmin = min(kmin, x[e]);
+    kmax = max(kmax, x[e]);
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
   const float r = static_cast<float>(B) * kWarpSamples / static_cast<float>(n);
   const float delta = 4.f * sqrtf(r * (1.f - r / kWarpSamples)) + 8.f;
   const int r_hi = static_cast<int>(floorf(r - delta)), r_lo = static_cast<int>(ceilf(r + delta));
-  const uint32_t U = r_hi >= 1 ? S.hist[kWarpSamples - r_hi] : 0xffffffffu;
-  const uint32_t L0 = r_lo <= kWarpSamples ? S.hist[kWarpSamples - r_lo] : 0u;
+  // the r_hi-th and r_lo-th largest samples (ranks counted from the top)
+  const uint32_t U = r_hi >= 1 ? warp_kth_smallest(x, kmin, kmax, kWarpSamples + 1 - r_hi) : 0xffffffffu;
+  const uint32_t L0 = r_lo <= kWarpSamples ? warp_kth_smallest(x, kmin, kmax, kWarpSamples + 1 - r_lo) : 0u;
   // rows that evict few keys (no lower bound; also when the bound is NaN's key)
   const bool few = L0 == 0u;
   // the same bounds as floats: above U is v > uf (NaN never is), in [L, U] is
@@ -191,58 +186,76 @@ __device__ __forceinline__ bool warp_select_row(const float* __restrict__ row, i
   const float uf = U == 0xffffffffu ? INFINITY : key_value(U);
   const float lf = key_value(L0);
 
-  // 2. one pass: count the keys above U, gather those in [L, U]; the loads of
-  // kWarpBatch chunks are issued before any of them is used
-  uint32_t above = 0, base = 0, cmin = 0xffffffffu, cmax = 0u;
-  for (int j0 = 0; j0 < chunks; j0 += kWarpBatch) {
-    float4 xb[kWarpBatch];
+  // 2. one pass gathers the candidates, in index order: every key up to U
+  // (rows that evict few keys: all the others are kept, so `above` is n minus
+  // the candidates), else the keys in [L, U], counting those above U.  The
+  // candidates are stored as float bits (with their indices when few) and
+  // turned into keys afterwards; the loads of kWarpBatch chunks are issued
+  // before any of them is used.
+  uint32_t base = 0, upc = 0;
+  auto collect = [&](auto few_c) {
+    constexpr bool kFew = decltype(few_c)::value;
+    for (int j0 = 0; j0 < chunks; j0 += kWarpBatch) {
+      float4 xb[kWarpBatch];
 #pragma unroll
-    for (int i = 0; i < kWarpBatch; ++i)
-      if (j0 + i < chunks) xb[i] = row_chunk(row, n, full, j0 + i, lane);
+      for (int i = 0; i < kWarpBatch; ++i)
+        if (j0 + i < chunks) xb[i] = row_chunk(row, n, full, j0 + i, lane);
 #pragma unroll
-    for (int i = 0; i < kWarpBatch; ++i) {
-      const int j = j0 + i;
-      if (j >= chunks) break;                      // warp-uniform
-      const float v[4] = {xb[i].x, xb[i].y, xb[i].z, xb[i].w};
-      bool in[4];
-      uint32_t before = 0, total = 0;
+      for (int i = 0; i < kWarpBatch; ++i) {
+        const int j = j0 + i;
+        if (j >= chunks) break;                    // warp-uniform
+        const float v[4] = {xb[i].x, xb[i].y, xb[i].z, xb[i].w};
+        bool in[4];
+        uint32_t cnt = 0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const bool vq = valid(j, q);
-        const bool up = v[q] > uf;
-        above += vq && up;
-        in[q] = vq && !up && (few || v[q] >= lf);
-        const uint32_t m = __ballot_sync(0xffffffffu, in[q]);
-        before += __popc(m & lt);
-        total += __popc(m);
-      }
-      uint32_t pos = base + before;                // index order: lanes, then q within a lane
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (in[q]) {
-          if (pos < static_cast<uint32_t>(kWarpCand)) {
-            const uint32_t k = order_key(v[q]);
-            S.cand[pos] = k;
-            if (few) S.cidx[pos] = 128 * j + 4 * lane + q;
-            cmin = min(cmin, k);
-            cmax = max(cmax, k);
-          }
-          ++pos;
+        for (int q = 0; q < 4; ++q) {
+          const bool vq = valid(j, q);
+          const bool up = v[q] > uf;
+          in[q] = vq && !up && (kFew || v[q] >= lf);
+          if constexpr (!kFew) upc += __popc(__ballot_sync(0xffffffffu, vq && up));
+          cnt += in[q];
         }
-      base += total;
+        // index order is lanes, then q: the lane's first slot is the
+        // candidates of the lanes before it (cnt <= 4, summed by bit planes)
+        const uint32_t b0 = __ballot_sync(0xffffffffu, cnt & 1u), b1 = __ballot_sync(0xffffffffu, cnt & 2u),
+                       b2 = __ballot_sync(0xffffffffu, cnt & 4u);
+        uint32_t pos = base + __popc(b0 & lt) + 2u * __popc(b1 & lt) + 4u * __popc(b2 & lt);
+        base += __popc(b0) + 2u * __popc(b1) + 4u * __popc(b2);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (in[q]) {
+            if (pos < static_cast<uint32_t>(kWarpCand)) {
+              S.cand[pos] = __float_as_uint(v[q]);
+              if (kFew) S.cidx[pos] = 128 * j + 4 * lane + q;
+            }
+            ++pos;
+          }
+      }
     }
-  }
-  above = __reduce_add_sync(0xffffffffu, above);
+  };
+  if (few)
+    collect(std::true_type());
+  else
+    collect(std::false_type());
+  const uint32_t above = few ? static_cast<uint32_t>(n) - base : upc;
   const bool ok = above < static_cast<uint32_t>(B) && static_cast<uint32_t>(B) <= above + base &&
                   base <= static_cast<uint32_t>(kWarpCand);
   uint32_t T, need;
   if (ok) {
     __syncwarp();
+    const int nc = static_cast<int>(base);
+    uint32_t cmin = 0xffffffffu, cmax = 0u;
+    for (int m = lane; m < nc; m += 32) {
+      const uint32_t k = order_key(__uint_as_float(S.cand[m]));
+      S.cand[m] = k;
+      cmin = min(cmin, k);
+      cmax = max(cmax, k);
+    }
     cmin = __reduce_min_sync(0xffffffffu, cmin);
     cmax = __reduce_max_sync(0xffffffffu, cmax);
+    __syncwarp();
     need = static_cast<uint32_t>(B) - above;       // 1 <= need <= base
     // 3. the exact threshold among the candidates; need becomes the ties to keep
-    const int nc = static_cast<int>(base);
     T = warp_radix_kth(
         [&](auto fn) {
           for (int m = lane; m < nc; m += 32) fn(S.cand[m]);
@@ -379,10 +392,18 @@ __device__ __forceinline__ bool warp_select_row(const float* __restrict__ row, i
 // above B the movers, and the r-th mover goes to the r-th hole -- the same
 // moves as compact::holefill_unit_warp, found without reading the kept list
 // back.  The holes are listed in `holes` (n - B ints of shared memory), in
-// order.  Half a warp copies K and the other half V, four rows in flight.
+// order.  The tail [B, n) is taken 128 positions at a time: every lane ranks
+// the movers among its 4 positions and, for a paged cache, looks up the
+// source and destination pages (all lookups of the chunk in flight at once),
+// into `lists` (3 x 128 ints of shared memory); then the chunk's rows are
+// copied 8 at a time, one 16-byte load per lane and row (lanes 0-15 K,
+// 16-31 V), all 8 loads in flight before the stores.
+constexpr int kFillChunk = 128;
+constexpr int kFillBatch = 8;
+
 __device__ __forceinline__ void warp_fill_row(const Geom& g, int l, int h, int b, const uint32_t* evb,
-                                              const uint32_t* ebw, int B, int n, int32_t* holes, uint16_t* k,
-                                              uint16_t* v) {
+                                              const uint32_t* ebw, int B, int n, int32_t* holes, int32_t* lists,
+                                              uint16_t* k, uint16_t* v) {
   const int lane = threadIdx.x & 31, l16 = lane & 15, hw = lane >> 4;
   const int wb = B >> 5, sb = B & 31;
   const int m = static_cast<int>(ebw[wb] + __popc(evb[wb] & ((1u << sb) - 1u)));   // holes below B
@@ -395,51 +416,69 @@ __device__ __forceinline__ void warp_fill_row(const Geom& g, int l, int h, int b
       bits &= bits - 1u;
     }
   }
-  __syncwarp();
+  const bool paged = g.layout == TRI_LAYOUT_PAGED;
+  const int32_t* table = paged ? g.block_table + static_cast<int64_t>(b) * g.max_blocks : nullptr;
+  int32_t* msrc = lists;                           // mover positions of the chunk, in mover order
+  int32_t* sblk = lists + kFillChunk;              // PAGED: their pages
+  int32_t* dblk = lists + 2 * kFillChunk;          // PAGED: their holes' pages
   uint16_t* const base = hw ? v : k;
-  int movers = 0;
-  for (int p0 = B; p0 < n; p0 += 32) {             // positions p0 + lane
-    const int p = p0 + lane;
-    bool mv = false;
-    int r = 0;
-    if (p < n) {
-      const uint32_t bits = evb[p >> 5];
-      const uint32_t below = bits & ((1u << (p & 31)) - 1u);
-      // kept positions in [B, p): (p - B) minus the evicted ones
-      r = (p - B) - (static_cast<int>(ebw[p >> 5] + __popc(below)) - m);
-      mv = ((bits >> (p & 31)) & 1u) == 0u && r < m;       // r < m unless the counts are off
+  // element offset of position i of this unit, given its page (PAGED)
+  auto elem = [&](int i, int blk) -> int64_t {
+    if (!paged) {
+      bool ok = true;
+      return row_elem(g, l, h, b, i, &ok);
     }
-    bool ok = true;
-    int64_t es = 0, ed = 0;
-    if (mv) {
-      es = row_elem(g, l, h, b, p, &ok);
-      ed = row_elem(g, l, h, b, holes[r], &ok);    // r < m
-      if (!ok) flag(TRI_DEVFLAG_BAD_PAGE);
-    }
-    movers += __popc(__ballot_sync(0xffffffffu, mv));
-    uint32_t rem = __ballot_sync(0xffffffffu, mv && ok);
-    while (rem) {                                  // warp-uniform
-      int sl[4];
+    return l * g.sL + static_cast<int64_t>(blk) * g.sB + static_cast<int64_t>((i % g.block_size) * g.H + h) * kD;
+  };
+  int r0 = 0;                                      // movers of the chunks before
+  for (int c0 = B; c0 < n; c0 += kFillChunk) {
+    __syncwarp();                                  // the holes, or the previous chunk's copies, are done
+    int mine = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        sl[i] = rem ? __ffs(rem) - 1 : -1;
-        rem &= rem - 1u;
+    for (int q = 0; q < 4; ++q) {
+      const int p = c0 + 4 * lane + q;
+      if (p < n) {
+        const uint32_t bits = evb[p >> 5];
+        // kept positions in [B, p): (p - B) minus the evicted ones
+        const int r = (p - B) - (static_cast<int>(ebw[p >> 5] + __popc(bits & ((1u << (p & 31)) - 1u))) - m);
+        const int i = r - r0;                      // < kFillChunk, and r < m, unless the counts are off
+        if (((bits >> (p & 31)) & 1u) == 0u && r < m && i < kFillChunk) {
+          msrc[i] = p;
+          if (paged) {
+            sblk[i] = table[p / g.block_size];
+            dblk[i] = table[holes[r] / g.block_size];
+          }
+          ++mine;
+        }
       }
-      uint4 x[4];
-      int64_t d[4];
+    }
+    const int mc = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<uint32_t>(mine)));
+    __syncwarp();
+    for (int i0 = 0; i0 < mc; i0 += kFillBatch) {
+      uint4 x[kFillBatch];
+      bool live[kFillBatch];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int from = sl[i] < 0 ? 0 : sl[i];
-        const int64_t s_i = __shfl_sync(0xffffffffu, es, from);
-        d[i] = __shfl_sync(0xffffffffu, ed, from);
-        if (sl[i] >= 0) x[i] = ld_nc_v4(base + s_i + l16 * 8);
+      for (int t = 0; t < kFillBatch; ++t) {
+        const int i = i0 + t;
+        live[t] = i < mc;
+        if (!live[t]) continue;
+        if (paged && (static_cast<unsigned>(sblk[i]) >= static_cast<unsigned>(g.num_blocks) ||
+                      static_cast<unsigned>(dblk[i]) >= static_cast<unsigned>(g.num_blocks))) {
+          live[t] = false;
+          if (lane == 0) flag(TRI_DEVFLAG_BAD_PAGE);
+          continue;
+        }
+        x[t] = ld_nc_v4(base + elem(msrc[i], paged ? sblk[i] : 0) + l16 * 8);
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (sl[i] >= 0) reinterpret_cast<uint4*>(base + d[i])[l16] = x[i];
+      for (int t = 0; t < kFillBatch; ++t) {
+        const int i = i0 + t;
+        if (live[t]) reinterpret_cast<uint4*>(base + elem(holes[r0 + i], paged ? dblk[i] : 0))[l16] = x[t];
+      }
     }
+    r0 += mc;
   }
-  if (lane == 0) TRI_CHECK(movers == m);           // as many movers as holes
+  if (lane == 0) TRI_CHECK(r0 == m);               // as many movers as holes
 }
 
 // One warp per unit, units [blockIdx.x * kWarpRows, ...): rows of at most
@@ -447,7 +486,7 @@ __device__ __forceinline__ void warp_fill_row(const Geom& g, int l, int h, int b
 // in-place hole fill of each row follows its selection in the same warp
 // (k, v: the cache), for launches whose rows move few keys.
 template <bool FILL>
-__global__ void __launch_bounds__(kWarpThreads) select_warp_kernel(const __grid_constant__ Geom g, const Args a,
+__global__ void __launch_bounds__(kWarpThreads, kWarpCtasPerSm) select_warp_kernel(const __grid_constant__ Geom g, const Args a,
                                                                    int units, uint16_t* k, uint16_t* v) {
   extern __shared__ float4 select_warp_dyn[];
   WarpScratch* scratch = reinterpret_cast<WarpScratch*>(select_warp_dyn);
@@ -470,7 +509,8 @@ __global__ void __launch_bounds__(kWarpThreads) select_warp_kernel(const __grid_
     compact::unit_coords(g, u, &l, &h, &b_);       // b_ == b
     __syncwarp();                                  // the kept list (global) and the bitmap (shared)
     if (bitmap && n - B <= kWarpCand)
-      warp_fill_row(g, l, h, b, scratch[w].hist, scratch[w].cand, B, n, scratch[w].cidx, k, v);
+      warp_fill_row(g, l, h, b, scratch[w].hist, scratch[w].cand, B, n, scratch[w].cidx,
+                    reinterpret_cast<int32_t*>(scratch[w].cand) + 128, k, v);
     else
       compact::holefill_unit_warp(g, kept, B, n, l, h, b, k, v);
   }
