@@ -19,6 +19,7 @@ struct Geom {
   int layout;                // tri_layout
   int L, H, batch;
   int block_size, max_blocks, num_blocks;
+  int block_shift;           // PAGED: log2(block_size) when it is a power of two, else -1
   int pages_per_tile;        // PAGED: consecutive pages of a sequence scored as one tile
   int64_t sL, sH, sB;        // layer / head / (seq for CONTIG, page for PAGED) strides, elements
   int64_t score_stride;      // floats per score row
@@ -60,13 +61,14 @@ __device__ __forceinline__ int64_t row_elem(const Geom& g, int l, int h, int b, 
     return l * g.sL + h * g.sH + b * g.sB + static_cast<int64_t>(i) * kD;
   if (g.layout == TRI_LAYOUT_RAGGED)
     return l * g.sL + h * g.sH + (static_cast<int64_t>(g.start[b]) + i) * kD;
-  int blk = g.block_table[static_cast<int64_t>(b) * g.max_blocks + i / g.block_size];
+  const int pg = g.block_shift >= 0 ? i >> g.block_shift : i / g.block_size;
+  const int blk = g.block_table[static_cast<int64_t>(b) * g.max_blocks + pg];
   if (static_cast<unsigned>(blk) >= static_cast<unsigned>(g.num_blocks)) {
     *ok = false;
     return 0;
   }
   return l * g.sL + static_cast<int64_t>(blk) * g.sB +
-         static_cast<int64_t>((i % g.block_size) * g.H + h) * kD;
+         static_cast<int64_t>((i - pg * g.block_size) * g.H + h) * kD;
 }
 
 // Largest b in [0, batch) with prefix[b] <= r (prefix non-decreasing, prefix[0] = 0).

@@ -57,9 +57,9 @@ constexpr int kWarpBatch = 4;                     // chunks whose loads are in f
 constexpr int kWarpCtasPerSm = 7;                 // register budget: 72 per thread
 
 struct __align__(16) WarpScratch {
-  uint32_t hist[256];                              // the radix digits, then the evicted bitmap
-  uint32_t cand[kWarpCand];                        // candidate keys (later: the evicted indices)
-  int32_t cidx[kWarpCand];                         // their indices (rows that evict few keys)
+  uint32_t hist[256];                              // the radix digits; then the evicted bitmap and its word counts
+  uint32_t cand[kWarpCand];                        // candidate keys (later: the fill's row offsets)
+  int32_t cidx[kWarpCand];                         // their indices (rows that evict few keys; later: the holes)
 };
 constexpr size_t kWarpSmemBytes = kWarpRows * sizeof(WarpScratch);
 
@@ -151,7 +151,7 @@ __device__ __forceinline__ uint32_t warp_radix_kth(Each each, uint32_t lo, uint3
 
 // Select one row of n > B scores (n <= kWarpMaxRow); kept gets the B indices.
 // Returns true when the evicted positions are left as a bitmap in S.hist
-// (word w: positions 32 w .. 32 w + 31) with, in S.cand, the count of
+// (word w: positions 32 w .. 32 w + 31) with, in S.hist + 128, the count of
 // evicted positions before each word.
 __device__ __forceinline__ bool warp_select_row(const float* __restrict__ row, int n, int B, WarpScratch& S,
                                                 int32_t* __restrict__ kept) {
@@ -282,7 +282,7 @@ __device__ __forceinline__ bool warp_select_row(const float* __restrict__ row, i
       }
       __syncwarp();
       // evicted positions before each word (lane l owns words 4 l .. 4 l + 3),
-      // written over the candidate keys
+      // in the second half of hist
       const uint4 wv = reinterpret_cast<const uint4*>(evb)[lane];
       const uint32_t c0 = __popc(wv.x), c1 = __popc(wv.y), c2 = __popc(wv.z), c3 = __popc(wv.w);
       const uint32_t mine = c0 + c1 + c2 + c3;
@@ -294,14 +294,14 @@ __device__ __forceinline__ bool warp_select_row(const float* __restrict__ row, i
       }
       const uint32_t ex = incl - mine;
       __syncwarp();                                // every lane has read its candidates
-      reinterpret_cast<uint4*>(S.cand)[lane] = make_uint4(ex, ex + c0, ex + c0 + c1, ex + c0 + c1 + c2);
+      reinterpret_cast<uint4*>(S.hist + 128)[lane] = make_uint4(ex, ex + c0, ex + c0 + c1, ex + c0 + c1 + c2);
       __syncwarp();
       const uint32_t evicted = __shfl_sync(0xffffffffu, incl, 31);
       if (lane == 0) TRI_CHECK(evicted == static_cast<uint32_t>(n - B));      // exactly B kept
       (void)evicted;
       // kept position p goes to slot p - #{evicted before p}: each lane takes
       // 4 consecutive positions of a 128-position chunk (one bitmap word)
-      const uint32_t* ebw = S.cand;
+      const uint32_t* ebw = S.hist + 128;
       const int sh = (4 * lane) & 31;
       for (int j = 0; j < chunks; ++j) {
         const int p0 = 128 * j + 4 * lane;
@@ -392,17 +392,17 @@ __device__ __forceinline__ bool warp_select_row(const float* __restrict__ row, i
 // above B the movers, and the r-th mover goes to the r-th hole -- the same
 // moves as compact::holefill_unit_warp, found without reading the kept list
 // back.  The holes are listed in `holes` (n - B ints of shared memory), in
-// order.  The tail [B, n) is taken 128 positions at a time: every lane ranks
-// the movers among its 4 positions and, for a paged cache, looks up the
-// source and destination pages (all lookups of the chunk in flight at once),
-// into `lists` (3 x 128 ints of shared memory); then the chunk's rows are
-// copied 8 at a time, one 16-byte load per lane and row (lanes 0-15 K,
-// 16-31 V), all 8 loads in flight before the stores.
+// order.  The tail [B, n) is taken kFillChunk positions at a time: every lane
+// ranks the movers among its 4 positions and computes their source and
+// destination offsets (for a paged cache all the chunk's page lookups are in
+// flight at once) into `offs` (2 x kFillChunk int64 of shared memory); then
+// the chunk's rows are copied kFillBatch at a time, one 16-byte load per
+// lane and row (lanes 0-15 K, 16-31 V), all loads in flight before the stores.
 constexpr int kFillChunk = 128;
 constexpr int kFillBatch = 8;
 
 __device__ __forceinline__ void warp_fill_row(const Geom& g, int l, int h, int b, const uint32_t* evb,
-                                              const uint32_t* ebw, int B, int n, int32_t* holes, int32_t* lists,
+                                              const uint32_t* ebw, int B, int n, int32_t* holes, int64_t* offs,
                                               uint16_t* k, uint16_t* v) {
   const int lane = threadIdx.x & 31, l16 = lane & 15, hw = lane >> 4;
   const int wb = B >> 5, sb = B & 31;
@@ -416,64 +416,57 @@ __device__ __forceinline__ void warp_fill_row(const Geom& g, int l, int h, int b
       bits &= bits - 1u;
     }
   }
-  const bool paged = g.layout == TRI_LAYOUT_PAGED;
-  const int32_t* table = paged ? g.block_table + static_cast<int64_t>(b) * g.max_blocks : nullptr;
-  int32_t* msrc = lists;                           // mover positions of the chunk, in mover order
-  int32_t* sblk = lists + kFillChunk;              // PAGED: their pages
-  int32_t* dblk = lists + 2 * kFillChunk;          // PAGED: their holes' pages
+  int64_t* const src = offs;                       // [kFillChunk] the chunk's movers, in mover order
+  int64_t* const dst = offs + kFillChunk;          // [kFillChunk] their holes
   uint16_t* const base = hw ? v : k;
-  // element offset of position i of this unit, given its page (PAGED)
-  auto elem = [&](int i, int blk) -> int64_t {
-    if (!paged) {
-      bool ok = true;
-      return row_elem(g, l, h, b, i, &ok);
-    }
-    return l * g.sL + static_cast<int64_t>(blk) * g.sB + static_cast<int64_t>((i % g.block_size) * g.H + h) * kD;
-  };
   int r0 = 0;                                      // movers of the chunks before
   for (int c0 = B; c0 < n; c0 += kFillChunk) {
     __syncwarp();                                  // the holes, or the previous chunk's copies, are done
-    int mine = 0;
+    int slot[4], pos[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int p = c0 + 4 * lane + q;
+      slot[q] = -1;
+      pos[q] = p;
       if (p < n) {
         const uint32_t bits = evb[p >> 5];
         // kept positions in [B, p): (p - B) minus the evicted ones
         const int r = (p - B) - (static_cast<int>(ebw[p >> 5] + __popc(bits & ((1u << (p & 31)) - 1u))) - m);
-        const int i = r - r0;                      // < kFillChunk, and r < m, unless the counts are off
-        if (((bits >> (p & 31)) & 1u) == 0u && r < m && i < kFillChunk) {
-          msrc[i] = p;
-          if (paged) {
-            sblk[i] = table[p / g.block_size];
-            dblk[i] = table[holes[r] / g.block_size];
-          }
-          ++mine;
-        }
+        // r < m and r - r0 < kFillChunk unless the counts are off
+        if (((bits >> (p & 31)) & 1u) == 0u && r < m && r - r0 < kFillChunk) slot[q] = r - r0;
       }
+    }
+    int64_t es[4], ed[4];
+    bool ok[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {                  // every lookup of the lane before any is used
+      ok[q] = slot[q] >= 0;
+      if (ok[q]) {
+        es[q] = row_elem(g, l, h, b, pos[q], &ok[q]);
+        ed[q] = row_elem(g, l, h, b, holes[r0 + slot[q]], &ok[q]);
+      }
+    }
+    int mine = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (slot[q] < 0) continue;
+      ++mine;
+      if (!ok[q]) flag(TRI_DEVFLAG_BAD_PAGE);
+      src[slot[q]] = ok[q] ? es[q] : -1;
+      dst[slot[q]] = ed[q];
     }
     const int mc = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<uint32_t>(mine)));
     __syncwarp();
     for (int i0 = 0; i0 < mc; i0 += kFillBatch) {
       uint4 x[kFillBatch];
-      bool live[kFillBatch];
 #pragma unroll
       for (int t = 0; t < kFillBatch; ++t) {
-        const int i = i0 + t;
-        live[t] = i < mc;
-        if (!live[t]) continue;
-        if (paged && (static_cast<unsigned>(sblk[i]) >= static_cast<unsigned>(g.num_blocks) ||
-                      static_cast<unsigned>(dblk[i]) >= static_cast<unsigned>(g.num_blocks))) {
-          live[t] = false;
-          if (lane == 0) flag(TRI_DEVFLAG_BAD_PAGE);
-          continue;
-        }
-        x[t] = ld_nc_v4(base + elem(msrc[i], paged ? sblk[i] : 0) + l16 * 8);
+        const int64_t e = i0 + t < mc ? src[i0 + t] : -1;
+        if (e >= 0) x[t] = ld_nc_v4(base + e + l16 * 8);
       }
 #pragma unroll
       for (int t = 0; t < kFillBatch; ++t) {
-        const int i = i0 + t;
-        if (live[t]) reinterpret_cast<uint4*>(base + elem(holes[r0 + i], paged ? dblk[i] : 0))[l16] = x[t];
+        if (i0 + t < mc && src[i0 + t] >= 0) reinterpret_cast<uint4*>(base + dst[i0 + t])[l16] = x[t];
       }
     }
     r0 += mc;
@@ -509,8 +502,8 @@ __global__ void __launch_bounds__(kWarpThreads, kWarpCtasPerSm) select_warp_kern
     compact::unit_coords(g, u, &l, &h, &b_);       // b_ == b
     __syncwarp();                                  // the kept list (global) and the bitmap (shared)
     if (bitmap && n - B <= kWarpCand)
-      warp_fill_row(g, l, h, b, scratch[w].hist, scratch[w].cand, B, n, scratch[w].cidx,
-                    reinterpret_cast<int32_t*>(scratch[w].cand) + 128, k, v);
+      warp_fill_row(g, l, h, b, scratch[w].hist, scratch[w].hist + 128, B, n, scratch[w].cidx,
+                    reinterpret_cast<int64_t*>(scratch[w].cand), k, v);
     else
       compact::holefill_unit_warp(g, kept, B, n, l, h, b, k, v);
   }

@@ -282,6 +282,7 @@ tri_status make_geom(const tri_cache_desc* c, bool need_v, Geom* g) {
         if (n > max_len) max_len = n;
       }
       g->block_size = c->block_size;
+      g->block_shift = (c->block_size & (c->block_size - 1)) == 0 ? __builtin_ctz(c->block_size) : -1;
       // as many consecutive pages per score tile as fill its 128 rows (at most 32)
       g->pages_per_tile = static_cast<int>(std::min<int64_t>(32, tri::score::kTileRows / (int64_t{c->block_size} * H)));
       g->max_blocks = c->max_blocks_per_seq;

@@ -7,6 +7,8 @@ import os
 import shutil
 import sys
 
+import torch
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 import bench  # noqa: E402
@@ -141,3 +143,10 @@ def test_bench_functions_read_only_names_they_can_see():
         missing += [(fn.name, n.lineno, n.id) for n in ast.walk(fn)
                     if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Load) and n.id not in seen]
     assert not missing, missing
+
+
+def test_flush_writes_then_reads_the_whole_buffer():
+    buf = torch.zeros(1000, dtype=torch.int32)
+    sink = torch.zeros((), dtype=torch.int64)
+    bench.flush_l2(buf, sink)
+    assert int(sink) == 1000 and bool((buf == 1).all())
