@@ -556,8 +556,9 @@ def run_paged(args, tri, dev, rank, ws):
     def steady(d, evs=None, score_alone=None):
         """A steady round: the fold, then tri_compress in place (score, then a
         warp per row that selects and fills the row's holes).  score_alone: a
-        score matrix; the scorer then runs once more on its own first, timed
-        (the breakdown round).  evs: events around each call."""
+        score matrix; the scorer and then the selection (without the fill) run
+        on their own first, each timed (the breakdown round; compress then
+        redoes both).  evs: events around each call."""
         nonlocal ws_buf
         need = tri.workspace_size(d, B)
         if ws_buf is None or ws_buf.numel() < need:
@@ -572,6 +573,8 @@ def run_paged(args, tri, dev, rank, ws):
         rec()
         if score_alone is not None:
             tri.score_keys(d, w, score_alone, stream=stream)
+            rec()
+            tri.select_topk(d, score_alone, B, kept, cnt, stream=stream)
             rec()
         tri.compress(d, w, B, tri.COMPACT_IN_PLACE_HOLEFILL, kept, cnt, None, None, ws_buf, stream=stream)
         rec()
@@ -634,9 +637,9 @@ def run_paged(args, tri, dev, rank, ws):
     for j in range(PAGED_BREAKDOWN_ROUNDS):
         gen.append_tokens(cache, PAGED_APPEND, step=1 + args.warmup + args.steps + j)
         d = tri.desc_paged(cache.k, cache.v, cache.block_table, cache.lens)
-        per1.append(timed(lambda evs: steady(d, evs, score_alone=scores), 4)[0])
+        per1.append(timed(lambda evs: steady(d, evs, score_alone=scores), 5)[0])
         gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
-    per1 = np.array(per1)                          # ms: fold, score alone, compress
+    per1 = np.array(per1)                          # ms: fold, score alone, select alone, compress
     st = tri.read_device_status()
     if st:
         raise RuntimeError(f"device status {st:#x} after the steady rounds")
@@ -677,11 +680,13 @@ def run_paged(args, tri, dev, rank, ws):
                              "written then read back (the write's dirty lines drain before the event)"},
             "step_breakdown_ms": {"fold": float(per[:, 0].mean()), "compress": float(per[:, 1].mean()),
                                   "score (alone)": score_ms,
+                                  "select alone (no fill, scores fresh in L2)": float(per1[:, 2].mean()),
                                   "select + hole fill (compress minus score alone)":
                                       float(per[:, 1].mean()) - score_ms,
-                                  "breakdown": f"score alone: {PAGED_BREAKDOWN_ROUNDS} more rounds, each with the "
-                                               "scorer run on its own (after the flush) before the compress "
-                                               "call; select + hole fill: the timed rounds' compress minus that"},
+                                  "breakdown": f"score alone, select alone: {PAGED_BREAKDOWN_ROUNDS} more rounds, "
+                                               "each with the scorer and then the selection run on their own "
+                                               "(after the flush) before the compress call; select + hole fill: "
+                                               "the timed rounds' compress minus the scorer alone"},
             "rows_moved_per_step": moved,
             "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_gbs,
                     "frac_of_measured": step_gbs / peak, "frac_of_8tbps_spec": step_gbs / SPEC_HBM_GBS},

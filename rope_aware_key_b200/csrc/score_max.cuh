@@ -11,13 +11,15 @@
 //    64-element boxes, 128-byte swizzle: the canonical K-major operand
 //    layout) into a ring of shared-memory stages;
 //  * warp 1 (one thread) issues tcgen05.mma kind::f16 (M = 128 keys,
-//    N = |D| rounded up to 16, K = 16 per instruction) with the keys as A and
-//    the weights as B.  bf16 weights alone would cost 2^-9 of relative
-//    accuracy, so every weight is split w = hi + lo into two bf16 parts and
-//    both products accumulate into the same fp32 accumulator in tensor memory
-//    (residual below 2^-16 of |w|); accumulators are double-buffered;
+//    K = 16 per instruction) with the keys as A and the weights as B.  bf16
+//    weights alone would cost 2^-9 of relative accuracy, so every weight is
+//    split w = hi + lo into two bf16 parts (residual below 2^-16 of |w|); B
+//    holds the hi rows and then the lo rows (N = 2 x |D| rounded up to 16),
+//    so 8 MMAs per tile give both products in fp32 tensor-memory columns;
+//    accumulators are double-buffered;
 //  * warps 2-5 read the accumulator rows (tcgen05.ld, one key per thread),
-//    take the max over the |D| columns and store the score.
+//    add the hi and lo columns, take the max over the |D| offsets and store
+//    the score.
 // The weights of a (layer, head) are converted and swizzled into shared memory
 // when a CTA's tile run reaches that head (runs are contiguous per CTA).
 #pragma once
@@ -37,6 +39,10 @@
 #ifndef TRI_SMAX_CTAS_PER_SM
 #define TRI_SMAX_CTAS_PER_SM 1
 #endif
+#ifndef TRI_SMAX_ACC_BUFS
+#define TRI_SMAX_ACC_BUFS 2
+#endif
+
 
 namespace tri {
 
@@ -60,12 +66,23 @@ constexpr int kStageBytes = kTileRows * kRowBytes;   // 32 KB: two 16 KB boxes
 constexpr int kBoxBytes = kStageBytes / 2;
 constexpr int kMaxOffsets = TRI_SMAX_MAX_OFFSETS;
 constexpr int kThreads = 6 * 32;
-constexpr int kAccCols = kMaxOffsets;             // columns per accumulator (N <= kMaxOffsets)
-constexpr uint32_t kTmemCols = 2 * kAccCols;
+// The B operand holds each offset's weights twice, as bf16 hi rows
+// [0, n_cols) and bf16 lo rows [n_cols, 2 n_cols), so one pass of 8 MMAs over
+// a key tile (N = 2 n_cols) gives both partial products side by side, and the
+// epilogue adds them.  (Accumulating hi and lo into the same columns took two
+// passes, 16 MMAs of half the width per tile, and held the kernel at 5.6 TB/s
+// with the key stream idle; the tensor pipe itself was 16 % busy.)
+constexpr int kAccCols = 2 * kMaxOffsets;          // columns per accumulator buffer
+// Accumulator buffers: the MMAs of a tile may run that many tiles ahead of
+// the epilogue.
+constexpr int kAccBufs = TRI_SMAX_ACC_BUFS;
+constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
+static_assert(kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "tensor memory columns");
 constexpr int kBBytesMax = 2 * kMaxOffsets * kRowBytes;   // hi and lo parts, N <= kMaxOffsets
 constexpr size_t kBOffset = static_cast<size_t>(kStages) * kStageBytes;
 constexpr size_t kBarOffset = kBOffset + kBBytesMax;
 constexpr size_t kSmemBytes = kBarOffset + 256 + 1024;    // barriers, slot, alignment slack
+static_assert((2 * kStages + 2 * kAccBufs) * 8 + 8 <= 256, "barrier area");
 
 struct Args {
   const float* w;        // [L*H][n_offsets][128]
@@ -134,20 +151,18 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// 32 consecutive fp32 columns of this warp's 32 tensor-memory lanes.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
+// 16 consecutive fp32 columns of this warp's 32 tensor-memory lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Byte offset of element (n, k) of a K-major operand with n_cols rows in two
@@ -162,13 +177,13 @@ __global__ void __launch_bounds__(kThreads, TRI_SMAX_CTAS_PER_SM)
 score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtensorMap kmap, const Args a) {
   extern __shared__ unsigned char smax_raw[];
   unsigned char* smem = align_shared<1024>(smax_raw);
-  unsigned char* bhi = smem + kBOffset;
-  unsigned char* blo = bhi + a.n_cols * kRowBytes;
+  unsigned char* bsm = smem + kBOffset;               // B: hi rows, then lo rows
+  const int n2 = 2 * a.n_cols;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* acc_empty = acc_full + kAccBufs;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + kAccBufs);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -177,7 +192,7 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kAccBufs; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
     }
@@ -199,7 +214,7 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
   const int t_begin = static_cast<int>(static_cast<int64_t>(a.ntiles) * blockIdx.x / gridDim.x);
   const int t_end = static_cast<int>(static_cast<int64_t>(a.ntiles) * (blockIdx.x + 1) / gridDim.x);
   const int per_lh = g.tile_prefix[g.batch];          // tiles of one (layer, head)
-  const uint32_t idesc = instr_desc(a.n_cols);
+  const uint32_t idesc = instr_desc(n2);
   const uint64_t policy = policy_evict_first();
   int k = 0, j = 0;                                   // stage-ring and accumulator counters
   for (int t0 = t_begin; t0 < t_end;) {
@@ -213,9 +228,8 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
         const float wv = n < a.n_offsets ? __ldg(a.w + (static_cast<int64_t>(lh) * a.n_offsets + n) * kD + kcol) : 0.f;
         const __nv_bfloat16 hi = __float2bfloat16_rn(wv);
         const __nv_bfloat16 lo = __float2bfloat16_rn(wv - __bfloat162float(hi));
-        const uint32_t off = sw128_offset(n, kcol, a.n_cols);
-        *reinterpret_cast<__nv_bfloat16*>(bhi + off) = hi;
-        *reinterpret_cast<__nv_bfloat16*>(blo + off) = lo;
+        *reinterpret_cast<__nv_bfloat16*>(bsm + sw128_offset(n, kcol, n2)) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(bsm + sw128_offset(a.n_cols + n, kcol, n2)) = lo;
       }
       fence_async_smem();
     }
@@ -245,7 +259,7 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
       if (lane == 0) {
         for (int t = t0; t < t1; ++t, ++k, ++j) {
           const int s = k % kStages, n = k / kStages;
-          const int ab = j & 1, na = j >> 1;
+          const int ab = j % kAccBufs, na = j / kAccBufs;
           if (!*abort_flag && !mbar_wait_bounded(&full[s], n & 1)) *abort_flag = 1;
           if (!*abort_flag && na > 0 && !mbar_wait_bounded(&acc_empty[ab], (na - 1) & 1)) *abort_flag = 1;
           if (*abort_flag) continue;
@@ -253,14 +267,10 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
           const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * kAccCols);
           const unsigned char* stage = smem + static_cast<size_t>(s) * kStageBytes;
 #pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            const unsigned char* b = part ? blo : bhi;
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint64_t da = sw128_desc(stage + (kk >> 2) * kBoxBytes + (kk & 3) * 32);
-              const uint64_t db = sw128_desc(b + (kk >> 2) * a.n_cols * 128 + (kk & 3) * 32);
-              mma_bf16(d_tmem, da, db, idesc, (part | kk) ? 1u : 0u);
-            }
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint64_t da = sw128_desc(stage + (kk >> 2) * kBoxBytes + (kk & 3) * 32);
+            const uint64_t db = sw128_desc(bsm + (kk >> 2) * n2 * 128 + (kk & 3) * 32);
+            mma_bf16(d_tmem, da, db, idesc, kk ? 1u : 0u);
           }
           mma_commit(&empty[s]);        // the stage is free once these MMAs have read it
           mma_commit(&acc_full[ab]);    // the accumulator is ready
@@ -274,30 +284,29 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
       const int quarter = warp & 3;                   // tensor-memory lanes 32*quarter ..
       const int r = quarter * 32 + lane;
       for (int t = t0; t < t1; ++t, ++j) {
-        const int ab = j & 1, na = j >> 1;
+        const int ab = j % kAccBufs, na = j / kAccBufs;
+        score::TileInfo T;                            // decoded while the MMAs run
+        int64_t src;
+        bool ok;
+        score::decode(g, t, a.scores, &T, &src, &ok);
         if (!*abort_flag && !mbar_wait_bounded(&acc_full[ab], na & 1)) *abort_flag = 1;
         if (*abort_flag) continue;
         tc_fence_after();
         const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(ab * kAccCols);
-        float v[32];
-        tmem_ld32(taddr, v);
-        float best = v[0];
+        float best = 0.f;
+        for (int c0 = 0; c0 < a.n_cols; c0 += 16) {  // 16 offsets at a time: hi + lo
+          float sum[16], v[16];
+          tmem_ld16(taddr + static_cast<uint32_t>(c0), sum);
+          tmem_ld16(taddr + static_cast<uint32_t>(a.n_cols + c0), v);
 #pragma unroll
-        for (int c = 1; c < 32; ++c)
-          if (c < a.n_offsets) best = fmaxf(best, v[c]);
-        if (a.n_cols > 32) {
-          tmem_ld32(taddr + 32, v);
+          for (int i = 0; i < 16; ++i) sum[i] += v[i];
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (32 + c < a.n_offsets) best = fmaxf(best, v[c]);
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < a.n_offsets) best = c0 + i == 0 ? sum[i] : fmaxf(best, sum[i]);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
-        score::TileInfo T;
-        int64_t src;
-        bool ok;
-        score::decode(g, t, a.scores, &T, &src, &ok);
         if (r < T.rows) T.out[r] = best;
       }
     }
