@@ -283,6 +283,28 @@ def test_compress_in_place_fills_holes_in_the_selection(lens, B):
     check_every_unit(cache, res, literal=False, before=before, after=after)
 
 
+@pytest.mark.parametrize("H,bs,B,lens", [
+    (8, 12, 2000, [2001, 2127, 2128, 2129, 2512, 1999]),   # pages of 12 tokens (no shift), B not a multiple of 32
+    (1, 32, 1000, [1512, 1129, 1001, 700]),                 # tails of 1..512 rows: several 128-position chunks
+    (2, 64, 3000, [3500, 3200, 3001, 3000]),
+])
+def test_compress_in_place_fill_page_shapes(H, bs, B, lens):
+    """The selection's in-kernel fill on paged caches of other page sizes and
+    head counts, tails that span several chunks and budgets that split a
+    bitmap word; every unit against the oracle, K and V before and after."""
+    t = tri()
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=H, batch=len(lens), budget=B,
+                    block_size=bs, spare_blocks_per_seq=1)
+    cache = gen.make_cache(wl, seed=40 + H + bs, device=DEV, lens=lens)
+    units = all_units(wl)
+    before = snapshot(cache, units)
+    n0 = t.kernel_launches()
+    res = parity.run_gpu(cache, mode=t.COMPACT_IN_PLACE_HOLEFILL, fused=True)
+    assert t.kernel_launches() - n0 == 3                       # fold, score, the selection with the fill
+    after = snapshot(cache, units)
+    check_every_unit(cache, res, literal=False, before=before, after=after)
+
+
 @pytest.mark.parametrize("dup", [1, 3])
 def test_compress_in_place_fill_after_the_whole_row_search(dup):
     """Rows whose scores take one or three values: the selection's bracket
