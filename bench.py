@@ -144,9 +144,9 @@ def ncu_traffic(workload, variant="mean"):
 
 class ClockSampler:
     """SM clock, power and throttle reasons sampled in the background while
-    the timed region runs: through NVML every 2 ms (so that even a timed
-    region of a few milliseconds gets a dozen samples), or, without NVML,
-    nvidia-smi every 100 ms.  Each sample is a row
+    the timed region runs: through NVML every 0.5 ms (so that a timed region
+    of 10 ms, 20 steps of the headline, gets about 20 samples), or, without
+    NVML, nvidia-smi every 100 ms.  Each sample is a row
     [time, index, sm MHz, max sm MHz, power W, reasons, hw_slowdown,
      hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap]."""
 
@@ -154,7 +154,7 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int, uuid: str = None, period_s: float = 0.002):
+    def __init__(self, gpu_index: int, uuid: str = None, period_s: float = 0.0005):
         self.samples = []
         self.proc = None
         self.source = None
@@ -607,7 +607,7 @@ def run_paged(args, tri, dev, rank, ws):
         raise RuntimeError(f"device status {st:#x} after the initial event")
 
     # steady rounds
-    sampler = ClockSampler(*gpu_identity(dev, local), period_s=0.001)
+    sampler = ClockSampler(*gpu_identity(dev, local))
     sampler.wait_first()
     scores = None
     rounds = []
