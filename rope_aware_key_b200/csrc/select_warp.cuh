@@ -53,7 +53,7 @@ constexpr int kWarpThreads = kWarpRows * 32;
 constexpr int kWarpSamples = 256;                  // 8 per lane
 constexpr int kWarpCand = 512;
 constexpr int kWarpMaxRow = 4096;
-constexpr int kWarpBatch = 4;                     // chunks whose loads are in flight together
+constexpr int kWarpBatch = 4;                     // chunks whose loads are in flight together (6 or 8: the same time)
 constexpr int kWarpCtasPerSm = 7;                 // register budget: 72 per thread
 
 struct __align__(16) WarpScratch {
