@@ -279,7 +279,13 @@ tri_status tri_workspace_size(const tri_cache_desc* desc, int B, size_t* bytes);
  * at most 8192 keys runs as ONE kernel: a cluster per unit scores its keys into
  * shared memory, selects across the cluster and copies the kept rows; its
  * scores, kept indices and compacted rows are identical, bit for bit, to the
- * three-kernel path's, which every other case takes. */
+ * three-kernel path's.
+ * IN_PLACE_HOLEFILL on rows of at most 4096 keys that each move at most 512
+ * rows (n - B <= 512: a serving cache re-compressed every window of new
+ * tokens) runs as TWO kernels: the scorer, then the selection with one warp
+ * per row, which fills the row's holes right after selecting it; kept,
+ * kept_count and the cache end up as the three calls leave them.  Every other
+ * case takes the three kernels. */
 tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B,
                         tri_compact_mode mode, int32_t* kept, int32_t* kept_count,
                         void* k_out, void* v_out, void* workspace, size_t workspace_bytes,
