@@ -71,30 +71,46 @@ __global__ void __launch_bounds__(kThreads) fold_kernel(const __grid_constant__ 
 
 // Per-offset weights for the max-over-offsets score (no averaging):
 //   a_{f,t} = E[q_f] e^{i w_f (delta0 + delta_t)},  w[c][t][re(f)] = Re, w[c][t][im(f)] = Im.
-// Grid: (band f, block of kThreads (center, offset) pairs); fp64, fp32 out.
+// The rotation depends only on (band, offset): a block takes one offset and
+// kFoldCenters centers, a thread one band and kFoldPer of those centers, so
+// each thread evaluates its rotation once (fp64 sincos) and applies it to its
+// centers (fp64 products, fp32 out), their loads issued together; loads and
+// stores of a center's bands are contiguous across the threads.
+constexpr int kFoldCenters = 32;                   // centers per block
+constexpr int kFoldRows = 4;                       // threads per band
+constexpr int kFoldPer = kFoldCenters / kFoldRows; // centers per thread
+
 template <int N>
-__global__ void __launch_bounds__(kThreads) fold_offsets_kernel(const __grid_constant__ Args<N> a) {
-  const int f = blockIdx.x;
-  const double omega = a.omega[f];
-  if (f == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+__global__ void __launch_bounds__(kBands * kFoldRows) fold_offsets_kernel(const __grid_constant__ Args<N> a) {
+  const int f = threadIdx.x, t = blockIdx.x;
+  if (t == 0 && blockIdx.y == 0 && f == 0 && threadIdx.y == 0) {
     bool finite = isfinite(a.theta) && isfinite(a.delta0);
-    for (int t = 0; t < a.n_offsets; ++t) finite = finite && isfinite(a.offsets[t]);
+    for (int o = 0; o < a.n_offsets; ++o) finite = finite && isfinite(a.offsets[o]);
     if (!finite) flag(TRI_DEVFLAG_NONFINITE);
   }
-  const int idx = blockIdx.y * kThreads + threadIdx.x;
-  if (idx >= a.n_centers * a.n_offsets) return;
-  const int c = idx / a.n_offsets, t = idx - c * a.n_offsets;
   const int re = a.pairing == TRI_PAIRING_HALF ? f : 2 * f;
   const int im = a.pairing == TRI_PAIRING_HALF ? f + kBands : 2 * f + 1;
-  const float* q = a.q + static_cast<int64_t>(c) * kD;
-  const float qr_f = q[re], qi_f = q[im];
-  if (!isfinite(qr_f) || !isfinite(qi_f)) flag(TRI_DEVFLAG_NONFINITE);
+  const int cb = blockIdx.y * kFoldCenters + threadIdx.y;
+  float qr[kFoldPer], qi[kFoldPer];
+#pragma unroll
+  for (int i = 0; i < kFoldPer; ++i) {
+    const int c = cb + i * kFoldRows;
+    const float* q = a.q + static_cast<int64_t>(c < a.n_centers ? c : 0) * kD;
+    qr[i] = q[re];
+    qi[i] = q[im];
+  }
   double sn, cs;
-  sincos(omega * (a.delta0 + a.offsets[t]), &sn, &cs);
-  const double qr = qr_f, qi = qi_f;
-  float* w = a.w + static_cast<int64_t>(idx) * kD;
-  w[re] = static_cast<float>(cs * qr - sn * qi);
-  w[im] = static_cast<float>(sn * qr + cs * qi);
+  sincos(a.omega[f] * (a.delta0 + a.offsets[t]), &sn, &cs);
+#pragma unroll
+  for (int i = 0; i < kFoldPer; ++i) {
+    const int c = cb + i * kFoldRows;
+    if (c >= a.n_centers) break;
+    if (!isfinite(qr[i]) || !isfinite(qi[i])) flag(TRI_DEVFLAG_NONFINITE);
+    const double dr = qr[i], di = qi[i];
+    float* w = a.w + (static_cast<int64_t>(c) * a.n_offsets + t) * kD;
+    w[re] = static_cast<float>(cs * dr - sn * di);
+    w[im] = static_cast<float>(sn * dr + cs * di);
+  }
 }
 
 }  // namespace fold

@@ -594,9 +594,8 @@ void launch_fold_offsets(const tri_fold_params* p, const float* q_center, int n_
   a.n_offsets = p->n_offsets;
   for (int f = 0; f < tri::fold::kBands; ++f) a.omega[f] = std::pow(p->theta, -2.0 * f / TRI_HEAD_DIM);
   std::memcpy(a.offsets, p->offsets, sizeof(double) * p->n_offsets);
-  const int pairs = n_centers * p->n_offsets;
-  const dim3 grid(tri::fold::kBands, (pairs + tri::fold::kThreads - 1) / tri::fold::kThreads);
-  tri::fold::fold_offsets_kernel<N><<<grid, tri::fold::kThreads, 0, s>>>(a);
+  const dim3 grid(p->n_offsets, (n_centers + tri::fold::kFoldCenters - 1) / tri::fold::kFoldCenters);
+  tri::fold::fold_offsets_kernel<N><<<grid, dim3(tri::fold::kBands, tri::fold::kFoldRows), 0, s>>>(a);
 }
 
 // Shared by the two fold calls: checks, then one launch with the schedule in
@@ -613,6 +612,9 @@ tri_status launch_fold(const tri_fold_params* p, const float* q_center, int n_ce
     if (!std::isfinite(p->offsets[t])) return TRI_ERR_INVALID_ARG;
   if (!aligned16(q_center) || !aligned16(w_out)) return TRI_ERR_INVALID_ARG;
   if (per_offset && int64_t{n_centers} * p->n_offsets > INT32_MAX / 2) return TRI_ERR_UNSUPPORTED;
+  // the per-offset kernel's grid: kFoldCenters centers per block along y (at most 65535 blocks)
+  if (per_offset && (int64_t{n_centers} + tri::fold::kFoldCenters - 1) / tri::fold::kFoldCenters > 65535)
+    return TRI_ERR_UNSUPPORTED;
   if (int64_t{n_centers} * TRI_HEAD_DIM > INT32_MAX / 2) return TRI_ERR_UNSUPPORTED;
   DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;

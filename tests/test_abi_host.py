@@ -256,6 +256,9 @@ def test_score_max_checks(L):
     assert L.tri_score_keys_max(ctypes.byref(pg), P(FAKE), 17, P(FAKE), None) == 2     # paged: not supported
     p = fold_params(offs=[1.0] * 3000)
     assert L.tri_fold_offset_weights(ctypes.byref(p), P(FAKE), 4, P(FAKE), None) == 2
+    # the per-offset fold takes 32 centers per block along the grid's y (at most 65535 blocks)
+    p = fold_params(offs=[1.0] * 2)
+    assert L.tri_fold_offset_weights(ctypes.byref(p), P(FAKE), 65535 * 32 + 1, P(FAKE), None) == 2
 
 
 def test_score_positions_checks(L):
