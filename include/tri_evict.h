@@ -117,7 +117,10 @@ typedef struct tri_cache_desc {
   int batch;               /* sequences, 1 .. TRI_MAX_BATCH */
   int max_seq_len;         /* capacity of a score row; 0 = the longest sequence */
   const void* k;           /* device bf16 key cache (16-byte aligned) */
-  const void* v;           /* device bf16 value cache; may be NULL for scoring/selection */
+  const void* v;           /* bf16 value cache on K's device; may be NULL for scoring/selection.  For an
+                              OUT_OF_PLACE compaction it may instead be pinned host memory mapped into
+                              the device at the same address (cudaHostAlloc): the gather then reads only
+                              the kept V rows over the bus.  Anything else: TRI_ERR_INVALID_ARG. */
   int64_t stride_layer;
   int64_t stride_head;     /* CONTIG / RAGGED */
   int64_t stride_seq;      /* CONTIG */

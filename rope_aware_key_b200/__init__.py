@@ -179,7 +179,9 @@ def _i32_host(values) -> ctypes.Array:
 
 
 def desc_contig(k: torch.Tensor, v: Optional[torch.Tensor] = None, max_seq_len: int = 0) -> Desc:
-    """k, v: bf16 [L][H][batch][N][128] with the last two dims packed."""
+    """k, v: bf16 [L][H][batch][N][128] with the last two dims packed.  k on
+    the device; v on the same device, or a pinned CPU tensor for out-of-place
+    compaction (the gather reads only the kept rows over the bus)."""
     assert k.dim() == 5 and k.dtype == torch.bfloat16 and k.shape[-1] == HEAD_DIM
     assert k.stride(-1) == 1 and k.stride(-2) == HEAD_DIM
     if v is not None:

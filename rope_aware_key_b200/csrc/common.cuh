@@ -20,6 +20,7 @@ struct Geom {
   int L, H, batch;
   int block_size, max_blocks, num_blocks;
   int block_shift;           // PAGED: log2(block_size) when it is a power of two, else -1
+  int v_host;                // V lives in pinned host memory mapped into the device (gather reads it over the bus)
   int pages_per_tile;        // PAGED: consecutive pages of a sequence scored as one tile
   int64_t sL, sH, sB;        // layer / head / (seq for CONTIG, page for PAGED) strides, elements
   int64_t score_stride;      // floats per score row
@@ -161,6 +162,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
       : "memory");
 }
+
+// 16-byte global load (plain: also right for pinned host memory mapped into
+// the device's address space).
+__device__ __forceinline__ uint4 ld_v4(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 
 // 16-byte global load that bypasses L1 (read-only data).
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {

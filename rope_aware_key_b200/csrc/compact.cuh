@@ -101,7 +101,7 @@ gather_kernel(const __grid_constant__ Geom g, const int32_t* __restrict__ kept,
           }
         }
         kx[q] = ld_nc_v4(g.k + e + l16 * 8);
-        vx[q] = ld_nc_v4(g.v + e + l16 * 8);
+        vx[q] = g.v_host ? ld_v4(g.v + e + l16 * 8) : ld_nc_v4(g.v + e + l16 * 8);   // warp-uniform
         live[q] = true;
       }
 #pragma unroll

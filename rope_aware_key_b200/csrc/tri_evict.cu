@@ -206,6 +206,30 @@ tri_status use_device_of(const void* ptr, int* dev_out, DeviceScope* scope) {
   return TRI_OK;
 }
 
+// Where V lives, for a compaction on device `dev`: device memory of that
+// device, or -- for OUT_OF_PLACE only, where V is read and never written --
+// pinned host memory mapped into the device's address space at the same
+// address (the gather then reads just the kept rows over the bus).  Sets
+// g->v_host.
+tri_status check_values(const tri_cache_desc* desc, int dev, tri_compact_mode mode, Geom* g) {
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, desc->v);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return TRI_ERR_INVALID_ARG;
+  }
+  if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) {
+    if (attr.device != dev) return TRI_ERR_INVALID_ARG;
+    g->v_host = 0;
+    return TRI_OK;
+  }
+  if (attr.type == cudaMemoryTypeHost && attr.devicePointer == desc->v && mode == TRI_COMPACT_OUT_OF_PLACE) {
+    g->v_host = 1;
+    return TRI_OK;
+  }
+  return TRI_ERR_INVALID_ARG;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Score matrix of tri_compress_noalloc: a fixed array in the module's device
@@ -850,6 +874,8 @@ tri_status tri_compact_kv(const tri_cache_desc* desc, const int32_t* kept, const
   int dev;
   st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
+  st = check_values(desc, dev, mode, &g);
+  if (st != TRI_OK) return st;
   return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -884,6 +910,8 @@ tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B, tri_c
   int dev;
   st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
+  st = check_values(desc, dev, mode, &g);
+  if (st != TRI_OK) return st;
   return run_compress(g, plan, w, B, mode, kept, kept_count, k_out, v_out, static_cast<float*>(workspace), dev,
                       reinterpret_cast<cudaStream_t>(stream));
 }
@@ -904,6 +932,8 @@ tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int 
   DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
   st = use_device_of(desc->k, &dev, &scope);   // makes the cache's device current
+  if (st != TRI_OK) return st;
+  st = check_values(desc, dev, mode, &g);
   if (st != TRI_OK) return st;
   float* scores = nullptr;
   {
