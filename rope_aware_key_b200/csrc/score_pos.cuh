@@ -123,7 +123,7 @@ __device__ __forceinline__ float2 hi_hi(uint32_t a, uint32_t b) {
 __device__ __forceinline__ uint32_t word(const uint4& x, int i) { return i == 0 ? x.x : i == 1 ? x.y : i == 2 ? x.z : x.w; }
 
 // Two bands (the x and y halves) of one key, added into acc:
-//   Re a conj(k) e^{i phi'} = (a_r k_r + a_i k_i) cos phi' + (a_r k_i - a_i k_r) sin phi'
+//   Re a conj(k) e^{i phi'} = k_r (a_r cos phi' - a_i sin phi') + k_i (a_r sin phi' + a_i cos phi')
 // with phi' the phase minus pi, built from the bits of |Delta| C_f (see the
 // top of the file).
 __device__ __forceinline__ float2 band_pair(float2 kr, float2 ki, float2 ar, float2 ai, uint32_t hi0, uint32_t lo0,
@@ -137,11 +137,13 @@ __device__ __forceinline__ float2 band_pair(float2 kr, float2 ki, float2 ar, flo
   float2 sn, cs;
   __sincosf(phi.x, &sn.x, &cs.x);
   __sincosf(phi.y, &sn.y, &cs.y);
-  const float2 u = __ffma2_rn(ar, kr, __fmul2_rn(ai, ki));
-  const float2 t = __fmul2_rn(ai, kr);
-  acc = __ffma2_rn(u, cs, acc);
-  acc = __ffma2_rn(__fmul2_rn(ar, ki), sn, acc);
-  return __ffma2_rn(make_float2(-t.x, -t.y), sn, acc);
+  // b = a e^{i phi'} first, then Re conj(k) b = k_r b_r + k_i b_i: six packed
+  // operations for the two bands
+  const float2 p = __fmul2_rn(ai, sn);
+  const float2 br = __ffma2_rn(ar, cs, make_float2(-p.x, -p.y));
+  const float2 bi = __ffma2_rn(ar, sn, __fmul2_rn(ai, cs));
+  acc = __ffma2_rn(kr, br, acc);
+  return __ffma2_rn(ki, bi, acc);
 }
 
 // Per-key distance terms shared by the scorers: whether t_b - p_i is in
