@@ -103,6 +103,37 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// A 5-D tiled load (the paged pool seen as [layer][page][token][head][128]).
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int x, int h, int t, int page,
+                                            int layer, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(h), "r"(t), "r"(page), "r"(layer), "r"(smem_addr(bar)),
+      "l"(policy)
+      : "memory");
+}
+
+// A 128-key tile of one unit (l, h, b) of a PAGED cache: tiles are numbered
+// per (layer, head), then sequence, then 128-key chunk (tile_prefix counts
+// 128-key chunks per sequence); its keys are the pages p0 .. of sequence b.
+struct HeadTile {
+  int l, h, b, i0, rows;
+  float* out;        // score of the tile's first key
+};
+__device__ __forceinline__ HeadTile head_tile(const Geom& g, int t, float* scores) {
+  HeadTile T;
+  const int per = g.tile_prefix[g.batch];
+  const int lh = t / per, r = t - lh * per;
+  T.b = find_seq(g.tile_prefix, g.batch, r);
+  T.i0 = (r - g.tile_prefix[T.b]) * kTileRows;
+  T.l = lh / g.H;
+  T.h = lh - T.l * g.H;
+  T.rows = min(kTileRows, g.len[T.b] - T.i0);
+  T.out = scores + (static_cast<int64_t>(lh) * g.batch + T.b) * g.score_stride + T.i0;
+  return T;
+}
+
 // K-major, 128-byte-swizzled operand: 8-row atoms of 1024 bytes (SBO), 16-byte
 // units along K; version 1 for sm_100.
 __device__ __forceinline__ uint64_t sw128_desc(const void* p) {
@@ -242,14 +273,36 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
           const int s = k % kStages, n = k / kStages;
           if (n > 0 && !*abort_flag && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) *abort_flag = 1;
           if (*abort_flag) continue;
-          score::TileInfo T;
-          int64_t src;
-          bool ok;
-          score::decode(g, t, a.scores, &T, &src, &ok);
-          const int row = static_cast<int>(src / kD);
-          mbar_arrive_expect_tx(&full[s], kStageBytes);
-          tma_load_2d(smem + static_cast<size_t>(s) * kStageBytes, &kmap, 0, row, &full[s], policy);
-          tma_load_2d(smem + static_cast<size_t>(s) * kStageBytes + kBoxBytes, &kmap, 64, row, &full[s], policy);
+          unsigned char* stage = smem + static_cast<size_t>(s) * kStageBytes;
+          if (g.layout == TRI_LAYOUT_PAGED) {
+            // one box pair per page of the tile (block_size is a power of two
+            // >= 8, so a tile is whole pages and each page's rows are whole
+            // 1 KB swizzle atoms); pages outside the pool are left out
+            const HeadTile T = head_tile(g, t, a.scores);
+            const int bs = g.block_size;
+            const int p0 = T.i0 >> g.block_shift, np = (T.rows + bs - 1) >> g.block_shift;
+            const int32_t* tab = g.block_table + static_cast<int64_t>(T.b) * g.max_blocks + p0;
+            uint32_t ok = 0u;
+            for (int p = 0; p < np; ++p)
+              if (static_cast<unsigned>(tab[p]) < static_cast<unsigned>(g.num_blocks)) ok |= 1u << p;
+            if (ok != (np >= 32 ? 0xffffffffu : (1u << np) - 1u)) flag(TRI_DEVFLAG_BAD_PAGE);
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(ok)) * bs * kRowBytes);
+            for (int p = 0; p < np; ++p) {
+              if (!((ok >> p) & 1u)) continue;
+              const uint32_t off = static_cast<uint32_t>(p * bs) * 128u;
+              tma_load_5d(stage + off, &kmap, 0, T.h, 0, tab[p], T.l, &full[s], policy);
+              tma_load_5d(stage + kBoxBytes + off, &kmap, 64, T.h, 0, tab[p], T.l, &full[s], policy);
+            }
+          } else {
+            score::TileInfo T;
+            int64_t src;
+            bool ok;
+            score::decode(g, t, a.scores, &T, &src, &ok);
+            const int row = static_cast<int>(src / kD);
+            mbar_arrive_expect_tx(&full[s], kStageBytes);
+            tma_load_2d(stage, &kmap, 0, row, &full[s], policy);
+            tma_load_2d(stage + kBoxBytes, &kmap, 64, row, &full[s], policy);
+          }
         }
       } else {
         k += t1 - t0;
@@ -285,10 +338,28 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
       const int r = quarter * 32 + lane;
       for (int t = t0; t < t1; ++t, ++j) {
         const int ab = j % kAccBufs, na = j / kAccBufs;
-        score::TileInfo T;                            // decoded while the MMAs run
-        int64_t src;
-        bool ok;
-        score::decode(g, t, a.scores, &T, &src, &ok);
+        // the tile's output, decoded while the MMAs run (PAGED: keys in pages
+        // outside the pool are not written)
+        float* out;
+        int rows;
+        bool live;
+        if (g.layout == TRI_LAYOUT_PAGED) {
+          const HeadTile T = head_tile(g, t, a.scores);
+          out = T.out;
+          rows = T.rows;
+          live = r < rows &&
+                 static_cast<unsigned>(g.block_table[static_cast<int64_t>(T.b) * g.max_blocks +
+                                                     ((T.i0 + r) >> g.block_shift)]) <
+                     static_cast<unsigned>(g.num_blocks);
+        } else {
+          score::TileInfo T;
+          int64_t src;
+          bool ok;
+          score::decode(g, t, a.scores, &T, &src, &ok);
+          out = T.out;
+          rows = T.rows;
+          live = r < rows;
+        }
         if (!*abort_flag && !mbar_wait_bounded(&acc_full[ab], na & 1)) *abort_flag = 1;
         if (*abort_flag) continue;
         tc_fence_after();
@@ -307,7 +378,7 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
-        if (r < T.rows) T.out[r] = best;
+        if (live) out[r] = best;
       }
     }
     t0 = t1;

@@ -713,6 +713,40 @@ tri_status encode_key_map(const tri_cache_desc* desc, int64_t rows, CUtensorMap*
   return cr == CUDA_SUCCESS ? TRI_OK : TRI_ERR_INVALID_ARG;
 }
 
+// A PAGED key pool as a 5-D bf16 tensor [layer][page][token][head][128] for
+// tiled TMA loads of one page of one head: boxes of 64 elements x block_size
+// tokens, 128-byte swizzle (the same shared-memory layout as the packed map's
+// 128-row boxes, a page's rows filling whole 1 KB swizzle atoms).
+tri_status encode_paged_key_map(const tri_cache_desc* desc, CUtensorMap* map) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return TRI_ERR_UNSUPPORTED;
+  const cuuint64_t H = static_cast<cuuint64_t>(desc->num_kv_heads);
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(TRI_HEAD_DIM), H, static_cast<cuuint64_t>(desc->block_size),
+                        static_cast<cuuint64_t>(desc->num_blocks), static_cast<cuuint64_t>(desc->num_layers)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(tri::kRowBytes), H * tri::kRowBytes,
+                           static_cast<cuuint64_t>(desc->stride_block) * 2,
+                           static_cast<cuuint64_t>(desc->stride_layer) * 2};
+  cuuint32_t box[5] = {64, 1, static_cast<cuuint32_t>(desc->block_size), 1, 1};
+  cuuint32_t elem[5] = {1, 1, 1, 1, 1};
+  CUresult cr = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(desc->k), dims, strides, box,
+                       elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return cr == CUDA_SUCCESS ? TRI_OK : TRI_ERR_INVALID_ARG;
+}
+
+// 128-key tiles per (layer, head), then sequence, whatever the layout (the
+// max scorer's tiles); returns the tile count.
+int64_t fill_head_tile_prefix(Geom* g) {
+  int64_t acc = 0;
+  for (int b = 0; b < g->batch; ++b) {
+    g->tile_prefix[b] = static_cast<int32_t>(acc);
+    acc += (g->len[b] + tri::score::kTileRows - 1) / tri::score::kTileRows;
+    if (acc > INT32_MAX) return INT64_MAX;
+  }
+  g->tile_prefix[g->batch] = static_cast<int32_t>(acc);
+  return int64_t{g->L} * g->H * acc;
+}
+
 }  // namespace
 
 extern "C" {
@@ -734,9 +768,16 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   if (st != TRI_OK) return st;
   if (!w || !scores || !aligned16(w) || !aligned16(scores) || n_offsets < 1) return TRI_ERR_INVALID_ARG;
   if (n_offsets > tri::smax::kMaxOffsets) return TRI_ERR_UNSUPPORTED;
-  const int64_t rows = packed_rows(desc);
-  if (rows <= 0 || rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
-  const int64_t ntiles = fill_tile_prefix(&g);
+  const bool paged = desc->layout == TRI_LAYOUT_PAGED;
+  int64_t rows = 0;
+  if (paged) {
+    // a tile is whole pages, each page whole swizzle atoms: a power of two >= 8
+    if (g.block_shift < 3) return TRI_ERR_UNSUPPORTED;
+  } else {
+    rows = packed_rows(desc);
+    if (rows <= 0 || rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  }
+  const int64_t ntiles = paged ? fill_head_tile_prefix(&g) : fill_tile_prefix(&g);
   if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
   if (ntiles == 0) return TRI_OK;
   DeviceScope scope;   // the caller's current device comes back when the call returns
@@ -744,7 +785,7 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
   CUtensorMap map;
-  st = encode_key_map(desc, rows, &map);
+  st = paged ? encode_paged_key_map(desc, &map) : encode_key_map(desc, rows, &map);
   if (st != TRI_OK) return st;
   tri::smax::Args a{w, scores, static_cast<int>(ntiles), n_offsets, (n_offsets + 15) & ~15};
   const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].smax_blocks_per_sm;

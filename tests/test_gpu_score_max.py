@@ -95,6 +95,39 @@ def test_score_max_ragged_edges():
                 check_unit_max(cache, scores, w64, l, h, b, GEO17, 0.0, 0)
 
 
+@pytest.mark.parametrize("H,bs", [(4, 16), (8, 8), (1, 128), (2, 32)])
+def test_score_max_paged(H, bs):
+    """Paged pools: a tile is 128 keys of one head, one 2-box load per page."""
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=H, batch=4, block_size=bs,
+                    spare_blocks_per_seq=1)
+    cache = gen.make_cache(wl, seed=24 + H + bs, device=DEV, with_values=False, lens=[1, 127, 300, 1000])
+    w, scores, status = run_max(cache, GEO17)
+    assert status == 0
+    w64 = check_offset_weights(w, cache, GEO17, 0.0, 0)
+    for l in range(wl.num_layers):
+        for h in range(H):
+            for b in range(wl.batch):
+                check_unit_max(cache, scores, w64, l, h, b, GEO17, 0.0, 0)
+
+
+def test_score_max_paged_bad_page_is_flagged_not_fatal():
+    import rope_aware_key_b200 as tri
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=1, num_kv_heads=4, batch=2, spare_blocks_per_seq=0)
+    cache = gen.make_cache(wl, seed=29, device=DEV, with_values=False, lens=[200, 200])
+    nb = cache.k.shape[1]
+    cache.block_table[1, 3] = nb + 1000                     # tokens 48..63 of sequence 1: out of the pool
+    w, scores, status = run_max(cache, GEO17)
+    assert status & tri.DEVFLAG_BAD_PAGE
+    tri.read_device_status(clear=True)
+    assert tri.read_device_status() == 0
+    w64 = check_offset_weights(w, cache, GEO17, 0.0, 0)
+    for h in range(4):
+        check_unit_max(cache, scores, w64, 0, h, 0, GEO17, 0.0, 0)        # the intact sequence is right
+        u = parity.unit_id(wl, 0, h, 1)
+        assert torch.isnan(scores[u, 48:64]).all()                     # the bad page's keys are not written
+        assert not torch.isnan(scores[u, :48]).any() and not torch.isnan(scores[u, 64:200]).any()
+
+
 def test_score_max_selects_like_the_oracle():
     """The kept set under the max score, through the same selection kernel."""
     import rope_aware_key_b200 as tri
