@@ -266,43 +266,69 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
     }
     __syncthreads();
 
-    if (warp == 0) {
-      // ---------------- producer
+    if (warp == 0 && g.layout == TRI_LAYOUT_PAGED) {
+      // ---------------- producer, PAGED: the whole warp, lane p on page p of
+      // the tile (block_size is a power of two >= 8, so a tile is whole pages,
+      // at most 16, and each page's rows are whole 1 KB swizzle atoms).  The
+      // page ids of the next tile are loaded before this tile's slot is
+      // awaited; pages outside the pool are left out.
+      const int bs = g.block_size;
+      auto page_of = [&](const HeadTile& T) -> int32_t {
+        const int np = (T.rows + bs - 1) >> g.block_shift;
+        return lane < np ? g.block_table[static_cast<int64_t>(T.b) * g.max_blocks + (T.i0 >> g.block_shift) + lane]
+                         : -1;
+      };
+      HeadTile Tn;
+      int32_t nxt = -1;
+      if (t0 < t1) {
+        Tn = head_tile(g, t0, a.scores);
+        nxt = page_of(Tn);
+      }
+      for (int t = t0; t < t1; ++t, ++k) {
+        const HeadTile T = Tn;
+        const int32_t cur = nxt;
+        if (t + 1 < t1) {
+          Tn = head_tile(g, t + 1, a.scores);
+          nxt = page_of(Tn);
+        }
+        const int s = k % kStages, n = k / kStages;
+        int stop = 0;
+        if (lane == 0) {
+          if (n > 0 && !*abort_flag && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) *abort_flag = 1;
+          stop = *abort_flag;
+        }
+        if (__shfl_sync(0xffffffffu, stop, 0)) continue;
+        const int np = (T.rows + bs - 1) >> g.block_shift;
+        const bool valid = lane < np && static_cast<unsigned>(cur) < static_cast<unsigned>(g.num_blocks);
+        const uint32_t ok = __ballot_sync(0xffffffffu, valid);
+        if (lane == 0) {
+          if (ok != (1u << np) - 1u) flag(TRI_DEVFLAG_BAD_PAGE);
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(ok)) * bs * kRowBytes);
+        }
+        __syncwarp();                                 // the expected bytes are set before any copy lands
+        if (valid) {
+          unsigned char* stage = smem + static_cast<size_t>(s) * kStageBytes;
+          const uint32_t off = static_cast<uint32_t>(lane * bs) * 128u;
+          tma_load_5d(stage + off, &kmap, 0, T.h, 0, cur, T.l, &full[s], policy);
+          tma_load_5d(stage + kBoxBytes + off, &kmap, 64, T.h, 0, cur, T.l, &full[s], policy);
+        }
+      }
+    } else if (warp == 0) {
+      // ---------------- producer, packed layouts: one thread
       if (lane == 0) {
         for (int t = t0; t < t1; ++t, ++k) {
           const int s = k % kStages, n = k / kStages;
           if (n > 0 && !*abort_flag && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) *abort_flag = 1;
           if (*abort_flag) continue;
           unsigned char* stage = smem + static_cast<size_t>(s) * kStageBytes;
-          if (g.layout == TRI_LAYOUT_PAGED) {
-            // one box pair per page of the tile (block_size is a power of two
-            // >= 8, so a tile is whole pages and each page's rows are whole
-            // 1 KB swizzle atoms); pages outside the pool are left out
-            const HeadTile T = head_tile(g, t, a.scores);
-            const int bs = g.block_size;
-            const int p0 = T.i0 >> g.block_shift, np = (T.rows + bs - 1) >> g.block_shift;
-            const int32_t* tab = g.block_table + static_cast<int64_t>(T.b) * g.max_blocks + p0;
-            uint32_t ok = 0u;
-            for (int p = 0; p < np; ++p)
-              if (static_cast<unsigned>(tab[p]) < static_cast<unsigned>(g.num_blocks)) ok |= 1u << p;
-            if (ok != (np >= 32 ? 0xffffffffu : (1u << np) - 1u)) flag(TRI_DEVFLAG_BAD_PAGE);
-            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(ok)) * bs * kRowBytes);
-            for (int p = 0; p < np; ++p) {
-              if (!((ok >> p) & 1u)) continue;
-              const uint32_t off = static_cast<uint32_t>(p * bs) * 128u;
-              tma_load_5d(stage + off, &kmap, 0, T.h, 0, tab[p], T.l, &full[s], policy);
-              tma_load_5d(stage + kBoxBytes + off, &kmap, 64, T.h, 0, tab[p], T.l, &full[s], policy);
-            }
-          } else {
-            score::TileInfo T;
-            int64_t src;
-            bool ok;
-            score::decode(g, t, a.scores, &T, &src, &ok);
-            const int row = static_cast<int>(src / kD);
-            mbar_arrive_expect_tx(&full[s], kStageBytes);
-            tma_load_2d(stage, &kmap, 0, row, &full[s], policy);
-            tma_load_2d(stage + kBoxBytes, &kmap, 64, row, &full[s], policy);
-          }
+          score::TileInfo T;
+          int64_t src;
+          bool ok;
+          score::decode(g, t, a.scores, &T, &src, &ok);
+          const int row = static_cast<int>(src / kD);
+          mbar_arrive_expect_tx(&full[s], kStageBytes);
+          tma_load_2d(stage, &kmap, 0, row, &full[s], policy);
+          tma_load_2d(stage + kBoxBytes, &kmap, 64, row, &full[s], policy);
         }
       } else {
         k += t1 - t0;
