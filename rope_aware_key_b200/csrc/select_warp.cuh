@@ -20,10 +20,11 @@
 //     scores; each is found by a bitwise search over the samples' key range
 //     (a step counts the samples below a trial key: one warp reduction);
 //  2. one pass over the row counts the keys above U (all kept) and gathers
-//     the keys in [L, U] into a candidate buffer (the comparisons are made
-//     on the floats; the candidates are stored as keys).  When L would fall
-//     below the sample (rows that evict few keys), every key up to U is a
-//     candidate and is gathered with its index, in index order;
+//     the keys in [L, U] into a candidate buffer, in index order (the
+//     comparisons are made on the floats; the candidates are stored as float
+//     bits and turned into keys afterwards).  When L would fall below the
+//     sample (rows that evict few keys), every key up to U is a candidate
+//     and is gathered with its index;
 //  3. if the B-th largest lies among the candidates (above < B <= above +
 //     candidates), a radix search over them (8-bit digits, a shared histogram
 //     per digit) gives it exactly: T, and `need`, how many keys equal to T
@@ -36,7 +37,9 @@
 //     second pass emits the kept keys in index order (ballots per 128-key
 //     chunk).
 // If the check fails (a pathological order, heavy duplication), the radix
-// search runs over the whole row instead (one pass per digit).
+// search runs over the whole row instead (one pass per digit).  In-place
+// compaction of rows that move few keys runs in the same kernel: the warp
+// fills the row's holes right after selecting it (warp_fill_row).
 #pragma once
 
 #include <type_traits>
