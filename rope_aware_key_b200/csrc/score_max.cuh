@@ -7,9 +7,10 @@
 // average being linear; a maximum over the offsets does not fold, so each
 // key needs one dot product per offset.  That is a skinny dense contraction
 // [keys x 128] x [128 x |D|], which is what the tensor cores are for:
-//  * warp 0 (one thread) streams 128-key tiles with 2-D TMA copies (two
-//    64-element boxes, 128-byte swizzle: the canonical K-major operand
-//    layout) into a ring of shared-memory stages;
+//  * warp 0 streams 128-key tiles with TMA copies (two 64-element boxes,
+//    128-byte swizzle: the canonical K-major operand layout) into a ring of
+//    shared-memory stages: one thread and 2-D copies for packed layouts, a
+//    lane per page and 5-D copies for paged pools;
 //  * warp 1 (one thread) issues tcgen05.mma kind::f16 (M = 128 keys,
 //    K = 16 per instruction) with the keys as A and the weights as B.  bf16
 //    weights alone would cost 2^-9 of relative accuracy, so every weight is
@@ -20,8 +21,9 @@
 //  * warps 2-5 read the accumulator rows (tcgen05.ld, one key per thread),
 //    add the hi and lo columns, take the max over the |D| offsets and store
 //    the score.
-// The weights of a (layer, head) are converted and swizzled into shared memory
-// when a CTA's tile run reaches that head (runs are contiguous per CTA).
+// The weights of a (layer, head), or of all heads of a layer for whole-page
+// paged tiles, are converted and swizzled into shared memory when a CTA's
+// tile run reaches them (runs are contiguous per CTA).
 #pragma once
 
 #include <cuda.h>
@@ -72,13 +74,20 @@ constexpr int kThreads = 6 * 32;
 // epilogue adds them.  (Accumulating hi and lo into the same columns took two
 // passes, 16 MMAs of half the width per tile, and held the kernel at 5.6 TB/s
 // with the key stream idle; the tensor pipe itself was 16 % busy.)
-constexpr int kAccCols = 2 * kMaxOffsets;          // columns per accumulator buffer
+// With a PAGED cache whose heads fit one MMA (H * n_cols <= 128), B holds the
+// weights of every head of the layer (head h: rows h * 2 n_cols ..) and a
+// tile is whole pages of all heads, one box pair per page, each page laid
+// head-major in the stage; every key's accumulator row then carries every
+// head's columns.  A warp's 32 rows hold one head, or 32 / block_size heads,
+// and the warp reads only those heads' columns.
+constexpr int kMaxB = 256;                         // B rows: 2 * heads * n_cols <= the MMA's largest N
+constexpr int kAccCols = kMaxB;                    // columns per accumulator buffer
 // Accumulator buffers: the MMAs of a tile may run that many tiles ahead of
 // the epilogue.
 constexpr int kAccBufs = TRI_SMAX_ACC_BUFS;
 constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
 static_assert(kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "tensor memory columns");
-constexpr int kBBytesMax = 2 * kMaxOffsets * kRowBytes;   // hi and lo parts, N <= kMaxOffsets
+constexpr int kBBytesMax = kMaxB * kRowBytes;             // hi and lo parts of every head in B
 constexpr size_t kBOffset = static_cast<size_t>(kStages) * kStageBytes;
 constexpr size_t kBarOffset = kBOffset + kBBytesMax;
 constexpr size_t kSmemBytes = kBarOffset + 256 + 1024;    // barriers, slot, alignment slack
@@ -90,6 +99,9 @@ struct Args {
   int ntiles;
   int n_offsets;         // 1 .. kMaxOffsets
   int n_cols;            // n_offsets rounded up to 16
+  int heads;             // heads in B: 1, or H for whole-page PAGED tiles
+  int head_shift;        // log2(heads)
+  int whole_pages;       // PAGED: tiles of whole pages of all heads (else of one head)
 };
 
 // ------------------------------------------------------------------ PTX
@@ -103,34 +115,88 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// A 5-D tiled load (the paged pool seen as [layer][page][token][head][128]).
-__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int x, int h, int t, int page,
+// A 5-D tiled load from a paged pool: coordinates (element, c1, c2, page,
+// layer), c1 / c2 the head / token (one-head map) or token / head (all-heads
+// map).
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int x, int c1, int c2, int page,
                                             int layer, uint64_t* bar, uint64_t policy) {
   asm volatile(
       "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
       "[%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(h), "r"(t), "r"(page), "r"(layer), "r"(smem_addr(bar)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(c1), "r"(c2), "r"(page), "r"(layer), "r"(smem_addr(bar)),
       "l"(policy)
       : "memory");
 }
 
-// A 128-key tile of one unit (l, h, b) of a PAGED cache: tiles are numbered
-// per (layer, head), then sequence, then 128-key chunk (tile_prefix counts
-// 128-key chunks per sequence); its keys are the pages p0 .. of sequence b.
-struct HeadTile {
-  int l, h, b, i0, rows;
+// Tiles are numbered outer index (a weight run), then sequence, then chunk
+// of the sequence; tile_prefix counts each sequence's chunks.  A CTA walks a
+// contiguous range of tiles, so the walk keeps (outer, b, j) and steps it,
+// searching tile_prefix only for the range's first tile.
+struct Cursor {
+  int outer, b, j;
+};
+__device__ __forceinline__ Cursor cursor_at(const Geom& g, int t) {
+  Cursor c;
+  const int per = g.tile_prefix[g.batch];
+  c.outer = t / per;
+  const int r = t - c.outer * per;
+  c.b = find_seq(g.tile_prefix, g.batch, r);
+  c.j = r - g.tile_prefix[c.b];
+  return c;
+}
+// The next tile (one must exist: sequences without tiles are passed over).
+__device__ __forceinline__ void cursor_next(const Geom& g, Cursor& c) {
+  ++c.j;
+  while (c.j >= g.tile_prefix[c.b + 1] - g.tile_prefix[c.b]) {
+    c.j = 0;
+    if (++c.b == g.batch) {
+      c.b = 0;
+      ++c.outer;
+    }
+  }
+}
+
+// A 128-key tile of a packed layout (CONTIG / RAGGED): chunk j of unit
+// (outer = l*H + h, b).
+struct PackedTile {
+  int rows;          // keys of the tile inside the sequence
+  int row;           // key row of the tile's first key in the [rows][128] view
   float* out;        // score of the tile's first key
 };
-__device__ __forceinline__ HeadTile head_tile(const Geom& g, int t, float* scores) {
-  HeadTile T;
-  const int per = g.tile_prefix[g.batch];
-  const int lh = t / per, r = t - lh * per;
-  T.b = find_seq(g.tile_prefix, g.batch, r);
-  T.i0 = (r - g.tile_prefix[T.b]) * kTileRows;
-  T.l = lh / g.H;
-  T.h = lh - T.l * g.H;
-  T.rows = min(kTileRows, g.len[T.b] - T.i0);
-  T.out = scores + (static_cast<int64_t>(lh) * g.batch + T.b) * g.score_stride + T.i0;
+__device__ __forceinline__ PackedTile packed_tile(const Geom& g, const Cursor& c, float* scores) {
+  PackedTile T;
+  const int l = c.outer / g.H, h = c.outer - l * g.H;
+  const int i0 = c.j * kTileRows;
+  T.rows = min(kTileRows, g.len[c.b] - i0);
+  bool ok = true;
+  T.row = static_cast<int>(row_elem(g, l, h, c.b, i0, &ok) / kD);
+  T.out = scores + (static_cast<int64_t>(c.outer) * g.batch + c.b) * g.score_stride + i0;
+  return T;
+}
+
+// A tile of a PAGED cache, in one of two forms:
+//  * whole pages (Args::whole_pages): pages_per_tile consecutive pages of
+//    sequence b in layer l = outer, all heads, each page head-major in the
+//    stage;
+//  * one head: 128 consecutive keys of unit (l, h, b), outer = l*H + h, a
+//    page's rows of that head after another's.
+struct PagedTile {
+  int l, h;          // layer; head (one-head tiles) or 0
+  int np;            // pages in the tile
+  int64_t tbl;       // block-table index of the tile's first page
+  int tvalid;        // tokens of the tile inside the sequence
+  float* out;        // score of the tile's first token (of head h, or of head 0)
+};
+__device__ __forceinline__ PagedTile paged_tile(const Geom& g, const Cursor& c, bool whole, float* scores) {
+  PagedTile T;
+  const int span = whole ? g.pages_per_tile << g.block_shift : kTileRows;
+  T.l = whole ? c.outer : c.outer / g.H;
+  T.h = whole ? 0 : c.outer - T.l * g.H;
+  const int i0 = c.j * span;
+  T.tvalid = min(span, g.len[c.b] - i0);
+  T.np = (T.tvalid + g.block_size - 1) >> g.block_shift;
+  T.tbl = static_cast<int64_t>(c.b) * g.max_blocks + (i0 >> g.block_shift);
+  T.out = scores + (static_cast<int64_t>(T.l * g.H + T.h) * g.batch + c.b) * g.score_stride + i0;
   return T;
 }
 
@@ -182,18 +248,48 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// 16 consecutive fp32 columns of this warp's 32 tensor-memory lanes.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
+// W consecutive fp32 columns at ta and W at tb of this warp's 32
+// tensor-memory lanes (one lane per thread): both loads are issued and then
+// awaited once, inside one asm statement, so no use of the registers can be
+// scheduled ahead of the wait.
+__device__ __forceinline__ void tmem_ld_pair(uint32_t ta, uint32_t tb, uint32_t (&x)[32], uint32_t (&y)[32]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+      "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, "
+      "%20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31"
+      "}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, "
+      "%50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63"
+      "}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7]),
+        "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]), "=r"(x[13]), "=r"(x[14]), "=r"(x[15]),
+        "=r"(x[16]), "=r"(x[17]), "=r"(x[18]), "=r"(x[19]), "=r"(x[20]), "=r"(x[21]), "=r"(x[22]), "=r"(x[23]),
+        "=r"(x[24]), "=r"(x[25]), "=r"(x[26]), "=r"(x[27]), "=r"(x[28]), "=r"(x[29]), "=r"(x[30]), "=r"(x[31]),
+        "=r"(y[0]), "=r"(y[1]), "=r"(y[2]), "=r"(y[3]), "=r"(y[4]), "=r"(y[5]), "=r"(y[6]), "=r"(y[7]),
+        "=r"(y[8]), "=r"(y[9]), "=r"(y[10]), "=r"(y[11]), "=r"(y[12]), "=r"(y[13]), "=r"(y[14]), "=r"(y[15]),
+        "=r"(y[16]), "=r"(y[17]), "=r"(y[18]), "=r"(y[19]), "=r"(y[20]), "=r"(y[21]), "=r"(y[22]), "=r"(y[23]),
+        "=r"(y[24]), "=r"(y[25]), "=r"(y[26]), "=r"(y[27]), "=r"(y[28]), "=r"(y[29]), "=r"(y[30]), "=r"(y[31])
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_pair(uint32_t ta, uint32_t tb, uint32_t (&x)[16], uint32_t (&y)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {"
+      "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15"
+      "}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {"
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31"
+      "}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7]),
+        "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]), "=r"(x[13]), "=r"(x[14]), "=r"(x[15]),
+        "=r"(y[0]), "=r"(y[1]), "=r"(y[2]), "=r"(y[3]), "=r"(y[4]), "=r"(y[5]), "=r"(y[6]), "=r"(y[7]),
+        "=r"(y[8]), "=r"(y[9]), "=r"(y[10]), "=r"(y[11]), "=r"(y[12]), "=r"(y[13]), "=r"(y[14]), "=r"(y[15])
+      : "r"(ta), "r"(tb)
+      : "memory");
 }
 
 // Byte offset of element (n, k) of a K-major operand with n_cols rows in two
@@ -208,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, TRI_SMAX_CTAS_PER_SM)
 score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtensorMap kmap, const Args a) {
   extern __shared__ unsigned char smax_raw[];
   unsigned char* smem = align_shared<1024>(smax_raw);
-  unsigned char* bsm = smem + kBOffset;               // B: hi rows, then lo rows
-  const int n2 = 2 * a.n_cols;
+  unsigned char* bsm = smem + kBOffset;               // B: per head, hi rows then lo rows
+  const int n2 = 2 * a.heads * a.n_cols;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
@@ -244,23 +340,26 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
   // this CTA's contiguous run of tiles
   const int t_begin = static_cast<int>(static_cast<int64_t>(a.ntiles) * blockIdx.x / gridDim.x);
   const int t_end = static_cast<int>(static_cast<int64_t>(a.ntiles) * (blockIdx.x + 1) / gridDim.x);
-  const int per_lh = g.tile_prefix[g.batch];          // tiles of one (layer, head)
+  const int per_run = g.tile_prefix[g.batch];         // tiles of one weight run: (layer, head), or a layer
   const uint32_t idesc = instr_desc(n2);
   const uint64_t policy = policy_evict_first();
   int k = 0, j = 0;                                   // stage-ring and accumulator counters
   for (int t0 = t_begin; t0 < t_end;) {
-    const int lh = t0 / per_lh;
-    const int t1 = min(t_end, (lh + 1) * per_lh);
+    const int run = t0 / per_run;
+    const int t1 = min(t_end, (run + 1) * per_run);
 
-    // weights of this head: bf16 hi / lo, swizzled (epilogue warps)
+    // weights of this run's heads: bf16 hi / lo, swizzled (epilogue warps)
     if (warp >= 2) {
       const int kcol = threadIdx.x - 64;              // 0..127: one element column
-      for (int n = 0; n < a.n_cols; ++n) {
-        const float wv = n < a.n_offsets ? __ldg(a.w + (static_cast<int64_t>(lh) * a.n_offsets + n) * kD + kcol) : 0.f;
+      for (int m = 0; m < a.heads * a.n_cols; ++m) {
+        const int hh = m / a.n_cols, n = m - hh * a.n_cols;
+        const int64_t lh = static_cast<int64_t>(run) * a.heads + hh;
+        const float wv = n < a.n_offsets ? __ldg(a.w + (lh * a.n_offsets + n) * kD + kcol) : 0.f;
         const __nv_bfloat16 hi = __float2bfloat16_rn(wv);
         const __nv_bfloat16 lo = __float2bfloat16_rn(wv - __bfloat162float(hi));
-        *reinterpret_cast<__nv_bfloat16*>(bsm + sw128_offset(n, kcol, n2)) = hi;
-        *reinterpret_cast<__nv_bfloat16*>(bsm + sw128_offset(a.n_cols + n, kcol, n2)) = lo;
+        const int row = hh * 2 * a.n_cols + n;
+        *reinterpret_cast<__nv_bfloat16*>(bsm + sw128_offset(row, kcol, n2)) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(bsm + sw128_offset(row + a.n_cols, kcol, n2)) = lo;
       }
       fence_async_smem();
     }
@@ -268,27 +367,26 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
 
     if (warp == 0 && g.layout == TRI_LAYOUT_PAGED) {
       // ---------------- producer, PAGED: the whole warp, lane p on page p of
-      // the tile (block_size is a power of two >= 8, so a tile is whole pages,
-      // at most 16, and each page's rows are whole 1 KB swizzle atoms).  The
-      // page ids of the next tile are loaded before this tile's slot is
-      // awaited; pages outside the pool are left out.
-      const int bs = g.block_size;
-      auto page_of = [&](const HeadTile& T) -> int32_t {
-        const int np = (T.rows + bs - 1) >> g.block_shift;
-        return lane < np ? g.block_table[static_cast<int64_t>(T.b) * g.max_blocks + (T.i0 >> g.block_shift) + lane]
-                         : -1;
-      };
-      HeadTile Tn;
+      // the tile (block_size is a power of two, a page's rows fill whole 1 KB
+      // swizzle atoms and a tile is whole pages, at most 16).  The page ids
+      // of the next tile are loaded before this tile's slot is awaited; pages
+      // outside the pool are left out.
+      const bool whole = a.whole_pages != 0;
+      const uint32_t page_rows = static_cast<uint32_t>(g.block_size) << a.head_shift;
+      auto page_of = [&](const PagedTile& T) -> int32_t { return lane < T.np ? g.block_table[T.tbl + lane] : -1; };
+      Cursor cn = cursor_at(g, t0);
+      PagedTile Tn;
       int32_t nxt = -1;
       if (t0 < t1) {
-        Tn = head_tile(g, t0, a.scores);
+        Tn = paged_tile(g, cn, whole, a.scores);
         nxt = page_of(Tn);
       }
       for (int t = t0; t < t1; ++t, ++k) {
-        const HeadTile T = Tn;
+        const PagedTile T = Tn;
         const int32_t cur = nxt;
         if (t + 1 < t1) {
-          Tn = head_tile(g, t + 1, a.scores);
+          cursor_next(g, cn);
+          Tn = paged_tile(g, cn, whole, a.scores);
           nxt = page_of(Tn);
         }
         const int s = k % kStages, n = k / kStages;
@@ -298,17 +396,16 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
           stop = *abort_flag;
         }
         if (__shfl_sync(0xffffffffu, stop, 0)) continue;
-        const int np = (T.rows + bs - 1) >> g.block_shift;
-        const bool valid = lane < np && static_cast<unsigned>(cur) < static_cast<unsigned>(g.num_blocks);
+        const bool valid = lane < T.np && static_cast<unsigned>(cur) < static_cast<unsigned>(g.num_blocks);
         const uint32_t ok = __ballot_sync(0xffffffffu, valid);
         if (lane == 0) {
-          if (ok != (1u << np) - 1u) flag(TRI_DEVFLAG_BAD_PAGE);
-          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(ok)) * bs * kRowBytes);
+          if (ok != (1u << T.np) - 1u) flag(TRI_DEVFLAG_BAD_PAGE);
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(ok)) * page_rows * kRowBytes);
         }
         __syncwarp();                                 // the expected bytes are set before any copy lands
         if (valid) {
           unsigned char* stage = smem + static_cast<size_t>(s) * kStageBytes;
-          const uint32_t off = static_cast<uint32_t>(lane * bs) * 128u;
+          const uint32_t off = static_cast<uint32_t>(lane) * page_rows * 128u;
           tma_load_5d(stage + off, &kmap, 0, T.h, 0, cur, T.l, &full[s], policy);
           tma_load_5d(stage + kBoxBytes + off, &kmap, 64, T.h, 0, cur, T.l, &full[s], policy);
         }
@@ -316,16 +413,14 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
     } else if (warp == 0) {
       // ---------------- producer, packed layouts: one thread
       if (lane == 0) {
+        Cursor c = cursor_at(g, t0);
         for (int t = t0; t < t1; ++t, ++k) {
+          if (t > t0) cursor_next(g, c);
+          const int row = packed_tile(g, c, a.scores).row;
           const int s = k % kStages, n = k / kStages;
           if (n > 0 && !*abort_flag && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) *abort_flag = 1;
           if (*abort_flag) continue;
           unsigned char* stage = smem + static_cast<size_t>(s) * kStageBytes;
-          score::TileInfo T;
-          int64_t src;
-          bool ok;
-          score::decode(g, t, a.scores, &T, &src, &ok);
-          const int row = static_cast<int>(src / kD);
           mbar_arrive_expect_tx(&full[s], kStageBytes);
           tma_load_2d(stage, &kmap, 0, row, &full[s], policy);
           tma_load_2d(stage + kBoxBytes, &kmap, 64, row, &full[s], policy);
@@ -362,53 +457,79 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
       // ---------------- epilogue: one key per thread
       const int quarter = warp & 3;                   // tensor-memory lanes 32*quarter ..
       const int r = quarter * 32 + lane;
+      // Row r of a tile.  Whole-page PAGED tiles hold each page head-major:
+      // page p = r >> (block_shift + head_shift), head (r >> block_shift) &
+      // (H - 1), token p * block_size + (r & (block_size - 1)) of the tile;
+      // a warp's 32 rows then hold min(H, 32 / block_size) heads (at least
+      // one), consecutive from h_first.  Otherwise one head, row r = token r.
+      const bool whole = a.whole_pages != 0;
+      int tok = r, hr = 0, h_first = 0, heads_in_warp = 1;
+      if (whole) {
+        hr = (r >> g.block_shift) & (g.H - 1);
+        tok = ((r >> (g.block_shift + a.head_shift)) << g.block_shift) | (r & (g.block_size - 1));
+        h_first = ((quarter * 32) >> g.block_shift) & (g.H - 1);
+        heads_in_warp = min(g.H, max(1, 32 >> g.block_shift));
+      }
+      Cursor c = cursor_at(g, t0);
       for (int t = t0; t < t1; ++t, ++j) {
+        if (t > t0) cursor_next(g, c);
         const int ab = j % kAccBufs, na = j / kAccBufs;
-        // the tile's output, decoded while the MMAs run (PAGED: keys in pages
-        // outside the pool are not written)
+        // the tile's output, decoded while the MMAs run; keys in pages outside
+        // the pool are not written
         float* out;
-        int rows;
         bool live;
         if (g.layout == TRI_LAYOUT_PAGED) {
-          const HeadTile T = head_tile(g, t, a.scores);
-          out = T.out;
-          rows = T.rows;
-          live = r < rows &&
-                 static_cast<unsigned>(g.block_table[static_cast<int64_t>(T.b) * g.max_blocks +
-                                                     ((T.i0 + r) >> g.block_shift)]) <
+          const PagedTile T = paged_tile(g, c, whole, a.scores);
+          out = T.out + hr * (static_cast<int64_t>(g.batch) * g.score_stride) + tok;
+          live = tok < T.tvalid &&
+                 static_cast<unsigned>(g.block_table[T.tbl + (tok >> g.block_shift)]) <
                      static_cast<unsigned>(g.num_blocks);
         } else {
-          score::TileInfo T;
-          int64_t src;
-          bool ok;
-          score::decode(g, t, a.scores, &T, &src, &ok);
-          out = T.out;
-          rows = T.rows;
-          live = r < rows;
+          const PackedTile T = packed_tile(g, c, a.scores);
+          out = T.out + tok;
+          live = tok < T.rows;
         }
         if (!*abort_flag && !mbar_wait_bounded(&acc_full[ab], na & 1)) *abort_flag = 1;
         if (*abort_flag) continue;
         tc_fence_after();
         const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(ab * kAccCols);
+        // tcgen05.ld reads the same columns in every lane: the warp goes
+        // through the columns of each head its rows hold, and each lane keeps
+        // its own head's max
         float best = 0.f;
-        for (int c0 = 0; c0 < a.n_cols; c0 += 16) {  // 16 offsets at a time: hi + lo
-          float sum[16], v[16];
-          tmem_ld16(taddr + static_cast<uint32_t>(c0), sum);
-          tmem_ld16(taddr + static_cast<uint32_t>(a.n_cols + c0), v);
+        for (int i = 0; i < heads_in_warp; ++i) {
+          const int hh = h_first + i;
+          const uint32_t hcol = taddr + static_cast<uint32_t>(hh * 2 * a.n_cols);
+          float m = 0.f;
+          for (int c0 = 0; c0 < a.n_cols; c0 += 32) {    // hi + lo, 32 (or the last 16) offsets at a time
+            if (c0 + 32 <= a.n_cols) {
+              uint32_t x[32], y[32];
+              tmem_ld_pair(hcol + static_cast<uint32_t>(c0), hcol + static_cast<uint32_t>(a.n_cols + c0), x, y);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) sum[i] += v[i];
+              for (int e = 0; e < 32; ++e) {
+                const float v = __uint_as_float(x[e]) + __uint_as_float(y[e]);
+                if (c0 + e < a.n_offsets) m = c0 + e == 0 ? v : fmaxf(m, v);
+              }
+            } else {
+              uint32_t x[16], y[16];
+              tmem_ld_pair(hcol + static_cast<uint32_t>(c0), hcol + static_cast<uint32_t>(a.n_cols + c0), x, y);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i < a.n_offsets) best = c0 + i == 0 ? sum[i] : fmaxf(best, sum[i]);
+              for (int e = 0; e < 16; ++e) {
+                const float v = __uint_as_float(x[e]) + __uint_as_float(y[e]);
+                if (c0 + e < a.n_offsets) m = c0 + e == 0 ? v : fmaxf(m, v);
+              }
+            }
+          }
+          if (hh == hr) best = m;
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[ab]);
-        if (live) out[r] = best;
+        if (live) *out = best;
       }
     }
     t0 = t1;
-    __syncthreads();   // the next head's weights overwrite bhi / blo
+    __syncthreads();   // the next run's weights overwrite B
   }
 
   // never exit with copies in flight (only possible after an abort)

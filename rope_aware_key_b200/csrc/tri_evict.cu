@@ -713,20 +713,28 @@ tri_status encode_key_map(const tri_cache_desc* desc, int64_t rows, CUtensorMap*
   return cr == CUDA_SUCCESS ? TRI_OK : TRI_ERR_INVALID_ARG;
 }
 
-// A PAGED key pool as a 5-D bf16 tensor [layer][page][token][head][128] for
-// tiled TMA loads of one page of one head: boxes of 64 elements x block_size
-// tokens, 128-byte swizzle (the same shared-memory layout as the packed map's
-// 128-row boxes, a page's rows filling whole 1 KB swizzle atoms).
-tri_status encode_paged_key_map(const tri_cache_desc* desc, CUtensorMap* map) {
+// A PAGED key pool as a 5-D bf16 tensor for tiled TMA loads of one page:
+//  * of one head (whole = false): dimensions [layer][page][token][head][128],
+//    boxes of 64 elements x block_size tokens of head h;
+//  * of all heads (whole = true): the token and head dimensions swapped,
+//    [layer][page][head][token][128] over the same memory, boxes of 64
+//    elements x block_size tokens x H heads, so that the page lands in shared
+//    memory head-major (head h's tokens in consecutive rows).
+// 128-byte swizzle: the same shared-memory layout as the packed map's 128-row
+// boxes, a page's rows filling whole 1 KB swizzle atoms.
+tri_status encode_paged_key_map(const tri_cache_desc* desc, bool whole, CUtensorMap* map) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return TRI_ERR_UNSUPPORTED;
   const cuuint64_t H = static_cast<cuuint64_t>(desc->num_kv_heads);
-  cuuint64_t dims[5] = {static_cast<cuuint64_t>(TRI_HEAD_DIM), H, static_cast<cuuint64_t>(desc->block_size),
+  const cuuint64_t bs = static_cast<cuuint64_t>(desc->block_size);
+  const cuuint64_t head_stride = tri::kRowBytes, token_stride = H * tri::kRowBytes;
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(TRI_HEAD_DIM), whole ? bs : H, whole ? H : bs,
                         static_cast<cuuint64_t>(desc->num_blocks), static_cast<cuuint64_t>(desc->num_layers)};
-  cuuint64_t strides[4] = {static_cast<cuuint64_t>(tri::kRowBytes), H * tri::kRowBytes,
+  cuuint64_t strides[4] = {whole ? token_stride : head_stride, whole ? head_stride : token_stride,
                            static_cast<cuuint64_t>(desc->stride_block) * 2,
                            static_cast<cuuint64_t>(desc->stride_layer) * 2};
-  cuuint32_t box[5] = {64, 1, static_cast<cuuint32_t>(desc->block_size), 1, 1};
+  cuuint32_t box[5] = {64, whole ? static_cast<cuuint32_t>(bs) : 1u,
+                       whole ? static_cast<cuuint32_t>(H) : static_cast<cuuint32_t>(bs), 1, 1};
   cuuint32_t elem[5] = {1, 1, 1, 1, 1};
   CUresult cr = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(desc->k), dims, strides, box,
                        elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -769,15 +777,21 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   if (!w || !scores || !aligned16(w) || !aligned16(scores) || n_offsets < 1) return TRI_ERR_INVALID_ARG;
   if (n_offsets > tri::smax::kMaxOffsets) return TRI_ERR_UNSUPPORTED;
   const bool paged = desc->layout == TRI_LAYOUT_PAGED;
+  const int n_cols = (n_offsets + 15) & ~15;
   int64_t rows = 0;
+  // PAGED: whole pages of all heads per tile when every head's weights fit
+  // one MMA (2 H n_cols <= 256) and a page of all heads fills whole swizzle
+  // atoms (H block_size a power of two >= 8, so whole pages fill the 128
+  // rows); else one head's rows per tile, pages of a power of two >= 8 tokens.
+  const bool whole = paged && g.block_shift >= 0 && g.H * n_cols <= tri::smax::kMaxB / 2 &&
+                     (g.block_size * g.H) >= 8;
   if (paged) {
-    // a tile is whole pages, each page whole swizzle atoms: a power of two >= 8
-    if (g.block_shift < 3) return TRI_ERR_UNSUPPORTED;
+    if (!whole && g.block_shift < 3) return TRI_ERR_UNSUPPORTED;
   } else {
     rows = packed_rows(desc);
     if (rows <= 0 || rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
   }
-  const int64_t ntiles = paged ? fill_head_tile_prefix(&g) : fill_tile_prefix(&g);
+  const int64_t ntiles = paged && !whole ? fill_head_tile_prefix(&g) : fill_tile_prefix(&g);
   if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
   if (ntiles == 0) return TRI_OK;
   DeviceScope scope;   // the caller's current device comes back when the call returns
@@ -785,9 +799,11 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
   CUtensorMap map;
-  st = paged ? encode_paged_key_map(desc, &map) : encode_key_map(desc, rows, &map);
+  st = paged ? encode_paged_key_map(desc, whole, &map) : encode_key_map(desc, rows, &map);
   if (st != TRI_OK) return st;
-  tri::smax::Args a{w, scores, static_cast<int>(ntiles), n_offsets, (n_offsets + 15) & ~15};
+  const int heads = whole ? g.H : 1;
+  tri::smax::Args a{w, scores, static_cast<int>(ntiles), n_offsets, n_cols, heads, __builtin_ctz(heads),
+                    whole ? 1 : 0};
   const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].smax_blocks_per_sm;
   const int grid = static_cast<int>(ntiles < resident ? ntiles : resident);
   tri::smax::score_max_kernel<<<grid, tri::smax::kThreads, tri::smax::kSmemBytes,

@@ -254,8 +254,13 @@ def test_score_max_checks(L):
     assert L.tri_score_keys_max(ctypes.byref(loose), P(FAKE), 17, P(FAKE), None) == 2  # units not packed
     pg = paged(block_size=12, stride_block=12 * 4 * 128, stride_layer=100 * 12 * 4 * 128)
     assert L.tri_score_keys_max(ctypes.byref(pg), P(FAKE), 17, P(FAKE), None) == 2     # pages not a power of two
-    pg = paged(block_size=4, stride_block=4 * 4 * 128, stride_layer=100 * 4 * 4 * 128, max_blocks_per_seq=16)
-    assert L.tri_score_keys_max(ctypes.byref(pg), P(FAKE), 17, P(FAKE), None) == 2     # pages under 8 tokens
+    # 8 heads x 32 weight columns exceed one MMA: one head per tile, and its pages are under 8 tokens
+    pg = paged(num_kv_heads=8, block_size=4, stride_block=4 * 8 * 128, stride_layer=100 * 4 * 8 * 128,
+               max_blocks_per_seq=16)
+    assert L.tri_score_keys_max(ctypes.byref(pg), P(FAKE), 17, P(FAKE), None) == 2
+    # a page of all 4 heads is 4 rows, under one 8-row swizzle atom
+    pg = paged(block_size=1, stride_block=4 * 128, stride_layer=100 * 4 * 128, max_blocks_per_seq=64)
+    assert L.tri_score_keys_max(ctypes.byref(pg), P(FAKE), 5, P(FAKE), None) == 2
     p = fold_params(offs=[1.0] * 3000)
     assert L.tri_fold_offset_weights(ctypes.byref(p), P(FAKE), 4, P(FAKE), None) == 2
     # the per-offset fold takes 32 centers per block along the grid's y (at most 65535 blocks)

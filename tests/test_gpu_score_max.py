@@ -95,24 +95,32 @@ def test_score_max_ragged_edges():
                 check_unit_max(cache, scores, w64, l, h, b, GEO17, 0.0, 0)
 
 
-@pytest.mark.parametrize("H,bs", [(4, 16), (8, 8), (1, 128), (2, 32)])
-def test_score_max_paged(H, bs):
-    """Paged pools: a tile is 128 keys of one head, one 2-box load per page."""
+@pytest.mark.parametrize("H,bs,n_off", [
+    (4, 16, 17), (1, 128, 17), (2, 32, 17), (4, 4, 17), (8, 2, 16), (8, 16, 5), (2, 64, 64),  # whole pages
+    (8, 8, 17), (8, 16, 33), (4, 32, 64),                                                     # one head
+])
+def test_score_max_paged(H, bs, n_off):
+    """Paged pools.  When every head's weights fit one MMA (H x n_cols <= 128)
+    a tile is whole pages of all heads, one 2-box load per page; otherwise 128
+    keys of one head, one 2-box load per page of that head."""
     wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=H, batch=4, block_size=bs,
                     spare_blocks_per_seq=1)
-    cache = gen.make_cache(wl, seed=24 + H + bs, device=DEV, with_values=False, lens=[1, 127, 300, 1000])
-    w, scores, status = run_max(cache, GEO17)
+    cache = gen.make_cache(wl, seed=24 + H + bs + n_off, device=DEV, with_values=False, lens=[1, 127, 300, 1000])
+    offsets = GEO17[:n_off] if n_off <= 17 else [float(1 + 37 * i) for i in range(n_off)]
+    w, scores, status = run_max(cache, offsets)
     assert status == 0
-    w64 = check_offset_weights(w, cache, GEO17, 0.0, 0)
+    w64 = check_offset_weights(w, cache, offsets, 0.0, 0)
     for l in range(wl.num_layers):
         for h in range(H):
             for b in range(wl.batch):
-                check_unit_max(cache, scores, w64, l, h, b, GEO17, 0.0, 0)
+                check_unit_max(cache, scores, w64, l, h, b, offsets, 0.0, 0)
+    assert torch.isnan(scores[:, 1000:]).all()          # row padding untouched
 
 
-def test_score_max_paged_bad_page_is_flagged_not_fatal():
+@pytest.mark.parametrize("H", [4, 8])                      # whole-page tiles, one-head tiles
+def test_score_max_paged_bad_page_is_flagged_not_fatal(H):
     import rope_aware_key_b200 as tri
-    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=1, num_kv_heads=4, batch=2, spare_blocks_per_seq=0)
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=1, num_kv_heads=H, batch=2, spare_blocks_per_seq=0)
     cache = gen.make_cache(wl, seed=29, device=DEV, with_values=False, lens=[200, 200])
     nb = cache.k.shape[1]
     cache.block_table[1, 3] = nb + 1000                     # tokens 48..63 of sequence 1: out of the pool
@@ -121,7 +129,7 @@ def test_score_max_paged_bad_page_is_flagged_not_fatal():
     tri.read_device_status(clear=True)
     assert tri.read_device_status() == 0
     w64 = check_offset_weights(w, cache, GEO17, 0.0, 0)
-    for h in range(4):
+    for h in range(H):
         check_unit_max(cache, scores, w64, 0, h, 0, GEO17, 0.0, 0)        # the intact sequence is right
         u = parity.unit_id(wl, 0, h, 1)
         assert torch.isnan(scores[u, 48:64]).all()                     # the bad page's keys are not written
