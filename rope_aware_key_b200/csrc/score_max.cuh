@@ -67,30 +67,39 @@ constexpr int kStages = TRI_SMAX_STAGES;
 constexpr int kStageBytes = kTileRows * kRowBytes;   // 32 KB: two 16 KB boxes
 constexpr int kBoxBytes = kStageBytes / 2;
 constexpr int kMaxOffsets = TRI_SMAX_MAX_OFFSETS;
-constexpr int kThreads = 6 * 32;
-// The B operand holds each offset's weights twice, as bf16 hi rows
-// [0, n_cols) and bf16 lo rows [n_cols, 2 n_cols), so one pass of 8 MMAs over
-// a key tile (N = 2 n_cols) gives both partial products side by side, and the
-// epilogue adds them.  (Accumulating hi and lo into the same columns took two
-// passes, 16 MMAs of half the width per tile, and held the kernel at 5.6 TB/s
-// with the key stream idle; the tensor pipe itself was 16 % busy.)
-// With a PAGED cache whose heads fit one MMA (H * n_cols <= 128), B holds the
-// weights of every head of the layer (head h: rows h * 2 n_cols ..) and a
-// tile is whole pages of all heads, one box pair per page, each page laid
+// The B operand holds each offset's weights twice, as a bf16 hi row and the
+// bf16 lo row after it (offset n: rows 2n and 2n + 1 of its head's block of
+// head_cols = 2 |D| rounded up to 16 rows), so one pass of 8 MMAs over a key
+// tile gives both partial products in adjacent columns, and the epilogue adds
+// each pair.  (Accumulating hi and lo into the same columns took two passes,
+// 16 MMAs of half the width per tile, and held the kernel at 5.6 TB/s with
+// the key stream idle; the tensor pipe itself was 16 % busy.)
+// With a PAGED cache whose heads fit one MMA (H * head_cols <= 256), B holds
+// the weights of every head of the layer (head h: rows h * head_cols ..) and
+// a tile is whole pages of all heads, one box pair per page, each page laid
 // head-major in the stage; every key's accumulator row then carries every
 // head's columns.  A warp's 32 rows hold one head, or 32 / block_size heads,
 // and the warp reads only those heads' columns.
-constexpr int kMaxB = 256;                         // B rows: 2 * heads * n_cols <= the MMA's largest N
+constexpr int kMaxB = 256;                         // B rows: heads * head_cols <= the MMA's largest N
 constexpr int kAccCols = kMaxB;                    // columns per accumulator buffer
 // Accumulator buffers: the MMAs of a tile may run that many tiles ahead of
 // the epilogue.
 constexpr int kAccBufs = TRI_SMAX_ACC_BUFS;
 constexpr uint32_t kTmemCols = kAccBufs * kAccCols;
+// Warps: 0 producer, 1 MMA issue, then one epilogue warpgroup per accumulator
+// buffer (tile t of a CTA's walk goes to buffer and warpgroup t mod kAccBufs),
+// so the epilogue works on kAccBufs tiles at once.
+constexpr int kEpiWarps = 4 * kAccBufs;
+constexpr int kThreads = (2 + kEpiWarps) * 32;
 static_assert(kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "tensor memory columns");
 constexpr int kBBytesMax = kMaxB * kRowBytes;             // hi and lo parts of every head in B
 constexpr size_t kBOffset = static_cast<size_t>(kStages) * kStageBytes;
 constexpr size_t kBarOffset = kBOffset + kBBytesMax;
-constexpr size_t kSmemBytes = kBarOffset + 256 + 1024;    // barriers, slot, alignment slack
+// PAGED: page ids of the producer's next tiles, [2][kIdTiles][kMaxPages]
+constexpr int kIdTiles = 32;                              // tiles decoded at once, a lane each
+constexpr int kMaxPages = 16;                             // pages of a tile: 128 rows of >= 8 per page
+constexpr size_t kIdsOffset = kBarOffset + 256;
+constexpr size_t kSmemBytes = kIdsOffset + 2 * kIdTiles * kMaxPages * 4 + 1024;   // + alignment slack
 static_assert((2 * kStages + 2 * kAccBufs) * 8 + 8 <= 256, "barrier area");
 
 struct Args {
@@ -98,7 +107,7 @@ struct Args {
   float* scores;
   int ntiles;
   int n_offsets;         // 1 .. kMaxOffsets
-  int n_cols;            // n_offsets rounded up to 16
+  int head_cols;         // B rows (accumulator columns) per head: 2 n_offsets rounded up to 16
   int heads;             // heads in B: 1, or H for whole-page PAGED tiles
   int head_shift;        // log2(heads)
   int whole_pages;       // PAGED: tiles of whole pages of all heads (else of one head)
@@ -248,10 +257,12 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// W consecutive fp32 columns at ta and W at tb of this warp's 32
-// tensor-memory lanes (one lane per thread): both loads are issued and then
-// awaited once, inside one asm statement, so no use of the registers can be
-// scheduled ahead of the wait.
+// Consecutive fp32 columns at ta (as many as x holds) and at tb (as many as
+// y holds) of this warp's 32 tensor-memory lanes, one lane per thread: both
+// loads are issued and then awaited once, inside one asm statement, so no use
+// of the registers can be scheduled ahead of the wait.  Callers start every
+// load of 32 columns on a multiple of 32 and every load of 16 on a multiple
+// of 16.
 __device__ __forceinline__ void tmem_ld_pair(uint32_t ta, uint32_t tb, uint32_t (&x)[32], uint32_t (&y)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
@@ -292,11 +303,63 @@ __device__ __forceinline__ void tmem_ld_pair(uint32_t ta, uint32_t tb, uint32_t 
       : "memory");
 }
 
-// Byte offset of element (n, k) of a K-major operand with n_cols rows in two
+__device__ __forceinline__ void tmem_ld_pair(uint32_t ta, uint32_t tb, uint32_t (&x)[32], uint32_t (&y)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+      "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, "
+      "%20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31"
+      "}, [%48];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {"
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47"
+      "}, [%49];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7]),
+        "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]), "=r"(x[13]), "=r"(x[14]), "=r"(x[15]),
+        "=r"(x[16]), "=r"(x[17]), "=r"(x[18]), "=r"(x[19]), "=r"(x[20]), "=r"(x[21]), "=r"(x[22]), "=r"(x[23]),
+        "=r"(x[24]), "=r"(x[25]), "=r"(x[26]), "=r"(x[27]), "=r"(x[28]), "=r"(x[29]), "=r"(x[30]), "=r"(x[31]),
+        "=r"(y[0]), "=r"(y[1]), "=r"(y[2]), "=r"(y[3]), "=r"(y[4]), "=r"(y[5]), "=r"(y[6]), "=r"(y[7]),
+        "=r"(y[8]), "=r"(y[9]), "=r"(y[10]), "=r"(y[11]), "=r"(y[12]), "=r"(y[13]), "=r"(y[14]), "=r"(y[15])
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_pair(uint32_t ta, uint32_t tb, uint32_t (&x)[16], uint32_t (&y)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {"
+      "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15"
+      "}, [%48];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, "
+      "%34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47"
+      "}, [%49];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7]),
+        "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]), "=r"(x[13]), "=r"(x[14]), "=r"(x[15]),
+        "=r"(y[0]), "=r"(y[1]), "=r"(y[2]), "=r"(y[3]), "=r"(y[4]), "=r"(y[5]), "=r"(y[6]), "=r"(y[7]),
+        "=r"(y[8]), "=r"(y[9]), "=r"(y[10]), "=r"(y[11]), "=r"(y[12]), "=r"(y[13]), "=r"(y[14]), "=r"(y[15]),
+        "=r"(y[16]), "=r"(y[17]), "=r"(y[18]), "=r"(y[19]), "=r"(y[20]), "=r"(y[21]), "=r"(y[22]), "=r"(y[23]),
+        "=r"(y[24]), "=r"(y[25]), "=r"(y[26]), "=r"(y[27]), "=r"(y[28]), "=r"(y[29]), "=r"(y[30]), "=r"(y[31])
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_one(uint32_t ta, uint32_t (&x)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {"
+      "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15"
+      "}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7]),
+        "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]), "=r"(x[13]), "=r"(x[14]), "=r"(x[15])
+      : "r"(ta)
+      : "memory");
+}
+
+// Byte offset of element (n, k) of a K-major operand with n_rows rows in two
 // 64-element boxes, 128-byte swizzle: 16-byte chunk index XOR (row mod 8).
-__device__ __forceinline__ uint32_t sw128_offset(int n, int k, int n_cols) {
+__device__ __forceinline__ uint32_t sw128_offset(int n, int k, int n_rows) {
   const int box = k >> 6, kk = k & 63;
-  return static_cast<uint32_t>(box * n_cols * 128 + (n >> 3) * 1024 + (n & 7) * 128 +
+  return static_cast<uint32_t>(box * n_rows * 128 + (n >> 3) * 1024 + (n & 7) * 128 +
                                ((((kk >> 3) ^ (n & 7)) & 7) << 4) + (kk & 7) * 2);
 }
 
@@ -305,7 +368,7 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
   extern __shared__ unsigned char smax_raw[];
   unsigned char* smem = align_shared<1024>(smax_raw);
   unsigned char* bsm = smem + kBOffset;               // B: per head, hi rows then lo rows
-  const int n2 = 2 * a.heads * a.n_cols;
+  const int n2 = a.heads * a.head_cols;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOffset);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
@@ -350,65 +413,91 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
 
     // weights of this run's heads: bf16 hi / lo, swizzled (epilogue warps)
     if (warp >= 2) {
-      const int kcol = threadIdx.x - 64;              // 0..127: one element column
-      for (int m = 0; m < a.heads * a.n_cols; ++m) {
-        const int hh = m / a.n_cols, n = m - hh * a.n_cols;
+      const int kcol = (threadIdx.x - 64) & (kD - 1);   // one element column
+      const int part = (threadIdx.x - 64) / kD;         // the warpgroups share the offsets
+      const int per_head = a.head_cols >> 1;          // offset slots per head (the last ones zero)
+      for (int m = part; m < a.heads * per_head; m += kAccBufs) {
+        const int hh = m / per_head, n = m - hh * per_head;
         const int64_t lh = static_cast<int64_t>(run) * a.heads + hh;
         const float wv = n < a.n_offsets ? __ldg(a.w + (lh * a.n_offsets + n) * kD + kcol) : 0.f;
         const __nv_bfloat16 hi = __float2bfloat16_rn(wv);
         const __nv_bfloat16 lo = __float2bfloat16_rn(wv - __bfloat162float(hi));
-        const int row = hh * 2 * a.n_cols + n;
+        const int row = hh * a.head_cols + 2 * n;
         *reinterpret_cast<__nv_bfloat16*>(bsm + sw128_offset(row, kcol, n2)) = hi;
-        *reinterpret_cast<__nv_bfloat16*>(bsm + sw128_offset(row + a.n_cols, kcol, n2)) = lo;
+        *reinterpret_cast<__nv_bfloat16*>(bsm + sw128_offset(row + 1, kcol, n2)) = lo;
       }
       fence_async_smem();
     }
     __syncthreads();
 
     if (warp == 0 && g.layout == TRI_LAYOUT_PAGED) {
-      // ---------------- producer, PAGED: the whole warp, lane p on page p of
-      // the tile (block_size is a power of two, a page's rows fill whole 1 KB
-      // swizzle atoms and a tile is whole pages, at most 16).  The page ids
-      // of the next tile are loaded before this tile's slot is awaited; pages
-      // outside the pool are left out.
+      // ---------------- producer, PAGED: the whole warp.  Lane i decodes
+      // tile tc + i of a group of 32 and loads its page ids (the pages of a
+      // tile are at most 16: block_size is a power of two, a page's rows fill
+      // whole 1 KB swizzle atoms and a tile is whole pages) while the previous
+      // group's copies are issued; each group's ids go to shared memory.  Per
+      // tile, lane p copies page p; pages outside the pool are left out.
       const bool whole = a.whole_pages != 0;
       const uint32_t page_rows = static_cast<uint32_t>(g.block_size) << a.head_shift;
-      auto page_of = [&](const PagedTile& T) -> int32_t { return lane < T.np ? g.block_table[T.tbl + lane] : -1; };
-      Cursor cn = cursor_at(g, t0);
-      PagedTile Tn;
-      int32_t nxt = -1;
-      if (t0 < t1) {
-        Tn = paged_tile(g, cn, whole, a.scores);
-        nxt = page_of(Tn);
-      }
-      for (int t = t0; t < t1; ++t, ++k) {
-        const PagedTile T = Tn;
-        const int32_t cur = nxt;
-        if (t + 1 < t1) {
-          cursor_next(g, cn);
-          Tn = paged_tile(g, cn, whole, a.scores);
-          nxt = page_of(Tn);
+      int32_t* ids = reinterpret_cast<int32_t*>(smem + kIdsOffset);
+      int32_t v[kMaxPages];
+      auto fetch = [&](int tc, int& l_, int& h_, int& np_) {
+        const int ti = tc + lane;
+        l_ = h_ = np_ = 0;
+        if (ti < t1) {
+          const PagedTile T = paged_tile(g, cursor_at(g, ti), whole, a.scores);
+          l_ = T.l;
+          h_ = T.h;
+          np_ = T.np;
+#pragma unroll
+          for (int p = 0; p < kMaxPages; ++p) v[p] = p < np_ ? g.block_table[T.tbl + p] : -1;
         }
-        const int s = k % kStages, n = k / kStages;
-        int stop = 0;
-        if (lane == 0) {
-          if (n > 0 && !*abort_flag && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) *abort_flag = 1;
-          stop = *abort_flag;
+      };
+      auto stash = [&](int buf) {
+#pragma unroll
+        for (int p = 0; p < kMaxPages; ++p) ids[(buf * kIdTiles + lane) * kMaxPages + p] = v[p];
+      };
+      int cl, ch, cnp;
+      fetch(t0, cl, ch, cnp);
+      stash(0);
+      __syncwarp();
+      for (int tc = t0, buf = 0; tc < t1; tc += kIdTiles, buf ^= 1) {
+        const bool more = tc + kIdTiles < t1;
+        int nl = 0, nh = 0, nnp = 0;
+        if (more) fetch(tc + kIdTiles, nl, nh, nnp);    // in flight while this group is issued
+        const int nt = min(kIdTiles, t1 - tc);
+        for (int i = 0; i < nt; ++i, ++k) {
+          const int l = __shfl_sync(0xffffffffu, cl, i), h = __shfl_sync(0xffffffffu, ch, i);
+          const int np = __shfl_sync(0xffffffffu, cnp, i);
+          const int32_t cur = lane < np ? ids[(buf * kIdTiles + i) * kMaxPages + lane] : -1;
+          const int s = k % kStages, n = k / kStages;
+          int stop = 0;
+          if (lane == 0) {
+            if (n > 0 && !*abort_flag && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) *abort_flag = 1;
+            stop = *abort_flag;
+          }
+          if (__shfl_sync(0xffffffffu, stop, 0)) continue;
+          const bool valid = lane < np && static_cast<unsigned>(cur) < static_cast<unsigned>(g.num_blocks);
+          const uint32_t ok = __ballot_sync(0xffffffffu, valid);
+          if (lane == 0) {
+            if (ok != (1u << np) - 1u) flag(TRI_DEVFLAG_BAD_PAGE);
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(ok)) * page_rows * kRowBytes);
+          }
+          __syncwarp();                               // the expected bytes are set before any copy lands
+          if (valid) {
+            unsigned char* stage = smem + static_cast<size_t>(s) * kStageBytes;
+            const uint32_t off = static_cast<uint32_t>(lane) * page_rows * 128u;
+            tma_load_5d(stage + off, &kmap, 0, h, 0, cur, l, &full[s], policy);
+            tma_load_5d(stage + kBoxBytes + off, &kmap, 64, h, 0, cur, l, &full[s], policy);
+          }
         }
-        if (__shfl_sync(0xffffffffu, stop, 0)) continue;
-        const bool valid = lane < T.np && static_cast<unsigned>(cur) < static_cast<unsigned>(g.num_blocks);
-        const uint32_t ok = __ballot_sync(0xffffffffu, valid);
-        if (lane == 0) {
-          if (ok != (1u << T.np) - 1u) flag(TRI_DEVFLAG_BAD_PAGE);
-          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(ok)) * page_rows * kRowBytes);
+        if (more) {
+          stash(buf ^ 1);
+          cl = nl;
+          ch = nh;
+          cnp = nnp;
         }
-        __syncwarp();                                 // the expected bytes are set before any copy lands
-        if (valid) {
-          unsigned char* stage = smem + static_cast<size_t>(s) * kStageBytes;
-          const uint32_t off = static_cast<uint32_t>(lane) * page_rows * 128u;
-          tma_load_5d(stage + off, &kmap, 0, T.h, 0, cur, T.l, &full[s], policy);
-          tma_load_5d(stage + kBoxBytes + off, &kmap, 64, T.h, 0, cur, T.l, &full[s], policy);
-        }
+        __syncwarp();                                 // the group's ids are read before they are replaced
       }
     } else if (warp == 0) {
       // ---------------- producer, packed layouts: one thread
@@ -454,7 +543,9 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
         j += t1 - t0;
       }
     } else {
-      // ---------------- epilogue: one key per thread
+      // ---------------- epilogue: one key per thread; warpgroup eg takes the
+      // tiles of accumulator buffer eg (every kAccBufs-th tile of the walk)
+      const int eg = (warp - 2) >> 2;
       const int quarter = warp & 3;                   // tensor-memory lanes 32*quarter ..
       const int r = quarter * 32 + lane;
       // Row r of a tile.  Whole-page PAGED tiles hold each page head-major:
@@ -470,20 +561,52 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
         h_first = ((quarter * 32) >> g.block_shift) & (g.H - 1);
         heads_in_warp = min(g.H, max(1, 32 >> g.block_shift));
       }
-      Cursor c = cursor_at(g, t0);
-      for (int t = t0; t < t1; ++t, ++j) {
-        if (t > t0) cursor_next(g, c);
-        const int ab = j % kAccBufs, na = j / kAccBufs;
+      // PAGED: the page id of this thread's key, loaded a tile of this
+      // warpgroup ahead (the load's latency under a saturated memory system
+      // is about a tile's time)
+      const bool paged = g.layout == TRI_LAYOUT_PAGED;
+      auto page_id = [&](const PagedTile& T) -> int32_t {
+        return tok < T.tvalid ? g.block_table[T.tbl + (tok >> g.block_shift)] : -1;
+      };
+      // cc at tile t moves to tile t + kAccBufs (as far as the walk goes)
+      auto step = [&](Cursor& cc, int t) {
+        for (int i = 1; i <= kAccBufs && t + i < t1; ++i) cursor_next(g, cc);
+      };
+      const int j0 = j;
+      const int first = t0 + (((eg - j0) % kAccBufs) + kAccBufs) % kAccBufs;
+      j = j0 + (t1 - t0);                             // every epilogue warp's count after this run
+      Cursor c{}, cn{};
+      PagedTile Tn{};
+      int32_t pg_n = -1;
+      if (first < t1) {
+        c = cursor_at(g, first);
+        cn = c;
+        step(cn, first);
+        if (paged) {
+          Tn = paged_tile(g, c, whole, a.scores);
+          pg_n = page_id(Tn);
+        }
+      }
+      for (int t = first; t < t1; t += kAccBufs) {
+        if (t > first) {
+          c = cn;
+          step(cn, t);
+        }
+        const PagedTile Tc = Tn;
+        const int32_t pg = pg_n;
+        if (paged && t + kAccBufs < t1) {
+          Tn = paged_tile(g, cn, whole, a.scores);
+          pg_n = page_id(Tn);
+        }
+        const int jt = j0 + (t - t0);
+        const int ab = jt % kAccBufs, na = jt / kAccBufs;
         // the tile's output, decoded while the MMAs run; keys in pages outside
         // the pool are not written
         float* out;
         bool live;
-        if (g.layout == TRI_LAYOUT_PAGED) {
-          const PagedTile T = paged_tile(g, c, whole, a.scores);
-          out = T.out + hr * (static_cast<int64_t>(g.batch) * g.score_stride) + tok;
-          live = tok < T.tvalid &&
-                 static_cast<unsigned>(g.block_table[T.tbl + (tok >> g.block_shift)]) <
-                     static_cast<unsigned>(g.num_blocks);
+        if (paged) {
+          out = Tc.out + hr * (static_cast<int64_t>(g.batch) * g.score_stride) + tok;
+          live = tok < Tc.tvalid && static_cast<unsigned>(pg) < static_cast<unsigned>(g.num_blocks);
         } else {
           const PackedTile T = packed_tile(g, c, a.scores);
           out = T.out + tok;
@@ -499,26 +622,50 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
         float best = 0.f;
         for (int i = 0; i < heads_in_warp; ++i) {
           const int hh = h_first + i;
-          const uint32_t hcol = taddr + static_cast<uint32_t>(hh * 2 * a.n_cols);
           float m = 0.f;
-          for (int c0 = 0; c0 < a.n_cols; c0 += 32) {    // hi + lo, 32 (or the last 16) offsets at a time
-            if (c0 + 32 <= a.n_cols) {
-              uint32_t x[32], y[32];
-              tmem_ld_pair(hcol + static_cast<uint32_t>(c0), hcol + static_cast<uint32_t>(a.n_cols + c0), x, y);
+          // columns 2n, 2n + 1 = offset n's hi and lo products
+          auto take = [&](const uint32_t* v, int cnt, int n0) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const float v = __uint_as_float(x[e]) + __uint_as_float(y[e]);
-                if (c0 + e < a.n_offsets) m = c0 + e == 0 ? v : fmaxf(m, v);
-              }
-            } else {
-              uint32_t x[16], y[16];
-              tmem_ld_pair(hcol + static_cast<uint32_t>(c0), hcol + static_cast<uint32_t>(a.n_cols + c0), x, y);
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const float v = __uint_as_float(x[e]) + __uint_as_float(y[e]);
-                if (c0 + e < a.n_offsets) m = c0 + e == 0 ? v : fmaxf(m, v);
-              }
+            for (int e = 0; e < cnt / 2; ++e) {
+              const float s2 = __uint_as_float(v[2 * e]) + __uint_as_float(v[2 * e + 1]);
+              if (n0 + e < a.n_offsets) m = n0 + e == 0 ? s2 : fmaxf(m, s2);
             }
+          };
+          // up to two loads per wait; a load of 32 columns only from a
+          // multiple of 32 (a head's block may start on an odd multiple of 16)
+          const int c_head = hh * a.head_cols, c_end = c_head + a.head_cols;
+          for (int col = c_head; col < c_end;) {
+            const int w1 = ((col & 31) == 0 && c_end - col >= 32) ? 32 : 16;
+            const int c2 = col + w1;
+            const int w2 = c2 >= c_end ? 0 : ((c2 & 31) == 0 && c_end - c2 >= 32) ? 32 : 16;
+            const uint32_t ca = taddr + static_cast<uint32_t>(col), cb = taddr + static_cast<uint32_t>(c2);
+            const int n0 = (col - c_head) >> 1, n1 = (c2 - c_head) >> 1;
+            if (w1 == 32 && w2 == 32) {
+              uint32_t x[32], y[32];
+              tmem_ld_pair(ca, cb, x, y);
+              take(x, 32, n0);
+              take(y, 32, n1);
+            } else if (w1 == 32 && w2 == 16) {
+              uint32_t x[32], y[16];
+              tmem_ld_pair(ca, cb, x, y);
+              take(x, 32, n0);
+              take(y, 16, n1);
+            } else if (w1 == 16 && w2 == 32) {
+              uint32_t x[16], y[32];
+              tmem_ld_pair(ca, cb, x, y);
+              take(x, 16, n0);
+              take(y, 32, n1);
+            } else if (w2 != 0 || w1 == 32) {     // 16 + 16, or 32 as two 16s
+              uint32_t x[16], y[16];
+              tmem_ld_pair(ca, ca + 16u, x, y);
+              take(x, 16, n0);
+              take(y, 16, n0 + 8);
+            } else {
+              uint32_t x[16];
+              tmem_ld_one(ca, x);
+              take(x, 16, n0);
+            }
+            col += w1 + (w2 != 0 ? w2 : 0);
           }
           if (hh == hr) best = m;
         }

@@ -777,13 +777,13 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   if (!w || !scores || !aligned16(w) || !aligned16(scores) || n_offsets < 1) return TRI_ERR_INVALID_ARG;
   if (n_offsets > tri::smax::kMaxOffsets) return TRI_ERR_UNSUPPORTED;
   const bool paged = desc->layout == TRI_LAYOUT_PAGED;
-  const int n_cols = (n_offsets + 15) & ~15;
+  const int head_cols = (2 * n_offsets + 15) & ~15;   // hi and lo column of every offset, per head
   int64_t rows = 0;
   // PAGED: whole pages of all heads per tile when every head's weights fit
-  // one MMA (2 H n_cols <= 256) and a page of all heads fills whole swizzle
+  // one MMA (H head_cols <= 256) and a page of all heads fills whole swizzle
   // atoms (H block_size a power of two >= 8, so whole pages fill the 128
   // rows); else one head's rows per tile, pages of a power of two >= 8 tokens.
-  const bool whole = paged && g.block_shift >= 0 && g.H * n_cols <= tri::smax::kMaxB / 2 &&
+  const bool whole = paged && g.block_shift >= 0 && g.H * head_cols <= tri::smax::kMaxB &&
                      (g.block_size * g.H) >= 8;
   if (paged) {
     if (!whole && g.block_shift < 3) return TRI_ERR_UNSUPPORTED;
@@ -802,7 +802,7 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   st = paged ? encode_paged_key_map(desc, whole, &map) : encode_key_map(desc, rows, &map);
   if (st != TRI_OK) return st;
   const int heads = whole ? g.H : 1;
-  tri::smax::Args a{w, scores, static_cast<int>(ntiles), n_offsets, n_cols, heads, __builtin_ctz(heads),
+  tri::smax::Args a{w, scores, static_cast<int>(ntiles), n_offsets, head_cols, heads, __builtin_ctz(heads),
                     whole ? 1 : 0};
   const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].smax_blocks_per_sm;
   const int grid = static_cast<int>(ntiles < resident ? ntiles : resident);
