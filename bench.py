@@ -125,7 +125,7 @@ def score_kernel_fingerprint(variant="mean"):
 def traffic_record(workload, variant="mean"):
     """The committed ncu traffic record of a variant's scorer on a workload."""
     if gen.WORKLOADS[workload].layout == "paged":
-        return f"score_keys_paged_{workload}_traffic.txt"
+        return f"{'score_max' if variant == 'max' else 'score_keys'}_paged_{workload}_traffic.txt"
     return SCORE_KERNELS[variant][2]
 
 
@@ -509,13 +509,18 @@ def run_paged(args, tri, dev, rank, ws):
     """The paged serving cache: an initial pruning event, then steady rounds
     (append PAGED_APPEND tokens per sequence, untimed; re-compress in place).
     The initial event is four calls (fold, score, select, in-place hole fill),
-    a steady round two (fold, tri_compress in place).  Every event is queued
-    behind a GPU sleep so that the launches are all waiting when the first one
-    runs, and timed with CUDA events on the launching stream; L2 is flushed
-    (a 512 MB fill) before every event."""
+    a steady round two (fold, tri_compress in place) for the folded score, and
+    four for the max over the offsets (per-offset fold, score_keys_max,
+    select, in-place hole fill: tri_compress runs the folded score only).
+    Every event is queued behind a GPU sleep so that the launches are all
+    waiting when the first one runs, and timed with CUDA events on the
+    launching stream; L2 is flushed (a 512 MB fill) before every event."""
     _, _, local = dist_env()
     if args.shard != "replicas":
         raise SystemExit("the paged workload runs as replicas (one cache per rank)")
+    if args.variant == "pos":
+        raise SystemExit("the paged workload runs the folded score (mean) or the max over the offsets (max)")
+    use_max = args.variant == "max"
     wl = gen.WORKLOADS[args.workload]
     B = wl.budget
     L, H = wl.num_layers, wl.num_kv_heads
@@ -527,7 +532,8 @@ def run_paged(args, tri, dev, rank, ws):
         f"({sum(cache.lens) * L * H / 1e6:.1f} M keys)")
     units = wl.units
     qc = cache.query_center.reshape(-1, wl.head_dim).to(dev).contiguous()
-    w = torch.empty_like(qc)
+    w = (torch.empty((qc.shape[0], len(wl.offsets), wl.head_dim), dtype=torch.float32, device=dev) if use_max
+         else torch.empty_like(qc))
     kept = torch.empty((units, B), dtype=torch.int32, device=dev)
     cnt = torch.empty((units,), dtype=torch.int32, device=dev)
     flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
@@ -537,6 +543,18 @@ def run_paged(args, tri, dev, rank, ws):
 
     ws_buf = None                                  # tri_compress's workspace (the score matrix)
 
+    def fold():
+        if use_max:
+            tri.fold_offset_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+        else:
+            tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+
+    def score(d, scores):
+        if use_max:
+            tri.score_keys_max(d, w, scores, stream=stream)
+        else:
+            tri.score_keys(d, w, scores, stream=stream)
+
     def event(d, scores, evs=None):
         """The initial pruning event, one call per stage: fold, score, select,
         in-place hole fill.  evs: five events around the four calls."""
@@ -544,9 +562,9 @@ def run_paged(args, tri, dev, rank, ws):
             if evs is not None:
                 evs[i].record(stream)
         rec(0)
-        tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+        fold()
         rec(1)
-        tri.score_keys(d, w, scores, stream=stream)
+        score(d, scores)
         rec(2)
         tri.select_topk(d, scores, B, kept, cnt, stream=stream)
         rec(3)
@@ -558,18 +576,31 @@ def run_paged(args, tri, dev, rank, ws):
         warp per row that selects and fills the row's holes).  score_alone: a
         score matrix; the scorer and then the selection (without the fill) run
         on their own first, each timed (the breakdown round; compress then
-        redoes both).  evs: events around each call."""
+        redoes both).  The max over the offsets: per-offset fold, then the
+        scorer, the selection and the in-place hole fill as three calls into
+        score_alone.  evs: events around each call."""
         nonlocal ws_buf
-        need = tri.workspace_size(d, B)
-        if ws_buf is None or ws_buf.numel() < need:
-            ws_buf = torch.empty(need, dtype=torch.uint8, device=dev)
         marks = iter(evs or [])
 
         def rec():
             if evs is not None:
                 next(marks).record(stream)
+        if use_max:
+            rec()
+            fold()
+            rec()
+            tri.score_keys_max(d, w, score_alone, stream=stream)
+            rec()
+            tri.select_topk(d, score_alone, B, kept, cnt, stream=stream)
+            rec()
+            tri.compact_kv(d, kept, cnt, B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None, stream=stream)
+            rec()
+            return
+        need = tri.workspace_size(d, B)
+        if ws_buf is None or ws_buf.numel() < need:
+            ws_buf = torch.empty(need, dtype=torch.uint8, device=dev)
         rec()
-        tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+        fold()
         rec()
         if score_alone is not None:
             tri.score_keys(d, w, score_alone, stream=stream)
@@ -595,8 +626,8 @@ def run_paged(args, tri, dev, rank, ws):
     scores0 = torch.empty((units, tri.score_row_stride(d0)), dtype=torch.float32, device=dev)
     keys0 = sum(cache.lens) * L * H
     for _ in range(args.warmup):
-        tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
-        tri.score_keys(d0, w, scores0, stream=stream)
+        fold()
+        score(d0, scores0)
         tri.select_topk(d0, scores0, B, kept, cnt, stream=stream)
     per0, moved0 = timed(lambda evs: event(d0, scores0, evs), 5)
     gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
@@ -623,7 +654,10 @@ def run_paged(args, tri, dev, rank, ws):
                 torch.distributed.barrier()
             t0 = time.time()
             launches0 = tri.kernel_launches()
-        per, moved = timed(lambda evs: steady(d, evs), 3)
+        if use_max:
+            per, moved = timed(lambda evs: steady(d, evs, score_alone=scores), 5)
+        else:
+            per, moved = timed(lambda evs: steady(d, evs), 3)
         if i >= args.warmup:
             rounds.append((per, moved, sum(cache.lens) * L * H))
         gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
@@ -632,9 +666,10 @@ def run_paged(args, tri, dev, rank, ws):
     sampler.stop()
     clocks = sampler.summary(t0, t1)
     clocks["window"] = "the steady rounds, appends between them included"
-    # breakdown rounds: the scorer alone, then the same round
+    # breakdown rounds (folded score): the scorer alone, then the same round;
+    # the max rounds are four calls, timed one by one already
     per1 = []
-    for j in range(PAGED_BREAKDOWN_ROUNDS):
+    for j in range(0 if use_max else PAGED_BREAKDOWN_ROUNDS):
         gen.append_tokens(cache, PAGED_APPEND, step=1 + args.warmup + args.steps + j)
         d = tri.desc_paged(cache.k, cache.v, cache.block_table, cache.lens)
         per1.append(timed(lambda evs: steady(d, evs, score_alone=scores), 5)[0])
@@ -644,7 +679,7 @@ def run_paged(args, tri, dev, rank, ws):
     if st:
         raise RuntimeError(f"device status {st:#x} after the steady rounds")
 
-    per = np.array([r[0] for r in rounds])       # ms: fold, compress
+    per = np.array([r[0] for r in rounds])       # ms: fold, compress (max: fold, score, select, hole fill)
     ms_rounds = float(per.sum())
     ms_max = max_over_ranks(ms_rounds, ws, dev)
     keys_round = rounds[0][2]
@@ -652,7 +687,7 @@ def run_paged(args, tri, dev, rank, ws):
     value = keys_round * len(rounds) * ws / (ms_max / 1e3)
     ms_step = ms_max / len(rounds)
     peak, peak_kind = measured_hbm_peak()
-    score_ms = float(per1[:, 1].mean())
+    score_ms = float(per[:, 1].mean()) if use_max else float(per1[:, 1].mean())
     score_bytes = keys_round * KEY_BYTES
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     step_bytes = keys_round * KEY_BYTES + moved * MOVE_BYTES
@@ -660,13 +695,14 @@ def run_paged(args, tri, dev, rank, ws):
     init_ms = float(sum(per0))
     init_bytes = keys0 * KEY_BYTES + moved0 * MOVE_BYTES
 
-    e2e = run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws, lambda dd: steady(dd))
+    e2e = run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws,
+                        lambda dd: steady(dd, score_alone=scores if use_max else None))
 
     result = None
     if rank == 0:
         cpu = cpu_baseline(wl, args) if ws == 1 and not args.no_cpu_baseline else None
         result = {
-            "metric": METRICS["mean"] + ", paged cache, in place",
+            "metric": METRICS[args.variant] + ", paged cache, in place",
             "value": value, "unit": "keys/s", "n_gpus": ws, "steps": len(rounds), "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16 keys/values, fp32 scores (fp64 fold)", "data": "synthetic (seeded generator)",
@@ -678,15 +714,18 @@ def run_paged(args, tri, dev, rank, ws):
                        "keys_per_gpu": keys_round, "budget": B, "parallelism": f"independent caches x{ws}",
                        "l2": "L2 flushed before every pruning event, outside the events: a 512 MB buffer "
                              "written then read back (the write's dirty lines drain before the event)"},
-            "step_breakdown_ms": {"fold": float(per[:, 0].mean()), "compress": float(per[:, 1].mean()),
-                                  "score (alone)": score_ms,
-                                  "select alone (no fill, scores fresh in L2)": float(per1[:, 2].mean()),
-                                  "select + hole fill (compress minus score alone)":
-                                      float(per[:, 1].mean()) - score_ms,
-                                  "breakdown": f"score alone, select alone: {PAGED_BREAKDOWN_ROUNDS} more rounds, "
-                                               "each with the scorer and then the selection run on their own "
-                                               "(after the flush) before the compress call; select + hole fill: "
-                                               "the timed rounds' compress minus the scorer alone"},
+            "step_breakdown_ms": ({"fold (per offset)": float(per[:, 0].mean()), "score": score_ms,
+                                   "select": float(per[:, 2].mean()), "hole fill": float(per[:, 3].mean()),
+                                   "breakdown": "the timed rounds' four calls, one event each"} if use_max else
+                                  {"fold": float(per[:, 0].mean()), "compress": float(per[:, 1].mean()),
+                                   "score (alone)": score_ms,
+                                   "select alone (no fill, scores fresh in L2)": float(per1[:, 2].mean()),
+                                   "select + hole fill (compress minus score alone)":
+                                       float(per[:, 1].mean()) - score_ms,
+                                   "breakdown": f"score alone, select alone: {PAGED_BREAKDOWN_ROUNDS} more "
+                                                "rounds, each with the scorer and then the selection run on "
+                                                "their own (after the flush) before the compress call; select + "
+                                                "hole fill: the timed rounds' compress minus the scorer alone"}),
             "rows_moved_per_step": moved,
             "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_gbs,
                     "frac_of_measured": step_gbs / peak, "frac_of_8tbps_spec": step_gbs / SPEC_HBM_GBS},
@@ -697,14 +736,17 @@ def run_paged(args, tri, dev, rank, ws):
                               "frac_of_8tbps_spec": init_bytes / (init_ms / 1e3) / 1e9 / SPEC_HBM_GBS,
                               "timing": "one event (it compacts the cache in place), after warm-up passes of "
                                         "the fold, score and select"},
-            "roofline": {"kernel": "score_kernel (paged)", "bound": "hbm", "achieved": achieved, "peak": peak,
+            "roofline": {"kernel": f"{SCORE_KERNELS[args.variant][0]} (paged)", "bound": "hbm",
+                         "achieved": achieved, "peak": peak,
                          "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": ncu_traffic(args.workload, "mean"),
+                         "traffic": ncu_traffic(args.workload, args.variant),
                          "algorithmic_bytes_per_launch": score_bytes},
             "clocks": clocks,
             "gpu_launches": int(launches),
-            "timing": "each round: plain launches queued behind a GPU sleep, CUDA events around the fold and "
-                      "the compress call",
+            "timing": ("each round: plain launches queued behind a GPU sleep, CUDA events around each of the "
+                       "four calls" if use_max else
+                       "each round: plain launches queued behind a GPU sleep, CUDA events around the fold and "
+                       "the compress call"),
             "e2e": e2e,
             "cpu_baseline": cpu,
         }

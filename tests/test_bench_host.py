@@ -75,6 +75,17 @@ def test_traffic_record_follows_the_sources(tmp_path, monkeypatch):
     assert bench.ncu_traffic("qwen3_full", "mean") is None
 
 
+def test_paged_records_are_kept_per_scorer(tmp_path, monkeypatch):
+    """The paged workload has a record for the folded scorer and one for the
+    max scorer; neither stands in for the other."""
+    _tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_record("qwen25_paged", "mean") != bench.traffic_record("qwen25_paged", "max")
+    _record(tmp_path, "max", "qwen25_paged", bench.score_kernel_fingerprint("max"), 777)
+    assert bench.ncu_traffic("qwen25_paged", "max") == 777
+    assert bench.ncu_traffic("qwen25_paged", "mean") is None
+
+
 def test_fingerprints_cover_each_scorers_sources(tmp_path, monkeypatch):
     csrc = _tree(tmp_path)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
