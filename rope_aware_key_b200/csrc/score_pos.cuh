@@ -123,9 +123,12 @@ __device__ __forceinline__ float2 hi_hi(uint32_t a, uint32_t b) {
 __device__ __forceinline__ uint32_t word(const uint4& x, int i) { return i == 0 ? x.x : i == 1 ? x.y : i == 2 ? x.z : x.w; }
 
 // Two bands (the x and y halves) of one key, added into acc:
-//   Re a conj(k) e^{i phi'} = k_r (a_r cos phi' - a_i sin phi') + k_i (a_r sin phi' + a_i cos phi')
+//   Re a conj(k) e^{i phi'} = cos phi' (a_r k_r + a_i k_i) + sin phi' (a_r k_i - a_i k_r)
 // with phi' the phase minus pi, built from the bits of |Delta| C_f (see the
-// top of the file).
+// top of the file).  The two products of the key and the weight do not
+// depend on the phase, so they are formed while the sine and cosine are in
+// flight, and one packed FMA each then adds them in: six packed operations
+// for the two bands.
 __device__ __forceinline__ float2 band_pair(float2 kr, float2 ki, float2 ar, float2 ai, uint32_t hi0, uint32_t lo0,
                                             uint32_t hi1, uint32_t lo1, uint32_t D, float2 sc, float2 off,
                                             float2 acc) {
@@ -137,13 +140,10 @@ __device__ __forceinline__ float2 band_pair(float2 kr, float2 ki, float2 ar, flo
   float2 sn, cs;
   __sincosf(phi.x, &sn.x, &cs.x);
   __sincosf(phi.y, &sn.y, &cs.y);
-  // b = a e^{i phi'} first, then Re conj(k) b = k_r b_r + k_i b_i: six packed
-  // operations for the two bands
-  const float2 p = __fmul2_rn(ai, sn);
-  const float2 br = __ffma2_rn(ar, cs, make_float2(-p.x, -p.y));
-  const float2 bi = __ffma2_rn(ar, sn, __fmul2_rn(ai, cs));
-  acc = __ffma2_rn(kr, br, acc);
-  return __ffma2_rn(ki, bi, acc);
+  const float2 P = __ffma2_rn(ar, kr, __fmul2_rn(ai, ki));                          // a_r k_r + a_i k_i
+  const float2 Q = __ffma2_rn(ar, ki, __fmul2_rn(make_float2(-ai.x, -ai.y), kr));   // a_r k_i - a_i k_r
+  acc = __ffma2_rn(cs, P, acc);
+  return __ffma2_rn(sn, Q, acc);
 }
 
 // Per-key distance terms shared by the scorers: whether t_b - p_i is in
