@@ -97,6 +97,7 @@ def test_score_max_ragged_edges():
 
 @pytest.mark.parametrize("H,bs,n_off", [
     (4, 16, 17), (1, 128, 17), (2, 32, 17), (4, 4, 17), (8, 2, 16), (8, 16, 5), (2, 64, 64),  # whole pages
+    (8, 1, 16), (2, 4, 17),                              # a page of all heads is one 8-row swizzle atom
     (8, 8, 17), (8, 16, 33), (4, 32, 64),                                                     # one head
 ])
 def test_score_max_paged(H, bs, n_off):
