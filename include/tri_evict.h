@@ -224,9 +224,12 @@ tri_status tri_score_keys_at_positions(const tri_cache_desc* desc, const float* 
  * to back (stride_seq = seq_len*128, stride_head = batch*stride_seq,
  * stride_layer = H*stride_head for CONTIG; stride_head = T*128 and
  * stride_layer = H*stride_head for RAGGED with T = cu_seqlens[batch]), and
- * PAGED caches whose block_size is a power of two >= 8 (a page id outside the
- * pool sets TRI_DEVFLAG_BAD_PAGE and that page's scores are not written);
- * anything else, or n_offsets > TRI_MAX_SCORE_OFFSETS, is TRI_ERR_UNSUPPORTED.
+ * PAGED caches whose block_size is a power of two and where either
+ * num_kv_heads * (2*n_offsets rounded up to 16) <= 256 and
+ * num_kv_heads * block_size >= 8 (tiles of whole pages of all heads), or
+ * block_size >= 8 (tiles of one head); a page id outside the pool sets
+ * TRI_DEVFLAG_BAD_PAGE and that page's scores are not written.  Anything
+ * else, or n_offsets > TRI_MAX_SCORE_OFFSETS, is TRI_ERR_UNSUPPORTED.
  * scores: as for tri_score_keys. */
 tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_offsets, float* scores,
                               tri_stream_t stream);
