@@ -17,8 +17,9 @@
 //  1. of 256 evenly spaced scores of the row (8 per lane), the ones at ranks
 //     B/n * 256 -/+ (4 sigma + 8) from the top give two keys U >= L that
 //     bracket the B-th largest key for any but a pathological order of the
-//     scores; each is found by a bitwise search over the samples' key range
-//     (a step counts the samples below a trial key: one warp reduction);
+//     scores; each is located to two 8-bit digits of the samples' key range
+//     (a shared histogram per digit), U at the top of its bin and L at the
+//     bottom, which only widens the bracket;
 //  2. one pass over the row counts the keys above U (all kept) and gathers
 //     the keys in [L, U] into a candidate buffer, in index order (the
 //     comparisons are made on the floats; the candidates are stored as float
@@ -78,33 +79,18 @@ __device__ __forceinline__ float4 row_chunk(const float* __restrict__ row, int n
   return x;
 }
 
-// The k-th smallest (1 <= k <= 256) of the 256 keys the lanes hold, 8 each,
-// whose range is [lo, hi]: the largest t in [lo, hi] with fewer than k keys
-// below it (the count never decreases with t), found bit by bit of t - lo.
-__device__ __forceinline__ uint32_t warp_kth_smallest(const uint32_t (&x)[8], uint32_t lo, uint32_t hi, uint32_t k) {
-  uint32_t t = lo;                                 // fewer than k keys below t
-  const uint32_t span = hi - lo;
-  for (int bit = span ? 31 - __clz(span) : -1; bit >= 0; --bit) {
-    const uint64_t trial = uint64_t{t} + (uint64_t{1} << bit);
-    if (trial > hi) continue;                      // warp-uniform
-    uint32_t c = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) c += x[e] < static_cast<uint32_t>(trial);
-    if (__reduce_add_sync(0xffffffffu, c) < k) t = static_cast<uint32_t>(trial);
-  }
-  return t;
-}
-
 // The need-th largest (need >= 1) of the keys in [lo, hi] among the keys the
 // lanes pass through `each` (at least `need` of them lie in [lo, hi]), by
 // 8-bit digits of key - lo, most significant first: each digit's histogram
 // (hist, 256 words) picks the bin that holds the rank.  *need becomes the
-// rank of the result among the keys equal to it.
+// rank of the result among the keys equal to it.  With max_digits, the search
+// stops after that many digits: the result is then in [returned, *hi_out].
 template <typename Each>
 __device__ __forceinline__ uint32_t warp_radix_kth(Each each, uint32_t lo, uint32_t hi, uint32_t* need,
-                                                   uint32_t* hist) {
+                                                   uint32_t* hist, int max_digits = 4,
+                                                   uint32_t* hi_out = nullptr) {
   const int lane = threadIdx.x & 31;
-  while (lo < hi) {
+  for (int digit = 0; lo < hi && digit < max_digits; ++digit) {
     const int bits = 32 - __clz(hi - lo);
     const int shift = bits > 8 ? bits - 8 : 0;
     __syncwarp();
@@ -149,6 +135,7 @@ __device__ __forceinline__ uint32_t warp_radix_kth(Each each, uint32_t lo, uint3
     const uint64_t top = static_cast<uint64_t>(lo) + ((uint64_t{1} << shift) - 1u);   // no wrap near 2^32
     hi = top < hi ? static_cast<uint32_t>(top) : hi;
   }
+  if (hi_out) *hi_out = hi;
   return lo;
 }
 
@@ -179,9 +166,23 @@ __device__ __forceinline__ bool warp_select_row(const float* __restrict__ row, i
   const float r = static_cast<float>(B) * kWarpSamples / static_cast<float>(n);
   const float delta = 4.f * sqrtf(r * (1.f - r / kWarpSamples)) + 8.f;
   const int r_hi = static_cast<int>(floorf(r - delta)), r_lo = static_cast<int>(ceilf(r + delta));
-  // the r_hi-th and r_lo-th largest samples (ranks counted from the top)
-  const uint32_t U = r_hi >= 1 ? warp_kth_smallest(x, kmin, kmax, kWarpSamples + 1 - r_hi) : 0xffffffffu;
-  const uint32_t L0 = r_lo <= kWarpSamples ? warp_kth_smallest(x, kmin, kmax, kWarpSamples + 1 - r_lo) : 0u;
+  // the r_hi-th and r_lo-th largest samples (ranks counted from the top), to
+  // two 8-bit digits of the samples' key range: U is taken at the top of its
+  // last bin and L at the bottom, so each bound only widens the bracket (by
+  // less than 2^-15 of the samples' key range)
+  auto each_sample = [&](auto fn) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) fn(x[e]);
+  };
+  uint32_t U = 0xffffffffu, L0 = 0u;
+  if (r_hi >= 1) {
+    uint32_t rank = static_cast<uint32_t>(r_hi);
+    warp_radix_kth(each_sample, kmin, kmax, &rank, S.hist, 2, &U);
+  }
+  if (r_lo <= kWarpSamples) {
+    uint32_t rank = static_cast<uint32_t>(r_lo);
+    L0 = warp_radix_kth(each_sample, kmin, kmax, &rank, S.hist, 2);
+  }
   // rows that evict few keys (no lower bound; also when the bound is NaN's key)
   const bool few = L0 == 0u;
   // the same bounds as floats: above U is v > uf (NaN never is), in [L, U] is
