@@ -451,6 +451,9 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
           np_ = T.np;
 #pragma unroll
           for (int p = 0; p < kMaxPages; ++p) v[p] = p < np_ ? g.block_table[T.tbl + p] : -1;
+        } else {
+#pragma unroll
+          for (int p = 0; p < kMaxPages; ++p) v[p] = -1;     // past the range: no pages
         }
       };
       auto stash = [&](int buf) {
