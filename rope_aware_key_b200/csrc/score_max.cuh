@@ -407,6 +407,7 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
   const uint32_t idesc = instr_desc(n2);
   const uint64_t policy = policy_evict_first();
   int k = 0, j = 0;                                   // stage-ring and accumulator counters
+  int j_last = -1;                                    // MMA thread: the last tile whose MMAs it committed
   for (int t0 = t_begin; t0 < t_end;) {
     const int run = t0 / per_run;
     const int t1 = min(t_end, (run + 1) * per_run);
@@ -473,6 +474,9 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
           const int l = __shfl_sync(0xffffffffu, cl, i), h = __shfl_sync(0xffffffffu, ch, i);
           const int np = __shfl_sync(0xffffffffu, cnp, i);
           const int32_t cur = lane < np ? ids[(buf * kIdTiles + i) * kMaxPages + lane] : -1;
+#ifdef TRI_TEST_HOOKS
+          if (tc + i == g.test_skip_tile) continue;   // test builds: no copy and no arrival for this tile
+#endif
           const int s = k % kStages, n = k / kStages;
           int stop = 0;
           if (lane == 0) {
@@ -509,6 +513,9 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
         for (int t = t0; t < t1; ++t, ++k) {
           if (t > t0) cursor_next(g, c);
           const int row = packed_tile(g, c, a.scores).row;
+#ifdef TRI_TEST_HOOKS
+          if (t == g.test_skip_tile) continue;        // test builds: no copy and no arrival for this tile
+#endif
           const int s = k % kStages, n = k / kStages;
           if (n > 0 && !*abort_flag && !mbar_wait_bounded(&empty[s], (n - 1) & 1)) *abort_flag = 1;
           if (*abort_flag) continue;
@@ -540,6 +547,7 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
           }
           mma_commit(&empty[s]);        // the stage is free once these MMAs have read it
           mma_commit(&acc_full[ab]);    // the accumulator is ready
+          j_last = j;
         }
       } else {
         k += t1 - t0;
@@ -682,10 +690,14 @@ score_max_kernel(const __grid_constant__ Geom g, const __grid_constant__ CUtenso
     __syncthreads();   // the next run's weights overwrite B
   }
 
-  // never exit with copies in flight (only possible after an abort)
+  // never exit with copies in flight, nor free tensor memory under MMAs still
+  // running (only possible after an abort): the producer waits for its
+  // copies, the MMA thread for its last commit (commits complete in order)
   if (warp == 0 && lane == 0 && *abort_flag) {
     for (int s = 0; s < kStages && s < k; ++s) mbar_wait_bounded(&full[s], ((k - 1 - s) / kStages) & 1);
   }
+  if (warp == 1 && lane == 0 && *abort_flag && j_last >= 0)
+    mbar_wait_bounded(&acc_full[j_last % kAccBufs], (j_last / kAccBufs) & 1);
   if (*abort_flag && threadIdx.x == 0) flag(TRI_DEVFLAG_TIMEOUT);
   tc_fence_before();
   __syncthreads();

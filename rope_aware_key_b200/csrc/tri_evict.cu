@@ -801,6 +801,9 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   CUtensorMap map;
   st = paged ? encode_paged_key_map(desc, whole, &map) : encode_key_map(desc, rows, &map);
   if (st != TRI_OK) return st;
+#ifdef TRI_TEST_HOOKS
+  g.test_skip_tile = g_test_skip_tile.load();
+#endif
   const int heads = whole ? g.H : 1;
   tri::smax::Args a{w, scores, static_cast<int>(ntiles), n_offsets, head_cols, heads, __builtin_ctz(heads),
                     whole ? 1 : 0};

@@ -3,8 +3,8 @@
 Two test-only builds of the library's sources (never the product library):
 
 * "hooks": every bounded wait gives up after 1 ms instead of about 2 s, and
-  the score producer can be told to leave one tile out -- no copy and no
-  arrival on its barrier.  The consumers of that tile then wait in vain,
+  the producer of the folded scorer or of the max scorer can be told to leave
+  one tile out -- no copy and no arrival on its barrier.  The consumers of that tile then wait in vain,
   give up, set TRI_DEVFLAG_TIMEOUT and leave the kernel; the producer's own
   waits end the same way, after it has waited for every copy it did issue,
   so no copy is in flight into an exiting CTA.  The host reads
@@ -70,6 +70,45 @@ def test_bounded_wait_runs_out_then_recovers(monkeypatch):
     assert res.status == 0
     _check_units(cache, res, [(0, 0, 0), (0, 3, 0), (0, 7, 0)])
     parity.check_all_units_properties(cache, res)
+
+
+@pytest.mark.parametrize("layout", ["contig", "paged"])
+def test_max_scorer_wait_runs_out_then_recovers(layout, monkeypatch):
+    """The tensor-core max scorer: its producer leaves one tile out; the MMA
+    thread's wait gives up, the epilogue and the producer stop, the producer
+    waits for the copies it did issue and the MMA thread for its last commit
+    before the tensor memory is freed; the next call is clean and right."""
+    from tests import test_gpu_score_max as tm
+    tri, V = _variant("hooks", monkeypatch)
+    if layout == "contig":
+        wl = gen.scaled(gen.WORKLOADS["qwen3_layer"], seq_len=32768)      # 2048 tiles, ~14 per CTA
+        cache = gen.make_cache(wl, seed=31, device=DEV, with_values=False)
+        skip = 20
+    else:                                                                # whole-page tiles of 4 heads
+        wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, batch=8, spare_blocks_per_seq=1)
+        cache = gen.make_cache(wl, seed=32, device=DEV, with_values=False, lens=[2176] * 8)
+        skip = 10
+    d = parity.make_desc(cache)
+    qc = cache.query_center.reshape(-1, wl.head_dim).to(DEV).contiguous()
+    w = tri.fold_offset_weights(qc, wl.theta, tm.GEO17)
+    assert tri.read_device_status() == 0
+    V.tri_test_skip_tile(skip)
+    try:
+        tri.score_keys_max(d, w)
+        flags = ctypes.c_uint32(0)
+        st = V.tri_read_device_status(tri._stream(None), ctypes.byref(flags), 1)
+    finally:
+        V.tri_test_skip_tile(-1)
+    assert st == 6                               # TRI_ERR_DEVICE_TIMEOUT
+    assert flags.value & tri.DEVFLAG_TIMEOUT
+    # the same device, the next call: clean and right
+    w2, scores, status = tm.run_max(cache, tm.GEO17)
+    assert status == 0
+    w64 = tm.check_offset_weights(w2, cache, tm.GEO17, 0.0, 0)
+    H = wl.num_kv_heads
+    for (l, h, b) in [(0, 0, 0), (wl.num_layers - 1, H - 1, wl.batch - 1)]:
+        tm.check_unit_max(cache, scores, w64, l, h, b, tm.GEO17, 0.0, 0, subset=1024)
+    assert not torch.isnan(scores[:, :max(cache.lens)]).any()
 
 
 def _same(a, b):
