@@ -163,6 +163,20 @@ def test_score_max_full_qwen3_sampled():
     assert not torch.isnan(scores).any()
 
 
+def test_score_max_paged_full_steady_rows_sampled():
+    """Config 5's steady-round rows as the bench scores them (28 layers x 4 KV
+    heads x 64 sequences x 2176 keys in 16-token pages, whole-page tiles):
+    sampled units against the oracle, and every key of every unit written."""
+    wl = gen.WORKLOADS["qwen25_paged"]
+    cache = gen.make_cache(wl, seed=5, device=DEV, with_values=False, lens=[2176] * wl.batch)
+    w, scores, status = run_max(cache, GEO17)
+    assert status == 0
+    w64 = check_offset_weights(w, cache, GEO17, 0.0, 0)
+    for (l, h, b) in [(0, 0, 0), (13, 2, 37), (27, 3, 63)]:
+        check_unit_max(cache, scores, w64, l, h, b, GEO17, 0.0, 0, subset=1024)
+    assert not torch.isnan(scores[:, :2176]).any()
+
+
 @pytest.mark.parametrize("group", [2, 4, 8])
 def test_gqa_group_aggregation(group):
     """Grouped-query attention: several query heads share a KV head.  The
