@@ -118,6 +118,26 @@ def test_score_max_paged(H, bs, n_off):
     assert torch.isnan(scores[:, 1000:]).all()          # row padding untouched
 
 
+@pytest.mark.parametrize("H,bs", [(4, 16), (1, 8), (8, 8)])    # whole pages x2, one head
+def test_score_max_paged_empty_sequences(H, bs):
+    """Sequences without keys among others: the tile walk steps past them."""
+    wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, num_kv_heads=H, batch=6, block_size=bs,
+                    spare_blocks_per_seq=1)
+    lens = [0, 300, 0, 0, 17, 129]
+    cache = gen.make_cache(wl, seed=40 + H + bs, device=DEV, with_values=False, lens=lens)
+    w, scores, status = run_max(cache, GEO17)
+    assert status == 0
+    w64 = check_offset_weights(w, cache, GEO17, 0.0, 0)
+    for l in range(wl.num_layers):
+        for h in range(H):
+            for b in range(wl.batch):
+                check_unit_max(cache, scores, w64, l, h, b, GEO17, 0.0, 0)
+    for b, n in enumerate(lens):                                  # nothing past each row's keys
+        for l in range(wl.num_layers):
+            for h in range(H):
+                assert torch.isnan(scores[parity.unit_id(wl, l, h, b), n:]).all()
+
+
 @pytest.mark.parametrize("H", [4, 8])                      # whole-page tiles, one-head tiles
 def test_score_max_paged_bad_page_is_flagged_not_fatal(H):
     import rope_aware_key_b200 as tri
