@@ -995,24 +995,37 @@ def run_reference(args):
     oracle_unit_pipeline(orc, kb, vb, qc, wl, min(wl.budget, probe_n), threads, args.variant)
     rate = probe_n / max(time.time() - t, 1e-6)
     per_step_s = min(1.0, 120.0 / max(1, args.steps + args.warmup))
-    n = int(min(32768, max(256, rate * per_step_s)))
+    paged = wl.layout == "paged"
+    if paged:
+        # a paged cache is timed in its steady rounds: units of B + PAGED_APPEND
+        # keys, as many per step as fill the step's time
+        n = wl.budget + PAGED_APPEND
+        units = int(min(64, max(1, rate * per_step_s / n)))
+    else:
+        n = int(min(32768, max(256, rate * per_step_s)))
+        units = 1
     kb, vb, qc = cpu_sample(wl, n, args.seed)
     B = min(wl.budget, n)
+
+    def step():
+        for _ in range(units):
+            oracle_unit_pipeline(orc, kb, vb, qc, wl, B, threads, args.variant)
     for _ in range(args.warmup):
-        oracle_unit_pipeline(orc, kb, vb, qc, wl, B, threads, args.variant)
+        step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_unit_pipeline(orc, kb, vb, qc, wl, B, threads, args.variant)
+        step()
     dt = time.perf_counter() - t0
-    value = n * args.steps / dt
+    value = n * units * args.steps / dt
     kind = {"mean": "literal average", "max": "literal max", "pos": "literal average at per-key distances"}
-    sample = (f"each step: one unit of {n} keys of the {args.workload} workload ({kind[args.variant]} over "
-              f"|D|={len(wl.offsets)} offsets, select B={B}, gather K and V), fp64")
+    sample = (f"each step: {units} unit(s) of {n} keys of the {args.workload} workload ({kind[args.variant]} "
+              f"over |D|={len(wl.offsets)} offsets, select B={B}, {'hole fill' if paged else 'gather'} K and V), "
+              f"fp64")
     return {"impl": "reference", "metric": METRICS[args.variant],
             "value": value, "unit": "keys/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)",
-            "config": {"workload": args.workload, "keys_per_step": n, "budget": B},
+            "config": {"workload": args.workload, "keys_per_step": n * units, "budget": B},
             "cpu_baseline": {"value": value, "unit": "keys/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
