@@ -509,9 +509,9 @@ def run_paged(args, tri, dev, rank, ws):
     """The paged serving cache: an initial pruning event, then steady rounds
     (append PAGED_APPEND tokens per sequence, untimed; re-compress in place).
     The initial event is four calls (fold, score, select, in-place hole fill),
-    a steady round two (fold, tri_compress in place) for the folded score, and
-    four for the max over the offsets (per-offset fold, score_keys_max,
-    select, in-place hole fill: tri_compress runs the folded score only).
+    a steady round two: the fold and tri_compress in place for the folded
+    score, the per-offset fold and tri_compress_max for the max over the
+    offsets.
     Every event is queued behind a GPU sleep so that the launches are all
     waiting when the first one runs, and timed with CUDA events on the
     launching stream; L2 is flushed (a 512 MB fill) before every event."""
@@ -572,30 +572,18 @@ def run_paged(args, tri, dev, rank, ws):
         rec(4)
 
     def steady(d, evs=None, score_alone=None):
-        """A steady round: the fold, then tri_compress in place (score, then a
-        warp per row that selects and fills the row's holes).  score_alone: a
-        score matrix; the scorer and then the selection (without the fill) run
-        on their own first, each timed (the breakdown round; compress then
-        redoes both).  The max over the offsets: per-offset fold, then the
-        scorer, the selection and the in-place hole fill as three calls into
-        score_alone.  evs: events around each call."""
+        """A steady round: the fold, then tri_compress (tri_compress_max for
+        the max over the offsets) in place: score, then a warp per row that
+        selects and fills the row's holes.  score_alone: a score matrix; the
+        scorer and then the selection (without the fill) run on their own
+        first, each timed (the breakdown round; the compress call then redoes
+        both).  evs: events around each call."""
         nonlocal ws_buf
         marks = iter(evs or [])
 
         def rec():
             if evs is not None:
                 next(marks).record(stream)
-        if use_max:
-            rec()
-            fold()
-            rec()
-            tri.score_keys_max(d, w, score_alone, stream=stream)
-            rec()
-            tri.select_topk(d, score_alone, B, kept, cnt, stream=stream)
-            rec()
-            tri.compact_kv(d, kept, cnt, B, tri.COMPACT_IN_PLACE_HOLEFILL, None, None, stream=stream)
-            rec()
-            return
         need = tri.workspace_size(d, B)
         if ws_buf is None or ws_buf.numel() < need:
             ws_buf = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -603,11 +591,14 @@ def run_paged(args, tri, dev, rank, ws):
         fold()
         rec()
         if score_alone is not None:
-            tri.score_keys(d, w, score_alone, stream=stream)
+            score(d, score_alone)
             rec()
             tri.select_topk(d, score_alone, B, kept, cnt, stream=stream)
             rec()
-        tri.compress(d, w, B, tri.COMPACT_IN_PLACE_HOLEFILL, kept, cnt, None, None, ws_buf, stream=stream)
+        if use_max:
+            tri.compress_max(d, w, B, tri.COMPACT_IN_PLACE_HOLEFILL, kept, cnt, None, None, ws_buf, stream=stream)
+        else:
+            tri.compress(d, w, B, tri.COMPACT_IN_PLACE_HOLEFILL, kept, cnt, None, None, ws_buf, stream=stream)
         rec()
 
     def timed(fn, n_events):
@@ -654,10 +645,7 @@ def run_paged(args, tri, dev, rank, ws):
                 torch.distributed.barrier()
             t0 = time.time()
             launches0 = tri.kernel_launches()
-        if use_max:
-            per, moved = timed(lambda evs: steady(d, evs, score_alone=scores), 5)
-        else:
-            per, moved = timed(lambda evs: steady(d, evs), 3)
+        per, moved = timed(lambda evs: steady(d, evs), 3)
         if i >= args.warmup:
             rounds.append((per, moved, sum(cache.lens) * L * H))
         gen.release_tail_blocks(cache, [min(B, n) for n in cache.lens])
@@ -666,10 +654,9 @@ def run_paged(args, tri, dev, rank, ws):
     sampler.stop()
     clocks = sampler.summary(t0, t1)
     clocks["window"] = "the steady rounds, appends between them included"
-    # breakdown rounds (folded score): the scorer alone, then the same round;
-    # the max rounds are four calls, timed one by one already
+    # breakdown rounds: the scorer alone, then the same round
     per1 = []
-    for j in range(0 if use_max else PAGED_BREAKDOWN_ROUNDS):
+    for j in range(PAGED_BREAKDOWN_ROUNDS):
         gen.append_tokens(cache, PAGED_APPEND, step=1 + args.warmup + args.steps + j)
         d = tri.desc_paged(cache.k, cache.v, cache.block_table, cache.lens)
         per1.append(timed(lambda evs: steady(d, evs, score_alone=scores), 5)[0])
@@ -679,7 +666,7 @@ def run_paged(args, tri, dev, rank, ws):
     if st:
         raise RuntimeError(f"device status {st:#x} after the steady rounds")
 
-    per = np.array([r[0] for r in rounds])       # ms: fold, compress (max: fold, score, select, hole fill)
+    per = np.array([r[0] for r in rounds])       # ms: fold, compress
     ms_rounds = float(per.sum())
     ms_max = max_over_ranks(ms_rounds, ws, dev)
     keys_round = rounds[0][2]
@@ -687,7 +674,7 @@ def run_paged(args, tri, dev, rank, ws):
     value = keys_round * len(rounds) * ws / (ms_max / 1e3)
     ms_step = ms_max / len(rounds)
     peak, peak_kind = measured_hbm_peak()
-    score_ms = float(per[:, 1].mean()) if use_max else float(per1[:, 1].mean())
+    score_ms = float(per1[:, 1].mean())
     score_bytes = keys_round * KEY_BYTES
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     step_bytes = keys_round * KEY_BYTES + moved * MOVE_BYTES
@@ -695,8 +682,7 @@ def run_paged(args, tri, dev, rank, ws):
     init_ms = float(sum(per0))
     init_bytes = keys0 * KEY_BYTES + moved0 * MOVE_BYTES
 
-    e2e = run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws,
-                        lambda dd: steady(dd, score_alone=scores if use_max else None))
+    e2e = run_paged_e2e(args, tri, cache, wl, qc, kept, cnt, stream, ws, lambda dd: steady(dd))
 
     result = None
     if rank == 0:
@@ -714,18 +700,16 @@ def run_paged(args, tri, dev, rank, ws):
                        "keys_per_gpu": keys_round, "budget": B, "parallelism": f"independent caches x{ws}",
                        "l2": "L2 flushed before every pruning event, outside the events: a 512 MB buffer "
                              "written then read back (the write's dirty lines drain before the event)"},
-            "step_breakdown_ms": ({"fold (per offset)": float(per[:, 0].mean()), "score": score_ms,
-                                   "select": float(per[:, 2].mean()), "hole fill": float(per[:, 3].mean()),
-                                   "breakdown": "the timed rounds' four calls, one event each"} if use_max else
-                                  {"fold": float(per[:, 0].mean()), "compress": float(per[:, 1].mean()),
-                                   "score (alone)": score_ms,
-                                   "select alone (no fill, scores fresh in L2)": float(per1[:, 2].mean()),
-                                   "select + hole fill (compress minus score alone)":
-                                       float(per[:, 1].mean()) - score_ms,
-                                   "breakdown": f"score alone, select alone: {PAGED_BREAKDOWN_ROUNDS} more "
-                                                "rounds, each with the scorer and then the selection run on "
-                                                "their own (after the flush) before the compress call; select + "
-                                                "hole fill: the timed rounds' compress minus the scorer alone"}),
+            "step_breakdown_ms": {("fold (per offset)" if use_max else "fold"): float(per[:, 0].mean()),
+                                  ("compress_max" if use_max else "compress"): float(per[:, 1].mean()),
+                                  "score (alone)": score_ms,
+                                  "select alone (no fill, scores fresh in L2)": float(per1[:, 2].mean()),
+                                  "select + hole fill (compress minus score alone)":
+                                      float(per[:, 1].mean()) - score_ms,
+                                  "breakdown": f"score alone, select alone: {PAGED_BREAKDOWN_ROUNDS} more "
+                                               "rounds, each with the scorer and then the selection run on "
+                                               "their own (after the flush) before the compress call; select + "
+                                               "hole fill: the timed rounds' compress minus the scorer alone"},
             "rows_moved_per_step": moved,
             "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_gbs,
                     "frac_of_measured": step_gbs / peak, "frac_of_8tbps_spec": step_gbs / SPEC_HBM_GBS},
@@ -743,10 +727,8 @@ def run_paged(args, tri, dev, rank, ws):
                          "algorithmic_bytes_per_launch": score_bytes},
             "clocks": clocks,
             "gpu_launches": int(launches),
-            "timing": ("each round: plain launches queued behind a GPU sleep, CUDA events around each of the "
-                       "four calls" if use_max else
-                       "each round: plain launches queued behind a GPU sleep, CUDA events around the fold and "
-                       "the compress call"),
+            "timing": "each round: plain launches queued behind a GPU sleep, CUDA events around the fold and "
+                      "the compress call",
             "e2e": e2e,
             "cpu_baseline": cpu,
         }

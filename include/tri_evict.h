@@ -305,6 +305,22 @@ tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B,
  * (16 MiB per device). */
 #define TRI_NOALLOC_MAX_SCORES (4 * 1024 * 1024)
 
+/* The three steps of tri_compress with the max-over-offsets score of
+ * tri_score_keys_max in place of the folded one (same page: "What it saves,
+ * and what it does not" for the score, which does not fold; opening section
+ * for keeping the highest-scoring keys and evicting the rest):
+ * w and n_offsets as for tri_score_keys_max (device fp32
+ * [L*H][n_offsets][128], from tri_fold_offset_weights); B, mode, kept,
+ * kept_count, k_out, v_out, the workspace (tri_workspace_size bytes, 256-byte
+ * aligned; it receives the score matrix), the results and the errors as for
+ * tri_compress, and the layouts those tri_score_keys_max takes.  Runs the max
+ * scorer, then the selection (in place, on rows that move at most 512 keys,
+ * with the hole fill in the same warp) and the compaction; every check is made
+ * on the host before the first launch. */
+tri_status tri_compress_max(const tri_cache_desc* desc, const float* w, int n_offsets, int B,
+                            tri_compact_mode mode, int32_t* kept, int32_t* kept_count, void* k_out, void* v_out,
+                            void* workspace, size_t workspace_bytes, tri_stream_t stream);
+
 /* tri_compress without a caller-provided workspace.  The pages have no
  * counterpart of this call: it exists for callers that cannot allocate
  * device memory where they compress -- for instance a serving engine that

@@ -104,6 +104,7 @@ def load(path: str) -> ctypes.CDLL:
     L.tri_compact_kv.argtypes = [D, P, P, I, I, P, P, P]
     L.tri_workspace_size.argtypes = [D, I, ctypes.POINTER(S)]
     L.tri_compress.argtypes = [D, P, I, I, P, P, P, P, P, S, P]
+    L.tri_compress_max.argtypes = [D, P, I, I, I, P, P, P, P, P, S, P]
     L.tri_read_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32), I]
     L.tri_status_string.argtypes = [I]
     L.tri_status_string.restype = ctypes.c_char_p
@@ -112,7 +113,7 @@ def load(path: str) -> ctypes.CDLL:
     L.tri_version.restype = ctypes.c_char_p
     for name in ("tri_fold_weights", "tri_fold_offset_weights", "tri_score_keys_max", "tri_score_keys",
                  "tri_score_keys_at_positions", "tri_select_topk", "tri_compact_kv", "tri_workspace_size",
-                 "tri_compress", "tri_read_device_status"):
+                 "tri_compress", "tri_compress_max", "tri_read_device_status"):
         getattr(L, name).restype = I
     return L
 
@@ -374,6 +375,33 @@ def compress(d: Desc, w: torch.Tensor, budget: int, mode: int = COMPACT_OUT_OF_P
     _check(lib().tri_compress(d.ref, _ptr(w), int(budget), int(mode), _ptr(kept), _ptr(kept_count), _ptr(k_out),
                               _ptr(v_out), _ptr(workspace), workspace.numel(), _stream(stream, dev)),
            "tri_compress")
+    return kept, kept_count
+
+
+def compress_max(d: Desc, w_offsets: torch.Tensor, budget: int, mode: int = COMPACT_OUT_OF_PLACE,
+                 kept: Optional[torch.Tensor] = None, kept_count: Optional[torch.Tensor] = None,
+                 k_out: Optional[torch.Tensor] = None, v_out: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None):
+    """max-over-offsets score -> select -> compact; returns (kept, kept_count)."""
+    dev = w_offsets.device
+    n_off = w_offsets.shape[-2]
+    if kept is None:
+        kept = torch.empty((d.units, budget), dtype=torch.int32, device=dev)
+    if kept_count is None:
+        kept_count = torch.empty((d.units,), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(workspace_size(d, budget), dtype=torch.uint8, device=dev)
+    nb = d.units * max(int(budget), 0)
+    _need(w_offsets, torch.float32, d.num_layers * d.num_kv_heads * n_off * HEAD_DIM, "w_offsets")
+    _need(kept, torch.int32, nb, "kept")
+    _need(kept_count, torch.int32, d.units, "kept_count")
+    _need(k_out, torch.bfloat16, nb * HEAD_DIM, "k_out")
+    _need(v_out, torch.bfloat16, nb * HEAD_DIM, "v_out")
+    _need(workspace, torch.uint8, 0, "workspace")      # its size goes to the library, which checks it
+    _check(lib().tri_compress_max(d.ref, _ptr(w_offsets), int(n_off), int(budget), int(mode), _ptr(kept),
+                                  _ptr(kept_count), _ptr(k_out), _ptr(v_out), _ptr(workspace), workspace.numel(),
+                                  _stream(stream, dev)),
+           "tri_compress_max")
     return kept, kept_count
 
 

@@ -755,6 +755,60 @@ int64_t fill_head_tile_prefix(Geom* g) {
   return int64_t{g->L} * g->H * acc;
 }
 
+// The max scorer's plan for a cache (host checks only, nothing launched):
+// tile form, accumulator columns per head and tile count; g receives the
+// tile prefix of that form.
+struct MaxPlan {
+  bool paged = false, whole = false;
+  int head_cols = 0;      // hi and lo column of every offset, per head, rounded up to 16
+  int64_t rows = 0;       // packed layouts: key rows of the [rows][128] view
+  int64_t ntiles = 0;
+};
+
+tri_status plan_max(const tri_cache_desc* desc, int n_offsets, Geom* g, MaxPlan* mp) {
+  if (n_offsets < 1) return TRI_ERR_INVALID_ARG;
+  if (n_offsets > tri::smax::kMaxOffsets) return TRI_ERR_UNSUPPORTED;
+  mp->paged = desc->layout == TRI_LAYOUT_PAGED;
+  mp->head_cols = (2 * n_offsets + 15) & ~15;
+  // PAGED: whole pages of all heads per tile when every head's weights fit
+  // one MMA (H head_cols <= 256) and a page of all heads fills whole swizzle
+  // atoms (H block_size a power of two >= 8, so whole pages fill the 128
+  // rows); else one head's rows per tile, pages of a power of two >= 8 tokens.
+  mp->whole = mp->paged && g->block_shift >= 0 && g->H * mp->head_cols <= tri::smax::kMaxB &&
+              (g->block_size * g->H) >= 8;
+  if (mp->paged) {
+    if (!mp->whole && g->block_shift < 3) return TRI_ERR_UNSUPPORTED;
+  } else {
+    mp->rows = packed_rows(desc);
+    if (mp->rows <= 0 || mp->rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  }
+  mp->ntiles = mp->paged && !mp->whole ? fill_head_tile_prefix(g) : fill_tile_prefix(g);
+  if (mp->ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+  return TRI_OK;
+}
+
+// Launch the max scorer planned by plan_max (g as plan_max left it).
+tri_status launch_max(const tri_cache_desc* desc, const Geom& g0, const MaxPlan& mp, const float* w, int n_offsets,
+                      float* scores, int dev, cudaStream_t s) {
+  if (mp.ntiles == 0) return TRI_OK;
+  Geom g = g0;
+  CUtensorMap map;
+  tri_status st = mp.paged ? encode_paged_key_map(desc, mp.whole, &map) : encode_key_map(desc, mp.rows, &map);
+  if (st != TRI_OK) return st;
+#ifdef TRI_TEST_HOOKS
+  g.test_skip_tile = g_test_skip_tile.load();
+#endif
+  const int heads = mp.whole ? g.H : 1;
+  tri::smax::Args a{w, scores, static_cast<int>(mp.ntiles), n_offsets, mp.head_cols, heads, __builtin_ctz(heads),
+                    mp.whole ? 1 : 0};
+  const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].smax_blocks_per_sm;
+  const int grid = static_cast<int>(mp.ntiles < resident ? mp.ntiles : resident);
+  tri::smax::score_max_kernel<<<grid, tri::smax::kThreads, tri::smax::kSmemBytes, s>>>(g, map, a);
+  ++g_launches;
+  TRI_CUDA(cudaGetLastError());
+  return TRI_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -774,46 +828,16 @@ tri_status tri_score_keys_max(const tri_cache_desc* desc, const float* w, int n_
   Geom g;
   tri_status st = make_geom(desc, false, &g);
   if (st != TRI_OK) return st;
-  if (!w || !scores || !aligned16(w) || !aligned16(scores) || n_offsets < 1) return TRI_ERR_INVALID_ARG;
-  if (n_offsets > tri::smax::kMaxOffsets) return TRI_ERR_UNSUPPORTED;
-  const bool paged = desc->layout == TRI_LAYOUT_PAGED;
-  const int head_cols = (2 * n_offsets + 15) & ~15;   // hi and lo column of every offset, per head
-  int64_t rows = 0;
-  // PAGED: whole pages of all heads per tile when every head's weights fit
-  // one MMA (H head_cols <= 256) and a page of all heads fills whole swizzle
-  // atoms (H block_size a power of two >= 8, so whole pages fill the 128
-  // rows); else one head's rows per tile, pages of a power of two >= 8 tokens.
-  const bool whole = paged && g.block_shift >= 0 && g.H * head_cols <= tri::smax::kMaxB &&
-                     (g.block_size * g.H) >= 8;
-  if (paged) {
-    if (!whole && g.block_shift < 3) return TRI_ERR_UNSUPPORTED;
-  } else {
-    rows = packed_rows(desc);
-    if (rows <= 0 || rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
-  }
-  const int64_t ntiles = paged && !whole ? fill_head_tile_prefix(&g) : fill_tile_prefix(&g);
-  if (ntiles > INT32_MAX) return TRI_ERR_UNSUPPORTED;
-  if (ntiles == 0) return TRI_OK;
+  if (!w || !scores || !aligned16(w) || !aligned16(scores)) return TRI_ERR_INVALID_ARG;
+  MaxPlan mp;
+  st = plan_max(desc, n_offsets, &g, &mp);
+  if (st != TRI_OK) return st;
+  if (mp.ntiles == 0) return TRI_OK;
   DeviceScope scope;   // the caller's current device comes back when the call returns
   int dev;
   st = use_device_of(desc->k, &dev, &scope);
   if (st != TRI_OK) return st;
-  CUtensorMap map;
-  st = paged ? encode_paged_key_map(desc, whole, &map) : encode_key_map(desc, rows, &map);
-  if (st != TRI_OK) return st;
-#ifdef TRI_TEST_HOOKS
-  g.test_skip_tile = g_test_skip_tile.load();
-#endif
-  const int heads = whole ? g.H : 1;
-  tri::smax::Args a{w, scores, static_cast<int>(ntiles), n_offsets, head_cols, heads, __builtin_ctz(heads),
-                    whole ? 1 : 0};
-  const int64_t resident = int64_t{g_dev[dev].sms} * g_dev[dev].smax_blocks_per_sm;
-  const int grid = static_cast<int>(ntiles < resident ? ntiles : resident);
-  tri::smax::score_max_kernel<<<grid, tri::smax::kThreads, tri::smax::kSmemBytes,
-                                reinterpret_cast<cudaStream_t>(stream)>>>(g, map, a);
-  ++g_launches;
-  TRI_CUDA(cudaGetLastError());
-  return TRI_OK;
+  return launch_max(desc, g, mp, w, n_offsets, scores, dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
 tri_status tri_score_keys_at_positions(const tri_cache_desc* desc, const float* w, double theta,
@@ -1007,6 +1031,43 @@ tri_status tri_compress_noalloc(const tri_cache_desc* desc, const float* w, int 
   }
   return run_compress(g, plan, w, B, mode, kept, kept_count, k_out, v_out, scores, dev,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+tri_status tri_compress_max(const tri_cache_desc* desc, const float* w, int n_offsets, int B,
+                            tri_compact_mode mode, int32_t* kept, int32_t* kept_count, void* k_out, void* v_out,
+                            void* workspace, size_t workspace_bytes, tri_stream_t stream) {
+  Geom g;
+  tri_status st = make_geom(desc, true, &g);
+  if (st != TRI_OK) return st;
+  if (!w || !aligned16(w)) return TRI_ERR_INVALID_ARG;
+  st = check_compact_args(desc, kept, kept_count, B, mode, k_out, v_out);
+  if (st != TRI_OK) return st;
+  size_t need = 0;
+  st = tri_workspace_size(desc, B, &need);
+  if (st != TRI_OK) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return TRI_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return TRI_ERR_WORKSPACE;
+  SelectPlan plan;
+  st = compress_checks(g, B, mode, &plan);
+  if (st != TRI_OK) return st;
+  Geom gm = g;
+  MaxPlan mp;
+  st = plan_max(desc, n_offsets, &gm, &mp);
+  if (st != TRI_OK) return st;
+  DeviceScope scope;   // the caller's current device comes back when the call returns
+  int dev;
+  st = use_device_of(desc->k, &dev, &scope);
+  if (st != TRI_OK) return st;
+  st = check_values(desc, dev, mode, &g);
+  if (st != TRI_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* scores = static_cast<float*>(workspace);
+  st = launch_max(desc, gm, mp, w, n_offsets, scores, dev, s);
+  if (st != TRI_OK) return st;
+  const bool fill = fill_in_select(g, plan, B, mode);
+  st = launch_select(g, plan, scores, B, kept, kept_count, s, fill);
+  if (st != TRI_OK || fill) return st;
+  return launch_compact(g, kept, kept_count, B, mode, k_out, v_out, dev, s);
 }
 
 tri_status tri_read_device_status(tri_stream_t stream, uint32_t* flags, int clear) {

@@ -156,6 +156,31 @@ def test_compress_workspace_checked_on_host(L):
     assert st == 1      # workspace not 256-byte aligned
 
 
+def test_compress_max_checked_on_host(L):
+    """tri_compress_max: its workspace, the max scorer's limits and the
+    compaction's checks are made before anything is launched (no GPU here)."""
+    d = contig()
+    P = ctypes.c_void_p
+    need = ctypes.c_size_t(0)
+    L.tri_workspace_size(ctypes.byref(d), 64, ctypes.byref(need))
+    n0 = L.tri_kernel_launches()
+    args = (P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE))
+    assert L.tri_compress_max(ctypes.byref(d), P(FAKE), 17, 64, 0, *args, need.value - 1, None) == 3
+    assert L.tri_compress_max(ctypes.byref(d), P(FAKE), 17, 64, 0, P(FAKE), P(FAKE), P(FAKE), P(FAKE),
+                              P(FAKE + 16), need.value, None) == 1      # workspace not 256-byte aligned
+    assert L.tri_compress_max(ctypes.byref(d), P(FAKE), 65, 64, 0, *args, need.value, None) == 2   # offsets
+    assert L.tri_compress_max(ctypes.byref(d), P(FAKE), 0, 64, 0, *args, need.value, None) == 1
+    assert L.tri_compress_max(ctypes.byref(d), P(FAKE), 17, 0, 0, *args, need.value, None) == 1    # B < 1
+    loose = contig(stride_head=1000 * 128 + 64, stride_layer=8 * (1000 * 128 + 64))
+    L.tri_workspace_size(ctypes.byref(loose), 64, ctypes.byref(need))
+    assert L.tri_compress_max(ctypes.byref(loose), P(FAKE), 17, 64, 0, *args, need.value, None) == 2  # not packed
+    pg = paged(block_size=12, stride_block=12 * 4 * 128, stride_layer=100 * 12 * 4 * 128)
+    L.tri_workspace_size(ctypes.byref(pg), 8, ctypes.byref(need))
+    assert L.tri_compress_max(ctypes.byref(pg), P(FAKE), 17, 8, 1, P(FAKE), P(FAKE), None, None, P(FAKE),
+                              need.value, None) == 2                                        # pages of 12
+    assert L.tri_kernel_launches() == n0
+
+
 def test_compress_refuses_before_any_launch(L):
     """More score tiles than an int32 counts (65536 heads x 2^24 keys) is
     refused by both compress calls before the scorer runs: the status is

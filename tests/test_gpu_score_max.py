@@ -197,6 +197,63 @@ def test_score_max_paged_full_steady_rows_sampled():
     assert not torch.isnan(scores[:, :2176]).any()
 
 
+def _max_calls(tri, d, w, B, mode, units, one_call):
+    kept = torch.full((units, B), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.full((units,), -1, dtype=torch.int32, device=DEV)
+    ko = vo = None
+    if mode == tri.COMPACT_OUT_OF_PLACE:
+        ko = torch.zeros((units, B, 128), dtype=torch.bfloat16, device=DEV)
+        vo = torch.zeros_like(ko)
+    if one_call:
+        tri.compress_max(d, w, B, mode, kept, cnt, ko, vo)
+    else:
+        sc = tri.score_keys_max(d, w)
+        tri.select_topk(d, sc, B, kept, cnt)
+        tri.compact_kv(d, kept, cnt, B, mode, ko, vo)
+    assert tri.read_device_status(clear=True) == 0
+    return kept, cnt, ko, vo
+
+
+@pytest.mark.parametrize("case", ["contig", "ragged", "paged_in_place", "paged_in_place_long"])
+def test_compress_max_equals_the_three_calls(case):
+    """tri_compress_max: the max scorer, then the selection (in place on short
+    rows with the hole fill in the same warp) and the compaction, bit for bit
+    the same as tri_score_keys_max + tri_select_topk + tri_compact_kv."""
+    import rope_aware_key_b200 as tri
+    mode = tri.COMPACT_OUT_OF_PLACE
+    lens = None
+    if case == "contig":
+        wl = gen.scaled(gen.WORKLOADS["qwen3_layer"], num_kv_heads=4, seq_len=4096, budget=700)
+    elif case == "ragged":
+        wl = gen.scaled(gen.WORKLOADS["qwen3_ragged"], num_layers=2, num_kv_heads=2, batch=5, budget=300)
+        lens = [900, 5000, 77, 0, 301]
+    else:
+        mode = tri.COMPACT_IN_PLACE_HOLEFILL
+        wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, batch=8, spare_blocks_per_seq=1)
+        # B + 128 keys per row (the fill runs in the selection), or rows that move more than 512
+        lens = [2176] * 8 if case == "paged_in_place" else [3000, 2176, 2047, 2900, 2600, 2048, 0, 3100]
+    res = []
+    for one_call in (True, False):
+        cache = gen.make_cache(wl, seed=71, device=DEV, lens=lens)
+        d = parity.make_desc(cache)
+        qc = cache.query_center.reshape(-1, wl.head_dim).to(DEV).contiguous()
+        w = tri.fold_offset_weights(qc, wl.theta, GEO17)
+        out = _max_calls(tri, d, w, wl.budget, mode, d.units, one_call)
+        torch.cuda.synchronize()
+        res.append((out, cache))
+    (a, ca), (b, cb) = res
+    assert torch.equal(a[1], b[1])
+    valid = torch.arange(wl.budget, device=DEV)[None, :] < a[1][:, None]
+    assert torch.equal(torch.where(valid, a[0], 0), torch.where(valid, b[0], 0))
+    if mode == tri.COMPACT_OUT_OF_PLACE:
+        v3 = valid[:, :, None]
+        for x, y in ((a[2], b[2]), (a[3], b[3])):
+            assert torch.equal(torch.where(v3, x.view(torch.int16), 0), torch.where(v3, y.view(torch.int16), 0))
+    else:                                   # the pools after the in-place fills
+        assert torch.equal(ca.k.view(torch.int16), cb.k.view(torch.int16))
+        assert torch.equal(ca.v.view(torch.int16), cb.v.view(torch.int16))
+
+
 @pytest.mark.parametrize("group", [2, 4, 8])
 def test_gqa_group_aggregation(group):
     """Grouped-query attention: several query heads share a KV head.  The
