@@ -335,7 +335,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     ws_buf = None
     if args.path == "compress":
-        assert args.variant == "mean", "--path compress runs the folded score"
+        assert args.variant != "pos", "--path compress runs the folded score or the max over the offsets"
         ws_buf = torch.empty(tri.workspace_size(d, B), dtype=torch.uint8, device=dev)
     positions = qpos = None
     if args.variant == "pos":
@@ -354,7 +354,11 @@ def run_ours(args):
             ev[1].record(st)
         if args.path == "compress":
             # one call: the single-kernel step when the units fit one wave of clusters, else three kernels
-            tri.compress(d, w, B, tri.COMPACT_OUT_OF_PLACE, kept, cnt, k_out, v_out, ws_buf, stream=st)
+            # (the max over the offsets: its scorer, then the selection and the gather)
+            if args.variant == "max":
+                tri.compress_max(d, w, B, tri.COMPACT_OUT_OF_PLACE, kept, cnt, k_out, v_out, ws_buf, stream=st)
+            else:
+                tri.compress(d, w, B, tri.COMPACT_OUT_OF_PLACE, kept, cnt, k_out, v_out, ws_buf, stream=st)
             if ev is not None:
                 for e in ev[2:]:
                     e.record(st)
@@ -489,7 +493,9 @@ def run_ours(args):
             "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_gbs,
                     "frac_of_measured": step_gbs / peak, "frac_of_8tbps_spec": step_gbs / SPEC_HBM_GBS},
             "roofline": {"kernel": (SCORE_KERNELS[args.variant][0] if args.path == "calls" else
-                                    f"tri_compress ({launches_per_step - 1} kernel(s))"), "bound": "hbm", "achieved": achieved, "peak": peak,
+                                    f"{'tri_compress_max' if args.variant == 'max' else 'tri_compress'} "
+                                    f"({launches_per_step - 1} kernel(s))"), "bound": "hbm", "achieved": achieved,
+                         "peak": peak,
                          "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic if args.path == "calls" else None,
                          "algorithmic_bytes_per_launch": score_bytes},
@@ -854,7 +860,10 @@ def run_e2e(args, tri, cache, d, wl, qc, w, kept, cnt, k_out, v_out, stream, job
         if hpos is not None:
             positions.copy_(hpos, non_blocking=True)
         stream.wait_event(copied[j])            # buffer j's previous copy-out is done
-        if args.path == "compress":
+        if args.path == "compress" and args.variant == "max":
+            tri.fold_offset_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
+            tri.compress_max(d, w, B, tri.COMPACT_OUT_OF_PLACE, kp, cn, ko, vo, ws_e2e, stream=stream)
+        elif args.path == "compress":
             tri.fold_weights(qc, wl.theta, wl.offsets, wl.delta0, tri.PAIRING_HALF, out=w, stream=stream)
             tri.compress(d, w, B, tri.COMPACT_OUT_OF_PLACE, kp, cn, ko, vo, ws_e2e, stream=stream)
         else:
@@ -1042,7 +1051,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time plain launches instead of a CUDA graph of the step")
     ap.add_argument("--path", default="calls", choices=["calls", "compress"],
-                    help="calls: fold, score, select, compact as four calls (default); compress: fold + tri_compress")
+                    help="calls: fold, score, select, compact as four calls (default); compress: fold + "
+                         "tri_compress (tri_compress_max with --variant max)")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "layers"],
                     help="N > 1: replicas (default): every rank compresses its own cache (weak scaling); "
                          "layers: one cache split by whole layers over the ranks (strong scaling)")
