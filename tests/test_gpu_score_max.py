@@ -214,7 +214,7 @@ def _max_calls(tri, d, w, B, mode, units, one_call):
     return kept, cnt, ko, vo
 
 
-@pytest.mark.parametrize("case", ["contig", "ragged", "paged_in_place", "paged_in_place_long"])
+@pytest.mark.parametrize("case", ["contig", "ragged", "paged_out_of_place", "paged_in_place", "paged_in_place_long"])
 def test_compress_max_equals_the_three_calls(case):
     """tri_compress_max: the max scorer, then the selection (in place on short
     rows with the hole fill in the same warp) and the compaction, bit for bit
@@ -227,6 +227,9 @@ def test_compress_max_equals_the_three_calls(case):
     elif case == "ragged":
         wl = gen.scaled(gen.WORKLOADS["qwen3_ragged"], num_layers=2, num_kv_heads=2, batch=5, budget=300)
         lens = [900, 5000, 77, 0, 301]
+    elif case == "paged_out_of_place":
+        wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, batch=4, budget=500, spare_blocks_per_seq=1)
+        lens = [2176, 300, 0, 1999]
     else:
         mode = tri.COMPACT_IN_PLACE_HOLEFILL
         wl = gen.scaled(gen.WORKLOADS["qwen25_paged"], num_layers=2, batch=8, spare_blocks_per_seq=1)
