@@ -299,12 +299,6 @@ tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B,
                         void* k_out, void* v_out, void* workspace, size_t workspace_bytes,
                         tri_stream_t stream);
 
-/* ---------------------------------------------------------------- no allocation */
-
-/* Capacity, in floats, of the built-in score scratch of tri_compress_noalloc
- * (16 MiB per device). */
-#define TRI_NOALLOC_MAX_SCORES (4 * 1024 * 1024)
-
 /* The three steps of tri_compress with the max-over-offsets score of
  * tri_score_keys_max in place of the folded one (same page: "What it saves,
  * and what it does not" for the score, which does not fold; opening section
@@ -320,6 +314,12 @@ tri_status tri_compress(const tri_cache_desc* desc, const float* w, int B,
 tri_status tri_compress_max(const tri_cache_desc* desc, const float* w, int n_offsets, int B,
                             tri_compact_mode mode, int32_t* kept, int32_t* kept_count, void* k_out, void* v_out,
                             void* workspace, size_t workspace_bytes, tri_stream_t stream);
+
+/* ---------------------------------------------------------------- no allocation */
+
+/* Capacity, in floats, of the built-in score scratch of tri_compress_noalloc
+ * (16 MiB per device). */
+#define TRI_NOALLOC_MAX_SCORES (4 * 1024 * 1024)
 
 /* tri_compress without a caller-provided workspace.  The pages have no
  * counterpart of this call: it exists for callers that cannot allocate
