@@ -281,8 +281,15 @@ def run_ours(args):
     import rope_aware_key_b200 as tri
     from rope_aware_key_b200 import build as tri_build
     if tri_build.needs_build():
-        log("building libtri_evict.so (missing or older than its sources)")
-        tri_build.build()
+        # one process builds (the ranks of a torchrun launch take turns on a
+        # lock; the later ones find the library current)
+        import fcntl
+        os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+        with open(os.path.join(ROOT, "_build", ".build.lock"), "w") as lock:
+            fcntl.flock(lock, fcntl.LOCK_EX)
+            if tri_build.needs_build():
+                log("building libtri_evict.so (missing or older than its sources)")
+                tri_build.build()
     ws, rank, local = dist_env()
     if ws > 1:
         import datetime
